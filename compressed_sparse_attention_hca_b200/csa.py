@@ -1,0 +1,223 @@
+"""Thin ctypes binding of libcsa_b200 (include/csa.h): argument marshalling only.
+
+Every function takes torch tensors that already live on the CUDA device,
+passes their data pointers and the current CUDA stream to the C ABI, and
+returns the output tensors.  All arithmetic runs in the library's kernels;
+there is no CPU fallback: if the shared library is missing or a call fails,
+an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+F32, BF16, KV_FP8MIX, IDX_NVFP4 = 0, 1, 2, 3
+_STATUS = {0: "CSA_OK", 1: "CSA_ERR_INVALID_ARG", 2: "CSA_ERR_UNSUPPORTED", 3: "CSA_ERR_CUDA",
+           4: "CSA_ERR_TIMEOUT"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa_b200.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "csa.h")
+_lib = None
+
+
+class CsaError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def header_functions():
+    """Names of the functions declared in include/csa.h."""
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(csa_\w+|hca_\w+)\s*\(", src)))
+
+
+def load():
+    """Load libcsa_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: run `python -m compressed_sparse_attention_hca_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i32, i64, sz, f32 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_float
+    sigs = {
+        "csa_last_error": (ctypes.c_char_p, []),
+        "csa_version": (i32, []),
+        "csa_row_bytes": (i64, [i32, i32]),
+        "csa_compress": (i32, [P, P, P, P, P, P, i32, i64, i64, i64, i64, i64, i32, i32, i32, P, P,
+                               i64, i32, P]),
+        "csa_index_topk_workspace_size": (sz, [i32, i32, i64, i32, i32, i32, i32]),
+        "csa_index_topk": (i32, [P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32, i32, P, P, P,
+                                 sz, P]),
+        "csa_sparse_mqa_workspace_size": (sz, [i32, i32, i32, i32, i32, i32, i32, i32]),
+        "csa_sparse_mqa": (i32, [P, i32, P, i64, P, i32, P, i64, P, P, i32, i32, P, f32, i32, i32,
+                                 i32, i32, i32, P, P, sz, P]),
+        "hca_dense_mqa_workspace_size": (sz, [i32, i32, i32, i32, i64, i32, i32, i32]),
+        "hca_dense_mqa": (i32, [P, i32, P, i64, P, i64, P, P, i32, i32, P, f32, i32, i32, i32, i32,
+                                i32, P, P, sz, P]),
+    }
+    for name, (res, args) in sigs.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    _lib = lib
+    return lib
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(status):
+    if status != 0:
+        raise CsaError(status, load().csa_last_error().decode())
+
+
+def _dt_of(t):
+    return F32 if t.dtype == torch.float32 else BF16
+
+
+def row_bytes(dt, dim):
+    return int(load().csa_row_bytes(dt, dim))
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None and (not t.is_cuda or not t.is_contiguous()):
+            raise ValueError("all tensors must be contiguous CUDA tensors")
+
+
+# --------------------------------------------------------------------- compress
+
+def compress(Ca, Za, Ba, m, Cb=None, Zb=None, Bb=None, *, tok0=0, e0=0, n_out=None, out_dt=None,
+             out=None, out_sf=None, out_row0=0, n_tok=None):
+    """Token-level compressor.  Ca/Za [batch, rows, dim] (F32 or BF16), Ba [m, dim] fp32.
+
+    Entry e0 + j of request b goes to row out_row0 + j of out[b] (out, out_sf:
+    [batch, rows, ...]; allocated when not given).  Returns out (and out_sf for
+    NVFP4)."""
+    _need_cuda(Ca, Za, Ba, Cb, Zb, Bb)
+    batch, rows, dim = Ca.shape
+    n_tok = rows if n_tok is None else n_tok
+    in_dt = _dt_of(Ca)
+    out_dt = in_dt if out_dt is None else out_dt
+    if n_out is None:
+        n_out = (tok0 + n_tok) // m - e0
+    if out is None:
+        stride = n_out + out_row0
+        if out_dt in (F32, BF16):
+            out = torch.empty(batch, stride, dim, device=Ca.device,
+                              dtype=torch.float32 if out_dt == F32 else torch.bfloat16)
+        else:
+            out = torch.empty(batch, stride, row_bytes(out_dt, dim), device=Ca.device, dtype=torch.uint8)
+        if out_dt == IDX_NVFP4:
+            out_sf = torch.empty(batch, stride, dim // 16, device=Ca.device, dtype=torch.uint8)
+    _need_cuda(out, out_sf)
+    stride = out.shape[1]
+    if out_row0 < 0 or out_row0 + n_out > stride:
+        raise ValueError("output rows out of range")
+    rb = out[0, 0].numel() * out.element_size()
+    optr = ctypes.c_void_p(out.data_ptr() + out_row0 * rb)
+    sptr = None if out_sf is None else ctypes.c_void_p(out_sf.data_ptr() + out_row0 * (dim // 16))
+    _check(load().csa_compress(_ptr(Ca), _ptr(Cb), _ptr(Za), _ptr(Zb), _ptr(Ba), _ptr(Bb), batch, n_tok,
+                               tok0, rows, e0, n_out, dim, m, in_dt, optr, sptr, stride, out_dt,
+                               _stream()))
+    return (out, out_sf) if out_dt == IDX_NVFP4 else out
+
+
+# ------------------------------------------------------------------- index top-k
+
+def index_topk_workspace_size(batch, n_q, n_entries, k, n_heads, dim, dt):
+    return int(load().csa_index_topk_workspace_size(batch, n_q, n_entries, k, n_heads, dim, dt))
+
+
+def index_topk(qI, wI, KI, q_pos, m, k, *, dt=None, qI_sf=None, KI_sf=None, n_heads=None,
+               scores=False, idx_out=None, ws=None):
+    """Lightning indexer + top-k.  qI [B, T, H, d] (or NVFP4 codes [B, T, H, d/2]),
+    wI [B, T, H] fp32, KI [B, E, d] (codes [B, E, d/2]), q_pos [B, T] int64.
+
+    Returns idx [B, T, k] int32 (and the score tensor when scores=True)."""
+    _need_cuda(qI, wI, KI, q_pos, qI_sf, KI_sf)
+    if dt is None:
+        dt = IDX_NVFP4 if qI.dtype == torch.uint8 else _dt_of(qI)
+    B, T, H = wI.shape
+    E = KI.shape[1]
+    dim = qI.shape[-1] * (2 if dt == IDX_NVFP4 else 1)
+    dev = qI.device
+    if idx_out is None:
+        idx_out = torch.empty(B, T, k, device=dev, dtype=torch.int32)
+    sc = None
+    if scores:
+        sc = torch.empty(B, T, E, device=dev, dtype=torch.float32 if dt == F32 else torch.bfloat16)
+    need = index_topk_workspace_size(B, T, E, k, H, dim, dt)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(need, device=dev, dtype=torch.uint8)
+    _check(load().csa_index_topk(_ptr(qI), _ptr(qI_sf), _ptr(wI), _ptr(KI), _ptr(KI_sf), _ptr(q_pos),
+                                 B, T, E, m, H, dim, k, dt, _ptr(idx_out), _ptr(sc), _ptr(ws),
+                                 ws.numel(), _stream()))
+    return (idx_out, sc) if scores else idx_out
+
+
+# -------------------------------------------------------------------- attention
+
+def _kv_dt(entries, kv_dt):
+    if kv_dt is not None:
+        return kv_dt
+    return KV_FP8MIX if entries.dtype == torch.uint8 else _dt_of(entries)
+
+
+def sparse_mqa_workspace_size(batch, n_q, n_heads, dim, k, window, q_dt, kv_dt):
+    return int(load().csa_sparse_mqa_workspace_size(batch, n_q, n_heads, dim, k, window, q_dt, kv_dt))
+
+
+def hca_dense_mqa_workspace_size(batch, n_q, n_heads, dim, n_entries, window, q_dt, kv_dt):
+    return int(load().hca_dense_mqa_workspace_size(batch, n_q, n_heads, dim, n_entries, window, q_dt,
+                                                   kv_dt))
+
+
+def sparse_mqa(Q, entries, idx, win, win_start, q_pos, window, m, sink, scale, *, kv_dt=None, O=None,
+               ws=None):
+    """CSA shared-KV MQA.  Q [B, T, H, c]; entries [B, E, row]; idx [B, T, k] int32;
+    win [B, Lw, row]; win_start [B] int64; q_pos [B, T] int64; sink [H] fp32."""
+    _need_cuda(Q, entries, idx, win, win_start, q_pos, sink)
+    B, T, H, c = Q.shape
+    kv_dt = _kv_dt(entries, kv_dt)
+    q_dt = _dt_of(Q)
+    k = idx.shape[-1]
+    if O is None:
+        O = torch.empty_like(Q)
+    need = sparse_mqa_workspace_size(B, T, H, c, k, window, q_dt, kv_dt)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(need, device=Q.device, dtype=torch.uint8)
+    _check(load().csa_sparse_mqa(_ptr(Q), q_dt, _ptr(entries), entries.shape[1], _ptr(idx), k, _ptr(win),
+                                 win.shape[1], _ptr(win_start), _ptr(q_pos), window, m, _ptr(sink),
+                                 float(scale), B, T, H, c, kv_dt, _ptr(O), _ptr(ws), ws.numel(),
+                                 _stream()))
+    return O
+
+
+def hca_dense_mqa(Q, entries, win, win_start, q_pos, window, m, sink, scale, *, kv_dt=None, O=None,
+                  ws=None):
+    """HCA dense shared-KV MQA over every visible entry plus the window."""
+    _need_cuda(Q, entries, win, win_start, q_pos, sink)
+    B, T, H, c = Q.shape
+    kv_dt = _kv_dt(entries, kv_dt)
+    q_dt = _dt_of(Q)
+    if O is None:
+        O = torch.empty_like(Q)
+    need = hca_dense_mqa_workspace_size(B, T, H, c, entries.shape[1], window, q_dt, kv_dt)
+    if ws is None or ws.numel() < need:
+        ws = torch.empty(need, device=Q.device, dtype=torch.uint8)
+    _check(load().hca_dense_mqa(_ptr(Q), q_dt, _ptr(entries), entries.shape[1], _ptr(win), win.shape[1],
+                                _ptr(win_start), _ptr(q_pos), window, m, _ptr(sink), float(scale), B, T,
+                                H, c, kv_dt, _ptr(O), _ptr(ws), ws.numel(), _stream()))
+    return O

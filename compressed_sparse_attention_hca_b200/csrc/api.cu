@@ -1,0 +1,245 @@
+// api.cu -- the C ABI of libcsa_b200 (declared and documented in include/csa.h):
+// host-side argument validation, workspace sizing and dispatch to the
+// kernels.  Nothing here allocates device memory, prints or aborts.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "csa_internal.cuh"
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+csa_status_t fail(csa_status_t st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+csa_status_t ok() {
+  g_err[0] = 0;
+  return CSA_OK;
+}
+
+csa_status_t cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return ok();
+  return fail(CSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+#define REQUIRE(cond, ...)                                  \
+  do {                                                      \
+    if (!(cond)) return fail(CSA_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+
+#define REQUIRE_PTR(p)                                                        \
+  do {                                                                        \
+    if ((p) == nullptr) return fail(CSA_ERR_INVALID_ARG, "%s is NULL", #p);   \
+    if (!aligned16(p)) return fail(CSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p); \
+  } while (0)
+
+#define REQUIRE_ALIGNED_OR_NULL(p)                                            \
+  do {                                                                        \
+    if ((p) != nullptr && !aligned16(p))                                      \
+      return fail(CSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p);     \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char* csa_last_error(void) { return g_err; }
+
+int csa_version(void) { return 100; }
+
+int64_t csa_row_bytes(csa_dtype_t dt, int dim) {
+  if (dim <= 0) return -1;
+  if (dt == CSA_KV_FP8MIX && (dim < 64 || (dim - 64) % 64 != 0)) return -1;
+  if (dt == CSA_IDX_NVFP4 && dim % 16 != 0) return -1;
+  return csa::row_bytes(dt, dim);
+}
+
+csa_status_t csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                          const float* Ba, const float* Bb, int batch, int64_t n_tok,
+                          int64_t tok0, int64_t in_batch_stride, int64_t e0, int64_t n_out,
+                          int dim, int m, csa_dtype_t in_dt, void* out, void* out_sf,
+                          int64_t out_batch_stride, csa_dtype_t out_dt, void* stream) {
+  REQUIRE(batch >= 0 && n_tok >= 0 && tok0 >= 0 && e0 >= 0 && n_out >= 0,
+          "negative size (batch=%d n_tok=%lld tok0=%lld e0=%lld n_out=%lld)", batch,
+          (long long)n_tok, (long long)tok0, (long long)e0, (long long)n_out);
+  REQUIRE(m >= 1 && m <= 4096, "m=%d out of range [1, 4096]", m);
+  REQUIRE(dim >= 8 && dim % 8 == 0, "dim=%d must be a positive multiple of 8", dim);
+  REQUIRE(in_dt == CSA_F32 || in_dt == CSA_BF16, "in_dt must be CSA_F32 or CSA_BF16");
+  REQUIRE(out_dt >= CSA_F32 && out_dt <= CSA_IDX_NVFP4, "unknown out_dt %d", (int)out_dt);
+  if (out_dt == CSA_KV_FP8MIX)
+    REQUIRE(dim >= 128 && (dim - 64) % 64 == 0, "KV_FP8MIX needs dim = 64 + 64*j (j >= 1), got %d", dim);
+  if (out_dt == CSA_IDX_NVFP4) REQUIRE(dim % 16 == 0, "NVFP4 needs dim %% 16 == 0");
+  REQUIRE(in_batch_stride >= n_tok, "in_batch_stride %lld < n_tok %lld", (long long)in_batch_stride,
+          (long long)n_tok);
+  REQUIRE(out_batch_stride >= n_out, "out_batch_stride %lld < n_out %lld",
+          (long long)out_batch_stride, (long long)n_out);
+  if ((int64_t)batch * n_out == 0) return ok();
+  REQUIRE_PTR(Ca);
+  REQUIRE_PTR(Za);
+  REQUIRE_PTR(Ba);
+  REQUIRE_PTR(out);
+  const bool overlap = Cb != nullptr;
+  if (overlap) {
+    REQUIRE_PTR(Zb);
+    REQUIRE_PTR(Bb);
+    REQUIRE_ALIGNED_OR_NULL(Cb);
+  }
+  if (out_dt == CSA_IDX_NVFP4) REQUIRE(out_sf != nullptr, "out_sf is NULL for NVFP4 output");
+  const int64_t first = (overlap && e0 >= 1) ? (int64_t)m * (e0 - 1) : (int64_t)m * e0;
+  const int64_t last = (int64_t)m * (e0 + n_out) - 1;
+  REQUIRE(first >= tok0 && last < tok0 + n_tok,
+          "entries [%lld, %lld) need tokens [%lld, %lld] but rows hold [%lld, %lld)",
+          (long long)e0, (long long)(e0 + n_out), (long long)first, (long long)last,
+          (long long)tok0, (long long)(tok0 + n_tok));
+  csa::CompressArgs a{Ca, Cb, Za, Zb, Ba, Bb, batch, n_tok, tok0, in_batch_stride, e0, n_out,
+                      dim, m, (int)in_dt, (int)out_dt, out, out_sf, out_batch_stride};
+  return cuda_status(csa::launch_compress(a, static_cast<cudaStream_t>(stream)), "csa_compress");
+}
+
+size_t csa_index_topk_workspace_size(int batch, int n_q, int64_t n_entries, int k, int n_heads,
+                                     int dim, csa_dtype_t dt) {
+  if (batch <= 0 || n_q <= 0 || n_entries <= 0 || k <= 0) return 256;
+  size_t s = csa::index_topk_workspace(batch, n_q, n_entries, k, n_heads, dim, (int)dt);
+  return s < 256 ? 256 : s;
+}
+
+csa_status_t csa_index_topk(const void* qI, const void* qI_sf, const float* wI, const void* KI,
+                            const void* KI_sf, const int64_t* q_pos, int batch, int n_q,
+                            int64_t n_entries, int m, int n_heads, int dim, int k, csa_dtype_t dt,
+                            int32_t* idx_out, void* scores_out, void* ws, size_t ws_bytes,
+                            void* stream) {
+  REQUIRE(batch >= 0 && n_q >= 0 && n_entries >= 0, "negative size");
+  REQUIRE(n_entries <= (int64_t)1 << 30, "n_entries=%lld too large", (long long)n_entries);
+  REQUIRE(m >= 1, "m=%d must be >= 1", m);
+  REQUIRE(k >= 1 && k <= 2048, "k=%d out of range [1, 2048]", k);
+  REQUIRE(n_heads >= 1 && n_heads <= 128, "n_heads=%d out of range [1, 128]", n_heads);
+  REQUIRE(dim >= 32 && dim <= 256 && dim % 32 == 0, "dim=%d must be a multiple of 32 in [32, 256]", dim);
+  REQUIRE(dt == CSA_F32 || dt == CSA_BF16 || dt == CSA_IDX_NVFP4, "dt must be F32, BF16 or IDX_NVFP4");
+  if ((int64_t)batch * n_q == 0) return ok();
+  REQUIRE_PTR(qI);
+  REQUIRE_PTR(wI);
+  REQUIRE_PTR(q_pos);
+  REQUIRE_PTR(idx_out);
+  REQUIRE_ALIGNED_OR_NULL(scores_out);
+  if (n_entries > 0) REQUIRE_PTR(KI);
+  if (dt == CSA_IDX_NVFP4) {
+    REQUIRE(qI_sf != nullptr && (KI_sf != nullptr || n_entries == 0), "NVFP4 needs qI_sf and KI_sf");
+  }
+  const size_t need = csa_index_topk_workspace_size(batch, n_q, n_entries, k, n_heads, dim, dt);
+  REQUIRE(ws_bytes >= need, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  REQUIRE_PTR(ws);
+  csa::IndexArgs a{qI, qI_sf, wI, KI, KI_sf, q_pos, batch, n_q, n_entries, m, n_heads, dim, k,
+                   (int)dt, idx_out, scores_out, ws, ws_bytes};
+  return cuda_status(csa::launch_index_topk(a, static_cast<cudaStream_t>(stream)), "csa_index_topk");
+}
+
+}  // extern "C"
+
+namespace {
+
+csa_status_t check_mqa(const csa::MqaArgs& a) {
+  REQUIRE(a.batch >= 0 && a.n_q >= 0 && a.n_entries >= 0 && a.win_len >= 0, "negative size");
+  REQUIRE(a.m >= 1, "m=%d must be >= 1", a.m);
+  REQUIRE(a.window >= 0 && a.window <= 4096, "window=%d out of range [0, 4096]", a.window);
+  REQUIRE(a.n_heads >= 1 && a.n_heads <= 128, "n_heads=%d out of range [1, 128]", a.n_heads);
+  REQUIRE(a.dim >= 64 && a.dim <= 512 && a.dim % 64 == 0, "dim=%d must be a multiple of 64 in [64, 512]",
+          a.dim);
+  REQUIRE(a.q_dt == CSA_F32 || a.q_dt == CSA_BF16, "q_dt must be F32 or BF16");
+  REQUIRE(a.kv_dt == CSA_F32 || a.kv_dt == CSA_BF16 || a.kv_dt == CSA_KV_FP8MIX,
+          "kv_dt must be F32, BF16 or KV_FP8MIX");
+  REQUIRE(a.idx == nullptr || (a.k >= 1 && a.k <= 2048), "k=%d out of range [1, 2048]", a.k);
+  return CSA_OK;
+}
+
+csa_status_t run_mqa(csa::MqaArgs& a, void* stream, const char* name) {
+  csa_status_t st = check_mqa(a);
+  if (st != CSA_OK) return st;
+  if ((int64_t)a.batch * a.n_q == 0) return ok();
+  REQUIRE_PTR(a.Q);
+  REQUIRE_PTR(a.O);
+  REQUIRE_PTR(a.q_pos);
+  REQUIRE_PTR(a.sink);
+  if (a.n_entries > 0) REQUIRE_PTR(a.entries);
+  if (a.window > 0) {
+    REQUIRE_PTR(a.win);
+    REQUIRE_PTR(a.win_start);
+  }
+  const size_t need = csa::mqa_workspace(a);
+  REQUIRE(a.ws_bytes >= need, "workspace too small: %zu < %zu bytes", a.ws_bytes, need);
+  if (need > 0) REQUIRE_PTR(a.ws);
+  return cuda_status(csa::launch_mqa(a, static_cast<cudaStream_t>(stream)), name);
+}
+
+csa::MqaArgs mqa_args(const void* Q, csa_dtype_t q_dt, const void* entries, int64_t n_entries,
+                      const int32_t* idx, int k, const void* win, int64_t win_len,
+                      const int64_t* win_start, const int64_t* q_pos, int window, int m,
+                      const float* sink, float scale, int batch, int n_q, int n_heads, int dim,
+                      csa_dtype_t kv_dt, void* O, void* ws, size_t ws_bytes) {
+  csa::MqaArgs a{};
+  a.Q = Q; a.q_dt = (int)q_dt; a.entries = entries; a.n_entries = n_entries; a.idx = idx; a.k = k;
+  a.win = win; a.win_len = win_len; a.win_start = win_start; a.q_pos = q_pos; a.window = window;
+  a.m = m; a.sink = sink; a.scale = scale; a.batch = batch; a.n_q = n_q; a.n_heads = n_heads;
+  a.dim = dim; a.kv_dt = (int)kv_dt; a.O = O; a.ws = ws; a.ws_bytes = ws_bytes;
+  return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t csa_sparse_mqa_workspace_size(int batch, int n_q, int n_heads, int dim, int k, int window,
+                                     csa_dtype_t q_dt, csa_dtype_t kv_dt) {
+  csa::MqaArgs a = mqa_args(nullptr, q_dt, nullptr, 0, reinterpret_cast<const int32_t*>(16), k,
+                            nullptr, 0, nullptr, nullptr, window, 1, nullptr, 1.f, batch, n_q,
+                            n_heads, dim, kv_dt, nullptr, nullptr, 0);
+  if (check_mqa(a) != CSA_OK || batch <= 0 || n_q <= 0) return 256;
+  const size_t s = csa::mqa_workspace(a);
+  return s < 256 ? 256 : s;
+}
+
+csa_status_t csa_sparse_mqa(const void* Q, csa_dtype_t q_dt, const void* entries,
+                            int64_t n_entries, const int32_t* idx, int k, const void* win,
+                            int64_t win_len, const int64_t* win_start, const int64_t* q_pos,
+                            int window, int m, const float* sink, float softmax_scale, int batch,
+                            int n_q, int n_heads, int dim, csa_dtype_t kv_dt, void* O, void* ws,
+                            size_t ws_bytes, void* stream) {
+  if (idx == nullptr && (int64_t)batch * n_q > 0) return fail(CSA_ERR_INVALID_ARG, "idx is NULL");
+  REQUIRE_ALIGNED_OR_NULL(idx);
+  csa::MqaArgs a = mqa_args(Q, q_dt, entries, n_entries, idx, k, win, win_len, win_start, q_pos,
+                            window, m, sink, softmax_scale, batch, n_q, n_heads, dim, kv_dt, O, ws,
+                            ws_bytes);
+  return run_mqa(a, stream, "csa_sparse_mqa");
+}
+
+size_t hca_dense_mqa_workspace_size(int batch, int n_q, int n_heads, int dim, int64_t n_entries,
+                                    int window, csa_dtype_t q_dt, csa_dtype_t kv_dt) {
+  csa::MqaArgs a = mqa_args(nullptr, q_dt, nullptr, n_entries, nullptr, 0, nullptr, 0, nullptr,
+                            nullptr, window, 1, nullptr, 1.f, batch, n_q, n_heads, dim, kv_dt,
+                            nullptr, nullptr, 0);
+  if (check_mqa(a) != CSA_OK || batch <= 0 || n_q <= 0) return 256;
+  const size_t s = csa::mqa_workspace(a);
+  return s < 256 ? 256 : s;
+}
+
+csa_status_t hca_dense_mqa(const void* Q, csa_dtype_t q_dt, const void* entries,
+                           int64_t n_entries, const void* win, int64_t win_len,
+                           const int64_t* win_start, const int64_t* q_pos, int window, int m,
+                           const float* sink, float softmax_scale, int batch, int n_q,
+                           int n_heads, int dim, csa_dtype_t kv_dt, void* O, void* ws,
+                           size_t ws_bytes, void* stream) {
+  csa::MqaArgs a = mqa_args(Q, q_dt, entries, n_entries, nullptr, 0, win, win_len, win_start, q_pos,
+                            window, m, sink, softmax_scale, batch, n_q, n_heads, dim, kv_dt, O, ws,
+                            ws_bytes);
+  return run_mqa(a, stream, "hca_dense_mqa");
+}
+
+}  // extern "C"

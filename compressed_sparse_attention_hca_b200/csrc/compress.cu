@@ -1,0 +1,200 @@
+// compress.cu -- Token-Level Compressor ("DeepSeek-V4 内部机制" 1.2 Step 1 and
+// 1.3; yunpan.plus write-up eq. 6-7 and 10-11).
+//
+// One thread owns one (request, entry, 8-channel chunk).  It streams the 2m
+// (CSA) or m' (HCA) token rows of its chunk once with 16-byte loads and keeps
+// an online softmax per channel in fp32, so every input byte is read exactly
+// once: the kernel is bound by HBM reads of C and Z.  Lanes that share an FP8
+// scale block (8 lanes = 64 dims) or an FP4 block (2 lanes = 16 dims) reduce
+// their amax with warp shuffles and quantise in the epilogue.
+#include "csa_internal.cuh"
+
+namespace csa {
+namespace {
+
+__device__ __forceinline__ void load8(const void* base, int dt, int64_t elem, float* v) {
+  if (dt == CSA_F32) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem);
+    float4 a = __ldg(p), b = __ldg(p + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + elem));
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  }
+}
+
+struct OnlineSoftmax8 {
+  float mx[8], den[8], acc[8];
+  __device__ void init() {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) { mx[j] = -INFINITY; den[j] = 0.f; acc[j] = 0.f; }
+  }
+  __device__ void add(const float* logit, const float* val) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (logit[j] > mx[j]) {
+        float r = expf(mx[j] - logit[j]);  // 0 on the first token
+        den[j] = den[j] * r + 1.f;
+        acc[j] = acc[j] * r + val[j];
+        mx[j] = logit[j];
+      } else {
+        float e = expf(logit[j] - mx[j]);
+        den[j] += e;
+        acc[j] = fmaf(e, val[j], acc[j]);
+      }
+    }
+  }
+};
+
+__global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
+  const int chunks = a.dim / 8;
+  const int64_t total = (int64_t)a.batch * a.n_out * chunks;
+  const int64_t gid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const bool valid = gid < total;
+  const int64_t g = valid ? gid : 0;
+  const int ch = (int)(g % chunks);
+  const int64_t ie = (g / chunks) % a.n_out;
+  const int b = (int)(g / chunks / a.n_out);
+  const int64_t i = a.e0 + ie;
+  const int d0 = ch * 8;
+
+  OnlineSoftmax8 sm;
+  sm.init();
+  float z[8], c[8], bias[8], logit[8];
+  const int64_t in_base = (int64_t)b * a.in_batch_stride;
+  if (valid) {
+    // current group (a-branch)
+    for (int j = 0; j < a.m; ++j) {
+      const int64_t r = a.m * i + j - a.tok0;
+      const int64_t off = (in_base + r) * a.dim + d0;
+      load8(a.Za, a.in_dt, off, z);
+      load8(a.Ca, a.in_dt, off, c);
+      const float4* bp = reinterpret_cast<const float4*>(a.Ba + (int64_t)j * a.dim + d0);
+      float4 b0 = __ldg(bp), b1 = __ldg(bp + 1);
+      bias[0] = b0.x; bias[1] = b0.y; bias[2] = b0.z; bias[3] = b0.w;
+      bias[4] = b1.x; bias[5] = b1.y; bias[6] = b1.z; bias[7] = b1.w;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) logit[q] = z[q] + bias[q];
+      sm.add(logit, c);
+    }
+    // previous group (b-branch), CSA only, absent for entry 0
+    if (a.Cb != nullptr && i >= 1) {
+      for (int j = 0; j < a.m; ++j) {
+        const int64_t r = a.m * (i - 1) + j - a.tok0;
+        const int64_t off = (in_base + r) * a.dim + d0;
+        load8(a.Zb, a.in_dt, off, z);
+        load8(a.Cb, a.in_dt, off, c);
+        const float4* bp = reinterpret_cast<const float4*>(a.Bb + (int64_t)j * a.dim + d0);
+        float4 b0 = __ldg(bp), b1 = __ldg(bp + 1);
+        bias[0] = b0.x; bias[1] = b0.y; bias[2] = b0.z; bias[3] = b0.w;
+        bias[4] = b1.x; bias[5] = b1.y; bias[6] = b1.z; bias[7] = b1.w;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) logit[q] = z[q] + bias[q];
+        sm.add(logit, c);
+      }
+    }
+  }
+  float x[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) x[q] = valid ? sm.acc[q] / sm.den[q] : 0.f;
+
+  const int64_t orow = (int64_t)b * a.out_batch_stride + ie;
+  const int64_t rb = row_bytes(a.out_dt, a.dim);
+  uint8_t* row = static_cast<uint8_t*>(a.out) + orow * rb;
+
+  if (a.out_dt == CSA_F32) {
+    if (valid) {
+      float4* p = reinterpret_cast<float4*>(row + 4 * d0);
+      p[0] = make_float4(x[0], x[1], x[2], x[3]);
+      p[1] = make_float4(x[4], x[5], x[6], x[7]);
+    }
+  } else if (a.out_dt == CSA_BF16) {
+    if (valid) {
+      uint32_t w[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
+        memcpy(&w[q], &h, 4);
+      }
+      *reinterpret_cast<uint4*>(row + 2 * d0) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else if (a.out_dt == CSA_KV_FP8MIX) {
+    const int n8 = a.dim - kRopeDims;
+    float amax = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) amax = fmaxf(amax, fabsf(x[q]));
+    // 8 consecutive lanes hold one 64-dim scale block
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    if (valid) {
+      if (d0 < n8) {
+        const float scale = amax > 0.f ? amax / 448.f : 1.f;
+        uint32_t w[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+              make_float2(x[4 * q] / scale, x[4 * q + 1] / scale), __NV_SATFINITE, __NV_E4M3);
+          __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+              make_float2(x[4 * q + 2] / scale, x[4 * q + 3] / scale), __NV_SATFINITE, __NV_E4M3);
+          w[q] = (uint32_t)lo | ((uint32_t)hi << 16);
+        }
+        *reinterpret_cast<uint2*>(row + d0) = make_uint2(w[0], w[1]);
+        if ((d0 % kFp8Block) == 0)
+          *reinterpret_cast<float*>(row + n8 + 2 * kRopeDims + 4 * (d0 / kFp8Block)) = scale;
+      } else {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
+          memcpy(&w[q], &h, 4);
+        }
+        *reinterpret_cast<uint4*>(row + n8 + 2 * (d0 - n8)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      if (ch == 0) {
+        for (int64_t p = n8 + 2 * kRopeDims + 4 * (n8 / kFp8Block); p < rb; ++p) row[p] = 0;
+      }
+    }
+  } else {  // CSA_IDX_NVFP4
+    float amax = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) amax = fmaxf(amax, fabsf(x[q]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));  // 2 lanes = 16 values
+    if (valid) {
+      const __nv_fp8_storage_t s8 = __nv_cvt_float_to_fp8(amax / 6.f, __NV_SATFINITE, __NV_E4M3);
+      const float s = e4m3_to_float((uint8_t)s8);
+      uint32_t packed = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        __nv_fp4x2_storage_t p2 = 0;
+        if (s > 0.f)
+          p2 = __nv_cvt_float2_to_fp4x2(make_float2(x[2 * q] / s, x[2 * q + 1] / s), __NV_E2M1,
+                                        cudaRoundNearest);
+        packed |= ((uint32_t)p2) << (8 * q);
+      }
+      *reinterpret_cast<uint32_t*>(row + d0 / 2) = packed;
+      if ((d0 % kFp4Block) == 0) {
+        uint8_t* sf = static_cast<uint8_t*>(a.out_sf) + orow * (a.dim / kFp4Block);
+        sf[d0 / kFp4Block] = (uint8_t)s8;
+      }
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s) {
+  const int64_t total = (int64_t)a.batch * a.n_out * (a.dim / 8);
+  if (total == 0) return cudaSuccess;
+  const int threads = 256;
+  const int64_t blocks = (total + threads - 1) / threads;
+  compress_kernel<<<(unsigned)blocks, threads, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

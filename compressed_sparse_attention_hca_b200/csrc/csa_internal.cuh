@@ -1,0 +1,188 @@
+// csa_internal.cuh -- device helpers and internal launcher declarations shared
+// by the CUDA translation units of libcsa_b200.  Nothing here is visible
+// through the C ABI (include/csa.h is the public surface).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_fp4.h>
+#include <stdint.h>
+
+#include "../../include/csa.h"
+
+namespace csa {
+
+// ---------------------------------------------------------------------------
+// Storage formats (byte layouts documented in include/csa.h).
+// ---------------------------------------------------------------------------
+constexpr int kRopeDims = 64;        // trailing RoPE dims kept in bf16 (FP8MIX)
+constexpr int kFp8Block = 64;        // FP8 dims sharing one fp32 scale
+constexpr int kFp4Block = 16;        // FP4 values sharing one E4M3 scale
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+__host__ __device__ inline int64_t row_bytes(int dt, int dim) {
+  switch (dt) {
+    case CSA_F32: return 4LL * dim;
+    case CSA_BF16: return 2LL * dim;
+    case CSA_KV_FP8MIX: {
+      int64_t n8 = dim - kRopeDims;
+      return (n8 + 2 * kRopeDims + 4 * (n8 / kFp8Block) + 15) / 16 * 16;
+    }
+    case CSA_IDX_NVFP4: return dim / 2;
+    default: return -1;
+  }
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t h) {
+  return __uint_as_float(((uint32_t)h) << 16);
+}
+
+// Two E4M3 codes (low byte = first element) -> two floats (hardware convert).
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint16_t codes) {
+  __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)codes, __NV_E4M3);
+  __half2 hh;
+  memcpy(&hh, &h, sizeof(hh));
+  return __half22float2(hh);
+}
+
+__device__ __forceinline__ float e4m3_to_float(uint8_t code) {
+  __half_raw h = __nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)code, __NV_E4M3);
+  __half hh;
+  memcpy(&hh, &h, sizeof(hh));
+  return __half2float(hh);
+}
+
+// Two E2M1 codes packed in one byte (low nibble = first element) -> floats.
+__device__ __forceinline__ float2 e2m1x2_to_float2(uint8_t byte) {
+  __half2_raw h = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)byte, __NV_E2M1);
+  __half2 hh;
+  memcpy(&hh, &h, sizeof(hh));
+  return __half22float2(hh);
+}
+
+// Decode `n` consecutive values [d0, d0+n) of one row of format dt into f32.
+// n and d0 are multiples of 8 (FP8MIX/BF16/F32) or 16 (NVFP4).
+__device__ __forceinline__ void decode_row_chunk8(const uint8_t* row, const uint8_t* sf_row, int dt,
+                                                  int dim, int d0, float* out8) {
+  if (dt == CSA_F32) {
+    const float4* p = reinterpret_cast<const float4*>(row + 4 * d0);
+    float4 a = p[0], b = p[1];
+    out8[0] = a.x; out8[1] = a.y; out8[2] = a.z; out8[3] = a.w;
+    out8[4] = b.x; out8[5] = b.y; out8[6] = b.z; out8[7] = b.w;
+  } else if (dt == CSA_BF16) {
+    uint4 v = *reinterpret_cast<const uint4*>(row + 2 * d0);
+    uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      out8[2 * j] = __uint_as_float(w[j] << 16);
+      out8[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  } else if (dt == CSA_KV_FP8MIX) {
+    const int n8 = dim - kRopeDims;
+    if (d0 < n8) {
+      uint2 v = *reinterpret_cast<const uint2*>(row + d0);
+      const float s = *reinterpret_cast<const float*>(row + n8 + 2 * kRopeDims + 4 * (d0 / kFp8Block));
+      uint32_t w[2] = {v.x, v.y};
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float2 lo = e4m3x2_to_float2((uint16_t)(w[j] & 0xFFFF));
+        float2 hi = e4m3x2_to_float2((uint16_t)(w[j] >> 16));
+        out8[4 * j + 0] = lo.x * s; out8[4 * j + 1] = lo.y * s;
+        out8[4 * j + 2] = hi.x * s; out8[4 * j + 3] = hi.y * s;
+      }
+    } else {
+      uint4 v = *reinterpret_cast<const uint4*>(row + n8 + 2 * (d0 - n8));
+      uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        out8[2 * j] = __uint_as_float(w[j] << 16);
+        out8[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+      }
+    }
+  } else {  // NVFP4: 8 values = 4 bytes, one scale per 16 values
+    uint32_t v = *reinterpret_cast<const uint32_t*>(row + d0 / 2);
+    const float s = e4m3_to_float(sf_row[d0 / kFp4Block]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      float2 f = e2m1x2_to_float2((uint8_t)(v >> (8 * j)));
+      out8[2 * j] = f.x * s;
+      out8[2 * j + 1] = f.y * s;
+    }
+  }
+}
+
+// Order-preserving key of a float score (larger score -> larger key).
+__device__ __forceinline__ uint32_t f32_key(float s) {
+  uint32_t u = __float_as_uint(s);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+// bf16 score -> key in the upper 16 bits (lower 16 bits zero).
+__device__ __forceinline__ uint32_t bf16_key(float s) {
+  __nv_bfloat16 b = __float2bfloat16_rn(s);
+  uint16_t h;
+  memcpy(&h, &b, 2);
+  uint32_t u = ((uint32_t)h) << 16;
+  return (u & 0x80000000u) ? (~u & 0xFFFF0000u) : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_to_f32(uint32_t k) {
+  uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
+  return __uint_as_float(u);
+}
+
+// ---------------------------------------------------------------------------
+// Internal launchers (one per translation unit); all return cudaError_t of the
+// launch (cudaGetLastError) and never allocate.
+// ---------------------------------------------------------------------------
+struct CompressArgs {
+  const void *Ca, *Cb, *Za, *Zb;
+  const float *Ba, *Bb;
+  int batch;
+  int64_t n_tok, tok0, in_batch_stride, e0, n_out;
+  int dim, m, in_dt, out_dt;
+  void *out, *out_sf;
+  int64_t out_batch_stride;
+};
+cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s);
+
+struct IndexArgs {
+  const void *qI, *qI_sf;
+  const float* wI;
+  const void *KI, *KI_sf;
+  const int64_t* q_pos;
+  int batch, n_q;
+  int64_t n_entries;
+  int m, n_heads, dim, k, dt;
+  int32_t* idx_out;
+  void* scores_out;
+  void* ws;
+  size_t ws_bytes;
+};
+size_t index_topk_workspace(int batch, int n_q, int64_t n_entries, int k, int n_heads, int dim, int dt);
+cudaError_t launch_index_topk(const IndexArgs& a, cudaStream_t s);
+
+struct MqaArgs {
+  const void* Q;
+  int q_dt;
+  const void* entries;
+  int64_t n_entries;
+  const int32_t* idx;  // nullptr: dense (HCA) over every visible entry
+  int k;
+  const void* win;
+  int64_t win_len;
+  const int64_t* win_start;
+  const int64_t* q_pos;
+  int window, m;
+  const float* sink;
+  float scale;
+  int batch, n_q, n_heads, dim, kv_dt;
+  void* O;
+  void* ws;
+  size_t ws_bytes;
+};
+size_t mqa_workspace(const MqaArgs& a);
+cudaError_t launch_mqa(const MqaArgs& a, cudaStream_t s);
+
+}  // namespace csa

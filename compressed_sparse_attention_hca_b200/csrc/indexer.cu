@@ -1,0 +1,180 @@
+// indexer.cu -- Lightning Indexer score fused with the top-k selector
+// ("DeepSeek-V4 内部机制" 1.2 Step 2: I[t,s] = sum_h w[t,h] ReLU(q[t,h].K[s]),
+// top-k over I[t,:]; section 6.2: fp32 score rounded to BF16 before top-k).
+//
+// Work split: the visible entries of a query are cut into slices; one CTA
+// scores one slice of one query into shared memory and selects the slice's
+// top k there (a radix select on the score keys, so the score row never goes
+// to HBM).  A query whose entries need several slices gets a second, small
+// merge kernel that selects the final k among the per-slice candidates.
+//
+// This file holds the SIMT score producer (fp32 FMA), used for F32 inputs
+// (exact-fp32 mode) and for shapes the tensor-core producer does not take;
+// indexer_tc.cu holds the tcgen05 producer for BF16 / NVFP4 inputs.
+#include "csa_internal.cuh"
+#include "topk_select.cuh"
+#include "indexer_plan.cuh"
+
+namespace csa {
+namespace {
+
+constexpr int kNT = 512;
+
+__global__ void __launch_bounds__(kNT) index_slice_simt_kernel(IndexArgs a, IndexPlan plan) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const int sl = blockIdx.x, t = blockIdx.y, b = blockIdx.z;
+  const int64_t bt = (int64_t)b * a.n_q + t;
+  float* q = reinterpret_cast<float*>(smem_raw);                 // [n_heads][dim]
+  float* w = q + a.n_heads * a.dim;                               // [n_heads]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(w + a.n_heads);    // [slice_len]
+  SelectSmem<kNT>& sm = *reinterpret_cast<SelectSmem<kNT>*>(keys + plan.slice_len);
+
+  const int64_t vis = visible_entries(a.q_pos[bt], a.m, a.n_entries);
+  const int64_t s0 = (int64_t)sl * plan.slice_len;
+  const int len = (int)min64(plan.slice_len, a.n_entries - s0);
+  const int n_valid = (int)max64(0, min64(len, vis - s0));
+
+  // decode the query heads and the head weights
+  const int qrb = (int)row_bytes(a.dt, a.dim);
+  const uint8_t* qbase = static_cast<const uint8_t*>(a.qI) + bt * a.n_heads * qrb;
+  const uint8_t* qsf = a.dt == CSA_IDX_NVFP4
+                           ? static_cast<const uint8_t*>(a.qI_sf) + bt * a.n_heads * (a.dim / 16)
+                           : nullptr;
+  for (int c = threadIdx.x; c < a.n_heads * (a.dim / 8); c += kNT) {
+    const int h = c / (a.dim / 8), d0 = (c % (a.dim / 8)) * 8;
+    decode_row_chunk8(qbase + (int64_t)h * qrb, qsf ? qsf + h * (a.dim / 16) : nullptr, a.dt, a.dim,
+                      d0, q + h * a.dim + d0);
+  }
+  for (int h = threadIdx.x; h < a.n_heads; h += kNT) w[h] = a.wI[bt * a.n_heads + h];
+  __syncthreads();
+
+  const bool f32mode = a.dt == CSA_F32;
+  const uint8_t* kbase = static_cast<const uint8_t*>(a.KI) + (int64_t)b * a.n_entries * qrb;
+  const uint8_t* ksf = a.dt == CSA_IDX_NVFP4
+                           ? static_cast<const uint8_t*>(a.KI_sf) + (int64_t)b * a.n_entries * (a.dim / 16)
+                           : nullptr;
+  for (int p = threadIdx.x; p < len; p += kNT) {
+    const int64_t e = s0 + p;
+    uint32_t key = 0;
+    float score = -INFINITY;
+    if (p < n_valid) {
+      const uint8_t* krow = kbase + e * qrb;
+      const uint8_t* ksrow = ksf ? ksf + e * (a.dim / 16) : nullptr;
+      float I = 0.f;
+      for (int h = 0; h < a.n_heads; ++h) {
+        float dot = 0.f;
+        for (int d0 = 0; d0 < a.dim; d0 += 8) {
+          float kv[8];
+          decode_row_chunk8(krow, ksrow, a.dt, a.dim, d0, kv);
+          const float* qh = q + h * a.dim + d0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) dot = fmaf(qh[j], kv[j], dot);
+        }
+        I = fmaf(w[h], fmaxf(dot, 0.f), I);
+      }
+      if (f32mode) {
+        score = I;
+        key = f32_key(I);
+      } else {
+        key = bf16_key(I);
+        score = key_to_f32(key);
+      }
+    }
+    if (p < n_valid) keys[p] = key;
+    if (a.scores_out) {
+      if (f32mode) static_cast<float*>(a.scores_out)[bt * a.n_entries + e] = score;
+      else static_cast<__nv_bfloat16*>(a.scores_out)[bt * a.n_entries + e] = __float2bfloat16_rn(score);
+    }
+  }
+  __syncthreads();
+
+  const int kk = min(a.k, n_valid);
+  const int passes = f32mode ? 4 : 2;
+  auto key_at = [&](int i) { return keys[i]; };
+  if (plan.n_slices == 1) {
+    int32_t* out = a.idx_out + bt * a.k;
+    block_select<kNT>(key_at, n_valid, kk, passes, sm,
+                      [&](int slot, int pos) { out[slot] = (int32_t)(s0 + pos); });
+    for (int j = kk + threadIdx.x; j < a.k; j += kNT) out[j] = -1;
+  } else {
+    const int64_t off = slice_cand_offset(plan, sl, vis, a.n_entries, a.k);
+    uint32_t* ck = plan_cand_keys(plan, a.ws, bt) + off;
+    int32_t* ci = plan_cand_idx(plan, a.ws, bt) + off;
+    block_select<kNT>(key_at, n_valid, kk, passes, sm, [&](int slot, int pos) {
+      ck[slot] = keys[pos];
+      ci[slot] = (int32_t)(s0 + pos);
+    });
+  }
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(kMergeNT) index_merge_kernel(IndexArgs a, IndexPlan plan) {
+  __shared__ SelectSmem<kMergeNT> sm;
+  const int t = blockIdx.x, b = blockIdx.y;
+  const int64_t bt = (int64_t)b * a.n_q + t;
+  const int64_t vis = visible_entries(a.q_pos[bt], a.m, a.n_entries);
+  const int64_t total = slice_cand_offset(plan, plan.n_slices, vis, a.n_entries, a.k);
+  const uint32_t* ck = plan_cand_keys(plan, a.ws, bt);
+  const int32_t* ci = plan_cand_idx(plan, a.ws, bt);
+  const int n = (int)total;
+  const int kk = (int)min64(min64(a.k, vis), n);
+  int32_t* out = a.idx_out + bt * a.k;
+  const int passes = a.dt == CSA_F32 ? 4 : 2;
+  block_select<kMergeNT>([&](int i) { return ck[i]; }, n, kk, passes, sm,
+                         [&](int slot, int pos) { out[slot] = ci[pos]; });
+  for (int j = kk + threadIdx.x; j < a.k; j += kMergeNT) out[j] = -1;
+}
+
+// Slices: enough CTAs to cover the GPU about twice, each slice at most
+// kMaxSlice entries (its keys live in shared memory).
+IndexPlan make_simt_plan(int batch, int n_q, int64_t n_entries, int k) {
+  constexpr int kMaxSlice = 16384;
+  IndexPlan p{};
+  p.n_rows = (int64_t)batch * n_q;
+  const int64_t rows = p.n_rows > 0 ? p.n_rows : 1;
+  const int64_t per_row = (296 + rows - 1) / rows;
+  int64_t len = (n_entries + per_row - 1) / per_row;
+  len = (len + 127) / 128 * 128;
+  const int64_t lo = ((n_entries < 1024 ? n_entries : 1024) + 127) / 128 * 128;
+  if (len < lo) len = lo;
+  if (len < 128) len = 128;
+  if (len > kMaxSlice) len = kMaxSlice;
+  p.slice_len = (int)len;
+  p.n_slices = (int)((n_entries + len - 1) / len);
+  if (p.n_slices < 1) p.n_slices = 1;
+  p.cand_cap = p.n_slices > 1 ? (int64_t)p.n_slices * k : 0;
+  return p;
+}
+
+size_t index_simt_smem(const IndexArgs& a, const IndexPlan& plan) {
+  return (size_t)a.n_heads * a.dim * 4 + (size_t)a.n_heads * 4 + (size_t)plan.slice_len * 4 +
+         sizeof(SelectSmem<kNT>) + 16;
+}
+
+cudaError_t launch_index_simt(const IndexArgs& a, const IndexPlan& plan, cudaStream_t s) {
+  const size_t smem = index_simt_smem(a, plan);
+  cudaError_t e = cudaFuncSetAttribute(index_slice_simt_kernel,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(plan.n_slices, a.n_q, a.batch);
+  index_slice_simt_kernel<<<grid, kNT, smem, s>>>(a, plan);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || plan.n_slices == 1) return e;
+  index_merge_kernel<<<dim3(a.n_q, a.batch), kMergeNT, 0, s>>>(a, plan);
+  return cudaGetLastError();
+}
+
+size_t index_topk_workspace(int batch, int n_q, int64_t n_entries, int k, int n_heads, int dim,
+                            int dt) {
+  (void)n_heads; (void)dim; (void)dt;
+  return plan_workspace_bytes(make_simt_plan(batch, n_q, n_entries, k));
+}
+
+cudaError_t launch_index_topk(const IndexArgs& a, cudaStream_t s) {
+  if ((int64_t)a.batch * a.n_q == 0) return cudaSuccess;
+  const IndexPlan plan = make_simt_plan(a.batch, a.n_q, a.n_entries, a.k);
+  return launch_index_simt(a, plan, s);
+}
+
+}  // namespace csa

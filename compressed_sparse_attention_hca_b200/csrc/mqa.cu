@@ -1,0 +1,212 @@
+// mqa.cu -- shared-KV multi-query attention with sliding window and attention
+// sink ("DeepSeek-V4 内部机制" 1.2 Step 2 "Shared-KV MQA", 1.3 HCA dense
+// attention, 1.4 window branch and sink equation; yunpan.plus eq. 9).
+//
+// Every head of a query attends the same rows (the selected compressed
+// entries, or all visible entries for HCA, followed by the window tokens) and
+// each row serves as both key and value.  The row list of a query is split
+// across CTAs (split-KV); each CTA keeps an online softmax per head and writes
+// an unnormalised partial (m, l, o); a combine kernel merges the partials in
+// split order (deterministic) and adds the sink to the denominator.  With one
+// split the CTA finishes the softmax itself.
+//
+// This file holds the SIMT kernel (fp32 FMA): it serves F32 mode (1e-5
+// parity) and every shape the tensor-core kernel (mqa_tc.cu) does not take.
+#include "csa_internal.cuh"
+#include "mqa_plan.cuh"
+
+namespace csa {
+namespace {
+
+constexpr int kRC = 32;  // rows per chunk (one per lane)
+
+__global__ void __launch_bounds__(256) mqa_simt_kernel(MqaArgs a, MqaPlan plan) {
+  extern __shared__ __align__(16) uint8_t smem_raw[];
+  const int split = blockIdx.x, hg = blockIdx.y;
+  const int64_t bt = blockIdx.z;
+  const int b = (int)(bt / a.n_q);
+  const int HG = plan.heads_per_cta;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = hg * HG + warp;
+  const int dim = a.dim;
+  const int stride = dim + 1;  // padded kv rows: lane r reads row r conflict-free
+
+  float* q = reinterpret_cast<float*>(smem_raw);  // [HG][dim]
+  float* kv = q + HG * dim;                        // [kRC][dim+1]
+
+  const int64_t t = a.q_pos[bt];
+  const RowList rl = make_row_list(a, bt, t);
+  const int64_t r_begin = (int64_t)split * plan.rows_per_split;
+  const int64_t r_end = min64(rl.n_rows, r_begin + plan.rows_per_split);
+
+  // query heads of this CTA in fp32
+  for (int i = threadIdx.x; i < HG * dim; i += blockDim.x) {
+    const int hh = i / dim, d = i % dim;
+    const int64_t off = (bt * a.n_heads + hg * HG + hh) * dim + d;
+    q[i] = a.q_dt == CSA_F32 ? static_cast<const float*>(a.Q)[off]
+                             : bf16_bits_to_float(static_cast<const uint16_t*>(a.Q)[off]);
+  }
+
+  const int per_lane = dim / 32;
+  float o[16];
+#pragma unroll
+  for (int j = 0; j < 16; ++j) o[j] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  const int64_t rb = row_bytes(a.kv_dt, dim);
+
+  for (int64_t c0 = r_begin; c0 < r_end; c0 += kRC) {
+    const int nr = (int)min64(kRC, r_end - c0);
+    __syncthreads();
+    // decode the chunk's rows into shared memory (invalid rows -> zeros)
+    for (int i = threadIdx.x; i < kRC * (dim / 8); i += blockDim.x) {
+      const int r = i / (dim / 8), d0 = (i % (dim / 8)) * 8;
+      float v[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+      if (r < nr) {
+        const uint8_t* src = row_ptr(a, rl, b, c0 + r, rb);
+        if (src) decode_row_chunk8(src, nullptr, a.kv_dt, dim, d0, v);
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) kv[r * stride + d0 + j] = v[j];
+    }
+    __syncthreads();
+    // logits: lane r scores row c0 + r for head h
+    float z = -INFINITY;
+    if (lane < nr && row_valid(a, rl, b, c0 + lane)) {
+      const float* qh = q + warp * dim;
+      const float* kr = kv + lane * stride;
+      float dot = 0.f;
+      for (int d = 0; d < dim; ++d) dot = fmaf(qh[d], kr[d], dot);
+      z = dot * a.scale;
+    }
+    float cmax = z;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, off));
+    const float m_new = fmaxf(m_run, cmax);
+    float p = 0.f, corr = 1.f;
+    if (m_new != -INFINITY) {
+      p = (z == -INFINITY) ? 0.f : expf(z - m_new);
+      corr = (m_run == -INFINITY) ? 0.f : expf(m_run - m_new);
+    }
+    float psum = p;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) psum += __shfl_xor_sync(0xffffffffu, psum, off);
+    l_run = l_run * corr + psum;
+    m_run = m_new;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) o[j] *= corr;
+    for (int r = 0; r < nr; ++r) {
+      const float pr = __shfl_sync(0xffffffffu, p, r);
+      const float* kr = kv + r * stride;
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        if (j < per_lane) o[j] = fmaf(pr, kr[lane + 32 * j], o[j]);
+    }
+  }
+
+  if (plan.n_splits == 1) {
+    const float sink = a.sink[h];
+    float M = fmaxf(m_run, sink);
+    float f = 0.f;
+    if (!(sink == INFINITY) && M != -INFINITY) {
+      const float em = (m_run == -INFINITY) ? 0.f : expf(m_run - M);
+      const float den = l_run * em + expf(sink - M);
+      f = em / den;
+    }
+    const int64_t ob = (bt * a.n_heads + h) * dim;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) {
+      if (j < per_lane) {
+        const float v = o[j] * f;
+        if (a.q_dt == CSA_F32) static_cast<float*>(a.O)[ob + lane + 32 * j] = v;
+        else static_cast<__nv_bfloat16*>(a.O)[ob + lane + 32 * j] = __float2bfloat16_rn(v);
+      }
+    }
+  } else {
+    float* po = plan_partial_o(plan, a, bt, split, h);
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (j < per_lane) po[lane + 32 * j] = o[j];
+    if (lane == 0) {
+      float* ml = plan_partial_ml(plan, a, bt, split, h);
+      ml[0] = m_run;
+      ml[1] = l_run;
+    }
+  }
+}
+
+}  // namespace
+
+// Merges the split partials of one (query, head) in split order and applies
+// the sink: O = sum_s e^{m_s-M} o_s / (sum_s e^{m_s-M} l_s + e^{sink-M}).
+__global__ void __launch_bounds__(128) mqa_combine_kernel(MqaArgs a, MqaPlan plan) {
+  const int h = blockIdx.x;
+  const int64_t bt = blockIdx.y;
+  const float sink = a.sink[h];
+  float M = sink;
+  for (int s = 0; s < plan.n_splits; ++s) M = fmaxf(M, plan_partial_ml(plan, a, bt, s, h)[0]);
+  float den = 0.f;
+  const bool zero = (sink == INFINITY) || (M == -INFINITY);
+  if (!zero) {
+    den = expf(sink - M);
+    for (int s = 0; s < plan.n_splits; ++s) {
+      const float* ml = plan_partial_ml(plan, a, bt, s, h);
+      if (ml[0] != -INFINITY) den += ml[1] * expf(ml[0] - M);
+    }
+  }
+  const int64_t ob = (bt * a.n_heads + h) * a.dim;
+  for (int d = threadIdx.x; d < a.dim; d += blockDim.x) {
+    float acc = 0.f;
+    if (!zero) {
+      for (int s = 0; s < plan.n_splits; ++s) {
+        const float* ml = plan_partial_ml(plan, a, bt, s, h);
+        if (ml[0] != -INFINITY) acc += plan_partial_o(plan, a, bt, s, h)[d] * expf(ml[0] - M);
+      }
+      acc /= den;
+    }
+    if (a.q_dt == CSA_F32) static_cast<float*>(a.O)[ob + d] = acc;
+    else static_cast<__nv_bfloat16*>(a.O)[ob + d] = __float2bfloat16_rn(acc);
+  }
+}
+
+MqaPlan make_simt_mqa_plan(const MqaArgs& a) {
+  MqaPlan p{};
+  p.heads_per_cta = (a.n_heads % 8 == 0) ? 8 : (a.n_heads % 4 == 0) ? 4 : (a.n_heads % 2 == 0) ? 2 : 1;
+  const int64_t rows_max = max_rows_per_query(a);
+  const int64_t units = (int64_t)a.batch * a.n_q * (a.n_heads / p.heads_per_cta);
+  int64_t splits = (296 + units - 1) / units;
+  const int64_t max_splits = (rows_max + kRC - 1) / kRC;
+  if (splits > max_splits) splits = max_splits;
+  if (splits < 1) splits = 1;
+  int64_t rps = (rows_max + splits - 1) / splits;
+  rps = (rps + kRC - 1) / kRC * kRC;
+  if (rps < kRC) rps = kRC;
+  p.rows_per_split = rps;
+  p.n_splits = (int)((rows_max + rps - 1) / rps);
+  if (p.n_splits < 1) p.n_splits = 1;
+  return p;
+}
+
+cudaError_t launch_mqa_simt(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) {
+  const size_t smem = ((size_t)p.heads_per_cta * a.dim + (size_t)kRC * (a.dim + 1)) * 4;
+  cudaError_t e = cudaFuncSetAttribute(mqa_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.n_splits, a.n_heads / p.heads_per_cta, (unsigned)((int64_t)a.batch * a.n_q));
+  mqa_simt_kernel<<<grid, 32 * p.heads_per_cta, smem, s>>>(a, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || p.n_splits == 1) return e;
+  mqa_combine_kernel<<<dim3(a.n_heads, (unsigned)((int64_t)a.batch * a.n_q)), 128, 0, s>>>(a, p);
+  return cudaGetLastError();
+}
+
+size_t mqa_workspace(const MqaArgs& a) {
+  const MqaPlan p = make_simt_mqa_plan(a);
+  return plan_mqa_workspace_bytes(p, a);
+}
+
+cudaError_t launch_mqa(const MqaArgs& a, cudaStream_t s) {
+  if ((int64_t)a.batch * a.n_q == 0) return cudaSuccess;
+  return launch_mqa_simt(a, make_simt_mqa_plan(a), s);
+}
+
+}  // namespace csa

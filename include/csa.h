@@ -1,0 +1,201 @@
+/*
+ * csa.h -- C ABI of libcsa_b200: the hybrid compressed attention forward pass
+ * of DeepSeek-V4 (CSA: Compressed Sparse Attention, HCA: Heavily Compressed
+ * Attention) on NVIDIA B200 (sm_100a).
+ *
+ * Passages defining the operations (page title, section, equation):
+ *   [P5] "DeepSeek-V4 内部机制" (LLM-101-CN deep dive):
+ *        1.2 Step 1 (compressor equations for S and C^Comp),
+ *        1.2 Step 2 (index score I[t,s], top-k, shared-KV MQA),
+ *        1.3 (HCA: m' tokens per entry, no overlap, no top-k),
+ *        1.4 table and sink equation (window branch of n_win = 128 raw
+ *        tokens, per-head sink logit in the softmax denominator),
+ *        1.5 (RoPE dims BF16, other dims FP8; FP4 indexer),
+ *        6.2 (FP4 indexer QK, scores quantised FP32 -> BF16 before top-k).
+ *   [P1] yunpan.plus write-up "CSA / HCA: 混合稀疏注意力机制", eq. (6)-(11).
+ *   [P2] admirer.cn article, CSA and HCA sections (top-k 512 / 1024,
+ *        window 128, sink, mixed FP8/BF16 KV).
+ *
+ * Conventions shared by every call
+ *   - All tensor arguments are DEVICE pointers owned by the caller; the
+ *     library allocates no memory.  Scratch space is passed explicitly as
+ *     (ws, ws_bytes); the matching *_workspace_size() call returns the
+ *     minimum size.  Scratch must not be shared by calls that may overlap.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream).  Host-side validation happens before any launch.
+ *   - Tensors are dense, row-major, batch-major, with the shapes given below.
+ *     Every device pointer must be 16-byte aligned.
+ *   - Errors: a call returns CSA_ERR_INVALID_ARG (bad shape, NULL or
+ *     misaligned pointer, workspace too small), CSA_ERR_UNSUPPORTED (a valid
+ *     combination this build does not implement), or CSA_ERR_CUDA (a launch
+ *     failed; the CUDA error string is in csa_last_error()).  Nothing aborts,
+ *     prints or exits.  csa_last_error() is per host thread.
+ *
+ * Row formats (csa_dtype_t)
+ *   CSA_F32        dim float32 values.
+ *   CSA_BF16       dim bfloat16 values.
+ *   CSA_KV_FP8MIX  KV entry / window row, dim = 64 * j + 64 (512 in the
+ *                  workloads): bytes [0, dim-64) E4M3 codes of dims
+ *                  0..dim-65; then 64 bf16 (128 bytes) for the RoPE dims
+ *                  dim-64..dim-1; then (dim-64)/64 fp32 scales, one per 64
+ *                  E4M3 dims; zero padding to a multiple of 16 bytes
+ *                  (608 bytes per row at dim 512).  value = code * scale.
+ *                  Writers use scale = amax/448 (1 when the block is zero)
+ *                  and round to nearest even, saturating at +-448.
+ *   CSA_IDX_NVFP4  indexer query/key rows as two arrays: codes
+ *                  [rows][dim/2] bytes (element 2j in the low nibble of byte
+ *                  j) and scales [rows][dim/16] unsigned E4M3, one per 16
+ *                  values.  value = e2m1 * scale.  Writers use
+ *                  scale = E4M3(amax/6) and codes = E2M1(x / scale), both
+ *                  rounded to nearest even with saturation.
+ */
+#ifndef CSA_B200_H
+#define CSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1,
+  CSA_ERR_UNSUPPORTED = 2,
+  CSA_ERR_CUDA = 3,
+  CSA_ERR_TIMEOUT = 4
+} csa_status_t;
+
+typedef enum {
+  CSA_F32 = 0,
+  CSA_BF16 = 1,
+  CSA_KV_FP8MIX = 2,
+  CSA_IDX_NVFP4 = 3
+} csa_dtype_t;
+
+/* Last error message of the calling host thread ("" after success). */
+const char* csa_last_error(void);
+
+/* Library ABI version (major * 100 + minor). */
+int csa_version(void);
+
+/* Bytes per row of format dt at dimension dim (codes only for NVFP4), or -1
+ * when dim is not valid for the format. */
+int64_t csa_row_bytes(csa_dtype_t dt, int dim);
+
+/*
+ * csa_compress -- Token-Level Compressor ([P5] 1.2 Step 1; [P1] eq. 6-7;
+ * HCA form [P5] 1.3, [P1] eq. 10-11).
+ *
+ * For entry i and channel d, the logits of the current group
+ * Z^a[m i + j, d] + B^a[j, d] (j < m) and, for CSA with i >= 1, of the
+ * previous group Z^b[m (i-1) + j, d] + B^b[j, d] are soft-maxed together over
+ * the token positions (per channel), and
+ *   C^Comp[i, d] = sum_j S^a_j C^a[m i + j, d] + sum_j S^b_j C^b[m (i-1) + j, d].
+ * Entry 0 has no previous group (its b-branch is absent).  Cb == NULL (and
+ * Zb, Bb ignored) selects the HCA form: one branch, no overlap.
+ *
+ *   Ca, Cb, Za, Zb  [batch][in_batch_stride rows][dim] of in_dt (F32/BF16);
+ *                   row r of request b holds absolute token tok0 + r, and
+ *                   rows 0..n_tok-1 are valid.
+ *   Ba, Bb          [m][dim] fp32, indexed by position inside the group.
+ *   e0, n_out       entries e0 .. e0+n_out-1 are produced; every token they
+ *                   need, m*(e0-1) (or m*e0 without overlap / at e0 = 0) up
+ *                   to m*(e0+n_out)-1, must lie in [tok0, tok0+n_tok).
+ *   out             [batch][out_batch_stride rows] of out_dt (F32, BF16,
+ *                   KV_FP8MIX, IDX_NVFP4); entry i of request b is written
+ *                   to row b*out_batch_stride + (i - e0).
+ *   out_sf          NVFP4 only: scales [batch][out_batch_stride][dim/16].
+ */
+csa_status_t csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                          const float* Ba, const float* Bb, int batch, int64_t n_tok,
+                          int64_t tok0, int64_t in_batch_stride, int64_t e0, int64_t n_out,
+                          int dim, int m, csa_dtype_t in_dt, void* out, void* out_sf,
+                          int64_t out_batch_stride, csa_dtype_t out_dt, void* stream);
+
+/*
+ * csa_index_topk -- Lightning Indexer fused with the top-k selector ([P5] 1.2
+ * Step 2; [P1] eq. 8; BF16 scores [P5] 6.2).
+ *
+ *   I[t, s] = sum_h wI[t, h] * ReLU(qI[t, h] . KI[s])
+ * over the entries visible to query t: s < floor((q_pos[t] + 1) / m) (an
+ * entry is visible once its whole group of m tokens is at or before t), and
+ * s < n_entries.  The score is accumulated in fp32 and, for BF16 / NVFP4
+ * inputs, rounded once to bf16 (nearest even) before selection; F32 inputs
+ * keep fp32 scores.  The k entries first in the order (score desc, index asc)
+ * are returned; with fewer than k visible entries the rest is -1.  The k
+ * indices of a query are written in ascending index order.
+ *
+ *   qI        [batch][n_q][n_heads][dim] of dt; NVFP4: codes, with qI_sf
+ *             [batch][n_q][n_heads][dim/16] scales.
+ *   wI        [batch][n_q][n_heads] fp32 head weights.
+ *   KI        [batch][n_entries][dim] of dt; NVFP4: codes, with KI_sf.
+ *   q_pos     [batch][n_q] int64 absolute position of each query.
+ *   idx_out   [batch][n_q][k] int32 entry indices (per request).
+ *   scores_out  optional (NULL in production): [batch][n_q][n_entries] of
+ *             the selection scores (bf16, or fp32 for F32 inputs), -inf for
+ *             entries not visible.  Used by tests to check selection.
+ *   dt        CSA_F32, CSA_BF16 or CSA_IDX_NVFP4 (qI and KI share it).
+ * Limits: 1 <= k <= 2048, dim a multiple of 32 (<= 256), n_heads <= 128.
+ */
+size_t csa_index_topk_workspace_size(int batch, int n_q, int64_t n_entries, int k, int n_heads,
+                                     int dim, csa_dtype_t dt);
+csa_status_t csa_index_topk(const void* qI, const void* qI_sf, const float* wI, const void* KI,
+                            const void* KI_sf, const int64_t* q_pos, int batch, int n_q,
+                            int64_t n_entries, int m, int n_heads, int dim, int k, csa_dtype_t dt,
+                            int32_t* idx_out, void* scores_out, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/*
+ * csa_sparse_mqa -- CSA core attention: shared-KV multi-query attention over
+ * the selected compressed entries plus the sliding window, with a per-head
+ * attention sink ([P5] 1.2 Step 2, 1.4 table rows "Sliding-Window" and
+ * "Attention Sink" and the sink equation; [P1] eq. 9; [P2] CSA section).
+ *
+ * For query t and head h, the attended rows J are the entries idx[t, :]
+ * (slots with -1 are unused) followed by the window tokens
+ * max(0, t-window+1) .. t (the query's own token included).  Each row is both
+ * key and value:
+ *   z_j = softmax_scale * <Q[t, h], row_j>,
+ *   O[t, h] = sum_j exp(z_j) row_j / (sum_j exp(z_j) + exp(sink[h])).
+ *
+ *   Q         [batch][n_q][n_heads][dim] of q_dt (F32 or BF16); O has the
+ *             same shape and dtype.
+ *   entries   [batch][n_entries] rows of kv_dt (F32, BF16, KV_FP8MIX).
+ *   idx       [batch][n_q][k] int32; an index outside
+ *             [0, min(n_entries, floor((q_pos+1)/m))) is ignored.
+ *   win       [batch][win_len] rows of kv_dt; row r holds absolute token
+ *             win_start[b] + r.  win_start [batch] int64 (device).  Every
+ *             window token of every query must be present.
+ *   q_pos     [batch][n_q] int64 (device); sink [n_heads] fp32 (device).
+ * Limits: dim a multiple of 64 (<= 512), n_heads <= 128, k <= 2048.
+ */
+size_t csa_sparse_mqa_workspace_size(int batch, int n_q, int n_heads, int dim, int k, int window,
+                                     csa_dtype_t q_dt, csa_dtype_t kv_dt);
+csa_status_t csa_sparse_mqa(const void* Q, csa_dtype_t q_dt, const void* entries,
+                            int64_t n_entries, const int32_t* idx, int k, const void* win,
+                            int64_t win_len, const int64_t* win_start, const int64_t* q_pos,
+                            int window, int m, const float* sink, float softmax_scale, int batch,
+                            int n_q, int n_heads, int dim, csa_dtype_t kv_dt, void* O, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/*
+ * hca_dense_mqa -- HCA core attention ([P5] 1.3: no top-k; every compressed
+ * entry is attended) over all visible entries s < floor((q_pos+1)/m) plus
+ * the window, with the sink, exactly as csa_sparse_mqa otherwise.
+ */
+size_t hca_dense_mqa_workspace_size(int batch, int n_q, int n_heads, int dim,
+                                    int64_t n_entries, int window, csa_dtype_t q_dt,
+                                    csa_dtype_t kv_dt);
+csa_status_t hca_dense_mqa(const void* Q, csa_dtype_t q_dt, const void* entries,
+                           int64_t n_entries, const void* win, int64_t win_len,
+                           const int64_t* win_start, const int64_t* q_pos, int window, int m,
+                           const float* sink, float softmax_scale, int batch, int n_q,
+                           int n_heads, int dim, csa_dtype_t kv_dt, void* O, void* ws,
+                           size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CSA_B200_H */

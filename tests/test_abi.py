@@ -1,0 +1,102 @@
+"""The C ABI library loads, exports what include/csa.h declares, and validates
+arguments on the host (CPU only: no call here reaches a kernel launch)."""
+import ctypes
+import subprocess
+
+import pytest
+
+from compressed_sparse_attention_hca_b200 import csa
+
+INVALID, UNSUPPORTED = 1, 2
+P = ctypes.c_void_p
+A = P(4096)  # a 16-byte aligned non-null address; never dereferenced by these calls
+
+
+def test_library_exports_every_declared_symbol():
+    lib = csa.load()
+    declared = csa.header_functions()
+    assert {"csa_compress", "csa_index_topk", "csa_sparse_mqa", "hca_dense_mqa"} <= set(declared)
+    out = subprocess.run(["nm", "-D", "--defined-only", csa.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared:
+        assert name in exported, name
+        getattr(lib, name)
+
+
+def test_version_and_row_bytes():
+    assert csa.load().csa_version() == 100
+    assert csa.row_bytes(csa.F32, 512) == 2048
+    assert csa.row_bytes(csa.BF16, 512) == 1024
+    assert csa.row_bytes(csa.KV_FP8MIX, 512) == 608
+    assert csa.row_bytes(csa.IDX_NVFP4, 128) == 64
+    assert csa.row_bytes(csa.KV_FP8MIX, 100) == -1
+    assert csa.row_bytes(csa.IDX_NVFP4, 40) == -1
+
+
+def _err():
+    return csa.load().csa_last_error().decode()
+
+
+def test_compress_rejects_bad_arguments():
+    lib = csa.load()
+    args = dict(Ca=A, Cb=A, Za=A, Zb=A, Ba=A, Bb=A, batch=1, n_tok=64, tok0=0, stride=64, e0=0, n_out=16,
+                dim=64, m=4, in_dt=csa.F32, out=A, out_sf=None, out_stride=16, out_dt=csa.F32)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.csa_compress(a["Ca"], a["Cb"], a["Za"], a["Zb"], a["Ba"], a["Bb"], a["batch"], a["n_tok"],
+                                a["tok0"], a["stride"], a["e0"], a["n_out"], a["dim"], a["m"], a["in_dt"],
+                                a["out"], a["out_sf"], a["out_stride"], a["out_dt"], None)
+    assert call(m=0) == INVALID and "m=0" in _err()
+    assert call(dim=60) == INVALID
+    assert call(in_dt=csa.KV_FP8MIX) == INVALID
+    assert call(out_dt=csa.KV_FP8MIX) == INVALID  # dim 64 has no FP8 dims
+    assert call(out_dt=csa.IDX_NVFP4) == INVALID and "out_sf" in _err()
+    assert call(Ca=None) == INVALID and "Ca is NULL" in _err()
+    assert call(Za=P(4100)) == INVALID and "aligned" in _err()
+    # entries 0..16 need tokens up to 67 but only 64 rows are present
+    assert call(n_out=17, out_stride=17) == INVALID and "need tokens" in _err()
+    # entry 5 with overlap needs token 16 onward; rows start at token 20
+    assert call(tok0=20, e0=5, n_out=1, n_tok=44, stride=44) == INVALID
+    assert call(out_stride=8) == INVALID
+    assert call(batch=0) == 0  # empty call is a no-op
+
+
+def test_index_topk_rejects_bad_arguments():
+    lib = csa.load()
+
+    def call(k=16, heads=2, dim=32, dt=csa.F32, ws_bytes=1 << 20, qsf=None, ksf=None, ws=A):
+        return lib.csa_index_topk(A, qsf, A, A, ksf, A, 1, 4, 64, 4, heads, dim, k, dt, A, None, ws,
+                                  ws_bytes, None)
+    assert call(k=0) == INVALID
+    assert call(k=4096) == INVALID
+    assert call(dim=48) == INVALID
+    assert call(heads=200) == INVALID
+    assert call(dt=csa.KV_FP8MIX) == INVALID
+    assert call(dt=csa.IDX_NVFP4) == INVALID and "NVFP4" in _err()
+    assert lib.csa_index_topk_workspace_size(1, 4, 64, 16, 2, 32, csa.F32) >= 256
+    big = lib.csa_index_topk_workspace_size(4, 1, 262144, 1024, 64, 128, csa.IDX_NVFP4)
+    assert call(ws_bytes=16) == INVALID or big <= 16
+
+
+def test_mqa_rejects_bad_arguments():
+    lib = csa.load()
+
+    def call(dim=64, heads=4, k=16, window=16, kv_dt=csa.F32, q_dt=csa.F32, idx=A):
+        return lib.csa_sparse_mqa(A, q_dt, A, 64, idx, k, A, 256, A, A, window, 4, A, 0.125, 1, 4, heads,
+                                  dim, kv_dt, A, A, 1 << 20, None)
+    assert call(dim=96) == INVALID
+    assert call(heads=0) == INVALID
+    assert call(k=0) == INVALID
+    assert call(window=-1) == INVALID
+    assert call(kv_dt=csa.IDX_NVFP4) == INVALID
+    assert call(q_dt=csa.KV_FP8MIX) == INVALID
+    assert call(idx=None) == INVALID
+    assert lib.hca_dense_mqa(A, csa.BF16, A, 64, A, 256, A, A, 16, 4, A, 0.1, 1, 4, 4, 100, csa.BF16,
+                             A, A, 1 << 20, None) == INVALID
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        csa.compress(torch.zeros(1, 8, 64), torch.zeros(1, 8, 64), torch.zeros(4, 64), 4)

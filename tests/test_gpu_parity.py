@@ -1,0 +1,309 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Inputs come from the seeded generators in compressed_sparse_attention_hca_b200.workloads
+(or are built in the test from plain random draws); expected values come from
+the oracle only.  Tolerances (spec contract):
+  * index scores: |g - o| <= 1e-2 |o| + 1e-3 rms(row) (BF16 scores);
+    bit-exact when every product and sum is exact in fp32 (integer inputs,
+    power-of-two weights): then top-k index sets are bit-exact too;
+  * attention outputs: 2e-2 max-abs for BF16 outputs, 1e-5 in F32 mode;
+  * compressor: F32 1e-5, BF16 one bf16 ulp (2^-8 relative); quantised
+    outputs (FP8MIX, NVFP4) within one code step of the oracle's value.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from compressed_sparse_attention_hca_b200 import csa
+from compressed_sparse_attention_hca_b200 import workloads as W
+from parity_util import assert_close, f64, raw, selection_from_scores
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.fail("the gpu tests need a CUDA device")
+    csa.load()
+
+
+def _cuda(d):
+    return {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in d.items()}
+
+
+# ---------------------------------------------------------------- compressor
+
+def _oracle_compress(orc, x, m, tok0, e0, n_out):
+    outs = []
+    for b in range(x["Ca"].shape[0]):
+        kw = {}
+        if x["Cb"] is not None:
+            kw = dict(Cb=f64(x["Cb"][b]), Zb=f64(x["Zb"][b]), Bb=f64(x["Bb"]))
+        outs.append(orc.compress(f64(x["Ca"][b]), f64(x["Za"][b]), f64(x["Ba"]), m, tok0=tok0, e0=e0,
+                                 n_out=n_out, **kw))
+    return np.stack(outs)
+
+
+@pytest.mark.parametrize("case", [
+    # batch, n_tok, dim, m, overlap, dtype, out_dt, tok0, e0, n_out
+    (1, 256, 64, 4, True, torch.float32, csa.F32, 0, 0, None),          # tiny prefill shape
+    (2, 4 * 37 + 3, 512, 4, True, torch.bfloat16, csa.BF16, 0, 0, None),  # ragged tail
+    (2, 128 * 5 + 17, 512, 128, False, torch.bfloat16, csa.F32, 0, 0, None),  # HCA
+    (3, 8, 512, 4, True, torch.bfloat16, csa.BF16, 4 * 1000, 1001, 1),   # decode: closing block
+    (1, 64, 128, 4, True, torch.float32, csa.F32, 0, 0, 16),
+])
+def test_compress_matches_oracle(orc, case):
+    batch, n_tok, dim, m, overlap, dtype, out_dt, tok0, e0, n_out = case
+    g = W.generator(100 + n_tok)
+    x = W.compress_inputs(g, batch, n_tok, dim, m, overlap, dtype)
+    if n_out is None:
+        n_out = (tok0 + n_tok) // m - e0
+    gx = _cuda(x)
+    out = csa.compress(gx["Ca"], gx["Za"], gx["Ba"], m, gx["Cb"], gx["Zb"], gx["Bb"], tok0=tok0, e0=e0,
+                       n_out=n_out, out_dt=out_dt)
+    want = _oracle_compress(orc, x, m, tok0, e0, n_out)
+    got = f64(out)
+    if out_dt == csa.F32:
+        assert_close(got, want, atol=1e-5, what="compress f32")
+    else:
+        assert_close(got, want, atol=1e-6, rtol=2.0 ** -8, what="compress bf16")
+
+
+def test_compress_writes_into_cache_row(orc):
+    """Decode: the entry closed by the last token lands at row E-1 of the cache."""
+    batch, dim, m, E = 2, 512, 4, 50
+    g = W.generator(7)
+    x = W.compress_inputs(g, batch, 2 * m, dim, m, True, torch.bfloat16)
+    gx = _cuda(x)
+    cache = torch.full((batch, E, dim), 7.0, device=DEV, dtype=torch.bfloat16)
+    csa.compress(gx["Ca"], gx["Za"], gx["Ba"], m, gx["Cb"], gx["Zb"], gx["Bb"], tok0=m * (E - 2), e0=E - 1,
+                 n_out=1, out=cache, out_row0=E - 1)
+    want = _oracle_compress(orc, x, m, m * (E - 2), E - 1, 1)
+    assert_close(f64(cache[:, E - 1:]), want, atol=1e-6, rtol=2.0 ** -8)
+    assert (cache[:, :E - 1] == 7.0).all()
+
+
+def test_compress_fp8mix_output(orc):
+    batch, n_tok, dim, m = 2, 4 * 40, 512, 4
+    x = W.compress_inputs(W.generator(5), batch, n_tok, dim, m, True, torch.bfloat16)
+    gx = _cuda(x)
+    out = csa.compress(gx["Ca"], gx["Za"], gx["Ba"], m, gx["Cb"], gx["Zb"], gx["Bb"], out_dt=csa.KV_FP8MIX)
+    want = _oracle_compress(orc, x, m, 0, 0, None)
+    got_bytes = raw(out)
+    assert got_bytes.shape == (batch, 40, 608)
+    assert (got_bytes[:, :, 604:] == 0).all()
+    for b in range(batch):
+        dec = orc.decode_rows(got_bytes[b], orc.FP8MIX, dim)
+        ref_bytes, _ = orc.encode_rows(want[b], orc.FP8MIX)
+        ref_scale = ref_bytes[:, 576:604].copy().view(np.float32)
+        got_scale = got_bytes[b, :, 576:604].copy().view(np.float32)
+        assert_close(got_scale, ref_scale, atol=0, rtol=1e-6, what="fp8 scales")
+        # one E4M3 step (relative 2^-3) or one subnormal step of the block scale
+        scale_per_dim = np.repeat(ref_scale, 64, axis=1)
+        bound = 2.0 ** -3 * np.abs(want[b, :, :448]) + 2.0 ** -9 * scale_per_dim + 1e-7
+        assert (np.abs(dec[:, :448] - want[b, :, :448]) <= bound).all()
+        assert_close(dec[:, 448:], want[b, :, 448:], atol=1e-6, rtol=2.0 ** -8, what="rope bf16")
+        codes_differ = (got_bytes[b, :, :448] != ref_bytes[:, :448]).mean()
+        assert codes_differ < 0.01, codes_differ
+
+
+def test_compress_nvfp4_output(orc):
+    batch, n_tok, dim, m = 2, 4 * 64, 128, 4
+    x = W.compress_inputs(W.generator(6), batch, n_tok, dim, m, True, torch.bfloat16)
+    gx = _cuda(x)
+    codes, sf = csa.compress(gx["Ca"], gx["Za"], gx["Ba"], m, gx["Cb"], gx["Zb"], gx["Bb"],
+                             out_dt=csa.IDX_NVFP4)
+    want = _oracle_compress(orc, x, m, 0, 0, None)
+    for b in range(batch):
+        dec = orc.decode_rows(raw(codes[b]), orc.NVFP4, dim, sf=raw(sf[b]))
+        ref_c, ref_sf = orc.encode_rows(want[b], orc.NVFP4)
+        ref_dec = orc.decode_rows(ref_c, orc.NVFP4, dim, sf=ref_sf)
+        s = np.repeat(np.array([[orc.e4m3_decode(int(v)) for v in row] for row in ref_sf]), 16, axis=1)
+        # at most one E2M1 step (<= 2 * scale) where fp32 and fp64 straddle a rounding boundary
+        assert (np.abs(dec - ref_dec) <= 2.0 * s * 1.13 + 1e-12).all()
+        assert (raw(sf[b]) != ref_sf).mean() < 0.02
+        assert (raw(codes[b]) != ref_c).mean() < 0.02
+
+
+# ------------------------------------------------------------- indexer + top-k
+
+def _exact_index_inputs(B, T, H, d, E, dt, seed):
+    """Integer-valued q, K and power-of-two weights: every score is exact in fp32."""
+    g = torch.Generator().manual_seed(seed)
+    wI = (2.0 ** torch.randint(-1, 2, (B, T, H), generator=g)).to(torch.float32)
+    if dt == csa.IDX_NVFP4:
+        qI, qsf = W.nvfp4_rows(g, (B, T, H), d)
+        KI, ksf = W.nvfp4_rows(g, (B, E), d)
+        p2 = torch.tensor([0.125, 0.25, 0.5, 1.0]).to(torch.float8_e4m3fn).view(torch.uint8)
+        qsf = p2[torch.randint(0, 4, qsf.shape, generator=g)]
+        ksf = p2[torch.randint(0, 4, ksf.shape, generator=g)]
+        return dict(qI=qI, qI_sf=qsf, KI=KI, KI_sf=ksf, wI=wI)
+    tdt = torch.float32 if dt == csa.F32 else torch.bfloat16
+    qI = torch.randint(-2, 3, (B, T, H, d), generator=g).to(tdt)
+    KI = torch.randint(-2, 3, (B, E, d), generator=g).to(tdt)
+    return dict(qI=qI, KI=KI, wI=wI, qI_sf=None, KI_sf=None)
+
+
+def _decode_idx_inputs(orc, x, dt, d):
+    if dt == csa.IDX_NVFP4:
+        B, T, H = x["wI"].shape
+        q = orc.decode_rows(raw(x["qI"]).reshape(-1, d // 2), orc.NVFP4, d,
+                            sf=raw(x["qI_sf"]).reshape(-1, d // 16)).reshape(B, T, H, d)
+        E = x["KI"].shape[1]
+        K = np.stack([orc.decode_rows(raw(x["KI"][b]), orc.NVFP4, d, sf=raw(x["KI_sf"][b]))
+                      for b in range(B)]).reshape(B, E, d)
+        return q, K
+    return f64(x["qI"]), f64(x["KI"])
+
+
+def _run_index(x, q_pos, m, k, dt):
+    gx = _cuda(x)
+    return csa.index_topk(gx["qI"], gx["wI"], gx["KI"], q_pos.to(DEV), m, k, dt=dt, qI_sf=gx["qI_sf"],
+                          KI_sf=gx["KI_sf"], scores=True)
+
+
+def _sorted_idx(idx):
+    """Oracle idx rows (score order) -> ascending index order, -1 at the end."""
+    out = np.full_like(idx, -1)
+    for r in np.ndindex(idx.shape[:-1]):
+        v = np.sort(idx[r][idx[r] >= 0])
+        out[r][:len(v)] = v
+    return out
+
+
+@pytest.mark.parametrize("dt,H,d,E,k", [
+    (csa.BF16, 64, 128, 3000, 512),
+    (csa.F32, 2, 32, 64, 16),
+    (csa.IDX_NVFP4, 64, 128, 2500, 512),
+    (csa.BF16, 8, 64, 700, 100),
+])
+def test_index_topk_bit_exact_on_exact_scores(orc, dt, H, d, E, k):
+    B, T, m = 2, 3, 4
+    x = _exact_index_inputs(B, T, H, d, E, dt, seed=E)
+    q_pos = torch.tensor([[4 * E - 1, 2999, 39], [4 * E + 50, 4 * 512 - 1, 6]], dtype=torch.int64)
+    idx, sc = _run_index(x, q_pos, m, k, dt)
+    q, K = _decode_idx_inputs(orc, x, dt, d)
+    want_sc, want_idx = orc.index_topk(q, f64(x["wI"]), K, q_pos.numpy(), m, k, round_bf16=(dt != csa.F32))
+    got_sc = f64(sc)
+    assert np.array_equal(np.isneginf(got_sc), np.isneginf(want_sc))
+    fin = ~np.isneginf(want_sc)
+    assert np.array_equal(got_sc[fin], want_sc[fin])
+    assert np.array_equal(raw(idx), _sorted_idx(want_idx))
+
+
+@pytest.mark.parametrize("dt,H,d,E,k,T", [
+    (csa.BF16, 64, 128, 5000, 512, 2),
+    (csa.IDX_NVFP4, 64, 128, 5000, 1024, 1),
+    (csa.F32, 2, 32, 64, 16, 256),
+])
+def test_index_topk_random_inputs(orc, dt, H, d, E, k, T):
+    B, m = 2, 4
+    g = W.generator(31 + E)
+    if dt == csa.IDX_NVFP4:
+        qI, qsf = W.nvfp4_rows(g, (B, T, H), d)
+        KI, ksf = W.nvfp4_rows(g, (B, E), d)
+        x = dict(qI=qI, qI_sf=qsf, KI=KI, KI_sf=ksf)
+    else:
+        tdt = torch.float32 if dt == csa.F32 else torch.bfloat16
+        x = dict(qI=W.normal(g, (B, T, H, d), 1.0, tdt), KI=W.normal(g, (B, E, d), 1.0, tdt), qI_sf=None,
+                 KI_sf=None)
+    x["wI"] = W.uniform(g, (B, T, H))
+    if T == 256:
+        q_pos = torch.arange(T, dtype=torch.int64).repeat(B, 1)
+    else:
+        q_pos = torch.tensor([[4 * E - 1] * T, [1500 + 4 * t for t in range(T)]], dtype=torch.int64)
+    idx, sc = _run_index(x, q_pos, m, k, dt)
+    q, K = _decode_idx_inputs(orc, x, dt, d)
+    want_sc, _ = orc.index_topk(q, f64(x["wI"]), K, q_pos.numpy(), m, k, round_bf16=False)
+    got_sc, got_idx = f64(sc), raw(idx)
+    for b in range(B):
+        for t in range(T):
+            vis = orc.visible_entries(int(q_pos[b, t]), m, E)
+            o, gsc = want_sc[b, t, :vis], got_sc[b, t, :vis]
+            rms = math.sqrt(float(np.mean(o * o))) if vis else 0.0
+            if dt == csa.F32:
+                assert_close(gsc, o, atol=1e-5 * (1 + rms), rtol=1e-5, what="f32 scores")
+            else:
+                assert_close(gsc, o, atol=1e-3 * rms, rtol=1e-2, what="scores")
+            assert np.isneginf(got_sc[b, t, vis:]).all()
+            # the GPU selection is exactly the top-k of its own score row ...
+            sel = got_idx[b, t][got_idx[b, t] >= 0]
+            assert np.array_equal(sel, selection_from_scores(gsc, vis, k))
+            assert (got_idx[b, t][len(sel):] == -1).all()
+            # ... and every selected entry is within tolerance of the oracle's k-th best
+            if 0 < k < vis:
+                kth = np.sort(o)[::-1][k - 1]
+                tol = 2e-2 * abs(kth) + 2e-3 * rms
+                assert o[sel].min() >= kth - tol
+
+
+# ------------------------------------------------------------------ attention
+
+def _random_selection(g, B, T, k, vis_rows, drop=0.1):
+    """Random distinct visible entries per query (some slots -1)."""
+    idx = torch.full((B, T, k), -1, dtype=torch.int32)
+    for b in range(B):
+        for t in range(T):
+            vis = int(vis_rows[b][t])
+            n = min(k, vis)
+            if n:
+                sel = torch.randperm(vis, generator=g)[:n].to(torch.int32)
+                keep = torch.rand(n, generator=g) >= drop
+                sel = torch.where(keep, sel, torch.full_like(sel, -1))
+                idx[b, t, torch.randperm(k, generator=g)[:n]] = sel
+    return idx
+
+
+def _mqa_case(orc, cfg_name, B, T, E, k, q0, sink_override=None, dense=False, seed=None):
+    cfg = dict(W.CONFIGS[cfg_name])
+    x = W.attention_inputs(cfg, "cpu", batch=B, ctx=E * cfg["m"], n_q=T, q0=q0, n_entries=E, seed=seed)
+    if sink_override is not None:
+        x["sink"] = torch.tensor(sink_override, dtype=torch.float32)
+    m, W_ = cfg["m"], cfg["window"]
+    scale = 1.0 / math.sqrt(cfg["dim"])
+    vis = [[orc.visible_entries(int(x["q_pos"][b, t]), m, E) for t in range(T)] for b in range(B)]
+    g = torch.Generator().manual_seed(77)
+    gx = _cuda(x)
+    if dense:
+        out = csa.hca_dense_mqa(gx["Q"], gx["entries"], gx["win"], gx["win_start"], gx["q_pos"], W_, m,
+                                gx["sink"], scale, kv_dt=cfg["kv_dt"])
+        want = orc.hca_dense_mqa(f64(x["Q"]), raw(x["entries"]), cfg["kv_dt"], raw(x["win"]),
+                                 raw(x["win_start"]), raw(x["q_pos"]), W_, m, f64(x["sink"]), scale)
+    else:
+        idx = _random_selection(g, B, T, k, vis)
+        out = csa.sparse_mqa(gx["Q"], gx["entries"], idx.to(DEV), gx["win"], gx["win_start"], gx["q_pos"], W_,
+                             m, gx["sink"], scale, kv_dt=cfg["kv_dt"])
+        want = orc.sparse_mqa(f64(x["Q"]), raw(x["entries"]), cfg["kv_dt"], raw(idx), raw(x["win"]),
+                              raw(x["win_start"]), raw(x["q_pos"]), W_, m, f64(x["sink"]), scale)
+    return f64(out), want, cfg
+
+
+@pytest.mark.parametrize("cfg_name,B,T,E,k,q0", [
+    ("tiny_prefill_f32", 1, 256, 64, 16, 0),             # the tiny prefill workload itself
+    ("csa_decode_bf16", 2, 1, 4000, 512, 4 * 4000 - 1),   # decode
+    ("csa_decode_1m_mixed", 2, 1, 3000, 1024, 4 * 3000 - 1),  # FP8MIX entries, 128 heads
+    ("csa_prefill_bf16", 1, 40, 300, 64, 0),              # early queries: t < window, t < m-1
+    ("csa_prefill_bf16", 1, 16, 300, 64, 1100),           # chunk of prefill queries
+])
+def test_sparse_mqa_matches_oracle(orc, cfg_name, B, T, E, k, q0):
+    got, want, cfg = _mqa_case(orc, cfg_name, B, T, E, k, q0)
+    atol = 1e-5 if cfg["q_dt"] == csa.F32 else 2e-2
+    assert_close(got, want, atol=atol, what=cfg_name)
+
+
+@pytest.mark.parametrize("B,T,E,q0", [(2, 1, 300, 128 * 300 - 1), (1, 8, 40, 128 * 30), (1, 3, 5, 0)])
+def test_hca_dense_mqa_matches_oracle(orc, B, T, E, q0):
+    got, want, _ = _mqa_case(orc, "hca_decode_bf16", B, T, E, 0, q0, dense=True)
+    assert_close(got, want, atol=2e-2, what="hca")
+
+
+def test_mqa_sink_limits(orc):
+    H = 4
+    got, want, _ = _mqa_case(orc, "tiny_prefill_f32", 1, 20, 64, 16, 10,
+                             sink_override=[float("inf"), float("-inf"), 30.0, -30.0])
+    assert_close(got, want, atol=1e-5, what="sink limits")
+    assert (got[0, :, 0] == 0).all()
