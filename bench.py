@@ -1,0 +1,514 @@
+"""Benchmark of the CSA / HCA decode (and prefill) hot path on B200.
+
+One step = one pass of the whole hot path over one batch:
+  csa_* workloads: compress the block closed by the newest token (KV entry and
+  indexer key) -> csa_index_topk -> csa_sparse_mqa;
+  hca_decode_bf16: compress the closed 128-token block -> hca_dense_mqa.
+Default workload: "csa_decode_1m_mixed" (4 requests x 1,048,576 tokens,
+262,144 entries each, NVFP4 indexer, FP8/BF16 KV, top-k 1024, 128 heads).
+
+Timing: W warm-up steps, then K timed steps between a barrier + synchronize.
+Before every step a 256 MiB buffer is written to flush L2 (outside the step's
+CUDA events); each step is bracketed by CUDA events on the launching stream,
+and the dominant kernel call (the indexer) by its own events.  Multi-GPU: one
+process per GPU, each rank runs its own independent requests (weak scaling,
+no collective on the data path); the step time is the max over ranks.
+
+`--impl reference` times the float64 CPU oracle (the reference for this
+method) on a bounded sample of the same workload on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from compressed_sparse_attention_hca_b200 import workloads as W  # noqa: E402
+
+METRIC = "CSA decode query-tokens/s at 1M ctx on 1 B200; % of HBM roofline (GB/s)"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(PEAKS_FALLBACK)
+    d["source"] = "fallback"
+    return d
+
+
+# ------------------------------------------------------------------ workload
+
+class Step:
+    """Device-resident inputs and outputs of one hot-path step."""
+
+    def __init__(self, name: str, device, seed_offset: int = 0):
+        from compressed_sparse_attention_hca_b200 import csa
+        self.csa = csa
+        self.name = name
+        self.cfg = cfg = dict(W.CONFIGS[name])
+        cfg["seed"] += 1000 * seed_offset
+        self.dev = device
+        self.kind = cfg["kind"]
+        x = W.attention_inputs(cfg, device)
+        self.x = x
+        m, c = cfg["m"], cfg["dim"]
+        self.scale = 1.0 / math.sqrt(c)
+        B, T, E = x["B"], x["T"], x["E"]
+        g = W.generator(cfg["seed"] + 17, device)
+        # newest tokens: the block closed by the last query token (decode), or
+        # every new token of the chunk (prefill)
+        if self.kind == "csa_prefill":
+            n_new = T
+            self.tok0 = x["q0"] - m
+            self.e0 = x["q0"] // m
+        else:
+            n_new = m
+            self.tok0 = E * m - (2 * m if self.kind.startswith("csa") else m)
+            self.e0 = E - 1
+        rows = n_new + (m if self.kind.startswith("csa") else 0)
+        overlap = self.kind.startswith("csa")
+        self.n_out = n_new // m if self.kind == "csa_prefill" else 1
+        self.tok = W.compress_inputs(g, B, rows, c, m, overlap, torch.bfloat16, c_std=cfg["kv_std"],
+                                     device=device)
+        if overlap:
+            dI = cfg["dI"]
+            self.itok = W.compress_inputs(g, B, rows, dI, m, True, torch.bfloat16, device=device)
+        self.idx = torch.empty(B, T, cfg.get("k", 1), device=device, dtype=torch.int32)
+        self.O = torch.empty_like(x["Q"])
+        self.ws_idx = None
+        self.ws_mqa = None
+        kv_dt = cfg["kv_dt"]
+        if overlap:
+            idt = cfg["idx_dt"]
+            H = cfg["n_hI"]
+            self.ws_idx = torch.empty(csa.index_topk_workspace_size(B, T, E, cfg["k"], H, cfg["dI"], idt),
+                                      device=device, dtype=torch.uint8)
+            self.ws_mqa = torch.empty(csa.sparse_mqa_workspace_size(B, T, cfg["n_h"], c, cfg["k"],
+                                                                    cfg["window"], cfg["q_dt"], kv_dt),
+                                      device=device, dtype=torch.uint8)
+        else:
+            self.ws_mqa = torch.empty(csa.hca_dense_mqa_workspace_size(B, T, cfg["n_h"], c, E, cfg["window"],
+                                                                       cfg["q_dt"], kv_dt),
+                                      device=device, dtype=torch.uint8)
+        self.launches = 0
+
+    def _compress(self):
+        csa, x, cfg, t = self.csa, self.x, self.cfg, self.tok
+        m = cfg["m"]
+        kv_dt = cfg["kv_dt"]
+        csa.compress(t["Ca"], t["Za"], t["Ba"], m, t["Cb"], t["Zb"], t["Bb"], tok0=self.tok0, e0=self.e0,
+                     n_out=self.n_out, out_dt=kv_dt, out=x["entries"], out_row0=self.e0)
+        n = csa.last_launch_count()
+        if self.kind.startswith("csa"):
+            it = self.itok
+            csa.compress(it["Ca"], it["Za"], it["Ba"], m, it["Cb"], it["Zb"], it["Bb"], tok0=self.tok0,
+                         e0=self.e0, n_out=self.n_out, out_dt=cfg["idx_dt"], out=x["KI"],
+                         out_sf=x.get("KI_sf"), out_row0=self.e0)
+            n += csa.last_launch_count()
+        return n
+
+    def index(self):
+        csa, x, cfg = self.csa, self.x, self.cfg
+        csa.index_topk(x["qI"], x["wI"], x["KI"], x["q_pos"], cfg["m"], cfg["k"], dt=cfg["idx_dt"],
+                       qI_sf=x.get("qI_sf"), KI_sf=x.get("KI_sf"), idx_out=self.idx, ws=self.ws_idx)
+        return csa.last_launch_count()
+
+    def attend(self):
+        csa, x, cfg = self.csa, self.x, self.cfg
+        if self.kind.startswith("csa"):
+            csa.sparse_mqa(x["Q"], x["entries"], self.idx, x["win"], x["win_start"], x["q_pos"], cfg["window"],
+                           cfg["m"], x["sink"], self.scale, kv_dt=cfg["kv_dt"], O=self.O, ws=self.ws_mqa)
+        else:
+            csa.hca_dense_mqa(x["Q"], x["entries"], x["win"], x["win_start"], x["q_pos"], cfg["window"],
+                              cfg["m"], x["sink"], self.scale, kv_dt=cfg["kv_dt"], O=self.O, ws=self.ws_mqa)
+        return csa.last_launch_count()
+
+    def run(self, ev=None):
+        """One step; ev = (start, after_compress, after_index, end) CUDA events."""
+        s = torch.cuda.current_stream()
+        if ev:
+            ev[0].record(s)
+        n = self._compress()
+        if ev:
+            ev[1].record(s)
+        if self.kind.startswith("csa"):
+            n += self.index()
+        if ev:
+            ev[2].record(s)
+        n += self.attend()
+        if ev:
+            ev[3].record(s)
+        self.launches = n
+
+    # per-step host<->device traffic for the end-to-end measurement: the new
+    # tokens' projections, the queries (attention + indexer) and the output;
+    # the compressed caches and the window are device-resident state.
+    def step_inputs(self):
+        x = self.x
+        ts = [self.tok[k] for k in ("Ca", "Za", "Cb", "Zb") if self.tok[k] is not None]
+        if self.kind.startswith("csa"):
+            ts += [self.itok[k] for k in ("Ca", "Za", "Cb", "Zb")]
+            ts += [x["qI"], x["wI"]] + ([x["qI_sf"]] if "qI_sf" in x else [])
+        ts += [x["Q"], x["q_pos"]]
+        return ts
+
+    def algorithmic_bytes(self):
+        """Minimum HBM bytes of one step (each byte the step must read or write once)."""
+        x, cfg = self.x, self.cfg
+        B, T, E = x["B"], x["T"], x["E"]
+        c, m = cfg["dim"], cfg["m"]
+        kvb = W.row_bytes(cfg["kv_dt"], c)
+        nb = lambda t: t.numel() * t.element_size()  # noqa: E731
+        comp = sum(nb(self.tok[k]) for k in ("Ca", "Za", "Cb", "Zb") if self.tok[k] is not None)
+        comp += nb(self.tok["Ba"]) + (nb(self.tok["Bb"]) if self.tok["Bb"] is not None else 0)
+        comp += B * self.n_out * kvb
+        if self.kind.startswith("csa"):
+            comp += sum(nb(self.itok[k]) for k in ("Ca", "Za", "Cb", "Zb"))
+            comp += B * self.n_out * (nb(x["KI"][0, 0]) + (nb(x["KI_sf"][0, 0]) if "KI_sf" in x else 0))
+        idx_bytes = self.index_bytes() if self.kind.startswith("csa") else 0
+        if self.kind.startswith("csa"):
+            if self.kind == "csa_prefill":
+                # every entry and window row at least once
+                att = B * (min(E, T * cfg["k"]) + x["Lw"]) * kvb + nb(self.idx)
+            else:
+                att = B * T * (cfg["k"] + cfg["window"]) * kvb + nb(self.idx)
+        else:
+            att = B * (E + cfg["window"]) * kvb
+        att += nb(x["Q"]) + nb(self.O)
+        return comp + idx_bytes + att
+
+    def index_bytes(self):
+        """Algorithmic bytes of one indexer call: every key once, queries, weights, idx."""
+        x = self.x
+        nb = lambda t: t.numel() * t.element_size()  # noqa: E731
+        b = nb(x["KI"]) + nb(x["qI"]) + nb(x["wI"]) + nb(self.idx)
+        if "KI_sf" in x:
+            b += nb(x["KI_sf"]) + nb(x["qI_sf"])
+        return b
+
+    def index_flops(self):
+        x, cfg = self.x, self.cfg
+        tot = 0
+        qp = x["q_pos"].cpu()
+        for b in range(x["B"]):
+            for t in range(x["T"]):
+                tot += min(x["E"], (int(qp[b, t]) + 1) // cfg["m"])
+        return 2.0 * tot * cfg["n_hI"] * cfg["dI"]
+
+
+def l2_flush_buffer(device):
+    return torch.empty(256 * 1024 * 1024 // 4, device=device, dtype=torch.float32)
+
+
+# ------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                       "-lms", "50", "-i", str(gpu_index)], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.seek(0)
+        rows = [ln.split(", ") for ln in self.f.read().strip().splitlines() if ln.count(",") >= 8]
+        os.unlink(self.f.name)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[5:9]):
+                if v.strip() == "Active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU side
+
+def cpu_oracle_step(name: str, sample_entries=None, seed_offset=0):
+    """Runs the oracle on one request of workload `name` (a bounded sample).
+
+    Returns (seconds, query tokens covered, description).  With sample_entries
+    set, the indexer is timed on that many entries and its time scaled to all
+    entries of the request (the indexer is linear in the entry count)."""
+    import numpy as np
+
+    import oracle as orc
+    cfg = dict(W.CONFIGS[name])
+    cfg["seed"] += 1000 * seed_offset
+    E_full = cfg["ctx"] // cfg["m"]
+    E = E_full if sample_entries is None else min(E_full, sample_entries)
+    x = W.attention_inputs(cfg, "cpu", batch=1, n_q=1, n_entries=E_full if cfg["kind"] == "hca_decode" else E,
+                           ctx=cfg["ctx"] if cfg["kind"] == "hca_decode" else E * cfg["m"])
+    m, c = cfg["m"], cfg["dim"]
+
+    def f64(t):
+        return t.detach().cpu().to(torch.float64).numpy()
+
+    def raw(t):
+        t = t.detach().cpu().contiguous()
+        return t.view(torch.int16).numpy().view(np.uint16) if t.dtype == torch.bfloat16 else t.numpy()
+
+    g = W.generator(cfg["seed"] + 17)
+    overlap = cfg["kind"].startswith("csa")
+    tok = W.compress_inputs(g, 1, 2 * m if overlap else m, c, m, overlap, torch.bfloat16, c_std=cfg["kv_std"])
+    t0 = time.perf_counter()
+    kw = dict(Cb=f64(tok["Cb"][0]), Zb=f64(tok["Zb"][0]), Bb=f64(tok["Bb"])) if overlap else {}
+    orc.compress(f64(tok["Ca"][0]), f64(tok["Za"][0]), f64(tok["Ba"]), m,
+                 tok0=(E - 2) * m if overlap else (E - 1) * m, e0=E - 1, n_out=1, **kw)
+    t_comp = time.perf_counter() - t0
+    t_idx = 0.0
+    scale = 1.0 / math.sqrt(c)
+    if overlap:
+        dI = cfg["dI"]
+        t0 = time.perf_counter()
+        if cfg["idx_dt"] == W.NVFP4:
+            q = orc.decode_rows(raw(x["qI"]).reshape(-1, dI // 2), orc.NVFP4, dI,
+                                sf=raw(x["qI_sf"]).reshape(-1, dI // 16)).reshape(1, 1, -1, dI)
+            K = orc.decode_rows(raw(x["KI"][0]), orc.NVFP4, dI, sf=raw(x["KI_sf"][0]))[None]
+        else:
+            q, K = f64(x["qI"]), f64(x["KI"])
+        _, idx = orc.index_topk(q, f64(x["wI"]), K, raw(x["q_pos"]), m, cfg["k"], want_scores=False)
+        t_idx = (time.perf_counter() - t0) * (E_full / E)
+        t0 = time.perf_counter()
+        orc.sparse_mqa(f64(x["Q"]), raw(x["entries"]), cfg["kv_dt"], idx, raw(x["win"]), raw(x["win_start"]),
+                       raw(x["q_pos"]), cfg["window"], m, f64(x["sink"]), scale)
+        t_att = time.perf_counter() - t0
+    else:
+        t0 = time.perf_counter()
+        orc.hca_dense_mqa(f64(x["Q"]), raw(x["entries"]), cfg["kv_dt"], raw(x["win"]), raw(x["win_start"]),
+                          raw(x["q_pos"]), cfg["window"], m, f64(x["sink"]), scale)
+        t_att = time.perf_counter() - t0
+    total = t_comp + t_idx + t_att
+    desc = (f"oracle (float64, single thread) on 1 request of {name}: compress 1 block, "
+            + (f"indexer over {E} of {E_full} entries scaled x{E_full / E:.1f}, " if overlap else "")
+            + ("top-k + sparse MQA" if overlap else "dense MQA over all entries"))
+    return total, 1, desc
+
+
+def reference_arm(args):
+    """`--impl reference`: the oracle on the host cores, same metric and workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    name = args.config
+    sample = 8192 if W.CONFIGS[name]["kind"].startswith("csa") else None
+    times = []
+    for i in range(args.warmup + args.steps):
+        t, n, desc = cpu_oracle_step(name, sample_entries=sample, seed_offset=i)
+        if i >= args.warmup:
+            times.append(t / n)
+    per_tok = statistics.mean(times)
+    value = 1.0 / per_tok
+    line = {
+        "impl": "reference", "metric": METRIC if name == "csa_decode_1m_mixed" else f"{name} query-tokens/s",
+        "value": value, "unit": "query-tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": per_tok * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": name},
+        "cpu_baseline": {"value": value, "unit": "query-tokens/s", "cores": 1, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "query-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU side
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--config", default="csa_decode_1m_mixed", choices=sorted(W.CONFIGS))
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    if args.impl == "reference":
+        reference_arm(args)
+        return
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from compressed_sparse_attention_hca_b200 import csa
+    csa.load()
+    peaks = load_peaks()
+    step = Step(args.config, dev, seed_offset=rank)
+    flush = l2_flush_buffer(dev)
+    for _ in range(args.warmup):
+        flush.zero_()
+        step.run()
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    launches = 0
+    for i in range(args.steps):
+        flush.zero_()
+        step.run(evs[i])
+        launches += step.launches
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    clk = clocks.stop()
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    idx_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    x = step.x
+    tokens_per_step = x["B"] * x["T"]
+    value = world * tokens_per_step / (ms_per_step / 1e3)
+
+    # dominant kernel roofline
+    kind = step.kind
+    if kind.startswith("csa"):
+        idx_avg_ms = statistics.mean(idx_ms)
+        if kind == "csa_prefill":
+            peak = peaks.get("bf16_tflops", PEAKS_FALLBACK["bf16_tflops"])
+            ach = step.index_flops() / (idx_avg_ms / 1e3) / 1e12
+            roof = {"kernel": "csa_index_topk", "bound": "tensor", "achieved": ach, "peak": peak,
+                    "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                    "note": f"bf16 dense peak, {peaks['source']}"}
+        else:
+            peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+            ach = step.index_bytes() / (idx_avg_ms / 1e3) / 1e9
+            roof = {"kernel": "csa_index_topk", "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+                    "frac": ach / peak, "traffic": None, "algorithmic_bytes": step.index_bytes(),
+                    "avg_launch_ms": idx_avg_ms, "note": f"HBM copy peak, {peaks['source']}"}
+    else:
+        att_ms = statistics.mean([e[2].elapsed_time(e[3]) for e in evs])
+        peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
+        b = step.algorithmic_bytes()
+        ach = b / (att_ms / 1e3) / 1e9
+        roof = {"kernel": "hca_dense_mqa", "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+                "frac": ach / peak, "traffic": None, "avg_launch_ms": att_ms,
+                "note": f"HBM copy peak, {peaks['source']}"}
+    step_bytes = step.algorithmic_bytes()
+    step_gbs = step_bytes / (ms_per_step / 1e3) / 1e9
+
+    # end to end through the public API with host buffers
+    e2e = measure_e2e(step, args, flush, dev, dist, world)
+
+    line = {
+        "metric": METRIC if args.config == "csa_decode_1m_mixed" else f"{args.config} query-tokens/s",
+        "value": value, "unit": "query-tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": dtype_label(step.cfg), "data": "synthetic",
+        "config": {"workload": args.config, "batch_per_gpu": x["B"], "ctx": step.cfg["ctx"],
+                   "entries_per_request": x["E"], "query_tokens_per_request": x["T"],
+                   "top_k": step.cfg.get("k"), "n_heads": step.cfg["n_h"], "window": step.cfg["window"],
+                   "parallelism": f"replicas x{world} (independent requests per GPU)",
+                   "l2": "flushed before every step (256 MiB write outside the step events)"},
+        "roofline": roof,
+        "step_hbm": {"algorithmic_bytes": step_bytes, "achieved_gbs": step_gbs,
+                     "frac": step_gbs / peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])},
+        "e2e": e2e,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t, n, desc = cpu_oracle_step(args.config, sample_entries=65536 if kind.startswith("csa") else None)
+        line["cpu_baseline"] = {"value": n / t, "unit": "query-tokens/s", "cores": 1, "kind": "oracle",
+                                "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def dtype_label(cfg):
+    names = {W.F32: "f32", W.BF16: "bf16", W.FP8MIX: "fp8e4m3+bf16", W.NVFP4: "nvfp4"}
+    parts = [f"kv {names[cfg['kv_dt']]}"]
+    if "idx_dt" in cfg:
+        parts.insert(0, f"indexer {names[cfg['idx_dt']]}")
+    return ", ".join(parts) + ", fp32 accumulate"
+
+
+def measure_e2e(step, args, flush, dev, dist, world):
+    """Same step through the public API with host buffers: each step copies its
+    inputs from pinned host memory and reads the output back."""
+    ins = step.step_inputs()
+    host = [t.detach().cpu().pin_memory() for t in ins]
+    out_host = torch.empty(step.O.shape, dtype=step.O.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for t in host)
+    d2h = out_host.numel() * out_host.element_size()
+    n = max(3, min(args.steps, 100))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    s = torch.cuda.current_stream()
+    for i in range(n + 2):
+        flush.zero_()
+        e = evs[i - 2] if i >= 2 else None
+        if e:
+            e[0].record(s)
+        for d, h in zip(ins, host):
+            d.copy_(h, non_blocking=True)
+        step.run()
+        out_host.copy_(step.O, non_blocking=True)
+        if e:
+            e[1].record(s)
+    torch.cuda.synchronize()
+    total = sum(a.elapsed_time(b) for a, b in evs)
+    if dist:
+        t = torch.tensor([total], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total = float(t.item())
+    ms = total / n
+    x = step.x
+    return {"value": world * x["B"] * x["T"] / (ms / 1e3), "unit": "query-tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms}
+
+
+if __name__ == "__main__":
+    main()

@@ -49,6 +49,7 @@ def load():
     sigs = {
         "csa_last_error": (ctypes.c_char_p, []),
         "csa_version": (i32, []),
+        "csa_last_launch_count": (i32, []),
         "csa_row_bytes": (i64, [i32, i32]),
         "csa_compress": (i32, [P, P, P, P, P, P, i32, i64, i64, i64, i64, i64, i32, i32, i32, P, P,
                                i64, i32, P]),
@@ -84,6 +85,11 @@ def _check(status):
 
 def _dt_of(t):
     return F32 if t.dtype == torch.float32 else BF16
+
+
+def last_launch_count():
+    """Kernels launched by this thread's last library call."""
+    return int(load().csa_last_launch_count())
 
 
 def row_bytes(dt, dim):

@@ -10,6 +10,7 @@
 namespace {
 
 thread_local char g_err[512] = "";
+thread_local int g_launches = 0;
 
 csa_status_t fail(csa_status_t st, const char* fmt, ...) {
   va_list ap;
@@ -50,9 +51,13 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 }  // namespace
 
+int& csa::launch_counter() { return g_launches; }
+
 extern "C" {
 
 const char* csa_last_error(void) { return g_err; }
+
+int csa_last_launch_count(void) { return g_launches; }
 
 int csa_version(void) { return 100; }
 
@@ -68,6 +73,7 @@ csa_status_t csa_compress(const void* Ca, const void* Cb, const void* Za, const 
                           int64_t tok0, int64_t in_batch_stride, int64_t e0, int64_t n_out,
                           int dim, int m, csa_dtype_t in_dt, void* out, void* out_sf,
                           int64_t out_batch_stride, csa_dtype_t out_dt, void* stream) {
+  g_launches = 0;
   REQUIRE(batch >= 0 && n_tok >= 0 && tok0 >= 0 && e0 >= 0 && n_out >= 0,
           "negative size (batch=%d n_tok=%lld tok0=%lld e0=%lld n_out=%lld)", batch,
           (long long)n_tok, (long long)tok0, (long long)e0, (long long)n_out);
@@ -117,6 +123,7 @@ csa_status_t csa_index_topk(const void* qI, const void* qI_sf, const float* wI, 
                             int64_t n_entries, int m, int n_heads, int dim, int k, csa_dtype_t dt,
                             int32_t* idx_out, void* scores_out, void* ws, size_t ws_bytes,
                             void* stream) {
+  g_launches = 0;
   REQUIRE(batch >= 0 && n_q >= 0 && n_entries >= 0, "negative size");
   REQUIRE(n_entries <= (int64_t)1 << 30, "n_entries=%lld too large", (long long)n_entries);
   REQUIRE(m >= 1, "m=%d must be >= 1", m);
@@ -161,6 +168,7 @@ csa_status_t check_mqa(const csa::MqaArgs& a) {
 }
 
 csa_status_t run_mqa(csa::MqaArgs& a, void* stream, const char* name) {
+  g_launches = 0;
   csa_status_t st = check_mqa(a);
   if (st != CSA_OK) return st;
   if ((int64_t)a.batch * a.n_q == 0) return ok();

@@ -194,6 +194,7 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s) {
   const int threads = 256;
   const int64_t blocks = (total + threads - 1) / threads;
   compress_kernel<<<(unsigned)blocks, threads, 0, s>>>(a);
+  ++launch_counter();
   return cudaGetLastError();
 }
 

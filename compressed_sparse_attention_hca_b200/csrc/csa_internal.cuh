@@ -134,8 +134,10 @@ __device__ __forceinline__ float key_to_f32(uint32_t k) {
 
 // ---------------------------------------------------------------------------
 // Internal launchers (one per translation unit); all return cudaError_t of the
-// launch (cudaGetLastError) and never allocate.
+// launch (cudaGetLastError) and never allocate.  Each kernel launch bumps the
+// calling thread's launch counter (reported by csa_last_launch_count).
 // ---------------------------------------------------------------------------
+int& launch_counter();
 struct CompressArgs {
   const void *Ca, *Cb, *Za, *Zb;
   const float *Ba, *Bb;

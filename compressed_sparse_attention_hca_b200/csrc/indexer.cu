@@ -159,9 +159,11 @@ cudaError_t launch_index_simt(const IndexArgs& a, const IndexPlan& plan, cudaStr
   if (e != cudaSuccess) return e;
   dim3 grid(plan.n_slices, a.n_q, a.batch);
   index_slice_simt_kernel<<<grid, kNT, smem, s>>>(a, plan);
+  ++launch_counter();
   e = cudaGetLastError();
   if (e != cudaSuccess || plan.n_slices == 1) return e;
   index_merge_kernel<<<dim3(a.n_q, a.batch), kMergeNT, 0, s>>>(a, plan);
+  ++launch_counter();
   return cudaGetLastError();
 }
 

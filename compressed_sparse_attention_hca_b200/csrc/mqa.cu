@@ -193,9 +193,11 @@ cudaError_t launch_mqa_simt(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) 
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_splits, a.n_heads / p.heads_per_cta, (unsigned)((int64_t)a.batch * a.n_q));
   mqa_simt_kernel<<<grid, 32 * p.heads_per_cta, smem, s>>>(a, p);
+  ++launch_counter();
   e = cudaGetLastError();
   if (e != cudaSuccess || p.n_splits == 1) return e;
   mqa_combine_kernel<<<dim3(a.n_heads, (unsigned)((int64_t)a.batch * a.n_q)), 128, 0, s>>>(a, p);
+  ++launch_counter();
   return cudaGetLastError();
 }
 

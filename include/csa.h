@@ -80,6 +80,10 @@ const char* csa_last_error(void);
 /* Library ABI version (major * 100 + minor). */
 int csa_version(void);
 
+/* Number of kernels the calling thread's last compute call launched (0 when
+ * it returned before launching). */
+int csa_last_launch_count(void);
+
 /* Bytes per row of format dt at dimension dim (codes only for NVFP4), or -1
  * when dim is not valid for the format. */
 int64_t csa_row_bytes(csa_dtype_t dt, int dim);
