@@ -53,6 +53,8 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 int& csa::launch_counter() { return g_launches; }
 
+csa_status_t csa::set_error(csa_status_t st, const char* msg) { return fail(st, "%s", msg); }
+
 extern "C" {
 
 const char* csa_last_error(void) { return g_err; }

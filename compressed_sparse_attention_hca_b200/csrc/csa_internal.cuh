@@ -138,6 +138,8 @@ __device__ __forceinline__ float key_to_f32(uint32_t k) {
 // calling thread's launch counter (reported by csa_last_launch_count).
 // ---------------------------------------------------------------------------
 int& launch_counter();
+// Records `msg` as the calling thread's last error and returns `st`.
+csa_status_t set_error(csa_status_t st, const char* msg);
 struct CompressArgs {
   const void *Ca, *Cb, *Za, *Zb;
   const float *Ba, *Bb;

@@ -152,6 +152,32 @@ csa_status_t csa_index_topk(const void* qI, const void* qI_sf, const float* wI, 
                             void* stream);
 
 /*
+ * csa_index_topk_noalloc -- csa_index_topk for callers that cannot allocate
+ * device memory.  The paper has no counterpart: this is a library service.
+ *
+ * Some callers have no allocator to draw a workspace from (a plugin inside a
+ * host that owns all device memory, or a serving loop that forbids
+ * cudaMalloc after start-up because it can synchronise the device).  This
+ * call takes the same inputs and outputs as csa_index_topk, minus the
+ * workspace, and runs the same kernels; its scratch is a 4 MiB array built
+ * into the library, resident on every GPU that loads the library until the
+ * process exits.  It calls no cudaMalloc, cudaFree or allocating routine.
+ *   - Shapes whose csa_index_topk_workspace_size exceeds 4 MiB (4194304
+ *     bytes) are rejected with CSA_ERR_INVALID_ARG before any launch.
+ *   - The first call on a device (with that device current) looks up the
+ *     array's device address; make that first call before any stream capture.
+ *   - All calls on a device share the one array and it keeps the previous
+ *     call's contents; calls that may overlap on the GPU (other streams or
+ *     host threads) race on it, so serialise them.  Nothing in it needs to
+ *     start at zero.
+ */
+csa_status_t csa_index_topk_noalloc(const void* qI, const void* qI_sf, const float* wI,
+                                    const void* KI, const void* KI_sf, const int64_t* q_pos,
+                                    int batch, int n_q, int64_t n_entries, int m, int n_heads,
+                                    int dim, int k, csa_dtype_t dt, int32_t* idx_out,
+                                    void* scores_out, void* stream);
+
+/*
  * csa_sparse_mqa -- CSA core attention: shared-KV multi-query attention over
  * the selected compressed entries plus the sliding window, with a per-head
  * attention sink ([P5] 1.2 Step 2, 1.4 table rows "Sliding-Window" and
