@@ -50,6 +50,7 @@ def load():
         "csa_last_error": (ctypes.c_char_p, []),
         "csa_version": (i32, []),
         "csa_last_launch_count": (i32, []),
+        "csa_check_device_status": (i32, []),
         "csa_row_bytes": (i64, [i32, i32]),
         "csa_compress": (i32, [P, P, P, P, P, P, i32, i64, i64, i64, i64, i64, i32, i32, i32, P, P,
                                i64, i32, P]),
@@ -85,6 +86,11 @@ def _check(status):
 
 def _dt_of(t):
     return F32 if t.dtype == torch.float32 else BF16
+
+
+def check_device_status():
+    """Synchronises the device; raises CsaError if a kernel wait timed out."""
+    _check(load().csa_check_device_status())
 
 
 def last_launch_count():

@@ -138,6 +138,9 @@ __device__ __forceinline__ float key_to_f32(uint32_t k) {
 // calling thread's launch counter (reported by csa_last_launch_count).
 // ---------------------------------------------------------------------------
 int& launch_counter();
+// Status words of the kernels with bounded waits (read and cleared; nonzero
+// means a wait gave up, 2 means the word could not be read).
+unsigned int take_status_indexer_tc();
 // Records `msg` as the calling thread's last error and returns `st`.
 csa_status_t set_error(csa_status_t st, const char* msg);
 struct CompressArgs {

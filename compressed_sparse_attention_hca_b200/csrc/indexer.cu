@@ -169,12 +169,23 @@ cudaError_t launch_index_simt(const IndexArgs& a, const IndexPlan& plan, cudaStr
 
 size_t index_topk_workspace(int batch, int n_q, int64_t n_entries, int k, int n_heads, int dim,
                             int dt) {
-  (void)n_heads; (void)dim; (void)dt;
+  IndexArgs probe{};
+  probe.batch = batch; probe.n_q = n_q; probe.n_entries = n_entries; probe.k = k;
+  probe.n_heads = n_heads; probe.dim = dim; probe.dt = dt;
+  if (index_tc_eligible(probe)) return plan_workspace_bytes(make_tc_plan(batch, n_q, n_entries, k));
   return plan_workspace_bytes(make_simt_plan(batch, n_q, n_entries, k));
 }
 
 cudaError_t launch_index_topk(const IndexArgs& a, cudaStream_t s) {
   if ((int64_t)a.batch * a.n_q == 0) return cudaSuccess;
+  if (index_tc_eligible(a)) {
+    const IndexPlan plan = make_tc_plan(a.batch, a.n_q, a.n_entries, a.k);
+    cudaError_t e = launch_index_tc(a, plan, s);
+    if (e != cudaSuccess || plan.n_slices == 1) return e;
+    index_merge_kernel<<<dim3(a.n_q, a.batch), kMergeNT, 0, s>>>(a, plan);
+    ++launch_counter();
+    return cudaGetLastError();
+  }
   const IndexPlan plan = make_simt_plan(a.batch, a.n_q, a.n_entries, a.k);
   return launch_index_simt(a, plan, s);
 }

@@ -56,4 +56,10 @@ inline size_t plan_workspace_bytes(const IndexPlan& p) {
   return (size_t)p.n_rows * (size_t)p.cand_cap * 8;
 }
 
+// Tensor-core producer (indexer_tc.cu): BF16 q / K with 64 heads of dim 128.
+struct IndexArgs;
+bool index_tc_eligible(const IndexArgs& a);
+IndexPlan make_tc_plan(int batch, int n_q, int64_t n_entries, int k);
+cudaError_t launch_index_tc(const IndexArgs& a, const IndexPlan& p, cudaStream_t s);
+
 }  // namespace csa

@@ -12,8 +12,21 @@
 
 namespace csa {
 
-// Device status word: bit 0 = a bounded wait gave up.
-extern __device__ unsigned int g_device_status;
+// Device status word of this translation unit: bit 0 = a bounded wait gave
+// up.  Each .cu file that includes this header gets its own word and exposes a
+// reader with CSA_DEFINE_STATUS_READER; csa_check_device_status collects them.
+static __device__ unsigned int g_device_status = 0;
+
+#define CSA_DEFINE_STATUS_READER(fname)                                              \
+  unsigned int fname() {                                                             \
+    unsigned int v = 0;                                                              \
+    if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v)) != cudaSuccess) return 2u; \
+    if (v != 0) {                                                                    \
+      const unsigned int z = 0;                                                      \
+      cudaMemcpyToSymbol(g_device_status, &z, sizeof(z));                            \
+    }                                                                                \
+    return v;                                                                        \
+  }
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
 

@@ -84,6 +84,12 @@ int csa_version(void);
  * it returned before launching). */
 int csa_last_launch_count(void);
 
+/* Synchronises the current device and reports whether any tensor-core kernel
+ * gave up a bounded pipeline wait since the last check (CSA_ERR_TIMEOUT: the
+ * results of the affected calls are invalid; the flag is cleared).  Kernels
+ * never spin without a limit, so a broken pipeline ends instead of hanging. */
+csa_status_t csa_check_device_status(void);
+
 /* Bytes per row of format dt at dimension dim (codes only for NVFP4), or -1
  * when dim is not valid for the format. */
 int64_t csa_row_bytes(csa_dtype_t dt, int dim);

@@ -175,17 +175,22 @@ def _sorted_idx(idx):
     return out
 
 
-@pytest.mark.parametrize("dt,H,d,E,k", [
-    (csa.BF16, 64, 128, 3000, 512),
-    (csa.F32, 2, 32, 64, 16),
-    (csa.IDX_NVFP4, 64, 128, 2500, 512),
-    (csa.BF16, 8, 64, 700, 100),
+@pytest.mark.parametrize("dt,H,d,E,k,T", [
+    (csa.BF16, 64, 128, 3000, 512, 3),      # tensor-core producer, 2 queries per CTA, merge
+    (csa.BF16, 64, 128, 20000, 1024, 1),    # tensor-core producer, decode slices, merge
+    (csa.BF16, 64, 128, 9000, 512, 16),     # tensor-core producer, prefill-like rows
+    (csa.F32, 2, 32, 64, 16, 3),
+    (csa.IDX_NVFP4, 64, 128, 2500, 512, 3),
+    (csa.BF16, 8, 64, 700, 100, 3),
 ])
-def test_index_topk_bit_exact_on_exact_scores(orc, dt, H, d, E, k):
-    B, T, m = 2, 3, 4
+def test_index_topk_bit_exact_on_exact_scores(orc, dt, H, d, E, k, T):
+    B, m = 2, 4
     x = _exact_index_inputs(B, T, H, d, E, dt, seed=E)
-    q_pos = torch.tensor([[4 * E - 1, 2999, 39], [4 * E + 50, 4 * 512 - 1, 6]], dtype=torch.int64)
+    base = [[4 * E - 1, 2999, 39], [4 * E + 50, 4 * 512 - 1, 6]]
+    q_pos = torch.tensor([[base[b][t % 3] - 13 * (t // 3) for t in range(T)] for b in range(B)],
+                         dtype=torch.int64).clamp(min=0)
     idx, sc = _run_index(x, q_pos, m, k, dt)
+    csa.check_device_status()
     q, K = _decode_idx_inputs(orc, x, dt, d)
     want_sc, want_idx = orc.index_topk(q, f64(x["wI"]), K, q_pos.numpy(), m, k, round_bf16=(dt != csa.F32))
     got_sc = f64(sc)
@@ -217,6 +222,7 @@ def test_index_topk_random_inputs(orc, dt, H, d, E, k, T):
     else:
         q_pos = torch.tensor([[4 * E - 1] * T, [1500 + 4 * t for t in range(T)]], dtype=torch.int64)
     idx, sc = _run_index(x, q_pos, m, k, dt)
+    csa.check_device_status()
     q, K = _decode_idx_inputs(orc, x, dt, d)
     want_sc, _ = orc.index_topk(q, f64(x["wI"]), K, q_pos.numpy(), m, k, round_bf16=False)
     got_sc, got_idx = f64(sc), raw(idx)
