@@ -172,14 +172,14 @@ size_t index_topk_workspace(int batch, int n_q, int64_t n_entries, int k, int n_
   IndexArgs probe{};
   probe.batch = batch; probe.n_q = n_q; probe.n_entries = n_entries; probe.k = k;
   probe.n_heads = n_heads; probe.dim = dim; probe.dt = dt;
-  if (index_tc_eligible(probe)) return plan_workspace_bytes(make_tc_plan(batch, n_q, n_entries, k));
+  if (index_tc_eligible(probe)) return plan_workspace_bytes(make_tc_plan(batch, n_q, n_entries, k, dt));
   return plan_workspace_bytes(make_simt_plan(batch, n_q, n_entries, k));
 }
 
 cudaError_t launch_index_topk(const IndexArgs& a, cudaStream_t s) {
   if ((int64_t)a.batch * a.n_q == 0) return cudaSuccess;
   if (index_tc_eligible(a)) {
-    const IndexPlan plan = make_tc_plan(a.batch, a.n_q, a.n_entries, a.k);
+    const IndexPlan plan = make_tc_plan(a.batch, a.n_q, a.n_entries, a.k, a.dt);
     cudaError_t e = launch_index_tc(a, plan, s);
     if (e != cudaSuccess || plan.n_slices == 1) return e;
     index_merge_kernel<<<dim3(a.n_q, a.batch), kMergeNT, 0, s>>>(a, plan);

@@ -59,7 +59,7 @@ inline size_t plan_workspace_bytes(const IndexPlan& p) {
 // Tensor-core producer (indexer_tc.cu): BF16 q / K with 64 heads of dim 128.
 struct IndexArgs;
 bool index_tc_eligible(const IndexArgs& a);
-IndexPlan make_tc_plan(int batch, int n_q, int64_t n_entries, int k);
+IndexPlan make_tc_plan(int batch, int n_q, int64_t n_entries, int k, int dt);
 cudaError_t launch_index_tc(const IndexArgs& a, const IndexPlan& p, cudaStream_t s);
 
 }  // namespace csa

@@ -180,7 +180,9 @@ def _sorted_idx(idx):
     (csa.BF16, 64, 128, 20000, 1024, 1),    # tensor-core producer, decode slices, merge
     (csa.BF16, 64, 128, 9000, 512, 16),     # tensor-core producer, prefill-like rows
     (csa.F32, 2, 32, 64, 16, 3),
-    (csa.IDX_NVFP4, 64, 128, 2500, 512, 3),
+    (csa.IDX_NVFP4, 64, 128, 2500, 512, 3),   # tensor-core producer (fp16 expansion)
+    (csa.IDX_NVFP4, 64, 128, 30000, 1024, 1),  # tensor-core producer, decode slices
+    (csa.IDX_NVFP4, 64, 128, 2501, 512, 3),   # odd entry count: SIMT producer
     (csa.BF16, 8, 64, 700, 100, 3),
 ])
 def test_index_topk_bit_exact_on_exact_scores(orc, dt, H, d, E, k, T):
