@@ -65,39 +65,40 @@ __global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
 
   OnlineSoftmax8 sm;
   sm.init();
-  float z[8], c[8], bias[8], logit[8];
   const int64_t in_base = (int64_t)b * a.in_batch_stride;
-  if (valid) {
-    // current group (a-branch)
-    for (int j = 0; j < a.m; ++j) {
-      const int64_t r = a.m * i + j - a.tok0;
-      const int64_t off = (in_base + r) * a.dim + d0;
-      load8(a.Za, a.in_dt, off, z);
-      load8(a.Ca, a.in_dt, off, c);
-      const float4* bp = reinterpret_cast<const float4*>(a.Ba + (int64_t)j * a.dim + d0);
-      float4 b0 = __ldg(bp), b1 = __ldg(bp + 1);
-      bias[0] = b0.x; bias[1] = b0.y; bias[2] = b0.z; bias[3] = b0.w;
-      bias[4] = b1.x; bias[5] = b1.y; bias[6] = b1.z; bias[7] = b1.w;
+  // One branch: tokens tok_first .. tok_first+m-1 with biases B[0..m).  Tokens
+  // are taken kTB at a time and all their loads are issued before any is used,
+  // so a thread waits one memory latency per batch rather than per token.
+  auto branch = [&](const void* C, const void* Z, const float* Bias, int64_t tok_first) {
+    constexpr int kTB = 4;
+    for (int j0 = 0; j0 < a.m; j0 += kTB) {
+      float z[kTB][8], c[kTB][8], bias[kTB][8];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) logit[q] = z[q] + bias[q];
-      sm.add(logit, c);
-    }
-    // previous group (b-branch), CSA only, absent for entry 0
-    if (a.Cb != nullptr && i >= 1) {
-      for (int j = 0; j < a.m; ++j) {
-        const int64_t r = a.m * (i - 1) + j - a.tok0;
-        const int64_t off = (in_base + r) * a.dim + d0;
-        load8(a.Zb, a.in_dt, off, z);
-        load8(a.Cb, a.in_dt, off, c);
-        const float4* bp = reinterpret_cast<const float4*>(a.Bb + (int64_t)j * a.dim + d0);
-        float4 b0 = __ldg(bp), b1 = __ldg(bp + 1);
-        bias[0] = b0.x; bias[1] = b0.y; bias[2] = b0.z; bias[3] = b0.w;
-        bias[4] = b1.x; bias[5] = b1.y; bias[6] = b1.z; bias[7] = b1.w;
+      for (int u = 0; u < kTB; ++u) {
+        if (j0 + u < a.m) {
+          const int64_t off = (in_base + tok_first + j0 + u - a.tok0) * a.dim + d0;
+          load8(Z, a.in_dt, off, z[u]);
+          load8(C, a.in_dt, off, c[u]);
+          const float4* bp = reinterpret_cast<const float4*>(Bias + (int64_t)(j0 + u) * a.dim + d0);
+          const float4 b0 = __ldg(bp), b1 = __ldg(bp + 1);
+          bias[u][0] = b0.x; bias[u][1] = b0.y; bias[u][2] = b0.z; bias[u][3] = b0.w;
+          bias[u][4] = b1.x; bias[u][5] = b1.y; bias[u][6] = b1.z; bias[u][7] = b1.w;
+        }
+      }
 #pragma unroll
-        for (int q = 0; q < 8; ++q) logit[q] = z[q] + bias[q];
-        sm.add(logit, c);
+      for (int u = 0; u < kTB; ++u) {
+        if (j0 + u < a.m) {
+          float logit[8];
+#pragma unroll
+          for (int q = 0; q < 8; ++q) logit[q] = z[u][q] + bias[u][q];
+          sm.add(logit, c[u]);
+        }
       }
     }
+  };
+  if (valid) {
+    branch(a.Ca, a.Za, a.Ba, a.m * i);                                       // current group
+    if (a.Cb != nullptr && i >= 1) branch(a.Cb, a.Zb, a.Bb, a.m * (i - 1));  // previous group (CSA)
   }
   float x[8];
 #pragma unroll

@@ -100,30 +100,85 @@ __global__ void __launch_bounds__(kNT) index_slice_simt_kernel(IndexArgs a, Inde
     const int64_t off = slice_cand_offset(plan, sl, vis, a.n_entries, a.k);
     uint32_t* ck = plan_cand_keys(plan, a.ws, bt) + off;
     int32_t* ci = plan_cand_idx(plan, a.ws, bt) + off;
-    block_select<kNT>(key_at, n_valid, kk, passes, sm, [&](int slot, int pos) {
-      ck[slot] = keys[pos];
-      ci[slot] = (int32_t)(s0 + pos);
-    });
+    uint32_t T = 0;
+    block_select<kNT>(
+        key_at, n_valid, kk, passes, sm,
+        [&](int slot, int pos) {
+          ck[slot] = keys[pos];
+          ci[slot] = (int32_t)(s0 + pos);
+        },
+        0u, &T);
+    if (threadIdx.x == 0) plan_cand_thr(plan, a.ws, bt)[sl] = T;
   }
 }
 
 }  // namespace
 
+// Final selection of one query row among the per-slice candidates.  The
+// candidate keys are first copied into shared memory with batches of
+// independent, coalesced loads (up to kMergeSmemKeys of them), so the
+// range-adaptive radix select runs on shared memory; the final k-th key is at
+// least every slice's own k-th key, which serves as the floor.
 __global__ void __launch_bounds__(kMergeNT) index_merge_kernel(IndexArgs a, IndexPlan plan) {
+  extern __shared__ __align__(16) uint32_t merge_keys[];
   __shared__ SelectSmem<kMergeNT> sm;
+  __shared__ uint32_t floor_s;
   const int t = blockIdx.x, b = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t bt = (int64_t)b * a.n_q + t;
   const int64_t vis = visible_entries(a.q_pos[bt], a.m, a.n_entries);
-  const int64_t total = slice_cand_offset(plan, plan.n_slices, vis, a.n_entries, a.k);
+  const int n = (int)slice_cand_offset(plan, plan.n_slices, vis, a.n_entries, a.k);
   const uint32_t* ck = plan_cand_keys(plan, a.ws, bt);
   const int32_t* ci = plan_cand_idx(plan, a.ws, bt);
-  const int n = (int)total;
   const int kk = (int)min64(min64(a.k, vis), n);
   int32_t* out = a.idx_out + bt * a.k;
-  const int passes = a.dt == CSA_F32 ? 4 : 2;
-  block_select<kMergeNT>([&](int i) { return ck[i]; }, n, kk, passes, sm,
-                         [&](int slot, int pos) { out[slot] = ci[pos]; });
+  if (warp == 0) {
+    const uint32_t* thr = plan_cand_thr(plan, a.ws, bt);
+    uint32_t f = 0;
+    for (int j = lane; j < plan.n_slices; j += 32) f = max(f, thr[j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) f = max(f, __shfl_xor_sync(0xffffffffu, f, o));
+    if (lane == 0) floor_s = f;
+  }
+  const bool staged = n <= kMergeSmemKeys;
+  if (staged) {
+    constexpr int kBatch = 8;
+    for (int base = 0; base < n; base += kMergeNT * kBatch) {
+      uint32_t kv[kBatch];
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = base + u * kMergeNT + threadIdx.x;
+        kv[u] = i < n ? ck[i] : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < kBatch; ++u) {
+        const int i = base + u * kMergeNT + threadIdx.x;
+        if (i < n) merge_keys[i] = kv[u];
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t floor = floor_s;
+  auto emit = [&](int slot, int pos) { out[slot] = ci[pos]; };
+  if (staged)
+    block_select<kMergeNT>([&](int i) { return merge_keys[i]; }, n, kk, 0, sm, emit, floor);
+  else
+    block_select<kMergeNT>([&](int i) { return ck[i]; }, n, kk, 0, sm, emit, floor);
   for (int j = kk + threadIdx.x; j < a.k; j += kMergeNT) out[j] = -1;
+}
+
+size_t index_merge_smem(const IndexPlan& plan) {
+  const int64_t cap = plan.cand_cap < kMergeSmemKeys ? plan.cand_cap : kMergeSmemKeys;
+  return (size_t)cap * 4;
+}
+
+cudaError_t launch_index_merge(const IndexArgs& a, const IndexPlan& plan, cudaStream_t s) {
+  const size_t smem = index_merge_smem(plan);
+  cudaError_t e = cudaFuncSetAttribute(index_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  index_merge_kernel<<<dim3(a.n_q, a.batch), kMergeNT, smem, s>>>(a, plan);
+  ++launch_counter();
+  return cudaGetLastError();
 }
 
 // Slices: enough CTAs to cover the GPU about twice, each slice at most
@@ -162,9 +217,7 @@ cudaError_t launch_index_simt(const IndexArgs& a, const IndexPlan& plan, cudaStr
   ++launch_counter();
   e = cudaGetLastError();
   if (e != cudaSuccess || plan.n_slices == 1) return e;
-  index_merge_kernel<<<dim3(a.n_q, a.batch), kMergeNT, 0, s>>>(a, plan);
-  ++launch_counter();
-  return cudaGetLastError();
+  return launch_index_merge(a, plan, s);
 }
 
 size_t index_topk_workspace(int batch, int n_q, int64_t n_entries, int k, int n_heads, int dim,
@@ -181,10 +234,8 @@ cudaError_t launch_index_topk(const IndexArgs& a, cudaStream_t s) {
   if (index_tc_eligible(a)) {
     const IndexPlan plan = make_tc_plan(a.batch, a.n_q, a.n_entries, a.k, a.dt);
     cudaError_t e = launch_index_tc(a, plan, s);
-    if (e != cudaSuccess || plan.n_slices == 1) return e;
-    index_merge_kernel<<<dim3(a.n_q, a.batch), kMergeNT, 0, s>>>(a, plan);
-    ++launch_counter();
-    return cudaGetLastError();
+    if (e != cudaSuccess || plan.n_slices == 1 || plan.coop) return e;
+    return launch_index_merge(a, plan, s);
   }
   const IndexPlan plan = make_simt_plan(a.batch, a.n_q, a.n_entries, a.k);
   return launch_index_simt(a, plan, s);

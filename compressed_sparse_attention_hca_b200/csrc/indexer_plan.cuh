@@ -7,6 +7,7 @@
 namespace csa {
 
 constexpr int kMergeNT = 1024;
+constexpr int kMergeSmemKeys = 40960;  // candidate keys the merge stages in shared memory (160 KB)
 
 // Entries visible to a query at absolute position t: an entry becomes visible
 // once its whole group of m tokens is at or before t, i.e. s < floor((t+1)/m)
@@ -22,7 +23,18 @@ struct IndexPlan {
   int n_slices;       // slices per query row
   int64_t cand_cap;   // candidate slots per query row (n_slices * k), 0 when n_slices == 1
   int64_t n_rows;     // batch * n_q
+  int coop;           // 1: the slices of a row select together (cooperative launch), no merge
 };
+
+// Cooperative selection workspace per query row: high-byte histogram [256],
+// low-byte histogram [256], barrier counter (+pad) [8], per-slice (gt, eq)
+// counts [2 * n_slices].  Zeroed before every launch.
+__host__ __device__ __forceinline__ int64_t plan_coop_stride(const IndexPlan& p) {
+  return (520 + 2 * (int64_t)p.n_slices + 7) / 8 * 8;
+}
+__host__ __device__ __forceinline__ uint32_t* plan_coop_row(const IndexPlan& p, void* ws, int64_t row) {
+  return static_cast<uint32_t*>(ws) + row * plan_coop_stride(p);
+}
 
 __host__ __device__ __forceinline__ int64_t slice_valid(const IndexPlan& p, int sl, int64_t vis,
                                                         int64_t n_entries) {
@@ -52,8 +64,17 @@ __host__ __device__ __forceinline__ int32_t* plan_cand_idx(const IndexPlan& p, v
   return reinterpret_cast<int32_t*>(static_cast<uint32_t*>(ws) + p.n_rows * p.cand_cap) + row * p.cand_cap;
 }
 
+// Per-slice k-th largest key (0 when the slice kept all its entries): the
+// final k-th key is at least the largest of them, so the merge ignores every
+// candidate below that floor.
+__host__ __device__ __forceinline__ uint32_t* plan_cand_thr(const IndexPlan& p, void* ws, int64_t row) {
+  return static_cast<uint32_t*>(ws) + 2 * p.n_rows * p.cand_cap + row * p.n_slices;
+}
+
 inline size_t plan_workspace_bytes(const IndexPlan& p) {
-  return (size_t)p.n_rows * (size_t)p.cand_cap * 8;
+  if (p.coop) return (size_t)p.n_rows * (size_t)plan_coop_stride(p) * 4;
+  if (p.cand_cap == 0) return 0;
+  return (size_t)p.n_rows * (size_t)p.cand_cap * 8 + (size_t)p.n_rows * (size_t)p.n_slices * 4;
 }
 
 // Tensor-core producer (indexer_tc.cu): BF16 q / K with 64 heads of dim 128.

@@ -173,7 +173,7 @@ __global__ void __launch_bounds__(TcCfg<NQ, FP4>::THREADS, 1)
       for (int i = 0; i < n_tiles; ++i) {
         const int row = (int)((int64_t)b * a.n_entries + s0 + (int64_t)i * kBM);
         if (FP4) {
-          const int s = i % C::RSTAGES, j = i / C::RSTAGES;
+          const int s = i % (FP4 ? C::RSTAGES : 1), j = i / (FP4 ? C::RSTAGES : 1);
           if (j > 0 && !mbar_wait(&rempty[s], (j - 1) & 1)) break;
           mbar_arrive_expect_tx(&rfull[s], C::R_STAGE);
           uint8_t* dst = rs + s * C::R_STAGE;
@@ -229,7 +229,7 @@ __global__ void __launch_bounds__(TcCfg<NQ, FP4>::THREADS, 1)
     __syncwarp();
     if (lane == 0) mbar_arrive(qconv);
     for (int i = 0; ok && i < n_tiles; ++i) {
-      const int rsi = i % C::RSTAGES, rj = i / C::RSTAGES;
+      const int rsi = i % (FP4 ? C::RSTAGES : 1), rj = i / (FP4 ? C::RSTAGES : 1);
       const int osi = i % C::STAGES, oj = i / C::STAGES;
       if (!mbar_wait(&rfull[rsi], rj & 1)) break;
       if (oj > 0 && !mbar_wait(&oempty[osi], (oj - 1) & 1)) break;
@@ -270,9 +270,11 @@ __global__ void __launch_bounds__(TcCfg<NQ, FP4>::THREADS, 1)
       const int pos = i * kBM + r;
 #pragma unroll
       for (int q = 0; q < NQ; ++q) {
-        float I = 0.f;
+        // four independent partial sums (heads h = 4i + j) keep the FMA pipe busy
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int h = 0; h < kHI; ++h) I = fmaf(wsm[q * kHI + h], fmaxf(acc[q][h], 0.f), I);
+        for (int h = 0; h < kHI; ++h) part[h & 3] = fmaf(wsm[q * kHI + h], fmaxf(acc[q][h], 0.f), part[h & 3]);
+        const float I = (part[0] + part[1]) + (part[2] + part[3]);
         const uint32_t key = bf16_key(I);
         const bool valid = pos < n_valid[q];
         keys[q * plan.slice_len + pos] = valid ? (uint16_t)(key >> 16) : (uint16_t)0;
@@ -313,10 +315,445 @@ __global__ void __launch_bounds__(TcCfg<NQ, FP4>::THREADS, 1)
       const int64_t off = slice_cand_offset(plan, sl, vis[q], a.n_entries, a.k);
       uint32_t* ck = plan_cand_keys(plan, a.ws, bt) + off;
       int32_t* ci = plan_cand_idx(plan, a.ws, bt) + off;
-      block_select<NT>(key_at, nv, kk, 2, sel, [&](int slot, int pos) {
-        ck[slot] = key_at(pos);
-        ci[slot] = (int32_t)(s0 + pos);
-      });
+      uint32_t T = 0;
+      block_select<NT>(
+          key_at, nv, kk, 2, sel,
+          [&](int slot, int pos) {
+            ck[slot] = key_at(pos);
+            ci[slot] = (int32_t)(s0 + pos);
+          },
+          0u, &T);
+      if (threadIdx.x == 0) plan_cand_thr(plan, a.ws, bt)[sl] = T;
+    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------------
+// Native NVFP4 producer: the packed E2M1 K and q tiles go straight from TMA
+// (64-byte swizzle) into tcgen05.mma kind::mxf4nvf4 with block16 scales.  The
+// scales reach TMEM through tcgen05.cp from 512-byte atoms in which byte
+// m0*16 + m1*4 + kk holds the scale of tile row m0 + 32*m1 for K-block kk;
+// warp 2 permutes each tile's row-major scales (8 per entry) into two such
+// atoms (one per 64-element K-block).  Nothing is expanded: per 128-entry tile
+// shared memory sees the 9 KB the TMA writes, 1 KB of permuted scales and the
+// 12 KB the tensor core reads.
+template <int NQ>
+struct Nvf4Cfg {
+  static constexpr int N = kHI * NQ;
+  static constexpr int THREADS = 384;  // warps: 0 TMA, 1 MMA, 2 scales, 4-7 and 8-11 epilogue
+  static constexpr int STAGES = 16;
+  static constexpr int CODES = kBM * kDI / 2;           // 8 KB of E2M1 per tile
+  static constexpr int RAWSF = kBM * kDI / 16;          // 1 KB of row-major scales
+  static constexpr int ATOMS = 2 * 512;                 // two permuted scale atoms
+  static constexpr int STAGE = CODES + RAWSF + ATOMS;   // 10 KB
+  static constexpr int QCODES = N * kDI / 2;
+  static constexpr int QRAWSF = N * kDI / 16;
+  static constexpr int QREG = (QCODES + QRAWSF + ATOMS + 1023) / 1024 * 1024;
+  static constexpr int ACC_COLS = 2 * N;                // double-buffered accumulator
+  static constexpr int SFA_COL = ACC_COLS;              // 8 columns
+  static constexpr int SFB_COL = ACC_COLS + 32;         // 8 columns
+  static constexpr int TMEM_COLS = ACC_COLS + 64 <= 256 ? 256 : 512;
+  static constexpr int FIXED_SMEM = 1024 + STAGES * STAGE + QREG + NQ * kHI * 4 + 512 +
+                                    (int)sizeof(SelectSmem<THREADS>) + 1024 /*local histogram*/;
+  static constexpr uint32_t IDESC = idesc_nvf4(kBM, N);
+};
+
+// rows [0, rows) of a row-major [rows][8] scale block -> two 512-byte atoms
+// (rows >= `rows` are zero).  One warp.
+__device__ __forceinline__ void permute_scales(const uint8_t* raw, uint8_t* atoms, int rows, int lane) {
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(raw);
+  uint32_t* dst = reinterpret_cast<uint32_t*>(atoms);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int w = lane + 32 * j;                 // output word: kb * 128 + m0 * 4 + m1
+    const int kb = w >> 7, m0 = (w & 127) >> 2, m1 = w & 3;
+    const int m = m0 + 32 * m1;
+    dst[w] = m < rows ? src[m * 2 + kb] : 0u;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Cooperative selection: the slice CTAs of one query row (all resident at once,
+// cooperative launch) pick the row's top k together, with no candidate lists
+// and no merge kernel.  Keys are 16-bit (bf16 score images):
+//   1. each CTA adds the high-byte histogram of its keys into the row's global
+//      histogram H1; barrier; every CTA finds the high byte d1 of the k-th key;
+//   2. the same for the low byte among keys whose high byte is d1 (H2); the
+//      k-th key T and the number of ties at T to take follow;
+//   3. each CTA publishes its counts of keys > T and == T; barrier; prefix
+//      sums over the slices give each CTA its output offset and its share of
+//      the ties (lowest entry indices first), and it writes its winners in
+//      index order straight into the output row.
+// Barriers are global counters polled with a bounded wait (the status word
+// records a timeout).
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void coop_barrier(uint32_t* ctr, uint32_t target) {
+  __threadfence();  // this thread's global atomics are visible device-wide first
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1u);
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1; ld_acquire_gpu(ctr) < target; ++it) {
+      if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        atomicOr(&g_device_status, 1u);
+        break;
+      }
+    }
+    __threadfence();
+  }
+  __syncthreads();
+}
+
+// Digit d (searched from 255 down) at which the running count of a 256-bin
+// histogram reaches `remaining`; returns (d, remaining - count above d) in
+// bc[0], bc[1].  One warp.
+__device__ __forceinline__ void digit_search(const uint32_t* hist, uint32_t remaining, uint32_t* bc, int lane) {
+  uint32_t c[8], s = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) { c[j] = __ldcg(hist + 255 - 8 * lane - j); s += c[j]; }
+  uint32_t inc = s;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  const uint32_t exc = inc - s;
+  const bool here = exc < remaining && remaining <= inc;
+  const unsigned ballot = __ballot_sync(0xffffffffu, here);
+  if (here && lane == __ffs(ballot) - 1) {
+    uint32_t above = exc;
+    int digit = 255 - 8 * lane;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (above + c[j] >= remaining) { digit = 255 - 8 * lane - j; break; }
+      above += c[j];
+    }
+    bc[0] = (uint32_t)digit;
+    bc[1] = remaining - above;
+  }
+}
+
+template <int NT>
+__device__ void coop_select(const uint16_t* kq, int nv, int64_t vis, int64_t s0, int sl, const IndexPlan& plan,
+                            const IndexArgs& a, int64_t bt, const uint32_t* h1_local, SelectSmem<NT>& sm) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int S = plan.n_slices;
+  int32_t* out = a.idx_out + bt * a.k;
+  const int kk = (int)min64(a.k, vis);
+  if (sl == 0)
+    for (int j = kk + threadIdx.x; j < a.k; j += NT) out[j] = -1;
+  if (vis <= a.k) {  // every visible entry is selected: offsets in closed form
+    const int64_t off = slice_cand_offset(plan, sl, vis, a.n_entries, a.k);
+    for (int p = threadIdx.x; p < nv; p += NT) out[off + p] = (int32_t)(s0 + p);
+    return;
+  }
+  uint32_t* row = plan_coop_row(plan, a.ws, bt);
+  uint32_t* H1 = row;
+  uint32_t* H2 = row + 256;
+  uint32_t* ctr = row + 512;
+  uint32_t* gtq = row + 520;
+  // 1. high byte
+  for (int d = threadIdx.x; d < 256; d += NT)
+    if (h1_local[d]) atomicAdd(&H1[d], h1_local[d]);
+  coop_barrier(ctr, (uint32_t)S);
+  if (warp == 0) digit_search(H1, (uint32_t)kk, sm.bcast, lane);
+  for (int d = threadIdx.x; d < 256; d += NT) sm.hist[d] = 0;
+  __syncthreads();
+  const uint32_t d1 = sm.bcast[0], rem1 = sm.bcast[1];
+  // 2. low byte among keys with high byte d1
+  for (int p = threadIdx.x; p < nv; p += NT) {
+    const uint32_t k16 = kq[p];
+    if ((k16 >> 8) == d1) atomicAdd(&sm.hist[k16 & 255u], 1u);
+  }
+  __syncthreads();
+  for (int d = threadIdx.x; d < 256; d += NT)
+    if (sm.hist[d]) atomicAdd(&H2[d], sm.hist[d]);
+  coop_barrier(ctr, 2u * (uint32_t)S);
+  if (warp == 0) digit_search(H2, rem1, sm.bcast + 2, lane);
+  __syncthreads();
+  const uint32_t T = (d1 << 8) | sm.bcast[2];
+  const int need_eq = (int)sm.bcast[3];
+  // 3. counts, offsets, ordered write
+  const unsigned lt = (1u << lane) - 1u;
+  const int span = ((nv + NW - 1) / NW + 31) / 32 * 32;
+  const int w0 = min(nv, warp * span), w1 = min(nv, w0 + span);
+  uint32_t c_gt = 0, c_eq = 0;
+  for (int base = w0; base < w1; base += 32) {
+    const int p = base + lane;
+    const uint32_t k16 = p < w1 ? kq[p] : 0u;
+    c_gt += __popc(__ballot_sync(0xffffffffu, p < w1 && k16 > T));
+    c_eq += __popc(__ballot_sync(0xffffffffu, p < w1 && k16 == T));
+  }
+  if (lane == 0) { sm.warp_tot[warp] = c_gt; }
+  __syncthreads();
+  uint32_t gt_before_w = 0, gt_tot = 0;
+  for (int w = 0; w < NW; ++w) { gt_before_w += w < warp ? sm.warp_tot[w] : 0u; gt_tot += sm.warp_tot[w]; }
+  __syncthreads();
+  if (lane == 0) sm.warp_tot[warp] = c_eq;
+  __syncthreads();
+  uint32_t eq_before_w = 0, eq_tot = 0;
+  for (int w = 0; w < NW; ++w) { eq_before_w += w < warp ? sm.warp_tot[w] : 0u; eq_tot += sm.warp_tot[w]; }
+  if (threadIdx.x == 0) {
+    gtq[2 * sl] = gt_tot;
+    gtq[2 * sl + 1] = eq_tot;
+  }
+  coop_barrier(ctr, 3u * (uint32_t)S);
+  // slices before this one: winners and ties taken
+  uint32_t off = 0, eq_prev = 0;
+  for (int j = 0; j < sl; ++j) {
+    const uint32_t g = ld_acquire_gpu(&gtq[2 * j]), e = ld_acquire_gpu(&gtq[2 * j + 1]);
+    int take = need_eq - (int)eq_prev;
+    take = take < 0 ? 0 : (take > (int)e ? (int)e : take);
+    off += g + (uint32_t)take;
+    eq_prev += e;
+  }
+  int eq_take_cta = need_eq - (int)eq_prev;
+  eq_take_cta = eq_take_cta < 0 ? 0 : (eq_take_cta > (int)eq_tot ? (int)eq_tot : eq_take_cta);
+  // this warp's share of the CTA's ties, then ordered compaction
+  int eq_take_w = eq_take_cta - (int)eq_before_w;
+  eq_take_w = eq_take_w < 0 ? 0 : (eq_take_w > (int)c_eq ? (int)c_eq : eq_take_w);
+  __syncthreads();
+  if (lane == 0) sm.warp_tot[warp] = c_gt + (uint32_t)eq_take_w;
+  __syncthreads();
+  uint32_t o = off;
+  for (int w = 0; w < warp; ++w) o += sm.warp_tot[w];
+  int eq_seen = 0;
+  for (int base = w0; base < w1; base += 32) {
+    const int p = base + lane;
+    const bool in = p < w1;
+    const uint32_t k16 = in ? kq[p] : 0u;
+    const unsigned eqm = __ballot_sync(0xffffffffu, in && k16 == T);
+    const bool take = in && (k16 > T || (k16 == T && eq_seen + __popc(eqm & lt) < eq_take_w));
+    const unsigned tm = __ballot_sync(0xffffffffu, take);
+    if (take) out[o + __popc(tm & lt)] = (int32_t)(s0 + p);
+    o += __popc(tm);
+    eq_seen += __popc(eqm);
+  }
+  (void)gt_before_w;
+}
+
+template <int NQ>
+__global__ void __launch_bounds__(Nvf4Cfg<NQ>::THREADS, 1)
+    index_nvf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
+                      const __grid_constant__ CUtensorMap tmKs, const __grid_constant__ CUtensorMap tmQs,
+                      IndexArgs a, IndexPlan plan) {
+  using C = Nvf4Cfg<NQ>;
+  constexpr int NT = C::THREADS;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* st = align1024(smem_raw);                          // stages
+  uint8_t* qreg = st + C::STAGES * C::STAGE;                  // q codes | q raw scales | q atoms
+  uint16_t* keys = reinterpret_cast<uint16_t*>(qreg + C::QREG);
+  float* wsm = reinterpret_cast<float*>(keys + NQ * plan.slice_len);
+  uint64_t* full = reinterpret_cast<uint64_t*>(wsm + NQ * kHI);
+  uint64_t* sfr = full + C::STAGES;
+  uint64_t* empty = sfr + C::STAGES;
+  uint64_t* accf = empty + C::STAGES;
+  uint64_t* acce = accf + 2;
+  uint64_t* qbar = acce + 2;
+  uint64_t* qsf = qbar + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qsf + 1);
+  SelectSmem<NT>& sel = *reinterpret_cast<SelectSmem<NT>*>(tmem_slot + 4);
+  uint32_t* h1s = reinterpret_cast<uint32_t*>(&sel + 1);  // [256] high-byte histogram (cooperative select)
+
+  const int sl = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
+  const int t0 = grp * NQ;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t s0 = (int64_t)sl * plan.slice_len;
+  const int len = (int)min64(plan.slice_len, a.n_entries - s0);
+  const bool coop = NQ == 1 && plan.coop;
+
+  int n_valid[NQ];
+  int64_t vis[NQ];
+  int max_valid = 0;
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int t = t0 + q;
+    vis[q] = t < a.n_q ? visible_entries(a.q_pos[(int64_t)b * a.n_q + t], a.m, a.n_entries) : 0;
+    n_valid[q] = (int)max64(0, min64(len, vis[q] - s0));
+    max_valid = max(max_valid, n_valid[q]);
+  }
+  const int n_tiles = (max_valid + kBM - 1) / kBM;
+
+  for (int i = threadIdx.x; i < NQ * kHI; i += NT) {
+    const int t = t0 + i / kHI;
+    wsm[i] = t < a.n_q ? a.wI[((int64_t)b * a.n_q + t) * kHI + (i % kHI)] : 0.f;
+  }
+  for (int i = threadIdx.x; i < 256; i += NT) h1s[i] = 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&sfr[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int i = 0; i < 2; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 4); }
+    mbar_init(qbar, 1);
+    mbar_init(qsf, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const int qrow = (b * a.n_q + t0) * kHI;
+      mbar_arrive_expect_tx(qbar, C::QCODES + C::QRAWSF);
+      tma_load_2d(qreg, &tmQ, qbar, 0, qrow);
+      tma_load_2d(qreg + C::QCODES, &tmQs, qbar, 0, qrow / 2);
+      for (int i = 0; i < n_tiles; ++i) {
+        const int s = i % C::STAGES, j = i / C::STAGES;
+        if (j > 0 && !mbar_wait(&empty[s], (j - 1) & 1)) break;
+        mbar_arrive_expect_tx(&full[s], C::CODES + C::RAWSF);
+        const int row = (int)((int64_t)b * a.n_entries + s0 + (int64_t)i * kBM);
+        uint8_t* dst = st + s * C::STAGE;
+        tma_load_2d(dst, &tmK, &full[s], 0, row);
+        tma_load_2d(dst + C::CODES, &tmKs, &full[s], 0, row / 2);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(qbar, 0) && mbar_wait(qsf, 0);
+      const uint32_t qa = smem_u32(qreg);
+      if (ok) {
+        tc_fence_after();
+        for (int kb = 0; kb < 2; ++kb)
+          tc_cp_32x128b_warpx4(tmem + C::SFB_COL + kb * 4,
+                               umma_desc_rows16(qa + C::QCODES + C::QRAWSF + kb * 512));
+      }
+      for (int i = 0; ok && i < n_tiles; ++i) {
+        const int s = i % C::STAGES, j = i / C::STAGES, buf = i & 1, u = i >> 1;
+        if (!mbar_wait(&full[s], j & 1) || !mbar_wait(&sfr[s], j & 1)) break;
+        if (u > 0 && !mbar_wait(&acce[buf], (u - 1) & 1)) break;
+        tc_fence_after();
+        const uint32_t base = smem_u32(st + s * C::STAGE);
+        for (int kb = 0; kb < 2; ++kb)
+          tc_cp_32x128b_warpx4(tmem + C::SFA_COL + kb * 4, umma_desc_rows16(base + C::CODES + C::RAWSF + kb * 512));
+        const uint32_t d = tmem + (uint32_t)(buf * C::N);
+        for (int kb = 0; kb < 2; ++kb)
+          tc_mma_nvf4(d, umma_desc_sw64(base + kb * 32), umma_desc_sw64(qa + kb * 32), C::IDESC,
+                      tmem + C::SFA_COL + kb * 4, tmem + C::SFB_COL + kb * 4, kb > 0 ? 1u : 0u);
+        tc_commit(&empty[s]);
+        tc_commit(&accf[buf]);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------ scale permutation into atoms
+    bool ok = mbar_wait(qbar, 0);
+    if (ok) permute_scales(qreg + C::QCODES, qreg + C::QCODES + C::QRAWSF, C::N, lane);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(qsf);
+    for (int i = 0; ok && i < n_tiles; ++i) {
+      const int s = i % C::STAGES, j = i / C::STAGES;
+      if (!mbar_wait(&full[s], j & 1)) break;
+      uint8_t* stage = st + s * C::STAGE;
+      permute_scales(stage + C::CODES, stage + C::CODES + C::RAWSF, kBM, lane);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sfr[s]);
+    }
+  } else if (warp >= 4) {
+    // --------------------------------------------------------------- epilogue
+    // Two groups of four warps; group g drains accumulator buffer g, i.e. the
+    // tiles i with i % 2 == g.  Warp w reads TMEM lanes 32 * (w % 4) ...
+    const int quarter = warp & 3, grp_e = (warp - 4) >> 2;
+    const int r = quarter * 32 + lane;
+    float wreg[NQ == 1 ? kHI : 1];
+    if (NQ == 1) {
+#pragma unroll
+      for (int h = 0; h < kHI; ++h) wreg[h] = wsm[h];
+    }
+    for (int i = grp_e; i < n_tiles; i += 2) {
+      const int buf = i & 1, u = i >> 1;
+      if (!mbar_wait(&accf[buf], u & 1)) break;
+      tc_fence_after();
+      float acc[NQ][kHI];
+      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::N);
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        tmem_ld_32x32b_x32(taddr + q * kHI, &acc[q][0]);
+        tmem_ld_32x32b_x32(taddr + q * kHI + 32, &acc[q][32]);
+      }
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acce[buf]);
+      const int pos = i * kBM + r;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int h = 0; h < kHI; ++h)
+          part[h & 3] = fmaf(NQ == 1 ? wreg[h % (NQ == 1 ? kHI : 1)] : wsm[q * kHI + h], fmaxf(acc[q][h], 0.f),
+                             part[h & 3]);
+        const float I = (part[0] + part[1]) + (part[2] + part[3]);
+        const uint32_t key = bf16_key(I);
+        const bool valid = pos < n_valid[q];
+        keys[q * plan.slice_len + pos] = valid ? (uint16_t)(key >> 16) : (uint16_t)0;
+        if (coop && valid) atomicAdd(&h1s[key >> 24], 1u);
+        if (a.scores_out != nullptr && pos < len && t0 + q < a.n_q) {
+          const float sc = valid ? key_to_f32(key) : -INFINITY;
+          static_cast<__nv_bfloat16*>(a.scores_out)[((int64_t)b * a.n_q + t0 + q) * a.n_entries + s0 + pos] =
+              __float2bfloat16_rn(sc);
+        }
+      }
+    }
+  }
+  if (a.scores_out != nullptr) {
+    for (int q = 0; q < NQ; ++q) {
+      if (t0 + q >= a.n_q) continue;
+      for (int pos = n_tiles * kBM + threadIdx.x; pos < len; pos += NT)
+        static_cast<__nv_bfloat16*>(a.scores_out)[((int64_t)b * a.n_q + t0 + q) * a.n_entries + s0 + pos] =
+            __float2bfloat16_rn(-INFINITY);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (coop) {
+    if (t0 < a.n_q) coop_select<NT>(keys, n_valid[0], vis[0], s0, sl, plan, a, (int64_t)b * a.n_q + t0, h1s, sel);
+    __syncthreads();
+  }
+  for (int q = 0; q < NQ && !coop; ++q) {
+    const int t = t0 + q;
+    if (t >= a.n_q) break;
+    const int64_t bt = (int64_t)b * a.n_q + t;
+    const int nv = n_valid[q];
+    const int kk = min(a.k, nv);
+    const uint16_t* kq = keys + q * plan.slice_len;
+    auto key_at = [&](int i) { return ((uint32_t)kq[i]) << 16; };
+    if (plan.n_slices == 1) {
+      int32_t* out = a.idx_out + bt * a.k;
+      block_select<NT>(key_at, nv, kk, 2, sel, [&](int slot, int pos) { out[slot] = (int32_t)(s0 + pos); });
+      for (int j = kk + threadIdx.x; j < a.k; j += NT) out[j] = -1;
+    } else {
+      const int64_t off = slice_cand_offset(plan, sl, vis[q], a.n_entries, a.k);
+      uint32_t* ck = plan_cand_keys(plan, a.ws, bt) + off;
+      int32_t* ci = plan_cand_idx(plan, a.ws, bt) + off;
+      uint32_t T = 0;
+      block_select<NT>(
+          key_at, nv, kk, 2, sel,
+          [&](int slot, int pos) {
+            ck[slot] = key_at(pos);
+            ci[slot] = (int32_t)(s0 + pos);
+          },
+          0u, &T);
+      if (threadIdx.x == 0) plan_cand_thr(plan, a.ws, bt)[sl] = T;
     }
     __syncthreads();
   }
@@ -394,7 +831,57 @@ cudaError_t launch_tc(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <int NQ>
+cudaError_t launch_nvf4(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) {
+  using C = Nvf4Cfg<NQ>;
+  CUtensorMap tmK, tmQ, tmKs, tmQs;
+  const uint64_t krows = (uint64_t)a.batch * a.n_entries, qrows = (uint64_t)a.batch * a.n_q * kHI;
+  // packed E2M1 rows of 64 bytes in the 64-byte swizzle; scales as 16-byte
+  // lines holding two entries each
+  const bool ok =
+      make_map_2d(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.KI, krows, kDI / 2, kDI / 2, kBM,
+                  CU_TENSOR_MAP_SWIZZLE_64B) &&
+      make_map_2d(&tmKs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.KI_sf, krows / 2, 16, 16, kBM / 2,
+                  CU_TENSOR_MAP_SWIZZLE_NONE) &&
+      make_map_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.qI, qrows, kDI / 2, kDI / 2, C::N,
+                  CU_TENSOR_MAP_SWIZZLE_64B) &&
+      make_map_2d(&tmQs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.qI_sf, qrows / 2, 16, 16, C::N / 2,
+                  CU_TENSOR_MAP_SWIZZLE_NONE);
+  if (!ok) return cudaErrorInvalidValue;
+  const size_t smem = (size_t)C::FIXED_SMEM + (size_t)NQ * p.slice_len * 2;
+  cudaError_t e = cudaFuncSetAttribute(index_nvf4_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.n_slices, (a.n_q + NQ - 1) / NQ, a.batch);
+  if (p.coop) {
+    // the slices of a row wait on one another: zero their counters and
+    // histograms, and launch cooperatively so that every CTA is resident
+    e = cudaMemsetAsync(a.ws, 0, plan_workspace_bytes(p), s);
+    if (e != cudaSuccess) return e;
+    IndexArgs aa = a;
+    IndexPlan pp = p;
+    CUtensorMap m0 = tmK, m1 = tmQ, m2 = tmKs, m3 = tmQs;
+    void* args[] = {&m0, &m1, &m2, &m3, &aa, &pp};
+    e = cudaLaunchCooperativeKernel((const void*)index_nvf4_kernel<NQ>, grid, dim3(C::THREADS), args, smem, s);
+    ++launch_counter();
+    return e;
+  }
+  index_nvf4_kernel<NQ><<<grid, C::THREADS, smem, s>>>(tmK, tmQ, tmKs, tmQs, a, p);
+  ++launch_counter();
+  return cudaGetLastError();
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// SMs of the current device (148 when it cannot be queried, e.g. no GPU).
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 148;
+  }
+  return n;
+}
 
 }  // namespace
 
@@ -413,13 +900,14 @@ int index_tc_nq(int n_q) { return n_q >= 2 ? 2 : 1; }
 IndexPlan make_tc_plan(int batch, int n_q, int64_t n_entries, int k, int dt) {
   const int NQ = index_tc_nq(n_q);
   const bool fp4 = dt == CSA_IDX_NVFP4;
-  const int fixed = NQ == 1 ? (fp4 ? TcCfg<1, true>::FIXED_SMEM : TcCfg<1, false>::FIXED_SMEM)
-                            : (fp4 ? TcCfg<2, true>::FIXED_SMEM : TcCfg<2, false>::FIXED_SMEM);
+  const int fixed = NQ == 1 ? (fp4 ? Nvf4Cfg<1>::FIXED_SMEM : TcCfg<1, false>::FIXED_SMEM)
+                            : (fp4 ? Nvf4Cfg<2>::FIXED_SMEM : TcCfg<2, false>::FIXED_SMEM);
   constexpr int kSmemCap = 227 * 1024;
   int64_t max_slice = ((kSmemCap - fixed) / (2 * NQ)) / kBM * kBM;
   const int64_t groups = (n_q + NQ - 1) / NQ;
   const int64_t units = (int64_t)batch * groups;
-  const int64_t want = units >= 148 ? 1 : (148 + units - 1) / units;
+  // one wave: at most 148 CTAs (one per SM; the kernel's shared memory allows one)
+  const int64_t want = units >= 148 ? 1 : 148 / units;
   int64_t len = (n_entries + want - 1) / want;
   len = (len + kBM - 1) / kBM * kBM;
   if (len < kBM) len = kBM;
@@ -429,14 +917,17 @@ IndexPlan make_tc_plan(int batch, int n_q, int64_t n_entries, int k, int dt) {
   p.n_slices = (int)((n_entries + len - 1) / len);
   if (p.n_slices < 1) p.n_slices = 1;
   p.n_rows = (int64_t)batch * n_q;
-  p.cand_cap = p.n_slices > 1 ? (int64_t)p.n_slices * k : 0;
+  // NVFP4 decode rows split over several slices select cooperatively when the
+  // whole grid fits on the GPU at once (one CTA per SM)
+  p.coop = (fp4 && NQ == 1 && p.n_slices > 1 && units * p.n_slices <= sm_count()) ? 1 : 0;
+  p.cand_cap = (p.n_slices > 1 && !p.coop) ? (int64_t)p.n_slices * k : 0;
   return p;
 }
 
 cudaError_t launch_index_tc(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) {
   const bool fp4 = a.dt == CSA_IDX_NVFP4;
-  if (index_tc_nq(a.n_q) == 1) return fp4 ? launch_tc<1, true>(a, p, s) : launch_tc<1, false>(a, p, s);
-  return fp4 ? launch_tc<2, true>(a, p, s) : launch_tc<2, false>(a, p, s);
+  if (index_tc_nq(a.n_q) == 1) return fp4 ? launch_nvf4<1>(a, p, s) : launch_tc<1, false>(a, p, s);
+  return fp4 ? launch_nvf4<2>(a, p, s) : launch_tc<2, false>(a, p, s);
 }
 
 }  // namespace csa

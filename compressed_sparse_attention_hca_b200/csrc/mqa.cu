@@ -138,33 +138,94 @@ __global__ void __launch_bounds__(256) mqa_simt_kernel(MqaArgs a, MqaPlan plan) 
 
 // Merges the split partials of one (query, head) in split order and applies
 // the sink: O = sum_s e^{m_s-M} o_s / (sum_s e^{m_s-M} l_s + e^{sink-M}).
+//
+// The per-split weights e^{m_s-M}/den are computed once into shared memory
+// (kMaxCombineSplits of them; more splits loop over chunks of partials), then
+// every thread sums its output dims over the splits with independent loads.
+constexpr int kMaxCombineSplits = 256;
+
 __global__ void __launch_bounds__(128) mqa_combine_kernel(MqaArgs a, MqaPlan plan) {
+  __shared__ float wgt[kMaxCombineSplits];
+  __shared__ float red[4];
   const int h = blockIdx.x;
   const int64_t bt = blockIdx.y;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const float sink = a.sink[h];
+  const int S = plan.n_splits;
+  // M = max(sink, m_s)
   float M = sink;
-  for (int s = 0; s < plan.n_splits; ++s) M = fmaxf(M, plan_partial_ml(plan, a, bt, s, h)[0]);
-  float den = 0.f;
+  for (int s = threadIdx.x; s < S; s += 128) M = fmaxf(M, plan_partial_ml(plan, a, bt, s, h)[0]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) red[warp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+  __syncthreads();
   const bool zero = (sink == INFINITY) || (M == -INFINITY);
-  if (!zero) {
-    den = expf(sink - M);
-    for (int s = 0; s < plan.n_splits; ++s) {
-      const float* ml = plan_partial_ml(plan, a, bt, s, h);
-      if (ml[0] != -INFINITY) den += ml[1] * expf(ml[0] - M);
+  // den = e^{sink-M} + sum_s l_s e^{m_s-M}, summed in split order by one warp
+  if (warp == 0) {
+    float den = 0.f;
+    if (!zero) {
+      for (int s0 = 0; s0 < S; s0 += 32) {
+        const int s = s0 + lane;
+        float v = 0.f;
+        if (s < S) {
+          const float* ml = plan_partial_ml(plan, a, bt, s, h);
+          v = ml[0] == -INFINITY ? 0.f : ml[1] * expf(ml[0] - M);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        den += v;
+      }
+      den += expf(sink - M);
+    }
+    if (lane == 0) red[0] = den;
+  }
+  __syncthreads();
+  const float den = red[0];
+  const int64_t ob = (bt * a.n_heads + h) * a.dim;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};  // dims threadIdx.x + 128 j (dim <= 512)
+  for (int c0 = 0; c0 < S; c0 += kMaxCombineSplits) {
+    const int cn = min(kMaxCombineSplits, S - c0);
+    __syncthreads();
+    for (int s = threadIdx.x; s < cn; s += 128) {
+      const float* ml = plan_partial_ml(plan, a, bt, c0 + s, h);
+      wgt[s] = (zero || ml[0] == -INFINITY) ? 0.f : expf(ml[0] - M) / den;
+    }
+    __syncthreads();
+    // splits in groups of 4 so that 16 independent loads are in flight
+    int s = 0;
+    for (; s + 4 <= cn; s += 4) {
+      float v[4][4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float* po = plan_partial_o(plan, a, bt, c0 + s + u, h);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int d = threadIdx.x + 128 * j;
+          v[u][j] = d < a.dim ? po[d] : 0.f;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[j] = fmaf(wgt[s + u], v[u][j], acc[j]);
+    }
+    for (; s < cn; ++s) {
+      const float* po = plan_partial_o(plan, a, bt, c0 + s, h);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int d = threadIdx.x + 128 * j;
+        if (d < a.dim) acc[j] = fmaf(wgt[s], po[d], acc[j]);
+      }
     }
   }
-  const int64_t ob = (bt * a.n_heads + h) * a.dim;
-  for (int d = threadIdx.x; d < a.dim; d += blockDim.x) {
-    float acc = 0.f;
-    if (!zero) {
-      for (int s = 0; s < plan.n_splits; ++s) {
-        const float* ml = plan_partial_ml(plan, a, bt, s, h);
-        if (ml[0] != -INFINITY) acc += plan_partial_o(plan, a, bt, s, h)[d] * expf(ml[0] - M);
-      }
-      acc /= den;
-    }
-    if (a.q_dt == CSA_F32) static_cast<float*>(a.O)[ob + d] = acc;
-    else static_cast<__nv_bfloat16*>(a.O)[ob + d] = __float2bfloat16_rn(acc);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int d = threadIdx.x + 128 * j;
+    if (d >= a.dim) continue;
+    if (a.q_dt == CSA_F32) static_cast<float*>(a.O)[ob + d] = acc[j];
+    else static_cast<__nv_bfloat16*>(a.O)[ob + d] = __float2bfloat16_rn(acc[j]);
   }
 }
 
@@ -201,13 +262,18 @@ cudaError_t launch_mqa_simt(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) 
   return cudaGetLastError();
 }
 
+bool mqa_tc_eligible(const MqaArgs& a);
+MqaPlan make_tc_mqa_plan(const MqaArgs& a);
+cudaError_t launch_mqa_tc(const MqaArgs& a, const MqaPlan& p, cudaStream_t s);
+
 size_t mqa_workspace(const MqaArgs& a) {
-  const MqaPlan p = make_simt_mqa_plan(a);
+  const MqaPlan p = mqa_tc_eligible(a) ? make_tc_mqa_plan(a) : make_simt_mqa_plan(a);
   return plan_mqa_workspace_bytes(p, a);
 }
 
 cudaError_t launch_mqa(const MqaArgs& a, cudaStream_t s) {
   if ((int64_t)a.batch * a.n_q == 0) return cudaSuccess;
+  if (mqa_tc_eligible(a)) return launch_mqa_tc(a, make_tc_mqa_plan(a), s);
   return launch_mqa_simt(a, make_simt_mqa_plan(a), s);
 }
 

@@ -71,12 +71,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 // Waits for the phase with the given parity to complete; false on timeout.
+// The timer is read only every 256 polls so that waiting warps take few issue
+// slots from the warps doing work (each try_wait already blocks for a while).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
-  while (true) {
+  for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+    if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitTimeoutNs) {
       atomicOr(&g_device_status, 1u);
       return false;
     }
@@ -124,6 +126,24 @@ __device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t a_desc, uin
       ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[smem] * B[smem]^T with NVFP4 operands: packed E2M1 A and B,
+// one unsigned-E4M3 scale per 16 K-elements for each row of A (sfa) and B
+// (sfb) read from TMEM; K = 64 per instruction; fp32 accumulate.
+__device__ __forceinline__ void tc_mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}"
+      ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+// Copies a 32-row x 16-byte shared-memory block (described by `src_desc`) into
+// TMEM columns [dst, dst+4) of lanes 0..31 and broadcasts it to the other three
+// lane quarters (the layout block-scaled MMAs read their scale factors from).
+__device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t dst_tmem, uint64_t src_desc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(dst_tmem), "l"(src_desc) : "memory");
+}
 // Arrives once on the mbarrier when every tcgen05.mma issued so far by this
 // thread has completed.
 __device__ __forceinline__ void tc_commit(uint64_t* bar) {
@@ -166,6 +186,36 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t smem_addr) {
   d |= (uint64_t)1 << 46;               // version
   d |= (uint64_t)2 << 61;               // SWIZZLE_128B
   return d;
+}
+
+// K-major operand with 64-byte rows and the 64-byte swizzle (TMA
+// CU_TENSOR_MAP_SWIZZLE_64B): 8-row groups 512 bytes apart, layout 4 = SW64.
+// The atom base must be 512-byte aligned.
+__device__ __forceinline__ uint64_t umma_desc_sw64(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(512 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)4 << 61;
+  return d;
+}
+// Unswizzled block of rows 16 bytes apart (8-row groups 128 bytes apart), the
+// source form of tcgen05.cp 32x128b.
+__device__ __forceinline__ uint64_t umma_desc_rows16(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFF);
+  d |= (uint64_t)1 << 16;
+  d |= (uint64_t)(128 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+// Instruction descriptor, kind::mxf4nvf4 block-scaled: E2M1 A and B (format
+// 1), K-major, unsigned-E4M3 scales (scale format 0), scale-factor ids 0,
+// dense K = 64, M x N tile, fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_nvf4(int M, int N) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // Instruction descriptor, kind::f16: fp32 accumulator, bf16 A and B, both
