@@ -181,7 +181,7 @@ class Step:
         comp += B * self.n_out * kvb
         if self.kind.startswith("csa"):
             comp += sum(nb(self.itok[k]) for k in ("Ca", "Za", "Cb", "Zb"))
-            comp += B * self.n_out * (nb(x["KI"][0, 0]) + (nb(x["KI_sf"][0, 0]) if "KI_sf" in x else 0))
+            comp += B * self.n_out * (nb(x["KI"][0, 0]) + (cfg["dI"] // 16 if "KI_sf" in x else 0))
         idx_bytes = self.index_bytes() if self.kind.startswith("csa") else 0
         if self.kind.startswith("csa"):
             if self.kind == "csa_prefill":
@@ -298,7 +298,7 @@ def cpu_oracle_step(name: str, sample_entries=None, seed_offset=0):
         if cfg["idx_dt"] == W.NVFP4:
             q = orc.decode_rows(raw(x["qI"]).reshape(-1, dI // 2), orc.NVFP4, dI,
                                 sf=raw(x["qI_sf"]).reshape(-1, dI // 16)).reshape(1, 1, -1, dI)
-            K = orc.decode_rows(raw(x["KI"][0]), orc.NVFP4, dI, sf=raw(x["KI_sf"][0]))[None]
+            K = orc.decode_rows(raw(x["KI"][0]), orc.NVFP4, dI, sf=raw(x["KI_sf"][0]), sf_blocked=True)[None]
         else:
             q, K = f64(x["qI"]), f64(x["KI"])
         _, idx = orc.index_topk(q, f64(x["wI"]), K, raw(x["q_pos"]), m, cfg["k"], want_scores=False)

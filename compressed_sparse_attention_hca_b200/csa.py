@@ -52,8 +52,9 @@ def load():
         "csa_last_launch_count": (i32, []),
         "csa_check_device_status": (i32, []),
         "csa_row_bytes": (i64, [i32, i32]),
+        "csa_nvfp4_key_scale_bytes": (i64, [i64, i32]),
         "csa_compress": (i32, [P, P, P, P, P, P, i32, i64, i64, i64, i64, i64, i32, i32, i32, P, P,
-                               i64, i32, P]),
+                               i64, i64, i32, P]),
         "csa_index_topk_workspace_size": (sz, [i32, i32, i64, i32, i32, i32, i32]),
         "csa_index_topk": (i32, [P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32, i32, P, P, P,
                                  sz, P]),
@@ -102,6 +103,11 @@ def row_bytes(dt, dim):
     return int(load().csa_row_bytes(dt, dim))
 
 
+def nvfp4_key_scale_bytes(n_rows, dim):
+    """Bytes of one request's blocked NVFP4 key-scale array."""
+    return int(load().csa_nvfp4_key_scale_bytes(n_rows, dim))
+
+
 def _need_cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
@@ -114,9 +120,10 @@ def compress(Ca, Za, Ba, m, Cb=None, Zb=None, Bb=None, *, tok0=0, e0=0, n_out=No
              out=None, out_sf=None, out_row0=0, n_tok=None):
     """Token-level compressor.  Ca/Za [batch, rows, dim] (F32 or BF16), Ba [m, dim] fp32.
 
-    Entry e0 + j of request b goes to row out_row0 + j of out[b] (out, out_sf:
-    [batch, rows, ...]; allocated when not given).  Returns out (and out_sf for
-    NVFP4)."""
+    Entry e0 + j of request b goes to row out_row0 + j of out[b] (out:
+    [batch, rows, ...]; NVFP4 out_sf: the blocked key scales [batch,
+    nvfp4_key_scale_bytes(rows, dim)]; allocated when not given).  Returns out
+    (and out_sf for NVFP4)."""
     _need_cuda(Ca, Za, Ba, Cb, Zb, Bb)
     batch, rows, dim = Ca.shape
     n_tok = rows if n_tok is None else n_tok
@@ -132,17 +139,14 @@ def compress(Ca, Za, Ba, m, Cb=None, Zb=None, Bb=None, *, tok0=0, e0=0, n_out=No
         else:
             out = torch.empty(batch, stride, row_bytes(out_dt, dim), device=Ca.device, dtype=torch.uint8)
         if out_dt == IDX_NVFP4:
-            out_sf = torch.empty(batch, stride, dim // 16, device=Ca.device, dtype=torch.uint8)
+            out_sf = torch.zeros(batch, nvfp4_key_scale_bytes(stride, dim), device=Ca.device, dtype=torch.uint8)
     _need_cuda(out, out_sf)
     stride = out.shape[1]
-    if out_row0 < 0 or out_row0 + n_out > stride:
-        raise ValueError("output rows out of range")
-    rb = out[0, 0].numel() * out.element_size()
-    optr = ctypes.c_void_p(out.data_ptr() + out_row0 * rb)
-    sptr = None if out_sf is None else ctypes.c_void_p(out_sf.data_ptr() + out_row0 * (dim // 16))
+    if out_dt == IDX_NVFP4 and out_sf.numel() < batch * nvfp4_key_scale_bytes(stride, dim):
+        raise ValueError("out_sf smaller than the blocked key-scale arrays of the cache")
     _check(load().csa_compress(_ptr(Ca), _ptr(Cb), _ptr(Za), _ptr(Zb), _ptr(Ba), _ptr(Bb), batch, n_tok,
-                               tok0, rows, e0, n_out, dim, m, in_dt, optr, sptr, stride, out_dt,
-                               _stream()))
+                               tok0, rows, e0, n_out, dim, m, in_dt, _ptr(out), _ptr(out_sf), stride,
+                               out_row0, out_dt, _stream()))
     return (out, out_sf) if out_dt == IDX_NVFP4 else out
 
 

@@ -70,7 +70,7 @@ csa_status_t csa_check_device_status(void) {
   return ok();
 }
 
-int csa_version(void) { return 100; }
+int csa_version(void) { return 200; }
 
 int64_t csa_row_bytes(csa_dtype_t dt, int dim) {
   if (dim <= 0) return -1;
@@ -79,26 +79,32 @@ int64_t csa_row_bytes(csa_dtype_t dt, int dim) {
   return csa::row_bytes(dt, dim);
 }
 
+int64_t csa_nvfp4_key_scale_bytes(int64_t n_rows, int dim) {
+  if (n_rows < 0 || dim <= 0 || dim % 64 != 0) return -1;
+  return csa::nvfp4_blocked_sf_bytes(n_rows, dim);
+}
+
 csa_status_t csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
                           const float* Ba, const float* Bb, int batch, int64_t n_tok,
                           int64_t tok0, int64_t in_batch_stride, int64_t e0, int64_t n_out,
                           int dim, int m, csa_dtype_t in_dt, void* out, void* out_sf,
-                          int64_t out_batch_stride, csa_dtype_t out_dt, void* stream) {
+                          int64_t out_batch_stride, int64_t out_row0, csa_dtype_t out_dt,
+                          void* stream) {
   g_launches = 0;
-  REQUIRE(batch >= 0 && n_tok >= 0 && tok0 >= 0 && e0 >= 0 && n_out >= 0,
-          "negative size (batch=%d n_tok=%lld tok0=%lld e0=%lld n_out=%lld)", batch,
-          (long long)n_tok, (long long)tok0, (long long)e0, (long long)n_out);
+  REQUIRE(batch >= 0 && n_tok >= 0 && tok0 >= 0 && e0 >= 0 && n_out >= 0 && out_row0 >= 0,
+          "negative size (batch=%d n_tok=%lld tok0=%lld e0=%lld n_out=%lld out_row0=%lld)", batch,
+          (long long)n_tok, (long long)tok0, (long long)e0, (long long)n_out, (long long)out_row0);
   REQUIRE(m >= 1 && m <= 4096, "m=%d out of range [1, 4096]", m);
   REQUIRE(dim >= 8 && dim % 8 == 0, "dim=%d must be a positive multiple of 8", dim);
   REQUIRE(in_dt == CSA_F32 || in_dt == CSA_BF16, "in_dt must be CSA_F32 or CSA_BF16");
   REQUIRE(out_dt >= CSA_F32 && out_dt <= CSA_IDX_NVFP4, "unknown out_dt %d", (int)out_dt);
   if (out_dt == CSA_KV_FP8MIX)
     REQUIRE(dim >= 128 && (dim - 64) % 64 == 0, "KV_FP8MIX needs dim = 64 + 64*j (j >= 1), got %d", dim);
-  if (out_dt == CSA_IDX_NVFP4) REQUIRE(dim % 16 == 0, "NVFP4 needs dim %% 16 == 0");
+  if (out_dt == CSA_IDX_NVFP4) REQUIRE(dim % 64 == 0, "NVFP4 output needs dim %% 64 == 0, got %d", dim);
   REQUIRE(in_batch_stride >= n_tok, "in_batch_stride %lld < n_tok %lld", (long long)in_batch_stride,
           (long long)n_tok);
-  REQUIRE(out_batch_stride >= n_out, "out_batch_stride %lld < n_out %lld",
-          (long long)out_batch_stride, (long long)n_out);
+  REQUIRE(out_batch_stride >= out_row0 + n_out, "out_batch_stride %lld < out_row0 %lld + n_out %lld",
+          (long long)out_batch_stride, (long long)out_row0, (long long)n_out);
   if ((int64_t)batch * n_out == 0) return ok();
   REQUIRE_PTR(Ca);
   REQUIRE_PTR(Za);
@@ -110,7 +116,10 @@ csa_status_t csa_compress(const void* Ca, const void* Cb, const void* Za, const 
     REQUIRE_PTR(Bb);
     REQUIRE_ALIGNED_OR_NULL(Cb);
   }
-  if (out_dt == CSA_IDX_NVFP4) REQUIRE(out_sf != nullptr, "out_sf is NULL for NVFP4 output");
+  if (out_dt == CSA_IDX_NVFP4) {
+    REQUIRE(out_sf != nullptr, "out_sf is NULL for NVFP4 output");
+    REQUIRE_ALIGNED_OR_NULL(out_sf);
+  }
   const int64_t first = (overlap && e0 >= 1) ? (int64_t)m * (e0 - 1) : (int64_t)m * e0;
   const int64_t last = (int64_t)m * (e0 + n_out) - 1;
   REQUIRE(first >= tok0 && last < tok0 + n_tok,
@@ -118,7 +127,7 @@ csa_status_t csa_compress(const void* Ca, const void* Cb, const void* Za, const 
           (long long)e0, (long long)(e0 + n_out), (long long)first, (long long)last,
           (long long)tok0, (long long)(tok0 + n_tok));
   csa::CompressArgs a{Ca, Cb, Za, Zb, Ba, Bb, batch, n_tok, tok0, in_batch_stride, e0, n_out,
-                      dim, m, (int)in_dt, (int)out_dt, out, out_sf, out_batch_stride};
+                      dim, m, (int)in_dt, (int)out_dt, out, out_sf, out_batch_stride, out_row0};
   return cuda_status(csa::launch_compress(a, static_cast<cudaStream_t>(stream)), "csa_compress");
 }
 
@@ -151,6 +160,8 @@ csa_status_t csa_index_topk(const void* qI, const void* qI_sf, const float* wI, 
   if (n_entries > 0) REQUIRE_PTR(KI);
   if (dt == CSA_IDX_NVFP4) {
     REQUIRE(qI_sf != nullptr && (KI_sf != nullptr || n_entries == 0), "NVFP4 needs qI_sf and KI_sf");
+    REQUIRE(dim % 64 == 0, "NVFP4 needs dim %% 64 == 0 (blocked key scales), got %d", dim);
+    REQUIRE_ALIGNED_OR_NULL(KI_sf);
   }
   const size_t need = csa_index_topk_workspace_size(batch, n_q, n_entries, k, n_heads, dim, dt);
   REQUIRE(ws_bytes >= need, "workspace too small: %zu < %zu bytes", ws_bytes, need);

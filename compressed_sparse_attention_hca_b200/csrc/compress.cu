@@ -104,7 +104,7 @@ __global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
 #pragma unroll
   for (int q = 0; q < 8; ++q) x[q] = valid ? sm.acc[q] / sm.den[q] : 0.f;
 
-  const int64_t orow = (int64_t)b * a.out_batch_stride + ie;
+  const int64_t orow = (int64_t)b * a.out_batch_stride + a.out_row0 + ie;
   const int64_t rb = row_bytes(a.out_dt, a.dim);
   uint8_t* row = static_cast<uint8_t*>(a.out) + orow * rb;
 
@@ -180,8 +180,11 @@ __global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {
       }
       *reinterpret_cast<uint32_t*>(row + d0 / 2) = packed;
       if ((d0 % kFp4Block) == 0) {
-        uint8_t* sf = static_cast<uint8_t*>(a.out_sf) + orow * (a.dim / kFp4Block);
-        sf[d0 / kFp4Block] = (uint8_t)s8;
+        // key-cache scales live in the blocked scale-factor atom layout
+        const int j = d0 / kFp4Block;
+        const int64_t off = (int64_t)b * nvfp4_blocked_sf_bytes(a.out_batch_stride, a.dim) +
+                            nvfp4_blocked_sf_offset(a.out_row0 + ie, a.dim) + (j / 4) * 512 + (j % 4);
+        static_cast<uint8_t*>(a.out_sf)[off] = (uint8_t)s8;
       }
     }
   }

@@ -65,8 +65,12 @@ __device__ __forceinline__ float2 e2m1x2_to_float2(uint8_t byte) {
 
 // Decode `n` consecutive values [d0, d0+n) of one row of format dt into f32.
 // n and d0 are multiples of 8 (FP8MIX/BF16/F32) or 16 (NVFP4).
+// NVFP4 scales come either row-major (sf_row[j] for values 16j..16j+15) or,
+// for key-cache rows, in the blocked atom layout (sf_blocked: sf_row from
+// nvfp4_blocked_sf_row, scale j at sf_row[(j / 4) * 512 + j % 4]).
 __device__ __forceinline__ void decode_row_chunk8(const uint8_t* row, const uint8_t* sf_row, int dt,
-                                                  int dim, int d0, float* out8) {
+                                                  int dim, int d0, float* out8,
+                                                  bool sf_blocked = false) {
   if (dt == CSA_F32) {
     const float4* p = reinterpret_cast<const float4*>(row + 4 * d0);
     float4 a = p[0], b = p[1];
@@ -104,7 +108,8 @@ __device__ __forceinline__ void decode_row_chunk8(const uint8_t* row, const uint
     }
   } else {  // NVFP4: 8 values = 4 bytes, one scale per 16 values
     uint32_t v = *reinterpret_cast<const uint32_t*>(row + d0 / 2);
-    const float s = e4m3_to_float(sf_row[d0 / kFp4Block]);
+    const int j = d0 / kFp4Block;
+    const float s = e4m3_to_float(sf_row[sf_blocked ? (j >> 2) * 512 + (j & 3) : j]);
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       float2 f = e2m1x2_to_float2((uint8_t)(v >> (8 * j)));
@@ -112,6 +117,17 @@ __device__ __forceinline__ void decode_row_chunk8(const uint8_t* row, const uint
       out8[2 * j + 1] = f.y * s;
     }
   }
+}
+
+// Start of row r's scales in a blocked NVFP4 key-scale array of dimension
+// dim: 128-row blocks of dim/64 atoms of 512 bytes; inside an atom, row r
+// owns bytes (r % 32) * 16 + (r % 128 / 32) * 4 .. +3.
+__host__ __device__ __forceinline__ int64_t nvfp4_blocked_sf_offset(int64_t r, int dim) {
+  return (r / 128) * (dim / 64) * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4;
+}
+// Bytes of the blocked scale array of one request with n_rows rows.
+__host__ __device__ __forceinline__ int64_t nvfp4_blocked_sf_bytes(int64_t n_rows, int dim) {
+  return (n_rows + 127) / 128 * (dim / 64) * 512;
 }
 
 // Order-preserving key of a float score (larger score -> larger key).
@@ -150,7 +166,7 @@ struct CompressArgs {
   int64_t n_tok, tok0, in_batch_stride, e0, n_out;
   int dim, m, in_dt, out_dt;
   void *out, *out_sf;
-  int64_t out_batch_stride;
+  int64_t out_batch_stride, out_row0;
 };
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s);
 

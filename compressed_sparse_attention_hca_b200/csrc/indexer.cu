@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(kNT) index_slice_simt_kernel(IndexArgs a, Inde
   const bool f32mode = a.dt == CSA_F32;
   const uint8_t* kbase = static_cast<const uint8_t*>(a.KI) + (int64_t)b * a.n_entries * qrb;
   const uint8_t* ksf = a.dt == CSA_IDX_NVFP4
-                           ? static_cast<const uint8_t*>(a.KI_sf) + (int64_t)b * a.n_entries * (a.dim / 16)
+                           ? static_cast<const uint8_t*>(a.KI_sf) + (int64_t)b * nvfp4_blocked_sf_bytes(a.n_entries, a.dim)
                            : nullptr;
   for (int p = threadIdx.x; p < len; p += kNT) {
     const int64_t e = s0 + p;
@@ -59,13 +59,13 @@ __global__ void __launch_bounds__(kNT) index_slice_simt_kernel(IndexArgs a, Inde
     float score = -INFINITY;
     if (p < n_valid) {
       const uint8_t* krow = kbase + e * qrb;
-      const uint8_t* ksrow = ksf ? ksf + e * (a.dim / 16) : nullptr;
+      const uint8_t* ksrow = ksf ? ksf + nvfp4_blocked_sf_offset(e, a.dim) : nullptr;
       float I = 0.f;
       for (int h = 0; h < a.n_heads; ++h) {
         float dot = 0.f;
         for (int d0 = 0; d0 < a.dim; d0 += 8) {
           float kv[8];
-          decode_row_chunk8(krow, ksrow, a.dt, a.dim, d0, kv);
+          decode_row_chunk8(krow, ksrow, a.dt, a.dim, d0, kv, true);
           const float* qh = q + h * a.dim + d0;
 #pragma unroll
           for (int j = 0; j < 8; ++j) dot = fmaf(qh[j], kv[j], dot);

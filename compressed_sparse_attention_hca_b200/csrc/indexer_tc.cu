@@ -1,28 +1,30 @@
-// indexer_tc.cu -- tensor-core producer of the Lightning Indexer score
+// indexer_tc.cu -- tensor-core producers of the Lightning Indexer score
 // ("DeepSeek-V4 内部机制" 1.2 Step 2: I[t,s] = sum_h w[t,h] ReLU(q[t,h].K[s]);
 // 6.2: FP4 q/K, fp32 score rounded to BF16 before top-k), fused with the
-// per-slice top-k selection.
+// top-k selection.
 //
 // One CTA owns a group of NQ queries of one request and a slice of that
 // request's entries.  The score tile is a dense contraction
 //     D[128 entries, 64*NQ heads] = K_tile[128 x 128] . Q_group[64*NQ x 128]^T
-// issued as tcgen05.mma (16-bit inputs, fp32 accumulate in TMEM) over operands
-// in the 128-byte-swizzled K-major shared-memory layout.
-//
-// BF16 inputs: TMA writes the K tiles straight into the operand ring.
-// NVFP4 inputs: TMA brings the packed E2M1 codes and E4M3 block scales (72
-//   bytes per entry, the HBM traffic) into a raw ring; converter warps expand
-//   them to fp16 in the swizzled layout.  Every e2m1 x e4m3 product is exact
-//   in fp16 (at most 6 significant bits, magnitudes 2^-10 .. 2688), so the
-//   fp16 MMA with fp32 accumulation sees exactly the decoded values.
-//
-// Warp roles: warp 0 TMA producer; warp 1 TMEM owner and MMA issuer (8 MMAs of
-// K = 16 per tile); warps 4-7 epilogue (each thread owns one entry row = one
-// TMEM lane, reads its 64 head scores per query, forms sum_h w_h relu(s_h),
-// rounds to bf16, stores the 16-bit order key in shared memory); NVFP4 only:
-// warps 2, 3, 8-11 convert.  The TMEM accumulator is double buffered.  After
-// the last tile the whole CTA runs the radix select on the slice's keys (the
-// score row never reaches HBM).
+// issued as tcgen05.mma with fp32 accumulation in TMEM:
+//   BF16 inputs:  kind::f16, K tiles TMA-staged in the 128-byte swizzle;
+//   NVFP4 inputs: kind::mxf4nvf4 block16 on the packed E2M1 tiles (64-byte
+//     swizzle), their E4M3 scales moved to TMEM by tcgen05.cp from 512-byte
+//     atoms (byte m0*16 + m1*4 + kk = scale of tile row m0 + 32*m1, K-block
+//     kk).  Key scales are stored in HBM in exactly that layout, so each
+//     tile's two atoms arrive by one 1 KB bulk copy; the query's row-major
+//     scales are permuted once per CTA.
+// Warp roles: 0 TMA producer; 1 TMEM owner and MMA issuer (NVFP4: even
+// tiles, warp 3 the odd ones); 2 query scale atoms (NVFP4); 4-7 and 8-11 two
+// epilogue groups.  The accumulator has NBUF TMEM buffers so that the MMAs
+// run several tiles ahead of the epilogue; epilogue group g drains the tiles
+// i with i % 2 == g: each thread owns one entry row
+// (one TMEM lane), reads its 64 head scores per query, forms
+// sum_h w_h relu(s_h), rounds to bf16 and stores the 16-bit order key in
+// shared memory.  After the last tile the CTA selects on those keys (the score
+// row never reaches HBM): alone when it holds the whole row, cooperatively
+// with the other slices of the row (NVFP4 decode), or by writing candidates
+// for the merge kernel.
 #include <cudaTypedefs.h>
 
 #include "csa_internal.cuh"
@@ -39,25 +41,50 @@ namespace {
 constexpr int kBM = 128;          // entries per tile (MMA M)
 constexpr int kDI = 128;          // indexer dim handled here
 constexpr int kHI = 64;           // indexer heads handled here
-constexpr int kAtom = kBM * 128;  // bytes of one 128-byte-wide K atom of a K tile
-constexpr int kConvWarps = 6;     // NVFP4 converter warps: 2, 3, 8, 9, 10, 11
+constexpr int kAtom = kBM * 128;  // bytes of one 128-byte-wide K atom of a bf16 K tile
+constexpr int kThreads = 384;
 
-template <int NQ, bool FP4>
-struct TcCfg {
-  static constexpr int N = kHI * NQ;                        // MMA N
-  static constexpr int THREADS = FP4 ? 384 : 256;
-  static constexpr int STAGES = FP4 ? 3 : (NQ == 1 ? 4 : 3);  // 16-bit operand ring
-  static constexpr int RSTAGES = FP4 ? 6 : 0;               // raw NVFP4 ring
-  static constexpr int Q_BYTES = N * 2 * kDI;               // two atoms of N rows x 128 B
-  static constexpr int K_STAGE = kBM * 2 * kDI;             // two atoms of 128 rows x 128 B
-  static constexpr int R_CODES = kBM * kDI / 2;             // 8 KB of E2M1 codes per tile
-  static constexpr int R_STAGE = R_CODES + kBM * kDI / 16;  // + 1 KB of scales
-  static constexpr int QRAW = FP4 ? (N * kDI / 2 + N * kDI / 16 + 1023) / 1024 * 1024 : 0;
-  static constexpr int TMEM_COLS = 2 * N;                   // double-buffered accumulator
-  static constexpr int FIXED_SMEM = 1024 /*align slack*/ + STAGES * K_STAGE + Q_BYTES + RSTAGES * R_STAGE +
-                                    QRAW + NQ * kHI * 4 + 512 /*barriers*/ +
-                                    (int)sizeof(SelectSmem<THREADS>);
-  static constexpr uint32_t IDESC = FP4 ? idesc_f16_f32(kBM, N) : idesc_bf16_f32(kBM, N);
+__host__ __device__ constexpr int pow2_cols(int c) {
+  return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512;
+}
+
+template <int NQ>
+struct Bf16Cfg {
+  static constexpr int N = kHI * NQ;
+  static constexpr int STAGES = NQ == 1 ? 4 : 3;
+  static constexpr int Q_BYTES = N * 2 * kDI;             // two atoms of N rows x 128 B
+  static constexpr int K_STAGE = kBM * 2 * kDI;           // two atoms of 128 rows x 128 B
+  static constexpr int NBUF = 512 / N;                    // 8 (NQ 1) or 4 (NQ 2)
+  static_assert(NBUF % 2 == 0, "one epilogue group per buffer");
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int FIXED_SMEM = 1024 + STAGES * K_STAGE + Q_BYTES + NQ * kHI * 4 + 1024 /*barriers*/ +
+                                    (int)sizeof(SelectSmem<kThreads>) + 1024 /*histogram*/;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(kBM, N);
+};
+
+template <int NQ>
+struct Nvf4Cfg {
+  static constexpr int N = kHI * NQ;
+  static constexpr int STAGES = 16;
+  static constexpr int CODES = kBM * kDI / 2;           // 8 KB of E2M1 per tile
+  static constexpr int ATOMS = 2 * 512;                 // the tile's two scale atoms
+  static constexpr int STAGE = CODES + ATOMS;           // 9 KB (1024-aligned stages)
+  static constexpr int QCODES = N * kDI / 2;
+  static constexpr int QRAWSF = N * kDI / 16;
+  static constexpr int QREG = (QCODES + QRAWSF + ATOMS + 1023) / 1024 * 1024;
+  // Even: buffer i % NBUF then always belongs to the same issuer (i % 2) and
+  // epilogue group (i % 2), so each side waits on every phase of its
+  // barriers in order (with an odd count a waiter could skip a phase and
+  // take the parity of an older one for the one it wants).
+  static constexpr int NBUF = NQ == 1 ? 6 : 2;
+  static_assert(NBUF % 2 == 0, "one issuer and one epilogue group per buffer");
+  static constexpr int ACC_COLS = NBUF * N;             // 384 or 256
+  static constexpr int SFA_COL = ACC_COLS;              // 2 x 8 columns (one set per issuer)
+  static constexpr int SFB_COL = ACC_COLS + 32;         // 2 x 8 columns
+  static constexpr int TMEM_COLS = pow2_cols(ACC_COLS + 64);
+  static constexpr int FIXED_SMEM = 1024 + STAGES * STAGE + QREG + NQ * kHI * 4 + 1024 +
+                                    (int)sizeof(SelectSmem<kThreads>) + 1024;
+  static constexpr uint32_t IDESC = idesc_nvf4(kBM, N);
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -65,315 +92,132 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return p + ((1024u - (a & 1023u)) & 1023u);
 }
 
-// 8 E2M1 values (4 bytes, element 2j in the low nibble of byte j) times their
-// E4M3 block scale -> 8 fp16 values (exact).
-__device__ __forceinline__ uint4 fp4x8_to_f16x8(uint32_t codes, uint8_t sf) {
-  const __half2_raw sr = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(sf | (sf << 8)), __NV_E4M3);
-  __half2 s;
-  memcpy(&s, &sr, 4);
-  uint32_t w[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const __half2_raw vr = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((codes >> (8 * j)) & 0xFFu), __NV_E2M1);
-    __half2 v;
-    memcpy(&v, &vr, 4);
-    const __half2 p = __hmul2(v, s);
-    memcpy(&w[j], &p, 4);
-  }
-  return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// Offset of 16-byte chunk c (elements 8c..8c+7) of row r inside a K-major
-// operand of `rows` rows stored as two 128-byte-swizzled atoms.
-__device__ __forceinline__ uint32_t sw128_chunk_offset(int r, int c, int rows) {
-  return (uint32_t)((c >> 3) * rows * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
-}
-
-template <int NQ, bool FP4>
-__global__ void __launch_bounds__(TcCfg<NQ, FP4>::THREADS, 1)
-    index_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
-                    const __grid_constant__ CUtensorMap tmKs, const __grid_constant__ CUtensorMap tmQs,
-                    IndexArgs a, IndexPlan plan) {
-  using C = TcCfg<NQ, FP4>;
-  constexpr int NT = C::THREADS;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* ks = align1024(smem_raw);                          // 16-bit operand ring
-  uint8_t* qs = ks + C::STAGES * C::K_STAGE;                  // 16-bit query tile
-  uint8_t* rs = qs + C::Q_BYTES;                              // raw NVFP4 ring
-  uint8_t* qraw = rs + C::RSTAGES * C::R_STAGE;               // raw NVFP4 query tile
-  uint16_t* keys = reinterpret_cast<uint16_t*>(qraw + C::QRAW);  // [NQ][slice_len]
-  float* wsm = reinterpret_cast<float*>(keys + NQ * plan.slice_len);
-  uint64_t* ofull = reinterpret_cast<uint64_t*>(wsm + NQ * kHI);
-  uint64_t* oempty = ofull + C::STAGES;
-  uint64_t* rfull = oempty + C::STAGES;
-  uint64_t* rempty = rfull + 8;
-  uint64_t* accf = rempty + 8;
-  uint64_t* acce = accf + 2;
-  uint64_t* qbar = acce + 2;
-  uint64_t* qconv = qbar + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qconv + 1);
-  SelectSmem<NT>& sel = *reinterpret_cast<SelectSmem<NT>*>(tmem_slot + 4);
-
-  const int sl = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
-  const int t0 = grp * NQ;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t s0 = (int64_t)sl * plan.slice_len;
-  const int len = (int)min64(plan.slice_len, a.n_entries - s0);
-
+// Per-CTA description of the slice and its queries.
+template <int NQ>
+struct SliceCtx {
+  int sl, t0, b, len, n_tiles;
+  int64_t s0;
   int n_valid[NQ];
   int64_t vis[NQ];
+};
+
+template <int NQ>
+__device__ __forceinline__ SliceCtx<NQ> slice_ctx(const IndexArgs& a, const IndexPlan& plan) {
+  SliceCtx<NQ> c;
+  c.sl = blockIdx.x;
+  c.t0 = blockIdx.y * NQ;
+  c.b = blockIdx.z;
+  c.s0 = (int64_t)c.sl * plan.slice_len;
+  c.len = (int)min64(plan.slice_len, a.n_entries - c.s0);
   int max_valid = 0;
 #pragma unroll
   for (int q = 0; q < NQ; ++q) {
-    const int t = t0 + q;
-    vis[q] = t < a.n_q ? visible_entries(a.q_pos[(int64_t)b * a.n_q + t], a.m, a.n_entries) : 0;
-    n_valid[q] = (int)max64(0, min64(len, vis[q] - s0));
-    max_valid = max(max_valid, n_valid[q]);
+    const int t = c.t0 + q;
+    c.vis[q] = t < a.n_q ? visible_entries(a.q_pos[(int64_t)c.b * a.n_q + t], a.m, a.n_entries) : 0;
+    c.n_valid[q] = (int)max64(0, min64(c.len, c.vis[q] - c.s0));
+    max_valid = max(max_valid, c.n_valid[q]);
   }
-  const int n_tiles = (max_valid + kBM - 1) / kBM;
+  c.n_tiles = (max_valid + kBM - 1) / kBM;
+  return c;
+}
 
-  for (int i = threadIdx.x; i < NQ * kHI; i += NT) {
-    const int t = t0 + i / kHI;
-    wsm[i] = t < a.n_q ? a.wI[((int64_t)b * a.n_q + t) * kHI + (i % kHI)] : 0.f;
+// Epilogue group `g` (warps 4-7: g = 0, warps 8-11: g = 1) drains the tiles
+// i with i % 2 == g from TMEM buffer i % NBUF.
+template <int NQ, int N, int NBUF>
+__device__ __forceinline__ void epilogue_group(const SliceCtx<NQ>& c, const IndexArgs& a, const IndexPlan& plan,
+                                               uint32_t tmem, uint64_t* accf, uint64_t* acce, const float* wsm,
+                                               uint16_t* keys, bool coop, uint32_t* h1s) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int quarter = warp & 3, g = (warp - 4) >> 2;
+  const int r = quarter * 32 + lane;
+  float wreg[NQ == 1 ? kHI : 1];
+  if (NQ == 1) {
+#pragma unroll
+    for (int h = 0; h < kHI; ++h) wreg[h] = wsm[h];
   }
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&ofull[s], FP4 ? kConvWarps : 1);
-      mbar_init(&oempty[s], 1);
-    }
-    for (int s = 0; s < C::RSTAGES; ++s) {
-      mbar_init(&rfull[s], 1);
-      mbar_init(&rempty[s], kConvWarps);
-    }
-    for (int i = 0; i < 2; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 4); }
-    mbar_init(qbar, 1);
-    mbar_init(qconv, kConvWarps);
-    fence_barrier_init();
-  }
-  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = *tmem_slot;
-  const bool conv_warp = FP4 && (warp == 2 || warp == 3 || warp >= 8);
-
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      const int qrow = (b * a.n_q + t0) * kHI;
-      if (FP4) {
-        mbar_arrive_expect_tx(qbar, C::N * kDI / 2 + C::N * kDI / 16);
-        tma_load_2d(qraw, &tmQ, qbar, 0, qrow);
-        tma_load_2d(qraw + C::N * kDI / 2, &tmQs, qbar, 0, qrow / 2);
-      } else {
-        mbar_arrive_expect_tx(qbar, C::Q_BYTES);
-        tma_load_2d(qs, &tmQ, qbar, 0, qrow);
-        tma_load_2d(qs + C::N * 128, &tmQ, qbar, 64, qrow);
-      }
-      for (int i = 0; i < n_tiles; ++i) {
-        const int row = (int)((int64_t)b * a.n_entries + s0 + (int64_t)i * kBM);
-        if (FP4) {
-          const int s = i % (FP4 ? C::RSTAGES : 1), j = i / (FP4 ? C::RSTAGES : 1);
-          if (j > 0 && !mbar_wait(&rempty[s], (j - 1) & 1)) break;
-          mbar_arrive_expect_tx(&rfull[s], C::R_STAGE);
-          uint8_t* dst = rs + s * C::R_STAGE;
-          tma_load_2d(dst, &tmK, &rfull[s], 0, row);
-          tma_load_2d(dst + C::R_CODES, &tmKs, &rfull[s], 0, row / 2);
-        } else {
-          const int s = i % C::STAGES, j = i / C::STAGES;
-          if (j > 0 && !mbar_wait(&oempty[s], (j - 1) & 1)) break;
-          mbar_arrive_expect_tx(&ofull[s], C::K_STAGE);
-          uint8_t* dst = ks + s * C::K_STAGE;
-          tma_load_2d(dst, &tmK, &ofull[s], 0, row);
-          tma_load_2d(dst + kAtom, &tmK, &ofull[s], 64, row);
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait(FP4 ? qconv : qbar, 0);
-      const uint32_t qa = smem_u32(qs);
-      for (int i = 0; ok && i < n_tiles; ++i) {
-        const int s = i % C::STAGES, j = i / C::STAGES, buf = i & 1, u = i >> 1;
-        if (!mbar_wait(&ofull[s], j & 1)) break;
-        if (u > 0 && !mbar_wait(&acce[buf], (u - 1) & 1)) break;
-        tc_fence_after();
-        const uint32_t ka = smem_u32(ks + s * C::K_STAGE);
-        const uint32_t d = tmem + (uint32_t)(buf * C::N);
+  for (int i = g; i < c.n_tiles; i += 2) {
+    const int buf = i % NBUF, u = i / NBUF;
+    if (!mbar_wait(&accf[buf], u & 1)) break;
+    tc_fence_after();
+    float acc[NQ][kHI];
+    const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * N);
 #pragma unroll
-        for (int kk = 0; kk < kDI / 16; ++kk) {
-          const uint32_t within = (uint32_t)(kk & 3) * 32u;  // 16 elements of 2 bytes
-          const uint32_t a_addr = ka + (uint32_t)(kk >> 2) * kAtom + within;
-          const uint32_t b_addr = qa + (uint32_t)(kk >> 2) * (C::N * 128) + within;
-          tc_mma_f16(d, umma_desc_sw128(a_addr), umma_desc_sw128(b_addr), C::IDESC, kk > 0 ? 1u : 0u);
-        }
-        tc_commit(&oempty[s]);
-        tc_commit(&accf[buf]);
-      }
-    }
-  } else if (conv_warp) {
-    // ------------------------------------------------- NVFP4 -> fp16 converters
-    const int ct = (warp < 4 ? warp - 2 : warp - 6) * 32 + lane;
-    constexpr int CT = kConvWarps * 32;
-    bool ok = mbar_wait(qbar, 0);
-    if (ok) {
-      for (int ch = ct; ch < C::N * 16; ch += CT) {
-        const int r = ch >> 4, c = ch & 15;
-        const uint32_t codes = *reinterpret_cast<const uint32_t*>(qraw + r * 64 + c * 4);
-        const uint8_t sf = qraw[C::N * kDI / 2 + r * 8 + (c >> 1)];
-        *reinterpret_cast<uint4*>(qs + sw128_chunk_offset(r, c, C::N)) = fp4x8_to_f16x8(codes, sf);
-      }
-    }
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(qconv);
-    for (int i = 0; ok && i < n_tiles; ++i) {
-      const int rsi = i % (FP4 ? C::RSTAGES : 1), rj = i / (FP4 ? C::RSTAGES : 1);
-      const int osi = i % C::STAGES, oj = i / C::STAGES;
-      if (!mbar_wait(&rfull[rsi], rj & 1)) break;
-      if (oj > 0 && !mbar_wait(&oempty[osi], (oj - 1) & 1)) break;
-      const uint8_t* src = rs + rsi * C::R_STAGE;
-      uint8_t* dst = ks + osi * C::K_STAGE;
-      for (int ch = ct; ch < kBM * 16; ch += CT) {
-        const int r = ch >> 4, c = ch & 15;
-        const uint32_t codes = *reinterpret_cast<const uint32_t*>(src + r * 64 + c * 4);
-        const uint8_t sf = src[C::R_CODES + r * 8 + (c >> 1)];
-        *reinterpret_cast<uint4*>(dst + sw128_chunk_offset(r, c, kBM)) = fp4x8_to_f16x8(codes, sf);
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&rempty[rsi]);
-        mbar_arrive(&ofull[osi]);
-      }
-    }
-  } else if (warp >= 4 && warp < 8) {
-    // --------------------------------------------------------------- epilogue
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    for (int i = 0; i < n_tiles; ++i) {
-      const int buf = i & 1, u = i >> 1;
-      if (!mbar_wait(&accf[buf], u & 1)) break;
-      tc_fence_after();
-      float acc[NQ][kHI];
-      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::N);
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        tmem_ld_32x32b_x32(taddr + q * kHI, &acc[q][0]);
-        tmem_ld_32x32b_x32(taddr + q * kHI + 32, &acc[q][32]);
-      }
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[buf]);
-      const int pos = i * kBM + r;
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        // four independent partial sums (heads h = 4i + j) keep the FMA pipe busy
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int h = 0; h < kHI; ++h) part[h & 3] = fmaf(wsm[q * kHI + h], fmaxf(acc[q][h], 0.f), part[h & 3]);
-        const float I = (part[0] + part[1]) + (part[2] + part[3]);
-        const uint32_t key = bf16_key(I);
-        const bool valid = pos < n_valid[q];
-        keys[q * plan.slice_len + pos] = valid ? (uint16_t)(key >> 16) : (uint16_t)0;
-        if (a.scores_out != nullptr && pos < len && t0 + q < a.n_q) {
-          const float sc = valid ? key_to_f32(key) : -INFINITY;
-          static_cast<__nv_bfloat16*>(a.scores_out)[((int64_t)b * a.n_q + t0 + q) * a.n_entries + s0 + pos] =
-              __float2bfloat16_rn(sc);
-        }
-      }
-    }
-  }
-  // debug scores of positions past the last computed tile
-  if (a.scores_out != nullptr) {
     for (int q = 0; q < NQ; ++q) {
-      if (t0 + q >= a.n_q) continue;
-      for (int pos = n_tiles * kBM + threadIdx.x; pos < len; pos += NT)
-        static_cast<__nv_bfloat16*>(a.scores_out)[((int64_t)b * a.n_q + t0 + q) * a.n_entries + s0 + pos] =
-            __float2bfloat16_rn(-INFINITY);
+      tmem_ld_32x32b_x32(taddr + q * kHI, &acc[q][0]);
+      tmem_ld_32x32b_x32(taddr + q * kHI + 32, &acc[q][32]);
+    }
+    tmem_ld_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&acce[buf]);
+    const int pos = i * kBM + r;
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      // four independent partial sums (heads h = 4i + j) keep the FMA pipe busy
+      float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int h = 0; h < kHI; ++h)
+        part[h & 3] = fmaf(NQ == 1 ? wreg[h % (NQ == 1 ? kHI : 1)] : wsm[q * kHI + h], fmaxf(acc[q][h], 0.f),
+                           part[h & 3]);
+      const float I = (part[0] + part[1]) + (part[2] + part[3]);
+      const uint32_t key = bf16_key(I);
+      const bool valid = pos < c.n_valid[q];
+      keys[q * plan.slice_len + pos] = valid ? (uint16_t)(key >> 16) : (uint16_t)0;
+      if (coop && valid) atomicAdd(&h1s[key >> 24], 1u);
+      if (a.scores_out != nullptr && pos < c.len && c.t0 + q < a.n_q) {
+        const float sc = valid ? key_to_f32(key) : -INFINITY;
+        static_cast<__nv_bfloat16*>(a.scores_out)[((int64_t)c.b * a.n_q + c.t0 + q) * a.n_entries + c.s0 + pos] =
+            __float2bfloat16_rn(sc);
+      }
     }
   }
-  tc_fence_before();
-  __syncthreads();
+}
 
-  // per-query top-k over this slice's keys
+// Debug score output (-inf) for the positions past the last computed tile.
+template <int NQ>
+__device__ __forceinline__ void scores_tail(const SliceCtx<NQ>& c, const IndexArgs& a) {
+  if (a.scores_out == nullptr) return;
   for (int q = 0; q < NQ; ++q) {
-    const int t = t0 + q;
+    if (c.t0 + q >= a.n_q) continue;
+    for (int pos = c.n_tiles * kBM + threadIdx.x; pos < c.len; pos += kThreads)
+      static_cast<__nv_bfloat16*>(a.scores_out)[((int64_t)c.b * a.n_q + c.t0 + q) * a.n_entries + c.s0 + pos] =
+          __float2bfloat16_rn(-INFINITY);
+  }
+}
+
+// Selection by one CTA over its own slice: final indices when it holds the
+// whole row, else the slice's top k as candidates (and its k-th key) for the
+// merge kernel.
+template <int NQ>
+__device__ void slice_select(const SliceCtx<NQ>& c, const IndexArgs& a, const IndexPlan& plan, const uint16_t* keys,
+                             SelectSmem<kThreads>& sel) {
+  for (int q = 0; q < NQ; ++q) {
+    const int t = c.t0 + q;
     if (t >= a.n_q) break;
-    const int64_t bt = (int64_t)b * a.n_q + t;
-    const int nv = n_valid[q];
+    const int64_t bt = (int64_t)c.b * a.n_q + t;
+    const int nv = c.n_valid[q];
     const int kk = min(a.k, nv);
     const uint16_t* kq = keys + q * plan.slice_len;
     auto key_at = [&](int i) { return ((uint32_t)kq[i]) << 16; };
     if (plan.n_slices == 1) {
       int32_t* out = a.idx_out + bt * a.k;
-      block_select<NT>(key_at, nv, kk, 2, sel, [&](int slot, int pos) { out[slot] = (int32_t)(s0 + pos); });
-      for (int j = kk + threadIdx.x; j < a.k; j += NT) out[j] = -1;
+      block_select<kThreads>(key_at, nv, kk, 0, sel, [&](int slot, int pos) { out[slot] = (int32_t)(c.s0 + pos); });
+      for (int j = kk + threadIdx.x; j < a.k; j += kThreads) out[j] = -1;
     } else {
-      const int64_t off = slice_cand_offset(plan, sl, vis[q], a.n_entries, a.k);
+      const int64_t off = slice_cand_offset(plan, c.sl, c.vis[q], a.n_entries, a.k);
       uint32_t* ck = plan_cand_keys(plan, a.ws, bt) + off;
       int32_t* ci = plan_cand_idx(plan, a.ws, bt) + off;
       uint32_t T = 0;
-      block_select<NT>(
-          key_at, nv, kk, 2, sel,
+      block_select<kThreads>(
+          key_at, nv, kk, 0, sel,
           [&](int slot, int pos) {
             ck[slot] = key_at(pos);
-            ci[slot] = (int32_t)(s0 + pos);
+            ci[slot] = (int32_t)(c.s0 + pos);
           },
           0u, &T);
-      if (threadIdx.x == 0) plan_cand_thr(plan, a.ws, bt)[sl] = T;
+      if (threadIdx.x == 0) plan_cand_thr(plan, a.ws, bt)[c.sl] = T;
     }
     __syncthreads();
-  }
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::TMEM_COLS);
-  }
-}
-
-// ------------------------------------------------------------------------
-// Native NVFP4 producer: the packed E2M1 K and q tiles go straight from TMA
-// (64-byte swizzle) into tcgen05.mma kind::mxf4nvf4 with block16 scales.  The
-// scales reach TMEM through tcgen05.cp from 512-byte atoms in which byte
-// m0*16 + m1*4 + kk holds the scale of tile row m0 + 32*m1 for K-block kk;
-// warp 2 permutes each tile's row-major scales (8 per entry) into two such
-// atoms (one per 64-element K-block).  Nothing is expanded: per 128-entry tile
-// shared memory sees the 9 KB the TMA writes, 1 KB of permuted scales and the
-// 12 KB the tensor core reads.
-template <int NQ>
-struct Nvf4Cfg {
-  static constexpr int N = kHI * NQ;
-  static constexpr int THREADS = 384;  // warps: 0 TMA, 1 MMA, 2 scales, 4-7 and 8-11 epilogue
-  static constexpr int STAGES = 16;
-  static constexpr int CODES = kBM * kDI / 2;           // 8 KB of E2M1 per tile
-  static constexpr int RAWSF = kBM * kDI / 16;          // 1 KB of row-major scales
-  static constexpr int ATOMS = 2 * 512;                 // two permuted scale atoms
-  static constexpr int STAGE = CODES + RAWSF + ATOMS;   // 10 KB
-  static constexpr int QCODES = N * kDI / 2;
-  static constexpr int QRAWSF = N * kDI / 16;
-  static constexpr int QREG = (QCODES + QRAWSF + ATOMS + 1023) / 1024 * 1024;
-  static constexpr int ACC_COLS = 2 * N;                // double-buffered accumulator
-  static constexpr int SFA_COL = ACC_COLS;              // 8 columns
-  static constexpr int SFB_COL = ACC_COLS + 32;         // 8 columns
-  static constexpr int TMEM_COLS = ACC_COLS + 64 <= 256 ? 256 : 512;
-  static constexpr int FIXED_SMEM = 1024 + STAGES * STAGE + QREG + NQ * kHI * 4 + 512 +
-                                    (int)sizeof(SelectSmem<THREADS>) + 1024 /*local histogram*/;
-  static constexpr uint32_t IDESC = idesc_nvf4(kBM, N);
-};
-
-// rows [0, rows) of a row-major [rows][8] scale block -> two 512-byte atoms
-// (rows >= `rows` are zero).  One warp.
-__device__ __forceinline__ void permute_scales(const uint8_t* raw, uint8_t* atoms, int rows, int lane) {
-  const uint32_t* src = reinterpret_cast<const uint32_t*>(raw);
-  uint32_t* dst = reinterpret_cast<uint32_t*>(atoms);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int w = lane + 32 * j;                 // output word: kb * 128 + m0 * 4 + m1
-    const int kb = w >> 7, m0 = (w & 127) >> 2, m1 = w & 3;
-    const int m = m0 + 32 * m1;
-    dst[w] = m < rows ? src[m * 2 + kb] : 0u;
   }
 }
 
@@ -381,14 +225,15 @@ __device__ __forceinline__ void permute_scales(const uint8_t* raw, uint8_t* atom
 // Cooperative selection: the slice CTAs of one query row (all resident at once,
 // cooperative launch) pick the row's top k together, with no candidate lists
 // and no merge kernel.  Keys are 16-bit (bf16 score images):
-//   1. each CTA adds the high-byte histogram of its keys into the row's global
-//      histogram H1; barrier; every CTA finds the high byte d1 of the k-th key;
+//   1. each CTA adds the high-byte histogram of its keys (built by the
+//      epilogue) into the row's global histogram H1; barrier; every CTA finds
+//      the high byte d1 of the k-th key;
 //   2. the same for the low byte among keys whose high byte is d1 (H2); the
 //      k-th key T and the number of ties at T to take follow;
 //   3. each CTA publishes its counts of keys > T and == T; barrier; prefix
 //      sums over the slices give each CTA its output offset and its share of
-//      the ties (lowest entry indices first), and it writes its winners in
-//      index order straight into the output row.
+//      the ties (lowest entry indices first); it writes its winners in index
+//      order straight into the output row.
 // Barriers are global counters polled with a bounded wait (the status word
 // records a timeout).
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
@@ -416,7 +261,7 @@ __device__ __forceinline__ void coop_barrier(uint32_t* ctr, uint32_t target) {
 }
 
 // Digit d (searched from 255 down) at which the running count of a 256-bin
-// histogram reaches `remaining`; returns (d, remaining - count above d) in
+// histogram reaches `remaining`; writes d and remaining - (count above d) to
 // bc[0], bc[1].  One warp.
 __device__ __forceinline__ void digit_search(const uint32_t* hist, uint32_t remaining, uint32_t* bc, int lane) {
   uint32_t c[8], s = 0;
@@ -444,19 +289,18 @@ __device__ __forceinline__ void digit_search(const uint32_t* hist, uint32_t rema
   }
 }
 
-template <int NT>
 __device__ void coop_select(const uint16_t* kq, int nv, int64_t vis, int64_t s0, int sl, const IndexPlan& plan,
-                            const IndexArgs& a, int64_t bt, const uint32_t* h1_local, SelectSmem<NT>& sm) {
-  constexpr int NW = NT / 32;
+                            const IndexArgs& a, int64_t bt, const uint32_t* h1_local, SelectSmem<kThreads>& sm) {
+  constexpr int NW = kThreads / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int S = plan.n_slices;
   int32_t* out = a.idx_out + bt * a.k;
   const int kk = (int)min64(a.k, vis);
   if (sl == 0)
-    for (int j = kk + threadIdx.x; j < a.k; j += NT) out[j] = -1;
+    for (int j = kk + threadIdx.x; j < a.k; j += kThreads) out[j] = -1;
   if (vis <= a.k) {  // every visible entry is selected: offsets in closed form
     const int64_t off = slice_cand_offset(plan, sl, vis, a.n_entries, a.k);
-    for (int p = threadIdx.x; p < nv; p += NT) out[off + p] = (int32_t)(s0 + p);
+    for (int p = threadIdx.x; p < nv; p += kThreads) out[off + p] = (int32_t)(s0 + p);
     return;
   }
   uint32_t* row = plan_coop_row(plan, a.ws, bt);
@@ -465,20 +309,20 @@ __device__ void coop_select(const uint16_t* kq, int nv, int64_t vis, int64_t s0,
   uint32_t* ctr = row + 512;
   uint32_t* gtq = row + 520;
   // 1. high byte
-  for (int d = threadIdx.x; d < 256; d += NT)
+  for (int d = threadIdx.x; d < 256; d += kThreads)
     if (h1_local[d]) atomicAdd(&H1[d], h1_local[d]);
   coop_barrier(ctr, (uint32_t)S);
   if (warp == 0) digit_search(H1, (uint32_t)kk, sm.bcast, lane);
-  for (int d = threadIdx.x; d < 256; d += NT) sm.hist[d] = 0;
+  for (int d = threadIdx.x; d < 256; d += kThreads) sm.hist[d] = 0;
   __syncthreads();
   const uint32_t d1 = sm.bcast[0], rem1 = sm.bcast[1];
   // 2. low byte among keys with high byte d1
-  for (int p = threadIdx.x; p < nv; p += NT) {
+  for (int p = threadIdx.x; p < nv; p += kThreads) {
     const uint32_t k16 = kq[p];
     if ((k16 >> 8) == d1) atomicAdd(&sm.hist[k16 & 255u], 1u);
   }
   __syncthreads();
-  for (int d = threadIdx.x; d < 256; d += NT)
+  for (int d = threadIdx.x; d < 256; d += kThreads)
     if (sm.hist[d]) atomicAdd(&H2[d], sm.hist[d]);
   coop_barrier(ctr, 2u * (uint32_t)S);
   if (warp == 0) digit_search(H2, rem1, sm.bcast + 2, lane);
@@ -496,10 +340,10 @@ __device__ void coop_select(const uint16_t* kq, int nv, int64_t vis, int64_t s0,
     c_gt += __popc(__ballot_sync(0xffffffffu, p < w1 && k16 > T));
     c_eq += __popc(__ballot_sync(0xffffffffu, p < w1 && k16 == T));
   }
-  if (lane == 0) { sm.warp_tot[warp] = c_gt; }
+  if (lane == 0) sm.warp_tot[warp] = c_gt;
   __syncthreads();
-  uint32_t gt_before_w = 0, gt_tot = 0;
-  for (int w = 0; w < NW; ++w) { gt_before_w += w < warp ? sm.warp_tot[w] : 0u; gt_tot += sm.warp_tot[w]; }
+  uint32_t gt_tot = 0;
+  for (int w = 0; w < NW; ++w) gt_tot += sm.warp_tot[w];
   __syncthreads();
   if (lane == 0) sm.warp_tot[warp] = c_eq;
   __syncthreads();
@@ -521,7 +365,6 @@ __device__ void coop_select(const uint16_t* kq, int nv, int64_t vis, int64_t s0,
   }
   int eq_take_cta = need_eq - (int)eq_prev;
   eq_take_cta = eq_take_cta < 0 ? 0 : (eq_take_cta > (int)eq_tot ? (int)eq_tot : eq_take_cta);
-  // this warp's share of the CTA's ties, then ordered compaction
   int eq_take_w = eq_take_cta - (int)eq_before_w;
   eq_take_w = eq_take_w < 0 ? 0 : (eq_take_w > (int)c_eq ? (int)c_eq : eq_take_w);
   __syncthreads();
@@ -541,63 +384,143 @@ __device__ void coop_select(const uint16_t* kq, int nv, int64_t vis, int64_t s0,
     o += __popc(tm);
     eq_seen += __popc(eqm);
   }
-  (void)gt_before_w;
+}
+
+// ----------------------------------------------------------------- BF16 kernel
+template <int NQ>
+__global__ void __launch_bounds__(kThreads, 1)
+    index_bf16_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ, IndexArgs a,
+                      IndexPlan plan) {
+  using C = Bf16Cfg<NQ>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* ks = align1024(smem_raw);                        // K ring
+  uint8_t* qs = ks + C::STAGES * C::K_STAGE;                // query tile
+  uint16_t* keys = reinterpret_cast<uint16_t*>(qs + C::Q_BYTES);
+  float* wsm = reinterpret_cast<float*>(keys + NQ * plan.slice_len);
+  uint64_t* full = reinterpret_cast<uint64_t*>(wsm + NQ * kHI);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* accf = empty + C::STAGES;
+  uint64_t* acce = accf + C::NBUF;
+  uint64_t* qbar = acce + C::NBUF;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qbar + 1);
+  SelectSmem<kThreads>& sel = *reinterpret_cast<SelectSmem<kThreads>*>(tmem_slot + 4);
+
+  const SliceCtx<NQ> c = slice_ctx<NQ>(a, plan);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < NQ * kHI; i += kThreads) {
+    const int t = c.t0 + i / kHI;
+    wsm[i] = t < a.n_q ? a.wI[((int64_t)c.b * a.n_q + t) * kHI + (i % kHI)] : 0.f;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int i = 0; i < C::NBUF; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 4); }
+    mbar_init(qbar, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      const int qrow = (c.b * a.n_q + c.t0) * kHI;
+      mbar_arrive_expect_tx(qbar, C::Q_BYTES);
+      tma_load_2d(qs, &tmQ, qbar, 0, qrow);
+      tma_load_2d(qs + C::N * 128, &tmQ, qbar, 64, qrow);
+      for (int i = 0; i < c.n_tiles; ++i) {
+        const int s = i % C::STAGES, j = i / C::STAGES;
+        if (j > 0 && !mbar_wait(&empty[s], (j - 1) & 1)) break;
+        mbar_arrive_expect_tx(&full[s], C::K_STAGE);
+        const int row = (int)((int64_t)c.b * a.n_entries + c.s0 + (int64_t)i * kBM);
+        uint8_t* dst = ks + s * C::K_STAGE;
+        tma_load_2d(dst, &tmK, &full[s], 0, row);
+        tma_load_2d(dst + kAtom, &tmK, &full[s], 64, row);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      bool ok = mbar_wait(qbar, 0);
+      const uint32_t qa = smem_u32(qs);
+      for (int i = 0; ok && i < c.n_tiles; ++i) {
+        const int s = i % C::STAGES, j = i / C::STAGES, buf = i % C::NBUF, u = i / C::NBUF;
+        if (!mbar_wait(&full[s], j & 1)) break;
+        if (u > 0 && !mbar_wait(&acce[buf], (u - 1) & 1)) break;
+        tc_fence_after();
+        const uint32_t ka = smem_u32(ks + s * C::K_STAGE);
+        const uint32_t d = tmem + (uint32_t)(buf * C::N);
+#pragma unroll
+        for (int kk = 0; kk < kDI / 16; ++kk) {
+          const uint32_t within = (uint32_t)(kk & 3) * 32u;  // 16 bf16 = 32 bytes
+          const uint32_t a_addr = ka + (uint32_t)(kk >> 2) * kAtom + within;
+          const uint32_t b_addr = qa + (uint32_t)(kk >> 2) * (C::N * 128) + within;
+          tc_mma_f16(d, umma_desc_sw128(a_addr), umma_desc_sw128(b_addr), C::IDESC, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&empty[s]);
+        tc_commit(&accf[buf]);
+      }
+    }
+  } else if (warp >= 4) {
+    epilogue_group<NQ, C::N, C::NBUF>(c, a, plan, tmem, accf, acce, wsm, keys, false, nullptr);
+  }
+  scores_tail<NQ>(c, a);
+  tc_fence_before();
+  __syncthreads();
+  slice_select<NQ>(c, a, plan, keys, sel);
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- NVFP4 kernel
+// rows [0, rows) of a row-major [rows][8] scale block -> two 512-byte atoms
+// (rows >= `rows` are zero).  One warp.
+__device__ __forceinline__ void permute_scales(const uint8_t* raw, uint8_t* atoms, int rows, int lane) {
+  const uint32_t* src = reinterpret_cast<const uint32_t*>(raw);
+  uint32_t* dst = reinterpret_cast<uint32_t*>(atoms);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int w = lane + 32 * j;                 // output word: kb * 128 + m0 * 4 + m1
+    const int kb = w >> 7, m0 = (w & 127) >> 2, m1 = w & 3;
+    const int m = m0 + 32 * m1;
+    dst[w] = m < rows ? src[m * 2 + kb] : 0u;
+  }
 }
 
 template <int NQ>
-__global__ void __launch_bounds__(Nvf4Cfg<NQ>::THREADS, 1)
+__global__ void __launch_bounds__(kThreads, 1)
     index_nvf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
-                      const __grid_constant__ CUtensorMap tmKs, const __grid_constant__ CUtensorMap tmQs,
-                      IndexArgs a, IndexPlan plan) {
+                      const __grid_constant__ CUtensorMap tmQs, IndexArgs a, IndexPlan plan) {
   using C = Nvf4Cfg<NQ>;
-  constexpr int NT = C::THREADS;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* st = align1024(smem_raw);                          // stages
+  uint8_t* st = align1024(smem_raw);                          // stages: codes | scale atoms
   uint8_t* qreg = st + C::STAGES * C::STAGE;                  // q codes | q raw scales | q atoms
   uint16_t* keys = reinterpret_cast<uint16_t*>(qreg + C::QREG);
   float* wsm = reinterpret_cast<float*>(keys + NQ * plan.slice_len);
   uint64_t* full = reinterpret_cast<uint64_t*>(wsm + NQ * kHI);
-  uint64_t* sfr = full + C::STAGES;
-  uint64_t* empty = sfr + C::STAGES;
+  uint64_t* empty = full + C::STAGES;
   uint64_t* accf = empty + C::STAGES;
-  uint64_t* acce = accf + 2;
-  uint64_t* qbar = acce + 2;
+  uint64_t* acce = accf + C::NBUF;
+  uint64_t* qbar = acce + C::NBUF;
   uint64_t* qsf = qbar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qsf + 1);
-  SelectSmem<NT>& sel = *reinterpret_cast<SelectSmem<NT>*>(tmem_slot + 4);
+  SelectSmem<kThreads>& sel = *reinterpret_cast<SelectSmem<kThreads>*>(tmem_slot + 4);
   uint32_t* h1s = reinterpret_cast<uint32_t*>(&sel + 1);  // [256] high-byte histogram (cooperative select)
 
-  const int sl = blockIdx.x, grp = blockIdx.y, b = blockIdx.z;
-  const int t0 = grp * NQ;
+  const SliceCtx<NQ> c = slice_ctx<NQ>(a, plan);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t s0 = (int64_t)sl * plan.slice_len;
-  const int len = (int)min64(plan.slice_len, a.n_entries - s0);
   const bool coop = NQ == 1 && plan.coop;
-
-  int n_valid[NQ];
-  int64_t vis[NQ];
-  int max_valid = 0;
-#pragma unroll
-  for (int q = 0; q < NQ; ++q) {
-    const int t = t0 + q;
-    vis[q] = t < a.n_q ? visible_entries(a.q_pos[(int64_t)b * a.n_q + t], a.m, a.n_entries) : 0;
-    n_valid[q] = (int)max64(0, min64(len, vis[q] - s0));
-    max_valid = max(max_valid, n_valid[q]);
+  for (int i = threadIdx.x; i < NQ * kHI; i += kThreads) {
+    const int t = c.t0 + i / kHI;
+    wsm[i] = t < a.n_q ? a.wI[((int64_t)c.b * a.n_q + t) * kHI + (i % kHI)] : 0.f;
   }
-  const int n_tiles = (max_valid + kBM - 1) / kBM;
-
-  for (int i = threadIdx.x; i < NQ * kHI; i += NT) {
-    const int t = t0 + i / kHI;
-    wsm[i] = t < a.n_q ? a.wI[((int64_t)b * a.n_q + t) * kHI + (i % kHI)] : 0.f;
-  }
-  for (int i = threadIdx.x; i < 256; i += NT) h1s[i] = 0;
+  for (int i = threadIdx.x; i < 256; i += kThreads) h1s[i] = 0;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&sfr[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int i = 0; i < 2; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 4); }
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int i = 0; i < C::NBUF; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 4); }
     mbar_init(qbar, 1);
     mbar_init(qsf, 1);
     fence_barrier_init();
@@ -611,151 +534,72 @@ __global__ void __launch_bounds__(Nvf4Cfg<NQ>::THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      const int qrow = (b * a.n_q + t0) * kHI;
+      const int qrow = (c.b * a.n_q + c.t0) * kHI;
       mbar_arrive_expect_tx(qbar, C::QCODES + C::QRAWSF);
       tma_load_2d(qreg, &tmQ, qbar, 0, qrow);
       tma_load_2d(qreg + C::QCODES, &tmQs, qbar, 0, qrow / 2);
-      for (int i = 0; i < n_tiles; ++i) {
+      // request b's blocked key scales: 1 KB (two atoms) per 128-entry block;
+      // slices start on block boundaries, so tile i is block s0/128 + i
+      const uint8_t* ksf = static_cast<const uint8_t*>(a.KI_sf) +
+                           (int64_t)c.b * nvfp4_blocked_sf_bytes(a.n_entries, kDI) + (c.s0 / kBM) * C::ATOMS;
+      for (int i = 0; i < c.n_tiles; ++i) {
         const int s = i % C::STAGES, j = i / C::STAGES;
         if (j > 0 && !mbar_wait(&empty[s], (j - 1) & 1)) break;
-        mbar_arrive_expect_tx(&full[s], C::CODES + C::RAWSF);
-        const int row = (int)((int64_t)b * a.n_entries + s0 + (int64_t)i * kBM);
+        mbar_arrive_expect_tx(&full[s], C::CODES + C::ATOMS);
+        const int row = (int)((int64_t)c.b * a.n_entries + c.s0 + (int64_t)i * kBM);
         uint8_t* dst = st + s * C::STAGE;
         tma_load_2d(dst, &tmK, &full[s], 0, row);
-        tma_load_2d(dst + C::CODES, &tmKs, &full[s], 0, row / 2);
+        bulk_load(dst + C::CODES, ksf + (int64_t)i * C::ATOMS, C::ATOMS, &full[s]);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------- MMA issuer
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------------ MMA issuers
+    // warp 1 issues the even tiles and warp 3 the odd ones, each with its own
+    // TMEM scale columns; tcgen05.commit tracks the issuing thread's work only.
     if (lane == 0) {
-      bool ok = mbar_wait(qbar, 0) && mbar_wait(qsf, 0);
+      const int w = warp == 1 ? 0 : 1;
+      const bool ok = mbar_wait(qsf, 0);
       const uint32_t qa = smem_u32(qreg);
+      const uint32_t sfa = tmem + C::SFA_COL + 8 * w, sfb = tmem + C::SFB_COL + 8 * w;
       if (ok) {
         tc_fence_after();
         for (int kb = 0; kb < 2; ++kb)
-          tc_cp_32x128b_warpx4(tmem + C::SFB_COL + kb * 4,
-                               umma_desc_rows16(qa + C::QCODES + C::QRAWSF + kb * 512));
+          tc_cp_32x128b_warpx4(sfb + kb * 4, umma_desc_rows16(qa + C::QCODES + C::QRAWSF + kb * 512));
       }
-      for (int i = 0; ok && i < n_tiles; ++i) {
-        const int s = i % C::STAGES, j = i / C::STAGES, buf = i & 1, u = i >> 1;
-        if (!mbar_wait(&full[s], j & 1) || !mbar_wait(&sfr[s], j & 1)) break;
+      for (int i = w; ok && i < c.n_tiles; i += 2) {
+        const int s = i % C::STAGES, j = i / C::STAGES, buf = i % C::NBUF, u = i / C::NBUF;
+        if (!mbar_wait(&full[s], j & 1)) break;
         if (u > 0 && !mbar_wait(&acce[buf], (u - 1) & 1)) break;
         tc_fence_after();
         const uint32_t base = smem_u32(st + s * C::STAGE);
         for (int kb = 0; kb < 2; ++kb)
-          tc_cp_32x128b_warpx4(tmem + C::SFA_COL + kb * 4, umma_desc_rows16(base + C::CODES + C::RAWSF + kb * 512));
+          tc_cp_32x128b_warpx4(sfa + kb * 4, umma_desc_rows16(base + C::CODES + kb * 512));
         const uint32_t d = tmem + (uint32_t)(buf * C::N);
         for (int kb = 0; kb < 2; ++kb)
-          tc_mma_nvf4(d, umma_desc_sw64(base + kb * 32), umma_desc_sw64(qa + kb * 32), C::IDESC,
-                      tmem + C::SFA_COL + kb * 4, tmem + C::SFB_COL + kb * 4, kb > 0 ? 1u : 0u);
+          tc_mma_nvf4(d, umma_desc_sw64(base + kb * 32), umma_desc_sw64(qa + kb * 32), C::IDESC, sfa + kb * 4,
+                      sfb + kb * 4, kb > 0 ? 1u : 0u);
         tc_commit(&empty[s]);
         tc_commit(&accf[buf]);
       }
     }
   } else if (warp == 2) {
-    // ------------------------------------------ scale permutation into atoms
-    bool ok = mbar_wait(qbar, 0);
-    if (ok) permute_scales(qreg + C::QCODES, qreg + C::QCODES + C::QRAWSF, C::N, lane);
+    // --------------------------------------- query scales into their atoms
+    if (mbar_wait(qbar, 0)) permute_scales(qreg + C::QCODES, qreg + C::QCODES + C::QRAWSF, C::N, lane);
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(qsf);
-    for (int i = 0; ok && i < n_tiles; ++i) {
-      const int s = i % C::STAGES, j = i / C::STAGES;
-      if (!mbar_wait(&full[s], j & 1)) break;
-      uint8_t* stage = st + s * C::STAGE;
-      permute_scales(stage + C::CODES, stage + C::CODES + C::RAWSF, kBM, lane);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sfr[s]);
-    }
   } else if (warp >= 4) {
-    // --------------------------------------------------------------- epilogue
-    // Two groups of four warps; group g drains accumulator buffer g, i.e. the
-    // tiles i with i % 2 == g.  Warp w reads TMEM lanes 32 * (w % 4) ...
-    const int quarter = warp & 3, grp_e = (warp - 4) >> 2;
-    const int r = quarter * 32 + lane;
-    float wreg[NQ == 1 ? kHI : 1];
-    if (NQ == 1) {
-#pragma unroll
-      for (int h = 0; h < kHI; ++h) wreg[h] = wsm[h];
-    }
-    for (int i = grp_e; i < n_tiles; i += 2) {
-      const int buf = i & 1, u = i >> 1;
-      if (!mbar_wait(&accf[buf], u & 1)) break;
-      tc_fence_after();
-      float acc[NQ][kHI];
-      const uint32_t taddr = tmem + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(buf * C::N);
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        tmem_ld_32x32b_x32(taddr + q * kHI, &acc[q][0]);
-        tmem_ld_32x32b_x32(taddr + q * kHI + 32, &acc[q][32]);
-      }
-      tmem_ld_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&acce[buf]);
-      const int pos = i * kBM + r;
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int h = 0; h < kHI; ++h)
-          part[h & 3] = fmaf(NQ == 1 ? wreg[h % (NQ == 1 ? kHI : 1)] : wsm[q * kHI + h], fmaxf(acc[q][h], 0.f),
-                             part[h & 3]);
-        const float I = (part[0] + part[1]) + (part[2] + part[3]);
-        const uint32_t key = bf16_key(I);
-        const bool valid = pos < n_valid[q];
-        keys[q * plan.slice_len + pos] = valid ? (uint16_t)(key >> 16) : (uint16_t)0;
-        if (coop && valid) atomicAdd(&h1s[key >> 24], 1u);
-        if (a.scores_out != nullptr && pos < len && t0 + q < a.n_q) {
-          const float sc = valid ? key_to_f32(key) : -INFINITY;
-          static_cast<__nv_bfloat16*>(a.scores_out)[((int64_t)b * a.n_q + t0 + q) * a.n_entries + s0 + pos] =
-              __float2bfloat16_rn(sc);
-        }
-      }
-    }
+    epilogue_group<NQ, C::N, C::NBUF>(c, a, plan, tmem, accf, acce, wsm, keys, coop, h1s);
   }
-  if (a.scores_out != nullptr) {
-    for (int q = 0; q < NQ; ++q) {
-      if (t0 + q >= a.n_q) continue;
-      for (int pos = n_tiles * kBM + threadIdx.x; pos < len; pos += NT)
-        static_cast<__nv_bfloat16*>(a.scores_out)[((int64_t)b * a.n_q + t0 + q) * a.n_entries + s0 + pos] =
-            __float2bfloat16_rn(-INFINITY);
-    }
-  }
+  scores_tail<NQ>(c, a);
   tc_fence_before();
   __syncthreads();
   if (coop) {
-    if (t0 < a.n_q) coop_select<NT>(keys, n_valid[0], vis[0], s0, sl, plan, a, (int64_t)b * a.n_q + t0, h1s, sel);
+    if (c.t0 < a.n_q)
+      coop_select(keys, c.n_valid[0], c.vis[0], c.s0, c.sl, plan, a, (int64_t)c.b * a.n_q + c.t0, h1s, sel);
     __syncthreads();
-  }
-  for (int q = 0; q < NQ && !coop; ++q) {
-    const int t = t0 + q;
-    if (t >= a.n_q) break;
-    const int64_t bt = (int64_t)b * a.n_q + t;
-    const int nv = n_valid[q];
-    const int kk = min(a.k, nv);
-    const uint16_t* kq = keys + q * plan.slice_len;
-    auto key_at = [&](int i) { return ((uint32_t)kq[i]) << 16; };
-    if (plan.n_slices == 1) {
-      int32_t* out = a.idx_out + bt * a.k;
-      block_select<NT>(key_at, nv, kk, 2, sel, [&](int slot, int pos) { out[slot] = (int32_t)(s0 + pos); });
-      for (int j = kk + threadIdx.x; j < a.k; j += NT) out[j] = -1;
-    } else {
-      const int64_t off = slice_cand_offset(plan, sl, vis[q], a.n_entries, a.k);
-      uint32_t* ck = plan_cand_keys(plan, a.ws, bt) + off;
-      int32_t* ci = plan_cand_idx(plan, a.ws, bt) + off;
-      uint32_t T = 0;
-      block_select<NT>(
-          key_at, nv, kk, 2, sel,
-          [&](int slot, int pos) {
-            ck[slot] = key_at(pos);
-            ci[slot] = (int32_t)(s0 + pos);
-          },
-          0u, &T);
-      if (threadIdx.x == 0) plan_cand_thr(plan, a.ws, bt)[sl] = T;
-    }
-    __syncthreads();
+  } else {
+    slice_select<NQ>(c, a, plan, keys, sel);
   }
   if (warp == 1) {
     tc_fence_after();
@@ -791,42 +635,19 @@ bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int esize, const v
             swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int NQ, bool FP4>
-size_t tc_smem(const IndexPlan& p) {
-  return (size_t)TcCfg<NQ, FP4>::FIXED_SMEM + (size_t)NQ * p.slice_len * 2;
-}
-
-template <int NQ, bool FP4>
-cudaError_t launch_tc(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) {
-  using C = TcCfg<NQ, FP4>;
-  CUtensorMap tmK, tmQ, tmKs, tmQs;
+template <int NQ>
+cudaError_t launch_bf16(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) {
+  using C = Bf16Cfg<NQ>;
+  CUtensorMap tmK, tmQ;
   const uint64_t krows = (uint64_t)a.batch * a.n_entries, qrows = (uint64_t)a.batch * a.n_q * kHI;
-  bool ok;
-  if (FP4) {
-    // codes [rows][64 B]; scales viewed as [rows/2][16 B] (two entries per line)
-    ok = make_map_2d(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.KI, krows, kDI / 2, kDI / 2, kBM,
-                     CU_TENSOR_MAP_SWIZZLE_NONE) &&
-         make_map_2d(&tmKs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.KI_sf, krows / 2, 16, 16, kBM / 2,
-                     CU_TENSOR_MAP_SWIZZLE_NONE) &&
-         make_map_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.qI, qrows, kDI / 2, kDI / 2, C::N,
-                     CU_TENSOR_MAP_SWIZZLE_NONE) &&
-         make_map_2d(&tmQs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.qI_sf, qrows / 2, 16, 16, C::N / 2,
-                     CU_TENSOR_MAP_SWIZZLE_NONE);
-  } else {
-    ok = make_map_2d(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.KI, krows, kDI, 64, kBM,
-                     CU_TENSOR_MAP_SWIZZLE_128B) &&
-         make_map_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.qI, qrows, kDI, 64, C::N,
-                     CU_TENSOR_MAP_SWIZZLE_128B);
-    tmKs = tmK;
-    tmQs = tmQ;
-  }
-  if (!ok) return cudaErrorInvalidValue;
-  const size_t smem = tc_smem<NQ, FP4>(p);
-  cudaError_t e = cudaFuncSetAttribute(index_tc_kernel<NQ, FP4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem);
+  if (!make_map_2d(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.KI, krows, kDI, 64, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+      !make_map_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.qI, qrows, kDI, 64, C::N, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  const size_t smem = (size_t)C::FIXED_SMEM + (size_t)NQ * p.slice_len * 2;
+  cudaError_t e = cudaFuncSetAttribute(index_bf16_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_slices, (a.n_q + NQ - 1) / NQ, a.batch);
-  index_tc_kernel<NQ, FP4><<<grid, C::THREADS, smem, s>>>(tmK, tmQ, tmKs, tmQs, a, p);
+  index_bf16_kernel<NQ><<<grid, kThreads, smem, s>>>(tmK, tmQ, a, p);
   ++launch_counter();
   return cudaGetLastError();
 }
@@ -834,15 +655,13 @@ cudaError_t launch_tc(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) {
 template <int NQ>
 cudaError_t launch_nvf4(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) {
   using C = Nvf4Cfg<NQ>;
-  CUtensorMap tmK, tmQ, tmKs, tmQs;
+  CUtensorMap tmK, tmQ, tmQs;
   const uint64_t krows = (uint64_t)a.batch * a.n_entries, qrows = (uint64_t)a.batch * a.n_q * kHI;
-  // packed E2M1 rows of 64 bytes in the 64-byte swizzle; scales as 16-byte
-  // lines holding two entries each
+  // packed E2M1 rows of 64 bytes in the 64-byte swizzle; query scales as
+  // 16-byte lines holding two head rows each (key scales are bulk-copied)
   const bool ok =
       make_map_2d(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.KI, krows, kDI / 2, kDI / 2, kBM,
                   CU_TENSOR_MAP_SWIZZLE_64B) &&
-      make_map_2d(&tmKs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.KI_sf, krows / 2, 16, 16, kBM / 2,
-                  CU_TENSOR_MAP_SWIZZLE_NONE) &&
       make_map_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.qI, qrows, kDI / 2, kDI / 2, C::N,
                   CU_TENSOR_MAP_SWIZZLE_64B) &&
       make_map_2d(&tmQs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.qI_sf, qrows / 2, 16, 16, C::N / 2,
@@ -859,13 +678,13 @@ cudaError_t launch_nvf4(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) 
     if (e != cudaSuccess) return e;
     IndexArgs aa = a;
     IndexPlan pp = p;
-    CUtensorMap m0 = tmK, m1 = tmQ, m2 = tmKs, m3 = tmQs;
-    void* args[] = {&m0, &m1, &m2, &m3, &aa, &pp};
-    e = cudaLaunchCooperativeKernel((const void*)index_nvf4_kernel<NQ>, grid, dim3(C::THREADS), args, smem, s);
+    CUtensorMap m0 = tmK, m1 = tmQ, m2 = tmQs;
+    void* args[] = {&m0, &m1, &m2, &aa, &pp};
+    e = cudaLaunchCooperativeKernel((const void*)index_nvf4_kernel<NQ>, grid, dim3(kThreads), args, smem, s);
     ++launch_counter();
     return e;
   }
-  index_nvf4_kernel<NQ><<<grid, C::THREADS, smem, s>>>(tmK, tmQ, tmKs, tmQs, a, p);
+  index_nvf4_kernel<NQ><<<grid, kThreads, smem, s>>>(tmK, tmQ, tmQs, a, p);
   ++launch_counter();
   return cudaGetLastError();
 }
@@ -890,9 +709,9 @@ bool index_tc_eligible(const IndexArgs& a) {
   if ((int64_t)a.batch * a.n_entries >= ((int64_t)1 << 31) || (int64_t)a.batch * a.n_q * kHI >= ((int64_t)1 << 31))
     return false;
   if (a.dt == CSA_BF16) return true;
-  // NVFP4: the scale arrays are streamed as 16-byte lines of two entries, so
-  // the entry count must be even and the scale arrays 16-byte aligned.
-  return a.dt == CSA_IDX_NVFP4 && a.n_entries % 2 == 0 && aligned16(a.KI_sf) && aligned16(a.qI_sf);
+  // NVFP4: key scale atoms are bulk-copied and query scales streamed as
+  // 16-byte lines, so both arrays must be 16-byte aligned.
+  return a.dt == CSA_IDX_NVFP4 && aligned16(a.KI_sf) && aligned16(a.qI_sf);
 }
 
 int index_tc_nq(int n_q) { return n_q >= 2 ? 2 : 1; }
@@ -900,14 +719,15 @@ int index_tc_nq(int n_q) { return n_q >= 2 ? 2 : 1; }
 IndexPlan make_tc_plan(int batch, int n_q, int64_t n_entries, int k, int dt) {
   const int NQ = index_tc_nq(n_q);
   const bool fp4 = dt == CSA_IDX_NVFP4;
-  const int fixed = NQ == 1 ? (fp4 ? Nvf4Cfg<1>::FIXED_SMEM : TcCfg<1, false>::FIXED_SMEM)
-                            : (fp4 ? Nvf4Cfg<2>::FIXED_SMEM : TcCfg<2, false>::FIXED_SMEM);
+  const int fixed = NQ == 1 ? (fp4 ? Nvf4Cfg<1>::FIXED_SMEM : Bf16Cfg<1>::FIXED_SMEM)
+                            : (fp4 ? Nvf4Cfg<2>::FIXED_SMEM : Bf16Cfg<2>::FIXED_SMEM);
   constexpr int kSmemCap = 227 * 1024;
   int64_t max_slice = ((kSmemCap - fixed) / (2 * NQ)) / kBM * kBM;
   const int64_t groups = (n_q + NQ - 1) / NQ;
   const int64_t units = (int64_t)batch * groups;
-  // one wave: at most 148 CTAs (one per SM; the kernel's shared memory allows one)
-  const int64_t want = units >= 148 ? 1 : 148 / units;
+  const int sms = sm_count();
+  // one wave: at most one CTA per SM (the kernels' shared memory allows one)
+  const int64_t want = units >= sms ? 1 : sms / units;
   int64_t len = (n_entries + want - 1) / want;
   len = (len + kBM - 1) / kBM * kBM;
   if (len < kBM) len = kBM;
@@ -918,16 +738,16 @@ IndexPlan make_tc_plan(int batch, int n_q, int64_t n_entries, int k, int dt) {
   if (p.n_slices < 1) p.n_slices = 1;
   p.n_rows = (int64_t)batch * n_q;
   // NVFP4 decode rows split over several slices select cooperatively when the
-  // whole grid fits on the GPU at once (one CTA per SM)
-  p.coop = (fp4 && NQ == 1 && p.n_slices > 1 && units * p.n_slices <= sm_count()) ? 1 : 0;
+  // whole grid fits on the GPU at once
+  p.coop = (fp4 && NQ == 1 && p.n_slices > 1 && units * p.n_slices <= sms) ? 1 : 0;
   p.cand_cap = (p.n_slices > 1 && !p.coop) ? (int64_t)p.n_slices * k : 0;
   return p;
 }
 
 cudaError_t launch_index_tc(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) {
   const bool fp4 = a.dt == CSA_IDX_NVFP4;
-  if (index_tc_nq(a.n_q) == 1) return fp4 ? launch_nvf4<1>(a, p, s) : launch_tc<1, false>(a, p, s);
-  return fp4 ? launch_nvf4<2>(a, p, s) : launch_tc<2, false>(a, p, s);
+  if (index_tc_nq(a.n_q) == 1) return fp4 ? launch_nvf4<1>(a, p, s) : launch_bf16<1>(a, p, s);
+  return fp4 ? launch_nvf4<2>(a, p, s) : launch_bf16<2>(a, p, s);
 }
 
 }  // namespace csa

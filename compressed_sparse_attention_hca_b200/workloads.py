@@ -133,6 +133,21 @@ def nvfp4_rows(g, shape, dim: int, device="cpu"):
     return codes.view(*shape, dim // 2), sf.contiguous().view(*shape, dim // 16)
 
 
+def block_scales(sf, dim: int):
+    """Row-major NVFP4 scales [..., rows, dim/16] -> the key-cache layout
+    [..., ceil(rows/128) * (dim/64) * 512]: 128-row blocks of 512-byte atoms,
+    byte m0*16 + m1*4 + kk of atom a holding the scale of block row m0 + 32*m1
+    for values 64*a + 16*kk .. +15 (a pure index permutation)."""
+    *lead, rows, ns = sf.shape
+    nb = (rows + 127) // 128
+    pad = torch.zeros(*lead, nb * 128, ns, dtype=sf.dtype, device=sf.device)
+    pad[..., :rows, :] = sf
+    x = pad.view(*lead, nb, 4, 32, dim // 64, 4)           # (block, m1, m0, atom, kk)
+    n = len(lead)
+    x = x.permute(*range(n), n, n + 3, n + 2, n + 1, n + 4)  # (block, atom, m0, m1, kk)
+    return x.contiguous().view(*lead, nb * (dim // 64) * 512)
+
+
 def compress_inputs(g, batch: int, n_tok: int, dim: int, m: int, overlap: bool, dtype,
                     c_std=1.0, z_std=1.0, b_std=0.1, device="cpu"):
     """Per-token C^a, C^b, Z^a, Z^b [batch, n_tok, dim] and biases B^a, B^b [m, dim] fp32."""
@@ -183,7 +198,8 @@ def attention_inputs(cfg: dict, device="cpu", batch=None, ctx=None, n_q=None, q0
         dI, HI = cfg["dI"], cfg["n_hI"]
         if cfg["idx_dt"] == NVFP4:
             out["qI"], out["qI_sf"] = nvfp4_rows(g, (B, T, HI), dI, device)
-            out["KI"], out["KI_sf"] = nvfp4_rows(g, (B, E), dI, device)
+            out["KI"], ksf = nvfp4_rows(g, (B, E), dI, device)
+            out["KI_sf"] = block_scales(ksf, dI)  # key-cache scale layout
         else:
             out["qI"] = normal(g, (B, T, HI, dI), 1.0, _torch_dtype(cfg["idx_dt"]), device)
             out["KI"] = normal(g, (B, E, dI), 1.0, _torch_dtype(cfg["idx_dt"]), device)

@@ -44,10 +44,20 @@
  *                  and round to nearest even, saturating at +-448.
  *   CSA_IDX_NVFP4  indexer query/key rows as two arrays: codes
  *                  [rows][dim/2] bytes (element 2j in the low nibble of byte
- *                  j) and scales [rows][dim/16] unsigned E4M3, one per 16
- *                  values.  value = e2m1 * scale.  Writers use
+ *                  j) and E4M3 scales, one per 16 values (dim a multiple of
+ *                  64).  value = e2m1 * scale.  Writers use
  *                  scale = E4M3(amax/6) and codes = E2M1(x / scale), both
  *                  rounded to nearest even with saturation.
+ *                  Query scales are row-major: [rows][dim/16].
+ *                  Key-cache scales are BLOCKED, in the tensor core's
+ *                  scale-factor atom layout, per request of n rows:
+ *                  ceil(n/128) blocks of dim/64 atoms of 512 bytes
+ *                  (csa_nvfp4_key_scale_bytes(n, dim) bytes); scale j of row
+ *                  r sits at byte
+ *                    (r/128)*(dim/64)*512 + (j/4)*512
+ *                      + (r%32)*16 + ((r%128)/32)*4 + j%4.
+ *                  Bytes of rows past n in the last block are never read
+ *                  into a result.
  */
 #ifndef CSA_B200_H
 #define CSA_B200_H
@@ -94,6 +104,10 @@ csa_status_t csa_check_device_status(void);
  * when dim is not valid for the format. */
 int64_t csa_row_bytes(csa_dtype_t dt, int dim);
 
+/* Bytes of one request's blocked NVFP4 key-scale array of n_rows rows, or -1
+ * when n_rows < 0 or dim is not a positive multiple of 64. */
+int64_t csa_nvfp4_key_scale_bytes(int64_t n_rows, int dim);
+
 /*
  * csa_compress -- Token-Level Compressor ([P5] 1.2 Step 1; [P1] eq. 6-7;
  * HCA form [P5] 1.3, [P1] eq. 10-11).
@@ -114,15 +128,23 @@ int64_t csa_row_bytes(csa_dtype_t dt, int dim);
  *                   need, m*(e0-1) (or m*e0 without overlap / at e0 = 0) up
  *                   to m*(e0+n_out)-1, must lie in [tok0, tok0+n_tok).
  *   out             [batch][out_batch_stride rows] of out_dt (F32, BF16,
- *                   KV_FP8MIX, IDX_NVFP4); entry i of request b is written
- *                   to row b*out_batch_stride + (i - e0).
- *   out_sf          NVFP4 only: scales [batch][out_batch_stride][dim/16].
+ *                   KV_FP8MIX, IDX_NVFP4): a cache of out_batch_stride rows
+ *                   per request; entry i of request b is written to row
+ *                   out_row0 + (i - e0) of request b (row
+ *                   b*out_batch_stride + out_row0 + i - e0); other rows are
+ *                   left untouched.  out_row0 + n_out <= out_batch_stride.
+ *   out_sf          NVFP4 only (dim a multiple of 64): the cache's blocked
+ *                   key scales, request b's array of
+ *                   csa_nvfp4_key_scale_bytes(out_batch_stride, dim) bytes
+ *                   starting at b times that size; only the written rows'
+ *                   scale bytes change.
  */
 csa_status_t csa_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
                           const float* Ba, const float* Bb, int batch, int64_t n_tok,
                           int64_t tok0, int64_t in_batch_stride, int64_t e0, int64_t n_out,
                           int dim, int m, csa_dtype_t in_dt, void* out, void* out_sf,
-                          int64_t out_batch_stride, csa_dtype_t out_dt, void* stream);
+                          int64_t out_batch_stride, int64_t out_row0, csa_dtype_t out_dt,
+                          void* stream);
 
 /*
  * csa_index_topk -- Lightning Indexer fused with the top-k selector ([P5] 1.2
@@ -140,14 +162,18 @@ csa_status_t csa_compress(const void* Ca, const void* Cb, const void* Za, const 
  *   qI        [batch][n_q][n_heads][dim] of dt; NVFP4: codes, with qI_sf
  *             [batch][n_q][n_heads][dim/16] scales.
  *   wI        [batch][n_q][n_heads] fp32 head weights.
- *   KI        [batch][n_entries][dim] of dt; NVFP4: codes, with KI_sf.
+ *   KI        [batch][n_entries][dim] of dt; NVFP4: codes, with KI_sf the
+ *             blocked key scales, request b's array of
+ *             csa_nvfp4_key_scale_bytes(n_entries, dim) bytes at b times
+ *             that size.
  *   q_pos     [batch][n_q] int64 absolute position of each query.
  *   idx_out   [batch][n_q][k] int32 entry indices (per request).
  *   scores_out  optional (NULL in production): [batch][n_q][n_entries] of
  *             the selection scores (bf16, or fp32 for F32 inputs), -inf for
  *             entries not visible.  Used by tests to check selection.
  *   dt        CSA_F32, CSA_BF16 or CSA_IDX_NVFP4 (qI and KI share it).
- * Limits: 1 <= k <= 2048, dim a multiple of 32 (<= 256), n_heads <= 128.
+ * Limits: 1 <= k <= 2048, dim a multiple of 32 (<= 256; NVFP4: of 64),
+ * n_heads <= 128.
  */
 size_t csa_index_topk_workspace_size(int batch, int n_q, int64_t n_entries, int k, int n_heads,
                                      int dim, csa_dtype_t dt);

@@ -58,6 +58,9 @@ def _load():
         "orc_row_bytes": (i64, [i32, i32]),
         "orc_decode_rows": (i32, [P, P, i32, i32, i64, P]),
         "orc_encode_rows": (i32, [P, i32, i32, i64, P, P]),
+        "orc_nvfp4_blocked_bytes": (i64, [i64, i32]),
+        "orc_nvfp4_unblock_scales": (i32, [P, i64, i32, P]),
+        "orc_nvfp4_block_scales": (i32, [P, i64, i32, P]),
         "orc_compress": (i32, [P, P, P, P, P, P, i64, i64, i64, i64, i32, i32, P]),
         "orc_index_scores": (None, [P, P, P, i32, i32, i64, P]),
         "orc_topk": (i32, [P, i64, i32, P]),
@@ -133,12 +136,33 @@ def row_bytes(dt: int, dim: int) -> int:
     return int(_load().orc_row_bytes(dt, dim))
 
 
-def decode_rows(buf, dt: int, dim: int, sf=None) -> np.ndarray:
-    """Decode rows of format dt into float64 [rows, dim] (exact)."""
+def unblock_scales(blocked, n_rows: int, dim: int) -> np.ndarray:
+    """NVFP4 key-cache scales (128-row blocks of tensor-core atoms) -> [rows, dim/16]."""
+    blocked = _c(blocked, np.uint8)
+    out = np.zeros((n_rows, dim // 16), np.uint8)
+    _check(_load().orc_nvfp4_unblock_scales(_p(blocked), n_rows, dim, _p(out)), "unblock_scales")
+    return out
+
+
+def block_scales(rowmajor, dim: int) -> np.ndarray:
+    """Row-major NVFP4 scales [rows, dim/16] -> 128-row blocked key-cache layout."""
+    rowmajor = _c(rowmajor, np.uint8)
+    n_rows = rowmajor.shape[0]
+    out = np.zeros(int(_load().orc_nvfp4_blocked_bytes(n_rows, dim)), np.uint8)
+    _check(_load().orc_nvfp4_block_scales(_p(rowmajor), n_rows, dim, _p(out)), "block_scales")
+    return out
+
+
+def decode_rows(buf, dt: int, dim: int, sf=None, sf_blocked=False) -> np.ndarray:
+    """Decode rows of format dt into float64 [rows, dim] (exact).  For NVFP4,
+    sf holds the scales row-major, or in the blocked key-cache layout when
+    sf_blocked is set."""
     buf = np.ascontiguousarray(buf)
     rb = row_bytes(dt, dim)
     n_rows = buf.nbytes // rb
     out = np.empty((n_rows, dim), np.float64)
+    if sf is not None and sf_blocked:
+        sf = unblock_scales(sf, n_rows, dim)
     sf = _c(sf, np.uint8)
     _check(_load().orc_decode_rows(_p(buf), _p(sf), dt, dim, n_rows, _p(out)), "decode_rows")
     return out

@@ -230,6 +230,39 @@ static void encode_nvfp4_row(const double* x, int dim, uint8_t* codes, uint8_t* 
     }
 }
 
+/* NVFP4 key-cache scale layout: rows are taken in blocks of 128; block b
+ * holds dim/64 atoms of 512 bytes, and byte m0*16 + m1*4 + kk of atom a is the
+ * scale of row 128*b + m0 + 32*m1 for values 64*a + 16*kk .. +15 (the layout
+ * in which the tensor cores read block scales).  These two functions convert
+ * between it and the row-major [rows][dim/16] layout; dim % 64 == 0. */
+static int64_t blocked_scale_offset(int64_t r, int j, int dim) {
+    int64_t blk = r / 128;
+    int m = (int)(r % 128), m0 = m % 32, m1 = m / 32, atom = j / 4, kk = j % 4;
+    return blk * (dim / 64) * 512 + (int64_t)atom * 512 + m0 * 16 + m1 * 4 + kk;
+}
+
+int64_t orc_nvfp4_blocked_bytes(int64_t n_rows, int dim) {
+    if (dim % 64 != 0 || n_rows < 0) return -1;
+    return (n_rows + 127) / 128 * (dim / 64) * 512;
+}
+
+int orc_nvfp4_unblock_scales(const uint8_t* blocked, int64_t n_rows, int dim, uint8_t* rowmajor) {
+    if (dim % 64 != 0) return ORC_EINVAL;
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int j = 0; j < dim / 16; ++j)
+            rowmajor[r * (dim / 16) + j] = blocked[blocked_scale_offset(r, j, dim)];
+    return ORC_OK;
+}
+
+int orc_nvfp4_block_scales(const uint8_t* rowmajor, int64_t n_rows, int dim, uint8_t* blocked) {
+    if (dim % 64 != 0) return ORC_EINVAL;
+    memset(blocked, 0, (size_t)orc_nvfp4_blocked_bytes(n_rows, dim));
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int j = 0; j < dim / 16; ++j)
+            blocked[blocked_scale_offset(r, j, dim)] = rowmajor[r * (dim / 16) + j];
+    return ORC_OK;
+}
+
 int orc_decode_rows(const void* base, const void* sf, int dt, int dim, int64_t n_rows, double* out) {
     int64_t rb = orc_row_bytes(dt, dim);
     if (rb < 0) return ORC_EINVAL;

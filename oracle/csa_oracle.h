@@ -27,6 +27,9 @@ uint8_t orc_e2m1_encode(double x);
 int64_t orc_row_bytes(int dt, int dim);
 int orc_decode_rows(const void* base, const void* sf, int dt, int dim, int64_t n_rows, double* out);
 int orc_encode_rows(const double* x, int dt, int dim, int64_t n_rows, void* out, void* sf);
+int64_t orc_nvfp4_blocked_bytes(int64_t n_rows, int dim);
+int orc_nvfp4_unblock_scales(const uint8_t* blocked, int64_t n_rows, int dim, uint8_t* rowmajor);
+int orc_nvfp4_block_scales(const uint8_t* rowmajor, int64_t n_rows, int dim, uint8_t* blocked);
 
 int orc_compress(const double* Ca, const double* Cb, const double* Za, const double* Zb,
                  const double* Ba, const double* Bb, int64_t tok0, int64_t n_tok,

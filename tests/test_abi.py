@@ -24,13 +24,20 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_row_bytes():
-    assert csa.load().csa_version() == 100
+    assert csa.load().csa_version() == 200
     assert csa.row_bytes(csa.F32, 512) == 2048
     assert csa.row_bytes(csa.BF16, 512) == 1024
     assert csa.row_bytes(csa.KV_FP8MIX, 512) == 608
     assert csa.row_bytes(csa.IDX_NVFP4, 128) == 64
     assert csa.row_bytes(csa.KV_FP8MIX, 100) == -1
     assert csa.row_bytes(csa.IDX_NVFP4, 40) == -1
+    # blocked key scales: 128-row blocks of dim/64 atoms of 512 bytes
+    assert csa.nvfp4_key_scale_bytes(1, 128) == 1024
+    assert csa.nvfp4_key_scale_bytes(128, 128) == 1024
+    assert csa.nvfp4_key_scale_bytes(129, 128) == 2048
+    assert csa.nvfp4_key_scale_bytes(262144, 128) == 262144 * 8
+    assert csa.nvfp4_key_scale_bytes(0, 128) == 0
+    assert csa.nvfp4_key_scale_bytes(10, 96) == -1
 
 
 def _err():
@@ -40,13 +47,13 @@ def _err():
 def test_compress_rejects_bad_arguments():
     lib = csa.load()
     args = dict(Ca=A, Cb=A, Za=A, Zb=A, Ba=A, Bb=A, batch=1, n_tok=64, tok0=0, stride=64, e0=0, n_out=16,
-                dim=64, m=4, in_dt=csa.F32, out=A, out_sf=None, out_stride=16, out_dt=csa.F32)
+                dim=64, m=4, in_dt=csa.F32, out=A, out_sf=None, out_stride=16, out_row0=0, out_dt=csa.F32)
 
     def call(**kw):
         a = dict(args, **kw)
         return lib.csa_compress(a["Ca"], a["Cb"], a["Za"], a["Zb"], a["Ba"], a["Bb"], a["batch"], a["n_tok"],
                                 a["tok0"], a["stride"], a["e0"], a["n_out"], a["dim"], a["m"], a["in_dt"],
-                                a["out"], a["out_sf"], a["out_stride"], a["out_dt"], None)
+                                a["out"], a["out_sf"], a["out_stride"], a["out_row0"], a["out_dt"], None)
     assert call(m=0) == INVALID and "m=0" in _err()
     assert call(dim=60) == INVALID
     assert call(in_dt=csa.KV_FP8MIX) == INVALID
@@ -59,6 +66,10 @@ def test_compress_rejects_bad_arguments():
     # entry 5 with overlap needs token 16 onward; rows start at token 20
     assert call(tok0=20, e0=5, n_out=1, n_tok=44, stride=44) == INVALID
     assert call(out_stride=8) == INVALID
+    assert call(out_stride=20, out_row0=5) == INVALID and "out_row0" in _err()  # 5 + 16 rows > 20
+    assert call(out_row0=-1) == INVALID
+    assert call(out_dt=csa.IDX_NVFP4, out_sf=P(4104)) == INVALID and "aligned" in _err()
+    assert call(out_dt=csa.IDX_NVFP4, out_sf=A, dim=32, n_tok=64) == INVALID and "64" in _err()
     assert call(batch=0) == 0  # empty call is a no-op
 
 
@@ -74,6 +85,8 @@ def test_index_topk_rejects_bad_arguments():
     assert call(heads=200) == INVALID
     assert call(dt=csa.KV_FP8MIX) == INVALID
     assert call(dt=csa.IDX_NVFP4) == INVALID and "NVFP4" in _err()
+    assert call(dt=csa.IDX_NVFP4, qsf=A, ksf=A, dim=96) == INVALID and "64" in _err()
+    assert call(dt=csa.IDX_NVFP4, qsf=A, ksf=P(4104), dim=128) == INVALID and "KI_sf" in _err()
     assert lib.csa_index_topk_workspace_size(1, 4, 64, 16, 2, 32, csa.F32) >= 256
     big = lib.csa_index_topk_workspace_size(4, 1, 262144, 1024, 64, 128, csa.IDX_NVFP4)
     assert call(ws_bytes=16) == INVALID or big <= 16

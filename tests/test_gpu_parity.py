@@ -111,6 +111,18 @@ def test_compress_fp8mix_output(orc):
         assert codes_differ < 0.01, codes_differ
 
 
+def _check_nvfp4_rows(orc, codes, sf_rowmajor, want, dim):
+    """Compressor NVFP4 rows against the oracle's encoding of its own fp64 entries."""
+    dec = orc.decode_rows(codes, orc.NVFP4, dim, sf=sf_rowmajor)
+    ref_c, ref_sf = orc.encode_rows(want, orc.NVFP4)
+    ref_dec = orc.decode_rows(ref_c, orc.NVFP4, dim, sf=ref_sf)
+    s = np.repeat(np.array([[orc.e4m3_decode(int(v)) for v in row] for row in ref_sf]), 16, axis=1)
+    # at most one E2M1 step (<= 2 * scale) where fp32 and fp64 straddle a rounding boundary
+    assert (np.abs(dec - ref_dec) <= 2.0 * s * 1.13 + 1e-12).all()
+    assert (sf_rowmajor != ref_sf).mean() < 0.02
+    assert (codes != ref_c).mean() < 0.02
+
+
 def test_compress_nvfp4_output(orc):
     batch, n_tok, dim, m = 2, 4 * 64, 128, 4
     x = W.compress_inputs(W.generator(6), batch, n_tok, dim, m, True, torch.bfloat16)
@@ -118,15 +130,39 @@ def test_compress_nvfp4_output(orc):
     codes, sf = csa.compress(gx["Ca"], gx["Za"], gx["Ba"], m, gx["Cb"], gx["Zb"], gx["Bb"],
                              out_dt=csa.IDX_NVFP4)
     want = _oracle_compress(orc, x, m, 0, 0, None)
+    n = codes.shape[1]
+    assert sf.shape == (batch, csa.nvfp4_key_scale_bytes(n, dim))
     for b in range(batch):
-        dec = orc.decode_rows(raw(codes[b]), orc.NVFP4, dim, sf=raw(sf[b]))
-        ref_c, ref_sf = orc.encode_rows(want[b], orc.NVFP4)
-        ref_dec = orc.decode_rows(ref_c, orc.NVFP4, dim, sf=ref_sf)
-        s = np.repeat(np.array([[orc.e4m3_decode(int(v)) for v in row] for row in ref_sf]), 16, axis=1)
-        # at most one E2M1 step (<= 2 * scale) where fp32 and fp64 straddle a rounding boundary
-        assert (np.abs(dec - ref_dec) <= 2.0 * s * 1.13 + 1e-12).all()
-        assert (raw(sf[b]) != ref_sf).mean() < 0.02
-        assert (raw(codes[b]) != ref_c).mean() < 0.02
+        _check_nvfp4_rows(orc, raw(codes[b]), orc.unblock_scales(raw(sf[b]), n, dim), want[b], dim)
+
+
+def test_compress_nvfp4_into_cache_rows(orc):
+    """Entries written at cache rows out_row0.. of a larger cache: the blocked
+    scale bytes land in the right 128-row block and atom byte (a run that
+    crosses a block boundary), and every other byte of the cache is unchanged."""
+    batch, dim, m, E = 2, 128, 4, 300
+    e0, n_out, row0 = 37, 120, 100  # rows 100..219 straddle the 128-row block boundary
+    tok0 = m * (e0 - 1)
+    x = W.compress_inputs(W.generator(8), batch, m * (n_out + 1), dim, m, True, torch.bfloat16)
+    gx = _cuda(x)
+    codes = torch.full((batch, E, dim // 2), 0xA5, dtype=torch.uint8, device=DEV)
+    sf = torch.full((batch, csa.nvfp4_key_scale_bytes(E, dim)), 0x5A, dtype=torch.uint8, device=DEV)
+    csa.compress(gx["Ca"], gx["Za"], gx["Ba"], m, gx["Cb"], gx["Zb"], gx["Bb"], tok0=tok0, e0=e0, n_out=n_out,
+                 out_dt=csa.IDX_NVFP4, out=codes, out_sf=sf, out_row0=row0)
+    want = _oracle_compress(orc, x, m, tok0, e0, n_out)
+    for b in range(batch):
+        c = raw(codes[b])
+        s = orc.unblock_scales(raw(sf[b]), E, dim)
+        rows = slice(row0, row0 + n_out)
+        _check_nvfp4_rows(orc, c[rows], s[rows], want[b], dim)
+        others = np.ones(E, bool)
+        others[rows] = False
+        assert (c[others] == 0xA5).all() and (s[others] == 0x5A).all()
+        # bytes of the blocked array that belong to no row (past E) are untouched too
+        full = raw(sf[b])
+        mask = np.ones(full.size, bool)
+        mask[orc.block_scales(np.zeros((E, dim // 16), np.uint8) + 1, dim) == 1] = False
+        assert (full[mask] == 0x5A).all()
 
 
 # ------------------------------------------------------------- indexer + top-k
@@ -141,7 +177,7 @@ def _exact_index_inputs(B, T, H, d, E, dt, seed):
         p2 = torch.tensor([0.125, 0.25, 0.5, 1.0]).to(torch.float8_e4m3fn).view(torch.uint8)
         qsf = p2[torch.randint(0, 4, qsf.shape, generator=g)]
         ksf = p2[torch.randint(0, 4, ksf.shape, generator=g)]
-        return dict(qI=qI, qI_sf=qsf, KI=KI, KI_sf=ksf, wI=wI)
+        return dict(qI=qI, qI_sf=qsf, KI=KI, KI_sf=W.block_scales(ksf, d), wI=wI)
     tdt = torch.float32 if dt == csa.F32 else torch.bfloat16
     qI = torch.randint(-2, 3, (B, T, H, d), generator=g).to(tdt)
     KI = torch.randint(-2, 3, (B, E, d), generator=g).to(tdt)
@@ -154,7 +190,7 @@ def _decode_idx_inputs(orc, x, dt, d):
         q = orc.decode_rows(raw(x["qI"]).reshape(-1, d // 2), orc.NVFP4, d,
                             sf=raw(x["qI_sf"]).reshape(-1, d // 16)).reshape(B, T, H, d)
         E = x["KI"].shape[1]
-        K = np.stack([orc.decode_rows(raw(x["KI"][b]), orc.NVFP4, d, sf=raw(x["KI_sf"][b]))
+        K = np.stack([orc.decode_rows(raw(x["KI"][b]), orc.NVFP4, d, sf=raw(x["KI_sf"][b]), sf_blocked=True)
                       for b in range(B)]).reshape(B, E, d)
         return q, K
     return f64(x["qI"]), f64(x["KI"])
@@ -180,9 +216,11 @@ def _sorted_idx(idx):
     (csa.BF16, 64, 128, 20000, 1024, 1),    # tensor-core producer, decode slices, merge
     (csa.BF16, 64, 128, 9000, 512, 16),     # tensor-core producer, prefill-like rows
     (csa.F32, 2, 32, 64, 16, 3),
-    (csa.IDX_NVFP4, 64, 128, 2500, 512, 3),   # tensor-core producer (fp16 expansion)
-    (csa.IDX_NVFP4, 64, 128, 30000, 1024, 1),  # tensor-core producer, decode slices
-    (csa.IDX_NVFP4, 64, 128, 2501, 512, 3),   # odd entry count: SIMT producer
+    (csa.IDX_NVFP4, 64, 128, 2500, 512, 3),   # block-scaled FP4 tensor cores, 2 queries per CTA
+    (csa.IDX_NVFP4, 64, 128, 30000, 1024, 1),  # decode slices, cooperative selection
+    (csa.IDX_NVFP4, 64, 128, 30000, 1024, 2),  # 2 queries per CTA, several tiles per slice, merge
+    (csa.IDX_NVFP4, 64, 128, 2501, 512, 3),   # odd entry count: partial last scale block
+    (csa.IDX_NVFP4, 2, 64, 700, 100, 3),      # SIMT producer on blocked key scales
     (csa.BF16, 8, 64, 700, 100, 3),
 ])
 def test_index_topk_bit_exact_on_exact_scores(orc, dt, H, d, E, k, T):
@@ -213,7 +251,7 @@ def test_index_topk_random_inputs(orc, dt, H, d, E, k, T):
     if dt == csa.IDX_NVFP4:
         qI, qsf = W.nvfp4_rows(g, (B, T, H), d)
         KI, ksf = W.nvfp4_rows(g, (B, E), d)
-        x = dict(qI=qI, qI_sf=qsf, KI=KI, KI_sf=ksf)
+        x = dict(qI=qI, qI_sf=qsf, KI=KI, KI_sf=W.block_scales(ksf, d))
     else:
         tdt = torch.float32 if dt == csa.F32 else torch.bfloat16
         x = dict(qI=W.normal(g, (B, T, H, d), 1.0, tdt), KI=W.normal(g, (B, E, d), 1.0, tdt), qI_sf=None,

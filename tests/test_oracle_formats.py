@@ -151,3 +151,30 @@ def test_nvfp4_exact_roundtrip_pins_nibble_order(orc):
     x2[0, 0], x2[0, 1] = 6.0, -0.5
     c2, s2 = orc.encode_rows(x2, orc.NVFP4)
     assert c2[0, 0] == (0x7 | (0x9 << 4)) and orc.e4m3_decode(int(s2[0, 0])) == 1.0
+
+
+def test_nvfp4_blocked_key_scale_layout(orc):
+    """The key-cache scale layout (128-row blocks of 512-byte atoms; byte
+    m0*16 + m1*4 + kk of atom a = scale of block row m0 + 32*m1, values
+    64a + 16kk ..) agrees between the oracle's permutation, the workload
+    generator's torch permutation and a direct evaluation of the definition,
+    and decodes to the same values as the row-major layout."""
+    from compressed_sparse_attention_hca_b200 import workloads as W
+    rng = np.random.default_rng(5)
+    for rows, dim in [(1, 64), (127, 128), (128, 128), (300, 128), (257, 256)]:
+        sf = rng.integers(0, 256, (rows, dim // 16)).astype(np.uint8)
+        blocked = orc.block_scales(sf, dim)
+        assert blocked.size == -(-rows // 128) * (dim // 64) * 512
+        by_gen = W.block_scales(torch.from_numpy(sf), dim).numpy()
+        assert np.array_equal(blocked, by_gen)
+        for r in range(0, rows, max(1, rows // 17)):
+            for j in range(dim // 16):
+                m = r % 128
+                off = (r // 128) * (dim // 64) * 512 + (j // 4) * 512 + (m % 32) * 16 + (m // 32) * 4 + j % 4
+                assert blocked[off] == sf[r, j]
+        assert np.array_equal(orc.unblock_scales(blocked, rows, dim), sf)
+        codes = rng.integers(0, 256, (rows, dim // 2)).astype(np.uint8)
+        sf_ok = np.full_like(sf, 0x38)  # keep scales finite (E4M3 1.0) for the decode comparison
+        sf_ok[:, ::2] = 0x30
+        assert np.array_equal(orc.decode_rows(codes, orc.NVFP4, dim, sf=orc.block_scales(sf_ok, dim), sf_blocked=True),
+                              orc.decode_rows(codes, orc.NVFP4, dim, sf=sf_ok))

@@ -42,6 +42,7 @@ def _inputs(dt, B, T, E, seed):
     if dt == csa.IDX_NVFP4:
         qI, qsf = W.nvfp4_rows(g, (B, T, H), d)
         KI, ksf = W.nvfp4_rows(g, (B, E), d)
+        ksf = W.block_scales(ksf, d)
     else:
         qI, qsf = W.normal(g, (B, T, H, d), 1.0, torch.bfloat16), None
         KI, ksf = W.normal(g, (B, E, d), 1.0, torch.bfloat16), None
