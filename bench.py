@@ -8,8 +8,8 @@ Default workload: "csa_decode_1m_mixed" (4 requests x 1,048,576 tokens,
 262,144 entries each, NVFP4 indexer, FP8/BF16 KV, top-k 1024, 128 heads).
 
 Timing: W warm-up steps, then K timed steps between a barrier + synchronize.
-Before every step a 256 MiB buffer is written to flush L2 (outside the step's
-CUDA events); each step is bracketed by CUDA events on the launching stream,
+Before every step a 256 MiB buffer is written and then read to flush L2
+(outside the step's CUDA events; the read leaves no dirty lines behind); each step is bracketed by CUDA events on the launching stream,
 and the dominant kernel call (the indexer) by its own events.  Multi-GPU: one
 process per GPU, each rank runs its own independent requests (weak scaling,
 no collective on the data path); the step time is the max over ranks.
@@ -108,21 +108,20 @@ class Step:
                                                                        cfg["q_dt"], kv_dt),
                                       device=device, dtype=torch.uint8)
         self.launches = 0
+        self.side = torch.cuda.Stream(device=device)
 
-    def _compress(self):
+    def _compress_kv(self):
         csa, x, cfg, t = self.csa, self.x, self.cfg, self.tok
-        m = cfg["m"]
-        kv_dt = cfg["kv_dt"]
-        csa.compress(t["Ca"], t["Za"], t["Ba"], m, t["Cb"], t["Zb"], t["Bb"], tok0=self.tok0, e0=self.e0,
-                     n_out=self.n_out, out_dt=kv_dt, out=x["entries"], out_row0=self.e0)
-        n = csa.last_launch_count()
-        if self.kind.startswith("csa"):
-            it = self.itok
-            csa.compress(it["Ca"], it["Za"], it["Ba"], m, it["Cb"], it["Zb"], it["Bb"], tok0=self.tok0,
-                         e0=self.e0, n_out=self.n_out, out_dt=cfg["idx_dt"], out=x["KI"],
-                         out_sf=x.get("KI_sf"), out_row0=self.e0)
-            n += csa.last_launch_count()
-        return n
+        csa.compress(t["Ca"], t["Za"], t["Ba"], cfg["m"], t["Cb"], t["Zb"], t["Bb"], tok0=self.tok0, e0=self.e0,
+                     n_out=self.n_out, out_dt=cfg["kv_dt"], out=x["entries"], out_row0=self.e0)
+        return csa.last_launch_count()
+
+    def _compress_index_keys(self):
+        csa, x, cfg, it = self.csa, self.x, self.cfg, self.itok
+        csa.compress(it["Ca"], it["Za"], it["Ba"], cfg["m"], it["Cb"], it["Zb"], it["Bb"], tok0=self.tok0,
+                     e0=self.e0, n_out=self.n_out, out_dt=cfg["idx_dt"], out=x["KI"],
+                     out_sf=x.get("KI_sf"), out_row0=self.e0)
+        return csa.last_launch_count()
 
     def index(self):
         csa, x, cfg = self.csa, self.x, self.cfg
@@ -141,17 +140,31 @@ class Step:
         return csa.last_launch_count()
 
     def run(self, ev=None):
-        """One step; ev = (start, after_compress, after_index, end) CUDA events."""
+        """One step; ev = (start, after_compress, after_index, end) CUDA events.
+
+        CSA: the KV-cache compression does not feed the indexer, so it runs on
+        a side stream (a parallel branch of the step's graph) while the index
+        keys are compressed and the indexer runs; attention waits for both."""
         s = torch.cuda.current_stream()
         if ev:
             ev[0].record(s)
-        n = self._compress()
+        n = 0
+        csa_kind = self.kind.startswith("csa")
+        if csa_kind:
+            self.side.wait_stream(s)
+            with torch.cuda.stream(self.side):
+                n += self._compress_kv()
+            n += self._compress_index_keys()
+        else:
+            n += self._compress_kv()
         if ev:
             ev[1].record(s)
-        if self.kind.startswith("csa"):
+        if csa_kind:
             n += self.index()
         if ev:
             ev[2].record(s)
+        if csa_kind:
+            s.wait_stream(self.side)
         n += self.attend()
         if ev:
             ev[3].record(s)
@@ -215,6 +228,15 @@ class Step:
 
 def l2_flush_buffer(device):
     return torch.empty(256 * 1024 * 1024 // 4, device=device, dtype=torch.float32)
+
+
+def flush_l2(buf):
+    """Writes then reads a buffer twice the L2 size: the write evicts the step's
+    data, the read evicts (and writes back) the dirty lines of the write, so
+    the next step starts with a cold and clean L2 and pays no write-back that
+    belongs to the flush."""
+    buf.zero_()
+    return buf.sum()
 
 
 # ------------------------------------------------------------------- clocks
@@ -380,26 +402,41 @@ def main():
     step = Step(args.config, dev, seed_offset=rank)
     flush = l2_flush_buffer(dev)
     for _ in range(args.warmup):
-        flush.zero_()
+        flush_l2(flush)
         step.run()
     torch.cuda.synchronize()
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    # The step runs as one CUDA graph (captured once, replayed every step): a
+    # decode step is a handful of short kernels, and launching them one by one
+    # from Python leaves the GPU idle between them.  Event record nodes inside
+    # the graph time the step and its phases on the device.
+    gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step.run(gev)
+    launches_per_step = step.launches
+    for _ in range(3):
+        flush_l2(flush)
+        graph.replay()
+    torch.cuda.synchronize()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
-    launches = 0
+    evs_ms = []
     for i in range(args.steps):
-        flush.zero_()
-        step.run(evs[i])
-        launches += step.launches
+        flush_l2(flush)
+        graph.replay()
+        gev[3].synchronize()
+        evs_ms.append([gev[0].elapsed_time(gev[j]) for j in (1, 2, 3)])
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     clk = clocks.stop()
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
-    idx_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    launches = launches_per_step * args.steps
+    step_ms = [e[2] for e in evs_ms]
+    idx_ms = [e[1] - e[0] for e in evs_ms]
+    eager = measure_eager(step, args, flush)
     total_ms = sum(step_ms)
     if dist:
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
@@ -427,7 +464,7 @@ def main():
                     "frac": ach / peak, "traffic": None, "algorithmic_bytes": step.index_bytes(),
                     "avg_launch_ms": idx_avg_ms, "note": f"HBM copy peak, {peaks['source']}"}
     else:
-        att_ms = statistics.mean([e[2].elapsed_time(e[3]) for e in evs])
+        att_ms = statistics.mean([e[2] - e[1] for e in evs_ms])
         peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
         b = step.algorithmic_bytes()
         ach = b / (att_ms / 1e3) / 1e9
@@ -436,6 +473,10 @@ def main():
                 "note": f"HBM copy peak, {peaks['source']}"}
     step_bytes = step.algorithmic_bytes()
     step_gbs = step_bytes / (ms_per_step / 1e3) / 1e9
+    # mean device time of each phase of the step (same events as above)
+    phases = {"compress": statistics.mean([e[0] for e in evs_ms]),
+              "index_topk": statistics.mean(idx_ms),
+              "attention": statistics.mean([e[2] - e[1] for e in evs_ms])}
 
     # end to end through the public API with host buffers
     e2e = measure_e2e(step, args, flush, dev, dist, world)
@@ -449,10 +490,15 @@ def main():
                    "entries_per_request": x["E"], "query_tokens_per_request": x["T"],
                    "top_k": step.cfg.get("k"), "n_heads": step.cfg["n_h"], "window": step.cfg["window"],
                    "parallelism": f"replicas x{world} (independent requests per GPU)",
-                   "l2": "flushed before every step (256 MiB write outside the step events)"},
+                   "l2": "flushed before every step (256 MiB write then read, outside the step events)"},
         "roofline": roof,
         "step_hbm": {"algorithmic_bytes": step_bytes, "achieved_gbs": step_gbs,
                      "frac": step_gbs / peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])},
+        "phases_ms": phases,
+        "phases_note": ("compress = index-key compression; the KV-cache compression runs beside it and the "
+                        "indexer on a side stream" if kind.startswith("csa") else "compress = KV-cache compression"),
+        "launch": "one CUDA graph per step",
+        "eager": eager,
         "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clk,
@@ -476,30 +522,53 @@ def dtype_label(cfg):
     return ", ".join(parts) + ", fp32 accumulate"
 
 
+def measure_eager(step, args, flush):
+    """The same step launched call by call from Python (no graph): device time
+    per step and per phase, host launch gaps included."""
+    n = max(3, min(args.steps, 100))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+    for i in range(n):
+        flush_l2(flush)
+        step.run(evs[i])
+    torch.cuda.synchronize()
+    return {"ms_per_step": statistics.mean([e[0].elapsed_time(e[3]) for e in evs]),
+            "phases_ms": {"compress": statistics.mean([e[0].elapsed_time(e[1]) for e in evs]),
+                          "index_topk": statistics.mean([e[1].elapsed_time(e[2]) for e in evs]),
+                          "attention": statistics.mean([e[2].elapsed_time(e[3]) for e in evs])}}
+
+
 def measure_e2e(step, args, flush, dev, dist, world):
     """Same step through the public API with host buffers: each step copies its
-    inputs from pinned host memory and reads the output back."""
+    inputs from pinned host memory and reads the output back (all inside the
+    step's graph)."""
     ins = step.step_inputs()
     host = [t.detach().cpu().pin_memory() for t in ins]
     out_host = torch.empty(step.O.shape, dtype=step.O.dtype, pin_memory=True)
     h2d = sum(t.numel() * t.element_size() for t in host)
     d2h = out_host.numel() * out_host.element_size()
     n = max(3, min(args.steps, 100))
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
-    s = torch.cuda.current_stream()
-    for i in range(n + 2):
-        flush.zero_()
-        e = evs[i - 2] if i >= 2 else None
-        if e:
-            e[0].record(s)
+    # one graph: pinned host -> device copies of the step's inputs, the step,
+    # and the device -> host copy of its output, timed by event nodes
+    e0, e1 = (torch.cuda.Event(enable_timing=True, external=True) for _ in range(2))
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        s = torch.cuda.current_stream()
+        e0.record(s)
         for d, h in zip(ins, host):
             d.copy_(h, non_blocking=True)
         step.run()
         out_host.copy_(step.O, non_blocking=True)
-        if e:
-            e[1].record(s)
+        e1.record(s)
+    for _ in range(2):
+        flush_l2(flush)
+        graph.replay()
     torch.cuda.synchronize()
-    total = sum(a.elapsed_time(b) for a, b in evs)
+    total = 0.0
+    for i in range(n):
+        flush_l2(flush)
+        graph.replay()
+        e1.synchronize()
+        total += e0.elapsed_time(e1)
     if dist:
         t = torch.tensor([total], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)

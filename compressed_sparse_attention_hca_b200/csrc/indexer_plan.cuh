@@ -26,11 +26,12 @@ struct IndexPlan {
   int coop;           // 1: the slices of a row select together (cooperative launch), no merge
 };
 
-// Cooperative selection workspace per query row: high-byte histogram [256],
-// low-byte histogram [256], barrier counter (+pad) [8], per-slice (gt, eq)
-// counts [2 * n_slices].  Zeroed before every launch.
+// Cooperative selection workspace per query row: 12-bit key-prefix histogram
+// [4096], barrier counter (+pad) [8], per-slice slots [17 * n_slices] (keys
+// above the k-th key's prefix, suffix histogram of keys inside it).  Zeroed
+// before every launch.
 __host__ __device__ __forceinline__ int64_t plan_coop_stride(const IndexPlan& p) {
-  return (520 + 2 * (int64_t)p.n_slices + 7) / 8 * 8;
+  return (4096 + 8 + 17 * (int64_t)p.n_slices + 7) / 8 * 8;
 }
 __host__ __device__ __forceinline__ uint32_t* plan_coop_row(const IndexPlan& p, void* ws, int64_t row) {
   return static_cast<uint32_t*>(ws) + row * plan_coop_stride(p);

@@ -43,6 +43,7 @@ constexpr int kDI = 128;          // indexer dim handled here
 constexpr int kHI = 64;           // indexer heads handled here
 constexpr int kAtom = kBM * 128;  // bytes of one 128-byte-wide K atom of a bf16 K tile
 constexpr int kThreads = 384;
+constexpr int kPrefixBins = 4096;  // 12-bit key prefixes (cooperative select)
 
 __host__ __device__ constexpr int pow2_cols(int c) {
   return c <= 32 ? 32 : c <= 64 ? 64 : c <= 128 ? 128 : c <= 256 ? 256 : 512;
@@ -57,33 +58,43 @@ struct Bf16Cfg {
   static constexpr int NBUF = 512 / N;                    // 8 (NQ 1) or 4 (NQ 2)
   static_assert(NBUF % 2 == 0, "one epilogue group per buffer");
   static constexpr int TMEM_COLS = 512;
+  static constexpr int NT = kThreads;
   static constexpr int FIXED_SMEM = 1024 + STAGES * K_STAGE + Q_BYTES + NQ * kHI * 4 + 1024 /*barriers*/ +
-                                    (int)sizeof(SelectSmem<kThreads>) + 1024 /*histogram*/;
+                                    (int)sizeof(SelectSmem<NT>) + 1024 /*histogram*/;
+  static constexpr int PER_ENTRY = 2 * NQ;
   static constexpr uint32_t IDESC = idesc_bf16_f32(kBM, N);
 };
 
 template <int NQ>
 struct Nvf4Cfg {
   static constexpr int N = kHI * NQ;
-  static constexpr int STAGES = 16;
+  static constexpr int TPS = 2;                         // tiles per stage: one 16 KB code copy
+  static constexpr int STAGES = 8;
   static constexpr int CODES = kBM * kDI / 2;           // 8 KB of E2M1 per tile
   static constexpr int ATOMS = 2 * 512;                 // the tile's two scale atoms
-  static constexpr int STAGE = CODES + ATOMS;           // 9 KB (1024-aligned stages)
+  static constexpr int STAGE = TPS * (CODES + ATOMS);   // 18 KB: codes of both tiles, then their atoms
   static constexpr int QCODES = N * kDI / 2;
   static constexpr int QRAWSF = N * kDI / 16;
   static constexpr int QREG = (QCODES + QRAWSF + ATOMS + 1023) / 1024 * 1024;
-  // Even: buffer i % NBUF then always belongs to the same issuer (i % 2) and
-  // epilogue group (i % 2), so each side waits on every phase of its
-  // barriers in order (with an odd count a waiter could skip a phase and
+  // MMA issue costs a thread more time per tile than the tile's data takes to
+  // arrive, so tiles are spread over NI issuer warps (tile i -> issuer i % NI).
+  static constexpr int NI = NQ == 1 ? 4 : 2;
+  static constexpr int NT = NQ == 1 ? 448 : 384;        // + issuer warps 12, 13
+  // NBUF a multiple of NI: buffer i % NBUF then always belongs to the same
+  // issuer (i % NI) and epilogue group (i % 2), so each side waits on every
+  // phase of its barriers in order (otherwise a waiter could skip a phase and
   // take the parity of an older one for the one it wants).
-  static constexpr int NBUF = NQ == 1 ? 6 : 2;
-  static_assert(NBUF % 2 == 0, "one issuer and one epilogue group per buffer");
-  static constexpr int ACC_COLS = NBUF * N;             // 384 or 256
-  static constexpr int SFA_COL = ACC_COLS;              // 2 x 8 columns (one set per issuer)
-  static constexpr int SFB_COL = ACC_COLS + 32;         // 2 x 8 columns
+  static constexpr int NBUF = NQ == 1 ? 4 : 2;
+  static_assert(NBUF % NI == 0 && NBUF % 2 == 0, "one issuer and one epilogue group per buffer");
+  static constexpr int ACC_COLS = NBUF * N;             // 256
+  static constexpr int SFA_COL = ACC_COLS;              // NI x 8 columns (one set per issuer)
+  static constexpr int SFB_COL = ACC_COLS + 32;         // NI x 8 columns
   static constexpr int TMEM_COLS = pow2_cols(ACC_COLS + 64);
+  static constexpr int HIST = NQ == 1 ? kPrefixBins * 4 : 0;  // prefix histogram (cooperative select)
   static constexpr int FIXED_SMEM = 1024 + STAGES * STAGE + QREG + NQ * kHI * 4 + 1024 +
-                                    (int)sizeof(SelectSmem<kThreads>) + 1024;
+                                    (int)sizeof(SelectSmem<NT>) + HIST;
+  // shared memory per slice entry: NQ keys, plus a candidate position (NQ 1)
+  static constexpr int PER_ENTRY = 2 * NQ + (NQ == 1 ? 2 : 0);
   static constexpr uint32_t IDESC = idesc_nvf4(kBM, N);
 };
 
@@ -126,15 +137,10 @@ __device__ __forceinline__ SliceCtx<NQ> slice_ctx(const IndexArgs& a, const Inde
 template <int NQ, int N, int NBUF>
 __device__ __forceinline__ void epilogue_group(const SliceCtx<NQ>& c, const IndexArgs& a, const IndexPlan& plan,
                                                uint32_t tmem, uint64_t* accf, uint64_t* acce, const float* wsm,
-                                               uint16_t* keys, bool coop, uint32_t* h1s) {
+                                               uint16_t* keys, bool coop, uint32_t* hist) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quarter = warp & 3, g = (warp - 4) >> 2;
   const int r = quarter * 32 + lane;
-  float wreg[NQ == 1 ? kHI : 1];
-  if (NQ == 1) {
-#pragma unroll
-    for (int h = 0; h < kHI; ++h) wreg[h] = wsm[h];
-  }
   for (int i = g; i < c.n_tiles; i += 2) {
     const int buf = i % NBUF, u = i / NBUF;
     if (!mbar_wait(&accf[buf], u & 1)) break;
@@ -153,17 +159,23 @@ __device__ __forceinline__ void epilogue_group(const SliceCtx<NQ>& c, const Inde
     const int pos = i * kBM + r;
 #pragma unroll
     for (int q = 0; q < NQ; ++q) {
-      // four independent partial sums (heads h = 4i + j) keep the FMA pipe busy
+      // four independent partial sums (heads h = 4i + j) keep the FMA pipe
+      // busy; the weights are warp-uniform shared-memory broadcasts
       float part[4] = {0.f, 0.f, 0.f, 0.f};
+      const float4* w4 = reinterpret_cast<const float4*>(wsm + q * kHI);
 #pragma unroll
-      for (int h = 0; h < kHI; ++h)
-        part[h & 3] = fmaf(NQ == 1 ? wreg[h % (NQ == 1 ? kHI : 1)] : wsm[q * kHI + h], fmaxf(acc[q][h], 0.f),
-                           part[h & 3]);
+      for (int h4 = 0; h4 < kHI / 4; ++h4) {
+        const float4 w = w4[h4];
+        part[0] = fmaf(w.x, fmaxf(acc[q][4 * h4 + 0], 0.f), part[0]);
+        part[1] = fmaf(w.y, fmaxf(acc[q][4 * h4 + 1], 0.f), part[1]);
+        part[2] = fmaf(w.z, fmaxf(acc[q][4 * h4 + 2], 0.f), part[2]);
+        part[3] = fmaf(w.w, fmaxf(acc[q][4 * h4 + 3], 0.f), part[3]);
+      }
       const float I = (part[0] + part[1]) + (part[2] + part[3]);
       const uint32_t key = bf16_key(I);
       const bool valid = pos < c.n_valid[q];
       keys[q * plan.slice_len + pos] = valid ? (uint16_t)(key >> 16) : (uint16_t)0;
-      if (coop && valid) atomicAdd(&h1s[key >> 24], 1u);
+      if (coop && valid) atomicAdd(&hist[key >> 20], 1u);
       if (a.scores_out != nullptr && pos < c.len && c.t0 + q < a.n_q) {
         const float sc = valid ? key_to_f32(key) : -INFINITY;
         static_cast<__nv_bfloat16*>(a.scores_out)[((int64_t)c.b * a.n_q + c.t0 + q) * a.n_entries + c.s0 + pos] =
@@ -174,12 +186,12 @@ __device__ __forceinline__ void epilogue_group(const SliceCtx<NQ>& c, const Inde
 }
 
 // Debug score output (-inf) for the positions past the last computed tile.
-template <int NQ>
+template <int NQ, int NT>
 __device__ __forceinline__ void scores_tail(const SliceCtx<NQ>& c, const IndexArgs& a) {
   if (a.scores_out == nullptr) return;
   for (int q = 0; q < NQ; ++q) {
     if (c.t0 + q >= a.n_q) continue;
-    for (int pos = c.n_tiles * kBM + threadIdx.x; pos < c.len; pos += kThreads)
+    for (int pos = c.n_tiles * kBM + threadIdx.x; pos < c.len; pos += NT)
       static_cast<__nv_bfloat16*>(a.scores_out)[((int64_t)c.b * a.n_q + c.t0 + q) * a.n_entries + c.s0 + pos] =
           __float2bfloat16_rn(-INFINITY);
   }
@@ -188,9 +200,9 @@ __device__ __forceinline__ void scores_tail(const SliceCtx<NQ>& c, const IndexAr
 // Selection by one CTA over its own slice: final indices when it holds the
 // whole row, else the slice's top k as candidates (and its k-th key) for the
 // merge kernel.
-template <int NQ>
+template <int NQ, int NT>
 __device__ void slice_select(const SliceCtx<NQ>& c, const IndexArgs& a, const IndexPlan& plan, const uint16_t* keys,
-                             SelectSmem<kThreads>& sel) {
+                             SelectSmem<NT>& sel) {
   for (int q = 0; q < NQ; ++q) {
     const int t = c.t0 + q;
     if (t >= a.n_q) break;
@@ -201,14 +213,14 @@ __device__ void slice_select(const SliceCtx<NQ>& c, const IndexArgs& a, const In
     auto key_at = [&](int i) { return ((uint32_t)kq[i]) << 16; };
     if (plan.n_slices == 1) {
       int32_t* out = a.idx_out + bt * a.k;
-      block_select<kThreads>(key_at, nv, kk, 0, sel, [&](int slot, int pos) { out[slot] = (int32_t)(c.s0 + pos); });
-      for (int j = kk + threadIdx.x; j < a.k; j += kThreads) out[j] = -1;
+      block_select<NT>(key_at, nv, kk, 0, sel, [&](int slot, int pos) { out[slot] = (int32_t)(c.s0 + pos); });
+      for (int j = kk + threadIdx.x; j < a.k; j += NT) out[j] = -1;
     } else {
       const int64_t off = slice_cand_offset(plan, c.sl, c.vis[q], a.n_entries, a.k);
       uint32_t* ck = plan_cand_keys(plan, a.ws, bt) + off;
       int32_t* ci = plan_cand_idx(plan, a.ws, bt) + off;
       uint32_t T = 0;
-      block_select<kThreads>(
+      block_select<NT>(
           key_at, nv, kk, 0, sel,
           [&](int slot, int pos) {
             ck[slot] = key_at(pos);
@@ -224,30 +236,44 @@ __device__ void slice_select(const SliceCtx<NQ>& c, const IndexArgs& a, const In
 // ---------------------------------------------------------------------------
 // Cooperative selection: the slice CTAs of one query row (all resident at once,
 // cooperative launch) pick the row's top k together, with no candidate lists
-// and no merge kernel.  Keys are 16-bit (bf16 score images):
-//   1. each CTA adds the high-byte histogram of its keys (built by the
-//      epilogue) into the row's global histogram H1; barrier; every CTA finds
-//      the high byte d1 of the k-th key;
-//   2. the same for the low byte among keys whose high byte is d1 (H2); the
-//      k-th key T and the number of ties at T to take follow;
-//   3. each CTA publishes its counts of keys > T and == T; barrier; prefix
-//      sums over the slices give each CTA its output offset and its share of
-//      the ties (lowest entry indices first); it writes its winners in index
-//      order straight into the output row.
-// Barriers are global counters polled with a bounded wait (the status word
-// records a timeout).
+// and no merge kernel.  Keys are 16-bit (bf16 score images), split into a
+// 12-bit prefix (sign, exponent, 3 mantissa bits) and a 4-bit suffix:
+//   1. each CTA adds its prefix histogram (built by the epilogue) into the
+//      row's global histogram H; barrier; every CTA finds the prefix d1 of the
+//      k-th key and how many keys (rem1) it still needs inside that prefix;
+//   2. each CTA publishes, in its own slot, its count of keys with prefix > d1
+//      and its 16-bin suffix histogram of keys with prefix d1 (each word
+//      stored as value + 1, so readers poll the slots instead of a barrier);
+//   3. every CTA reads all slots and derives the k-th key T, the ties at T to
+//      take (lowest entry indices first, i.e. lowest slices first), its output
+//      offset and its share of the ties, and writes its winners in index order
+//      straight into the output row.
+// The barrier is a global counter and the slots are polled, both with a
+// bounded wait (the status word records a timeout).
+constexpr int kSlotWords = 17;  // keys with prefix > d1, then suffix counts 0..15
+
 __device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
   uint32_t v;
   asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 
+__device__ __forceinline__ uint32_t ld_relaxed_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_relaxed_gpu(uint32_t* p, uint32_t v) {
+  asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 __device__ __forceinline__ void coop_barrier(uint32_t* ctr, uint32_t target) {
-  __threadfence();  // this thread's global atomics are visible device-wide first
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    atomicAdd(ctr, 1u);
+    // release: this CTA's global writes and atomics (ordered before by the
+    // CTA barrier) are visible to every CTA that acquires the counter
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t it = 1; ld_acquire_gpu(ctr) < target; ++it) {
       if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitTimeoutNs) {
@@ -255,127 +281,196 @@ __device__ __forceinline__ void coop_barrier(uint32_t* ctr, uint32_t target) {
         break;
       }
     }
-    __threadfence();
   }
   __syncthreads();
 }
 
-// Digit d (searched from 255 down) at which the running count of a 256-bin
-// histogram reaches `remaining`; writes d and remaining - (count above d) to
-// bc[0], bc[1].  One warp.
-__device__ __forceinline__ void digit_search(const uint32_t* hist, uint32_t remaining, uint32_t* bc, int lane) {
-  uint32_t c[8], s = 0;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) { c[j] = __ldcg(hist + 255 - 8 * lane - j); s += c[j]; }
-  uint32_t inc = s;
+// Exclusive prefix sum of v over the block's NT threads (thread order);
+// *total receives the block sum.  Ends with a block barrier.
+template <int NT>
+__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* warp_tot, uint32_t* total) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t inc = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
     if (lane >= o) inc += y;
   }
-  const uint32_t exc = inc - s;
-  const bool here = exc < remaining && remaining <= inc;
-  const unsigned ballot = __ballot_sync(0xffffffffu, here);
-  if (here && lane == __ffs(ballot) - 1) {
-    uint32_t above = exc;
-    int digit = 255 - 8 * lane;
+  if (lane == 31) warp_tot[warp] = inc;
+  __syncthreads();
+  uint32_t before = 0, all = 0;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (above + c[j] >= remaining) { digit = 255 - 8 * lane - j; break; }
-      above += c[j];
-    }
-    bc[0] = (uint32_t)digit;
-    bc[1] = remaining - above;
+  for (int w = 0; w < NW; ++w) {
+    before += w < warp ? warp_tot[w] : 0u;
+    all += warp_tot[w];
   }
+  *total = all;
+  __syncthreads();
+  return before + inc - v;
 }
 
-__device__ void coop_select(const uint16_t* kq, int nv, int64_t vis, int64_t s0, int sl, const IndexPlan& plan,
-                            const IndexArgs& a, int64_t bt, const uint32_t* h1_local, SelectSmem<kThreads>& sm) {
-  constexpr int NW = kThreads / 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// kq: the slice's 16-bit keys in position order; cand: scratch for up to nv
+// positions.  Warp w scans positions [w * span, (w + 1) * span).
+template <int NT>
+__device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t vis, int64_t s0, int sl,
+                            const IndexPlan& plan, const IndexArgs& a, int64_t bt, const uint32_t* hist_local,
+                            SelectSmem<NT>& sm) {
+  constexpr int NW = NT / 32;
+  constexpr int CH = (kPrefixBins + NT - 1) / NT;  // prefix bins per thread
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tid = threadIdx.x;
+  const unsigned lt = (1u << lane) - 1u;
   const int S = plan.n_slices;
   int32_t* out = a.idx_out + bt * a.k;
   const int kk = (int)min64(a.k, vis);
   if (sl == 0)
-    for (int j = kk + threadIdx.x; j < a.k; j += kThreads) out[j] = -1;
+    for (int j = kk + tid; j < a.k; j += NT) out[j] = -1;
   if (vis <= a.k) {  // every visible entry is selected: offsets in closed form
     const int64_t off = slice_cand_offset(plan, sl, vis, a.n_entries, a.k);
-    for (int p = threadIdx.x; p < nv; p += kThreads) out[off + p] = (int32_t)(s0 + p);
+    for (int p = tid; p < nv; p += NT) out[off + p] = (int32_t)(s0 + p);
     return;
   }
   uint32_t* row = plan_coop_row(plan, a.ws, bt);
-  uint32_t* H1 = row;
-  uint32_t* H2 = row + 256;
-  uint32_t* ctr = row + 512;
-  uint32_t* gtq = row + 520;
-  // 1. high byte
-  for (int d = threadIdx.x; d < 256; d += kThreads)
-    if (h1_local[d]) atomicAdd(&H1[d], h1_local[d]);
+  uint32_t* H = row;
+  uint32_t* ctr = row + kPrefixBins;
+  uint32_t* slots = row + kPrefixBins + 8;
+  uint32_t total;
+
+  // 1. prefix histogram -> prefix d1 of the k-th key
+  for (int d = tid; d < kPrefixBins; d += NT)
+    if (hist_local[d]) atomicAdd(&H[d], hist_local[d]);
   coop_barrier(ctr, (uint32_t)S);
-  if (warp == 0) digit_search(H1, (uint32_t)kk, sm.bcast, lane);
-  for (int d = threadIdx.x; d < 256; d += kThreads) sm.hist[d] = 0;
+  // thread t owns bins hi-CH*t-1 .. hi-CH*(t+1) (descending)
+  uint32_t c[CH], sum = 0;
+#pragma unroll
+  for (int j = 0; j < CH; ++j) {
+    const int d = kPrefixBins - 1 - CH * tid - j;
+    c[j] = d >= 0 ? __ldcg(H + d) : 0u;
+    sum += c[j];
+  }
+  const uint32_t above0 = block_exclusive_scan<NT>(sum, sm.warp_tot, &total);
+  if (above0 < (uint32_t)kk && (uint32_t)kk <= above0 + sum) {
+    uint32_t above = above0;
+#pragma unroll
+    for (int j = 0; j < CH; ++j) {
+      if (above + c[j] >= (uint32_t)kk) {
+        sm.bcast[0] = (uint32_t)(kPrefixBins - 1 - CH * tid - j);
+        sm.bcast[1] = (uint32_t)kk - above;
+        break;
+      }
+      above += c[j];
+    }
+  }
+  if (tid < 32) sm.hist[tid] = 0;
   __syncthreads();
   const uint32_t d1 = sm.bcast[0], rem1 = sm.bcast[1];
-  // 2. low byte among keys with high byte d1
-  for (int p = threadIdx.x; p < nv; p += kThreads) {
-    const uint32_t k16 = kq[p];
-    if ((k16 >> 8) == d1) atomicAdd(&sm.hist[k16 & 255u], 1u);
-  }
-  __syncthreads();
-  for (int d = threadIdx.x; d < 256; d += kThreads)
-    if (sm.hist[d]) atomicAdd(&H2[d], sm.hist[d]);
-  coop_barrier(ctr, 2u * (uint32_t)S);
-  if (warp == 0) digit_search(H2, rem1, sm.bcast + 2, lane);
-  __syncthreads();
-  const uint32_t T = (d1 << 8) | sm.bcast[2];
-  const int need_eq = (int)sm.bcast[3];
-  // 3. counts, offsets, ordered write
-  const unsigned lt = (1u << lane) - 1u;
+
+  // 2. one pass over the keys: count those above prefix d1, histogram the
+  //    suffixes of those inside it, and compact the positions of both (the
+  //    only possible winners) into the warp's part of cand, in order
   const int span = ((nv + NW - 1) / NW + 31) / 32 * 32;
   const int w0 = min(nv, warp * span), w1 = min(nv, w0 + span);
-  uint32_t c_gt = 0, c_eq = 0;
+  uint32_t n_cand = 0, gt1 = 0;
   for (int base = w0; base < w1; base += 32) {
     const int p = base + lane;
     const uint32_t k16 = p < w1 ? kq[p] : 0u;
-    c_gt += __popc(__ballot_sync(0xffffffffu, p < w1 && k16 > T));
-    c_eq += __popc(__ballot_sync(0xffffffffu, p < w1 && k16 == T));
+    const uint32_t pre = k16 >> 4;
+    const bool hi = p < w1 && pre > d1, mid = p < w1 && pre == d1;
+    const unsigned cm = __ballot_sync(0xffffffffu, hi || mid);
+    if (hi || mid) cand[w0 + n_cand + __popc(cm & lt)] = (uint16_t)p;
+    if (mid) atomicAdd(&sm.hist[k16 & 15u], 1u);
+    n_cand += __popc(cm);
+    gt1 += __popc(__ballot_sync(0xffffffffu, hi));
   }
-  if (lane == 0) sm.warp_tot[warp] = c_gt;
-  __syncthreads();
-  uint32_t gt_tot = 0;
-  for (int w = 0; w < NW; ++w) gt_tot += sm.warp_tot[w];
-  __syncthreads();
-  if (lane == 0) sm.warp_tot[warp] = c_eq;
-  __syncthreads();
-  uint32_t eq_before_w = 0, eq_tot = 0;
-  for (int w = 0; w < NW; ++w) { eq_before_w += w < warp ? sm.warp_tot[w] : 0u; eq_tot += sm.warp_tot[w]; }
-  if (threadIdx.x == 0) {
-    gtq[2 * sl] = gt_tot;
-    gtq[2 * sl + 1] = eq_tot;
+  block_exclusive_scan<NT>(lane == 0 ? gt1 : 0u, sm.warp_tot, &total);
+  // slot words are stored as value + 1 into a zeroed workspace, so a reader
+  // knows a word has arrived when it is nonzero: the exchange needs no
+  // barrier, only each reader's bounded poll of the slots it reads
+  if (tid == 0) st_relaxed_gpu(slots + sl * kSlotWords, total + 1u);
+  if (tid < 16) st_relaxed_gpu(slots + sl * kSlotWords + 1 + tid, sm.hist[tid] + 1u);
+
+  // 3. every slot -> k-th key T, ties to take, this slice's offset and ties
+  uint32_t h4[16], g1 = 0;
+#pragma unroll
+  for (int n = 0; n < 16; ++n) h4[n] = 0;
+  if (tid < S) {
+    const uint32_t* sj = slots + tid * kSlotWords;
+    const unsigned long long t0 = globaltimer_ns();
+    for (uint32_t it = 1;; ++it) {
+      bool all = true;
+      g1 = ld_relaxed_gpu(sj);
+      all = all && g1 != 0u;
+#pragma unroll
+      for (int n = 0; n < 16; ++n) {
+        h4[n] = ld_relaxed_gpu(sj + 1 + n);
+        all = all && h4[n] != 0u;
+      }
+      if (all) break;
+      if ((it & 15u) == 0 && globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        atomicOr(&g_device_status, 1u);
+        break;
+      }
+    }
+    g1 = g1 - 1u;
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      h4[n] = h4[n] - 1u;
+      if (h4[n]) atomicAdd(&sm.hist[16 + n], h4[n]);
+    }
   }
-  coop_barrier(ctr, 3u * (uint32_t)S);
-  // slices before this one: winners and ties taken
-  uint32_t off = 0, eq_prev = 0;
-  for (int j = 0; j < sl; ++j) {
-    const uint32_t g = ld_acquire_gpu(&gtq[2 * j]), e = ld_acquire_gpu(&gtq[2 * j + 1]);
-    int take = need_eq - (int)eq_prev;
-    take = take < 0 ? 0 : (take > (int)e ? (int)e : take);
-    off += g + (uint32_t)take;
-    eq_prev += e;
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t above = 0;
+    for (int n = 15; n >= 0; --n) {
+      if (above + sm.hist[16 + n] >= rem1) {
+        sm.bcast[2] = (uint32_t)n;
+        sm.bcast[3] = rem1 - above;
+        break;
+      }
+      above += sm.hist[16 + n];
+    }
   }
-  int eq_take_cta = need_eq - (int)eq_prev;
-  eq_take_cta = eq_take_cta < 0 ? 0 : (eq_take_cta > (int)eq_tot ? (int)eq_tot : eq_take_cta);
+  __syncthreads();
+  const uint32_t d2 = sm.bcast[2], need_eq = sm.bcast[3];
+  const uint32_t T = (d1 << 4) | d2;
+  uint32_t gt_j = g1, eq_j = 0;
+#pragma unroll
+  for (int n = 0; n < 16; ++n) {
+    gt_j += (uint32_t)n > d2 ? h4[n] : 0u;
+    eq_j += (uint32_t)n == d2 ? h4[n] : 0u;
+  }
+  if (tid >= S) gt_j = eq_j = 0;
+  const uint32_t eq_prev = block_exclusive_scan<NT>(eq_j, sm.warp_tot, &total);
+  const uint32_t take_j = need_eq > eq_prev ? min(need_eq - eq_prev, eq_j) : 0u;
+  const uint32_t off_j = block_exclusive_scan<NT>(gt_j + take_j, sm.warp_tot, &total);
+  if (tid == sl) {
+    sm.bcast[0] = off_j;
+    sm.bcast[1] = take_j;
+  }
+  __syncthreads();
+  const uint32_t off = sm.bcast[0];
+  const int eq_take_cta = (int)sm.bcast[1];
+
+  // 4. per-warp counts over the compacted candidates, offsets, ordered write
+  const uint16_t* cw = cand + w0;
+  uint32_t c_gt = 0, c_eq = 0;
+  for (int base = 0; base < (int)n_cand; base += 32) {
+    const int j = base + lane;
+    const uint32_t k16 = j < (int)n_cand ? kq[cw[j]] : 0u;
+    c_gt += __popc(__ballot_sync(0xffffffffu, j < (int)n_cand && k16 > T));
+    c_eq += __popc(__ballot_sync(0xffffffffu, j < (int)n_cand && k16 == T));
+  }
+  const uint32_t eq_before_w =
+      __shfl_sync(0xffffffffu, block_exclusive_scan<NT>(lane == 0 ? c_eq : 0u, sm.warp_tot, &total), 0);
   int eq_take_w = eq_take_cta - (int)eq_before_w;
   eq_take_w = eq_take_w < 0 ? 0 : (eq_take_w > (int)c_eq ? (int)c_eq : eq_take_w);
-  __syncthreads();
-  if (lane == 0) sm.warp_tot[warp] = c_gt + (uint32_t)eq_take_w;
-  __syncthreads();
-  uint32_t o = off;
-  for (int w = 0; w < warp; ++w) o += sm.warp_tot[w];
+  uint32_t o = off + block_exclusive_scan<NT>(lane == 0 ? c_gt + (uint32_t)eq_take_w : 0u, sm.warp_tot, &total);
+  o = __shfl_sync(0xffffffffu, o, 0);
   int eq_seen = 0;
-  for (int base = w0; base < w1; base += 32) {
-    const int p = base + lane;
-    const bool in = p < w1;
+  for (int base = 0; base < (int)n_cand; base += 32) {
+    const int j = base + lane;
+    const bool in = j < (int)n_cand;
+    const int p = in ? cw[j] : 0;
     const uint32_t k16 = in ? kq[p] : 0u;
     const unsigned eqm = __ballot_sync(0xffffffffu, in && k16 == T);
     const bool take = in && (k16 > T || (k16 == T && eq_seen + __popc(eqm & lt) < eq_take_w));
@@ -465,10 +560,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp >= 4) {
     epilogue_group<NQ, C::N, C::NBUF>(c, a, plan, tmem, accf, acce, wsm, keys, false, nullptr);
   }
-  scores_tail<NQ>(c, a);
+  scores_tail<NQ, kThreads>(c, a);
   tc_fence_before();
   __syncthreads();
-  slice_select<NQ>(c, a, plan, keys, sel);
+  slice_select<NQ, kThreads>(c, a, plan, keys, sel);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
@@ -491,15 +586,16 @@ __device__ __forceinline__ void permute_scales(const uint8_t* raw, uint8_t* atom
 }
 
 template <int NQ>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Nvf4Cfg<NQ>::NT, 1)
     index_nvf4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                       const __grid_constant__ CUtensorMap tmQs, IndexArgs a, IndexPlan plan) {
   using C = Nvf4Cfg<NQ>;
   extern __shared__ uint8_t smem_raw[];
-  uint8_t* st = align1024(smem_raw);                          // stages: codes | scale atoms
+  uint8_t* st = align1024(smem_raw);                          // stages: codes x2 | scale atoms x2
   uint8_t* qreg = st + C::STAGES * C::STAGE;                  // q codes | q raw scales | q atoms
   uint16_t* keys = reinterpret_cast<uint16_t*>(qreg + C::QREG);
-  float* wsm = reinterpret_cast<float*>(keys + NQ * plan.slice_len);
+  uint16_t* cand = keys + NQ * plan.slice_len;                // [slice_len] candidate positions (NQ 1)
+  float* wsm = reinterpret_cast<float*>(keys + (C::PER_ENTRY / 2) * plan.slice_len);
   uint64_t* full = reinterpret_cast<uint64_t*>(wsm + NQ * kHI);
   uint64_t* empty = full + C::STAGES;
   uint64_t* accf = empty + C::STAGES;
@@ -507,19 +603,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* qbar = acce + C::NBUF;
   uint64_t* qsf = qbar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qsf + 1);
-  SelectSmem<kThreads>& sel = *reinterpret_cast<SelectSmem<kThreads>*>(tmem_slot + 4);
-  uint32_t* h1s = reinterpret_cast<uint32_t*>(&sel + 1);  // [256] high-byte histogram (cooperative select)
+  SelectSmem<C::NT>& sel = *reinterpret_cast<SelectSmem<C::NT>*>(tmem_slot + 4);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(&sel + 1);  // [kPrefixBins] (cooperative select only)
 
   const SliceCtx<NQ> c = slice_ctx<NQ>(a, plan);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool coop = NQ == 1 && plan.coop;
-  for (int i = threadIdx.x; i < NQ * kHI; i += kThreads) {
+  const int n_stages = (c.n_tiles + C::TPS - 1) / C::TPS;
+  for (int i = threadIdx.x; i < NQ * kHI; i += C::NT) {
     const int t = c.t0 + i / kHI;
     wsm[i] = t < a.n_q ? a.wI[((int64_t)c.b * a.n_q + t) * kHI + (i % kHI)] : 0.f;
   }
-  for (int i = threadIdx.x; i < 256; i += kThreads) h1s[i] = 0;
+  if (coop)
+    for (int i = threadIdx.x; i < kPrefixBins; i += C::NT) hist[i] = 0;
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    // full: one arrival from each producer (codes, scales); empty: one
+    // commit from each issuer (the stage's two tiles)
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 2); mbar_init(&empty[s], C::TPS); }
     for (int i = 0; i < C::NBUF; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 4); }
     mbar_init(qbar, 1);
     mbar_init(qsf, 1);
@@ -532,32 +632,49 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------- producer: codes, 2 tiles per copy
     if (lane == 0) {
       const int qrow = (c.b * a.n_q + c.t0) * kHI;
       mbar_arrive_expect_tx(qbar, C::QCODES + C::QRAWSF);
       tma_load_2d(qreg, &tmQ, qbar, 0, qrow);
       tma_load_2d(qreg + C::QCODES, &tmQs, qbar, 0, qrow / 2);
+      for (int g = 0; g < n_stages; ++g) {
+        const int s = g % C::STAGES, j = g / C::STAGES;
+        if (j > 0 && !mbar_wait(&empty[s], (j - 1) & 1)) break;
+        // a 256-row box: rows past the tensor read as zero, rows of the next
+        // request are never valid positions here
+        mbar_arrive_expect_tx(&full[s], C::TPS * C::CODES);
+        const int row = (int)((int64_t)c.b * a.n_entries + c.s0 + (int64_t)g * C::TPS * kBM);
+        tma_load_2d(st + s * C::STAGE, &tmK, &full[s], 0, row);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------- query scales into their atoms, then producer: key scale atoms
+    if (mbar_wait(qbar, 0)) permute_scales(qreg + C::QCODES, qreg + C::QCODES + C::QRAWSF, C::N, lane);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(qsf);
       // request b's blocked key scales: 1 KB (two atoms) per 128-entry block;
       // slices start on block boundaries, so tile i is block s0/128 + i
       const uint8_t* ksf = static_cast<const uint8_t*>(a.KI_sf) +
                            (int64_t)c.b * nvfp4_blocked_sf_bytes(a.n_entries, kDI) + (c.s0 / kBM) * C::ATOMS;
-      for (int i = 0; i < c.n_tiles; ++i) {
-        const int s = i % C::STAGES, j = i / C::STAGES;
+      for (int g = 0; g < n_stages; ++g) {
+        const int s = g % C::STAGES, j = g / C::STAGES;
         if (j > 0 && !mbar_wait(&empty[s], (j - 1) & 1)) break;
-        mbar_arrive_expect_tx(&full[s], C::CODES + C::ATOMS);
-        const int row = (int)((int64_t)c.b * a.n_entries + c.s0 + (int64_t)i * kBM);
-        uint8_t* dst = st + s * C::STAGE;
-        tma_load_2d(dst, &tmK, &full[s], 0, row);
-        bulk_load(dst + C::CODES, ksf + (int64_t)i * C::ATOMS, C::ATOMS, &full[s]);
+        const int nt = min(C::TPS, c.n_tiles - g * C::TPS);  // blocks that exist
+        mbar_arrive_expect_tx(&full[s], nt * C::ATOMS);
+        bulk_load(st + s * C::STAGE + C::TPS * C::CODES, ksf + (int64_t)g * C::TPS * C::ATOMS, nt * C::ATOMS,
+                  &full[s]);
       }
     }
-  } else if (warp == 1 || warp == 3) {
+  } else if (warp == 1 || warp == 3 || warp >= 12) {
     // ------------------------------------------------------------ MMA issuers
-    // warp 1 issues the even tiles and warp 3 the odd ones, each with its own
-    // TMEM scale columns; tcgen05.commit tracks the issuing thread's work only.
+    // issuer w (warps 1, 3, 12, 13) issues the tiles i with i % NI == w, with
+    // its own TMEM scale columns; tcgen05.commit tracks the issuing thread's
+    // work only, so each stage's empty barrier takes one commit per tile.
     if (lane == 0) {
-      const int w = warp == 1 ? 0 : 1;
+      const int w = warp == 1 ? 0 : warp == 3 ? 1 : warp - 10;
       const bool ok = mbar_wait(qsf, 0);
       const uint32_t qa = smem_u32(qreg);
       const uint32_t sfa = tmem + C::SFA_COL + 8 * w, sfb = tmem + C::SFB_COL + 8 * w;
@@ -566,40 +683,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < 2; ++kb)
           tc_cp_32x128b_warpx4(sfb + kb * 4, umma_desc_rows16(qa + C::QCODES + C::QRAWSF + kb * 512));
       }
-      for (int i = w; ok && i < c.n_tiles; i += 2) {
-        const int s = i % C::STAGES, j = i / C::STAGES, buf = i % C::NBUF, u = i / C::NBUF;
+      for (int i = w; ok && i < c.n_tiles; i += C::NI) {
+        const int g = i / C::TPS, s = g % C::STAGES, j = g / C::STAGES, buf = i % C::NBUF, u = i / C::NBUF;
         if (!mbar_wait(&full[s], j & 1)) break;
         if (u > 0 && !mbar_wait(&acce[buf], (u - 1) & 1)) break;
         tc_fence_after();
-        const uint32_t base = smem_u32(st + s * C::STAGE);
-        for (int kb = 0; kb < 2; ++kb)
-          tc_cp_32x128b_warpx4(sfa + kb * 4, umma_desc_rows16(base + C::CODES + kb * 512));
+        const int h = i % C::TPS;  // tile within the stage
+        const uint32_t codes = smem_u32(st + s * C::STAGE) + (uint32_t)(h * C::CODES);
+        const uint32_t atoms = smem_u32(st + s * C::STAGE) + (uint32_t)(C::TPS * C::CODES + h * C::ATOMS);
+        for (int kb = 0; kb < 2; ++kb) tc_cp_32x128b_warpx4(sfa + kb * 4, umma_desc_rows16(atoms + kb * 512));
         const uint32_t d = tmem + (uint32_t)(buf * C::N);
         for (int kb = 0; kb < 2; ++kb)
-          tc_mma_nvf4(d, umma_desc_sw64(base + kb * 32), umma_desc_sw64(qa + kb * 32), C::IDESC, sfa + kb * 4,
+          tc_mma_nvf4(d, umma_desc_sw64(codes + kb * 32), umma_desc_sw64(qa + kb * 32), C::IDESC, sfa + kb * 4,
                       sfb + kb * 4, kb > 0 ? 1u : 0u);
         tc_commit(&empty[s]);
         tc_commit(&accf[buf]);
       }
     }
-  } else if (warp == 2) {
-    // --------------------------------------- query scales into their atoms
-    if (mbar_wait(qbar, 0)) permute_scales(qreg + C::QCODES, qreg + C::QCODES + C::QRAWSF, C::N, lane);
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(qsf);
-  } else if (warp >= 4) {
-    epilogue_group<NQ, C::N, C::NBUF>(c, a, plan, tmem, accf, acce, wsm, keys, coop, h1s);
+  } else if (warp >= 4 && warp < 12) {
+    epilogue_group<NQ, C::N, C::NBUF>(c, a, plan, tmem, accf, acce, wsm, keys, coop, hist);
   }
-  scores_tail<NQ>(c, a);
+  scores_tail<NQ, C::NT>(c, a);
   tc_fence_before();
   __syncthreads();
   if (coop) {
-    if (c.t0 < a.n_q)
-      coop_select(keys, c.n_valid[0], c.vis[0], c.s0, c.sl, plan, a, (int64_t)c.b * a.n_q + c.t0, h1s, sel);
+    coop_select<C::NT>(keys, cand, c.n_valid[0], c.vis[0], c.s0, c.sl, plan, a, (int64_t)c.b * a.n_q + c.t0, hist,
+                       sel);
     __syncthreads();
   } else {
-    slice_select<NQ>(c, a, plan, keys, sel);
+    slice_select<NQ, C::NT>(c, a, plan, keys, sel);
   }
   if (warp == 1) {
     tc_fence_after();
@@ -660,14 +772,14 @@ cudaError_t launch_nvf4(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) 
   // packed E2M1 rows of 64 bytes in the 64-byte swizzle; query scales as
   // 16-byte lines holding two head rows each (key scales are bulk-copied)
   const bool ok =
-      make_map_2d(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.KI, krows, kDI / 2, kDI / 2, kBM,
+      make_map_2d(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.KI, krows, kDI / 2, kDI / 2, C::TPS * kBM,
                   CU_TENSOR_MAP_SWIZZLE_64B) &&
       make_map_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.qI, qrows, kDI / 2, kDI / 2, C::N,
                   CU_TENSOR_MAP_SWIZZLE_64B) &&
       make_map_2d(&tmQs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.qI_sf, qrows / 2, 16, 16, C::N / 2,
                   CU_TENSOR_MAP_SWIZZLE_NONE);
   if (!ok) return cudaErrorInvalidValue;
-  const size_t smem = (size_t)C::FIXED_SMEM + (size_t)NQ * p.slice_len * 2;
+  const size_t smem = (size_t)C::FIXED_SMEM + (size_t)C::PER_ENTRY * p.slice_len;
   cudaError_t e = cudaFuncSetAttribute(index_nvf4_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_slices, (a.n_q + NQ - 1) / NQ, a.batch);
@@ -680,11 +792,11 @@ cudaError_t launch_nvf4(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) 
     IndexPlan pp = p;
     CUtensorMap m0 = tmK, m1 = tmQ, m2 = tmQs;
     void* args[] = {&m0, &m1, &m2, &aa, &pp};
-    e = cudaLaunchCooperativeKernel((const void*)index_nvf4_kernel<NQ>, grid, dim3(kThreads), args, smem, s);
+    e = cudaLaunchCooperativeKernel((const void*)index_nvf4_kernel<NQ>, grid, dim3(C::NT), args, smem, s);
     ++launch_counter();
     return e;
   }
-  index_nvf4_kernel<NQ><<<grid, kThreads, smem, s>>>(tmK, tmQ, tmQs, a, p);
+  index_nvf4_kernel<NQ><<<grid, C::NT, smem, s>>>(tmK, tmQ, tmQs, a, p);
   ++launch_counter();
   return cudaGetLastError();
 }
@@ -708,10 +820,12 @@ bool index_tc_eligible(const IndexArgs& a) {
   if (a.n_heads != kHI || a.dim != kDI || a.n_entries <= 0) return false;
   if ((int64_t)a.batch * a.n_entries >= ((int64_t)1 << 31) || (int64_t)a.batch * a.n_q * kHI >= ((int64_t)1 << 31))
     return false;
-  if (a.dt == CSA_BF16) return true;
+  // the key tensor must be at least one TMA box high (128 rows BF16, 256 NVFP4)
+  const int64_t krows = (int64_t)a.batch * a.n_entries;
+  if (a.dt == CSA_BF16) return krows >= kBM;
   // NVFP4: key scale atoms are bulk-copied and query scales streamed as
   // 16-byte lines, so both arrays must be 16-byte aligned.
-  return a.dt == CSA_IDX_NVFP4 && aligned16(a.KI_sf) && aligned16(a.qI_sf);
+  return a.dt == CSA_IDX_NVFP4 && krows >= 2 * kBM && aligned16(a.KI_sf) && aligned16(a.qI_sf);
 }
 
 int index_tc_nq(int n_q) { return n_q >= 2 ? 2 : 1; }
@@ -721,8 +835,10 @@ IndexPlan make_tc_plan(int batch, int n_q, int64_t n_entries, int k, int dt) {
   const bool fp4 = dt == CSA_IDX_NVFP4;
   const int fixed = NQ == 1 ? (fp4 ? Nvf4Cfg<1>::FIXED_SMEM : Bf16Cfg<1>::FIXED_SMEM)
                             : (fp4 ? Nvf4Cfg<2>::FIXED_SMEM : Bf16Cfg<2>::FIXED_SMEM);
+  const int per_entry = NQ == 1 ? (fp4 ? Nvf4Cfg<1>::PER_ENTRY : Bf16Cfg<1>::PER_ENTRY)
+                                : (fp4 ? Nvf4Cfg<2>::PER_ENTRY : Bf16Cfg<2>::PER_ENTRY);
   constexpr int kSmemCap = 227 * 1024;
-  int64_t max_slice = ((kSmemCap - fixed) / (2 * NQ)) / kBM * kBM;
+  int64_t max_slice = ((kSmemCap - fixed) / per_entry) / kBM * kBM;
   const int64_t groups = (n_q + NQ - 1) / NQ;
   const int64_t units = (int64_t)batch * groups;
   const int sms = sm_count();

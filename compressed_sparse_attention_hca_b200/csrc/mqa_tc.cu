@@ -14,15 +14,17 @@
 //   O += P V (warp = 16 heads x 256 dims, 128 fp32 accumulators per thread).
 // Every row is both key and value.  Shared-memory tiles use a 16-byte-chunk
 // XOR swizzle (chunk ^ row % 8) so ldmatrix row gathers are conflict free.
-// With one split the CTA adds the sink and writes O; otherwise it writes the
-// unnormalised partial (m, l, o) for mqa_combine_kernel.
+// With one split the CTA adds the sink and writes O.  A query whose rows are
+// split over CL CTAs (decode: few queries, many rows) runs them as one thread
+// block cluster: the CTAs exchange their per-head (max, sum) through
+// distributed shared memory, each scales its partial o to its share of the
+// final output and pushes it to the CTA that owns those heads, and the owner
+// adds the CL partials in rank order and writes O.  No partial result goes
+// through global memory and no second kernel runs.
 #include "csa_internal.cuh"
 #include "mqa_plan.cuh"
 
 namespace csa {
-
-__global__ void mqa_combine_kernel(MqaArgs a, MqaPlan plan);
-
 namespace {
 
 constexpr int kDim = 512;
@@ -67,6 +69,32 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 
+// ------------------------------------------------- thread block cluster (DSMEM)
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address in CTA `rank`'s shared memory of the variable at local address `addr`.
+__device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_dsmem(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_dsmem_v2(uint32_t addr, float x, float y) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");
+}
+// All threads of all CTAs of the cluster; orders shared-memory accesses
+// (local and remote) before the barrier with those after it.
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
 template <bool FP8>
 struct MqaTcSmem {
   static constexpr int Q = kHG * kRowBytes;                 // 64 KB
@@ -76,10 +104,14 @@ struct MqaTcSmem {
   static constexpr int RAW = FP8 ? kRC * RAW_ROW : 0;       // per raw buffer
   static constexpr int P = kHG * 128;                       // 8 KB
   static constexpr int RED = 4 * kHG * 4;
-  static constexpr int TOTAL = Q + NKV * KV + 2 * RAW + P + RED + kRC * 8 + 128;
+  static constexpr int STATS = 2 * kHG * 4;                 // cluster: per-head max and sum
+  static constexpr int TOTAL = Q + NKV * KV + 2 * RAW + P + RED + kRC * 8 + STATS + 128;
+  // cluster: the receive buffer [CL sources][64 / CL heads][512] fp32 reuses
+  // the query, chunk and raw buffers once every CTA of the cluster is done
+  static_assert(Q + NKV * KV + 2 * RAW >= kHG * kDim * 4, "receive buffer fits");
 };
 
-template <bool FP8>
+template <bool FP8, int CL>
 __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(MqaArgs a, MqaPlan plan) {
   using S = MqaTcSmem<FP8>;
   extern __shared__ __align__(128) uint8_t sm[];
@@ -89,6 +121,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(MqaArgs a, MqaPlan 
   uint8_t* ps = raws + 2 * S::RAW;
   float* red = reinterpret_cast<float*>(ps + S::P);          // [2][64] max, [2][64] l
   const uint8_t** rowp = reinterpret_cast<const uint8_t**>(red + 4 * kHG);  // [64] row pointers
+  float* st_m = reinterpret_cast<float*>(rowp + kRC);        // cluster: [64] max (log2 domain)
+  float* st_l = st_m + kHG;                                   // cluster: [64] sum
 
   const int split = blockIdx.x, hg = blockIdx.y;
   const int64_t bt = blockIdx.z;
@@ -99,8 +133,10 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(MqaArgs a, MqaPlan 
 
   const int64_t tq = a.q_pos[bt];
   const RowList rl = make_row_list(a, bt, tq);
-  const int64_t r_begin = (int64_t)split * plan.rows_per_split;
-  const int64_t r_end = min64(rl.n_rows, r_begin + plan.rows_per_split);
+  // split s of CL takes chunks [s * nch / CL, (s + 1) * nch / CL) of the rows
+  const int64_t nch = (rl.n_rows + kRC - 1) / kRC;
+  const int64_t r_begin = (int64_t)split * nch / CL * kRC;
+  const int64_t r_end = min64(rl.n_rows, ((int64_t)split + 1) * nch / CL * kRC);
   const int n_chunks = r_end > r_begin ? (int)((r_end - r_begin + kRC - 1) / kRC) : 0;
   const int64_t rb = row_bytes(a.kv_dt, kDim);
 
@@ -316,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(MqaArgs a, MqaPlan 
     l_tot[h] = red[2 * kHG + head] + red[3 * kHG + head];
   }
   const int hbase = hg * kHG + hb * 16 + g;
-  if (plan.n_splits == 1) {
+  if constexpr (CL == 1) {
     float f[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -339,20 +375,71 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(MqaArgs a, MqaPlan 
       }
     }
   } else {
+    // 1. per-head (max, sum) of every CTA of the cluster
+    if (half == 0 && t4 == 0) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        st_m[hb * 16 + g + 8 * h] = m_run[h];
+        st_l[hb * 16 + g + 8 * h] = l_tot[h];
+      }
+    }
+    cluster_sync();
+    // 2. the factor that turns this CTA's partial into its share of O:
+    //    O = sum_s o_s 2^(m_s - M) / (sum_s l_s 2^(m_s - M) + 2^(sink - M))
+    float f[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      float* po = plan_partial_o(plan, a, bt, split, hbase + 8 * h);
+      const int head = hb * 16 + g + 8 * h;
+      const uint32_t am = smem_u32_generic(st_m + head), al = smem_u32_generic(st_l + head);
+      float ms[CL];
+      float M = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < CL; ++r) {
+        ms[r] = ld_dsmem(mapa_shared(am, (uint32_t)r));
+        M = fmaxf(M, ms[r]);
+      }
+      const float sink = a.sink[hbase + 8 * h] * kLog2e;
+      const float Mt = fmaxf(M, sink);
+      f[h] = 0.f;
+      if (!(sink == INFINITY) && Mt != -INFINITY) {
+        float L = exp2f(sink - Mt);
+#pragma unroll
+        for (int r = 0; r < CL; ++r)
+          if (ms[r] != -INFINITY) L += ld_dsmem(mapa_shared(al, (uint32_t)r)) * exp2f(ms[r] - Mt);
+        f[h] = m_run[h] == -INFINITY ? 0.f : exp2f(m_run[h] - Mt) / L;
+      }
+    }
+    // 3. push the scaled partial to the owner of its heads: CTA r owns heads
+    //    [r * HPC, (r + 1) * HPC) and receives [CL sources][HPC heads][512]
+    constexpr int HPC = kHG / CL;
+    float* recv = reinterpret_cast<float*>(sm);
+    const uint32_t rank = cluster_ctarank();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int head = hb * 16 + g + 8 * h;
+      const uint32_t owner = (uint32_t)(head / HPC);
+      const uint32_t dst =
+          mapa_shared(smem_u32_generic(recv + ((int)rank * HPC + head % HPC) * kDim), owner);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int d = half * 256 + j * 8 + 2 * t4;
-        *reinterpret_cast<float2*>(po + d) = make_float2(o[j][2 * h], o[j][2 * h + 1]);
+        st_dsmem_v2(dst + 4u * (uint32_t)d, o[j][2 * h] * f[h], o[j][2 * h + 1] * f[h]);
       }
-      if (half == 0 && t4 == 0) {
-        float* ml = plan_partial_ml(plan, a, bt, split, hbase + 8 * h);
-        // partials are kept in the natural-log domain for the combine kernel
-        ml[0] = m_run[h] == -INFINITY ? -INFINITY : m_run[h] / kLog2e;
-        ml[1] = l_tot[h];
+    }
+    cluster_sync();
+    // 4. add the CL partials of the owned heads in rank order and write O
+    for (int i = threadIdx.x; i < HPC * kDim / 2; i += kThreads) {
+      const int hl = i / (kDim / 2), d = 2 * (i % (kDim / 2));
+      float x = 0.f, y = 0.f;
+#pragma unroll
+      for (int r = 0; r < CL; ++r) {
+        const float2 v = *reinterpret_cast<const float2*>(recv + (r * HPC + hl) * kDim + d);
+        x += v.x;
+        y += v.y;
       }
+      __nv_bfloat16* orow =
+          static_cast<__nv_bfloat16*>(a.O) + ((bt * a.n_heads + hg * kHG + (int)rank * HPC + hl) * kDim);
+      *reinterpret_cast<__nv_bfloat162*>(orow + d) = __floats2bfloat162_rn(x, y);
     }
   }
 }
@@ -367,36 +454,53 @@ bool mqa_tc_eligible(const MqaArgs& a) {
 MqaPlan make_tc_mqa_plan(const MqaArgs& a) {
   MqaPlan p{};
   p.heads_per_cta = kHG;
-  const int64_t rows_max = max_rows_per_query(a);
+  // rows of one query are split over a cluster of CL CTAs (a power of two up
+  // to the portable cluster size 8) while the grid stays within one wave
   const int64_t units = (int64_t)a.batch * a.n_q * (a.n_heads / kHG);
-  int64_t splits = (148 + units - 1) / units;
-  const int64_t max_splits = (rows_max + kRC - 1) / kRC;
-  if (splits > max_splits) splits = max_splits;
-  if (splits < 1) splits = 1;
-  int64_t rps = (rows_max + splits - 1) / splits;
-  rps = (rps + kRC - 1) / kRC * kRC;
-  if (rps < kRC) rps = kRC;
-  p.rows_per_split = rps;
-  p.n_splits = (int)((rows_max + rps - 1) / rps);
-  if (p.n_splits < 1) p.n_splits = 1;
+  const int64_t nch = (max_rows_per_query(a) + kRC - 1) / kRC;
+  int cl = 1;
+  while (cl < 8 && units * cl * 2 <= 148 && cl * 2 <= nch) cl *= 2;
+  p.n_splits = cl;
+  p.cluster = 1;
+  p.rows_per_split = 0;
   return p;
 }
 
-cudaError_t launch_mqa_tc(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) {
-  const bool fp8 = a.kv_dt == CSA_KV_FP8MIX;
-  const size_t smem = fp8 ? MqaTcSmem<true>::TOTAL : MqaTcSmem<false>::TOTAL;
-  cudaError_t e = fp8 ? cudaFuncSetAttribute(mqa_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)
-                      : cudaFuncSetAttribute(mqa_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+template <bool FP8, int CL>
+cudaError_t launch_tc(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) {
+  const size_t smem = MqaTcSmem<FP8>::TOTAL;
+  cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel<FP8, CL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.n_splits, a.n_heads / kHG, (unsigned)((int64_t)a.batch * a.n_q));
-  if (fp8) mqa_tc_kernel<true><<<grid, kThreads, smem, s>>>(a, p);
-  else mqa_tc_kernel<false><<<grid, kThreads, smem, s>>>(a, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CL, a.n_heads / kHG, (unsigned)((int64_t)a.batch * a.n_q));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = CL > 1 ? 1 : 0;
+  e = cudaLaunchKernelEx(&cfg, mqa_tc_kernel<FP8, CL>, a, p);
   ++launch_counter();
-  e = cudaGetLastError();
-  if (e != cudaSuccess || p.n_splits == 1) return e;
-  mqa_combine_kernel<<<dim3(a.n_heads, (unsigned)((int64_t)a.batch * a.n_q)), 128, 0, s>>>(a, p);
-  ++launch_counter();
-  return cudaGetLastError();
+  return e;
+}
+
+template <bool FP8>
+cudaError_t launch_tc_fmt(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) {
+  switch (p.n_splits) {
+    case 1: return launch_tc<FP8, 1>(a, p, s);
+    case 2: return launch_tc<FP8, 2>(a, p, s);
+    case 4: return launch_tc<FP8, 4>(a, p, s);
+    case 8: return launch_tc<FP8, 8>(a, p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_mqa_tc(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) {
+  return a.kv_dt == CSA_KV_FP8MIX ? launch_tc_fmt<true>(a, p, s) : launch_tc_fmt<false>(a, p, s);
 }
 
 }  // namespace csa

@@ -1,0 +1,67 @@
+"""The decode path captured in a CUDA graph and replayed gives exactly the
+results of the same calls made one by one (GPU only).
+
+A serving loop replays one captured step per token; every launch of the path
+(the workspace memset, the cooperative indexer launch, the attention kernels)
+must therefore be capture-safe and take all its inputs from device memory.
+"""
+import pytest
+import torch
+
+from compressed_sparse_attention_hca_b200 import csa
+from compressed_sparse_attention_hca_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("idx_dt", [csa.IDX_NVFP4, csa.BF16])
+def test_graph_replay_matches_eager(idx_dt):
+    if not torch.cuda.is_available():
+        pytest.fail("needs a CUDA device")
+    B, E, k, H, dI, m = 2, 30000, 1024, 64, 128, 4
+    g = W.generator(77)
+    if idx_dt == csa.IDX_NVFP4:
+        qI, qsf = W.nvfp4_rows(g, (B, 1, H), dI)
+        KI, ksf = W.nvfp4_rows(g, (B, E), dI)
+        ksf = W.block_scales(ksf, dI)
+    else:
+        qI, qsf = W.normal(g, (B, 1, H, dI), 1.0, torch.bfloat16), None
+        KI, ksf = W.normal(g, (B, E, dI), 1.0, torch.bfloat16), None
+    wI = W.uniform(g, (B, 1, H))
+    q_pos = torch.tensor([[m * E - 1], [m * E - 777]], dtype=torch.int64)
+    n_h, c, window = 16, 512, 128
+    Q = W.normal(g, (B, 1, n_h, c), 1.0, torch.bfloat16)
+    entries = W.normal(g, (B, E, c), 1.0, torch.bfloat16)
+    win = W.normal(g, (B, window, c), 1.0, torch.bfloat16)
+    win_start = (q_pos[:, 0] - window + 1).clamp(min=0)
+    sink = W.normal(g, (n_h,), 1.0, torch.float32)
+    dev = "cuda"
+    t = {n: (v.to(dev) if v is not None else None) for n, v in dict(
+        qI=qI, qsf=qsf, KI=KI, ksf=ksf, wI=wI, q_pos=q_pos, Q=Q, entries=entries, win=win,
+        win_start=win_start, sink=sink).items()}
+    ws_i = torch.empty(csa.index_topk_workspace_size(B, 1, E, k, H, dI, idx_dt), dtype=torch.uint8, device=dev)
+    ws_a = torch.empty(csa.sparse_mqa_workspace_size(B, 1, n_h, c, k, window, csa.BF16, csa.BF16),
+                       dtype=torch.uint8, device=dev)
+    idx = torch.empty(B, 1, k, dtype=torch.int32, device=dev)
+    O = torch.empty(B, 1, n_h, c, dtype=torch.bfloat16, device=dev)
+
+    def step():
+        csa.index_topk(t["qI"], t["wI"], t["KI"], t["q_pos"], m, k, dt=idx_dt, qI_sf=t["qsf"], KI_sf=t["ksf"],
+                       idx_out=idx, ws=ws_i)
+        csa.sparse_mqa(t["Q"], t["entries"], idx, t["win"], t["win_start"], t["q_pos"], window, m, t["sink"],
+                       c ** -0.5, O=O, ws=ws_a)
+
+    step()
+    torch.cuda.synchronize()
+    idx_eager, O_eager = idx.clone(), O.clone()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    for _ in range(3):
+        idx.fill_(-7)
+        O.zero_()
+        graph.replay()
+        torch.cuda.synchronize()
+        csa.check_device_status()
+        assert torch.equal(idx, idx_eager)
+        assert torch.equal(O, O_eager)

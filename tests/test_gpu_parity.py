@@ -55,6 +55,9 @@ def _oracle_compress(orc, x, m, tok0, e0, n_out):
     (2, 128 * 5 + 17, 512, 128, False, torch.bfloat16, csa.F32, 0, 0, None),  # HCA
     (3, 8, 512, 4, True, torch.bfloat16, csa.BF16, 4 * 1000, 1001, 1),   # decode: closing block
     (1, 64, 128, 4, True, torch.float32, csa.F32, 0, 0, 16),
+    (2, 4 * 4800, 64, 4, True, torch.float32, csa.F32, 0, 0, None),  # many entries: thread per entry
+    (1, 4 * 10, 72, 4, True, torch.float32, csa.F32, 0, 0, None),    # dim not a multiple of 64
+    (2, 40 * 6, 128, 40, True, torch.bfloat16, csa.BF16, 0, 0, None),  # 2m = 80 tokens over 32 lanes
 ])
 def test_compress_matches_oracle(orc, case):
     batch, n_tok, dim, m, overlap, dtype, out_dt, tok0, e0, n_out = case
@@ -353,3 +356,13 @@ def test_mqa_sink_limits(orc):
                              sink_override=[float("inf"), float("-inf"), 30.0, -30.0])
     assert_close(got, want, atol=1e-5, what="sink limits")
     assert (got[0, :, 0] == 0).all()
+
+
+def test_mqa_sink_limits_cluster_split(orc):
+    """Sink +inf / -inf / large values on the tensor-core path whose decode
+    rows are split over a thread block cluster (per-head max and sum are
+    exchanged between the cluster's CTAs before the partials are added)."""
+    sinks = [float("inf"), float("-inf"), 30.0, -30.0] + [0.5] * 60
+    got, want, _ = _mqa_case(orc, "csa_decode_bf16", 2, 1, 4000, 512, 4 * 4000 - 1, sink_override=sinks)
+    assert_close(got, want, atol=2e-2, what="sink limits, cluster split")
+    assert (got[:, :, 0] == 0).all()
