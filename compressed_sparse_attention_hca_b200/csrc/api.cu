@@ -64,7 +64,7 @@ int csa_last_launch_count(void) { return g_launches; }
 csa_status_t csa_check_device_status(void) {
   const cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_status(e, "csa_check_device_status");
-  const unsigned int st = csa::take_status_indexer_tc();
+  const unsigned int st = csa::take_status_indexer_tc() | csa::take_status_mqa_umma();
   if (st & 2u) return fail(CSA_ERR_CUDA, "csa_check_device_status: status word unreadable");
   if (st & 1u) return fail(CSA_ERR_TIMEOUT, "a kernel pipeline wait timed out; its results are invalid");
   return ok();

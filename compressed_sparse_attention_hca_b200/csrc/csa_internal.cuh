@@ -157,6 +157,7 @@ int& launch_counter();
 // Status words of the kernels with bounded waits (read and cleared; nonzero
 // means a wait gave up, 2 means the word could not be read).
 unsigned int take_status_indexer_tc();
+unsigned int take_status_mqa_umma();
 // Records `msg` as the calling thread's last error and returns `st`.
 csa_status_t set_error(csa_status_t st, const char* msg);
 struct CompressArgs {

@@ -317,7 +317,6 @@ __device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t 
                             const IndexPlan& plan, const IndexArgs& a, int64_t bt, const uint32_t* hist_local,
                             SelectSmem<NT>& sm) {
   constexpr int NW = NT / 32;
-  constexpr int CH = (kPrefixBins + NT - 1) / NT;  // prefix bins per thread
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tid = threadIdx.x;
   const unsigned lt = (1u << lane) - 1u;
   const int S = plan.n_slices;
@@ -333,32 +332,45 @@ __device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t 
   uint32_t* row = plan_coop_row(plan, a.ws, bt);
   uint32_t* H = row;
   uint32_t* ctr = row + kPrefixBins;
+  uint32_t* Hmax = row + kPrefixBins + 1;
   uint32_t* slots = row + kPrefixBins + 8;
   uint32_t total;
 
-  // 1. prefix histogram -> prefix d1 of the k-th key
+  // 1. prefix histogram (and the row's highest prefix) -> prefix d1 of the
+  //    k-th key; warp 0 walks the bins down from the highest prefix, 32 at a
+  //    time, so only the few bins above the k-th key are read
+  uint32_t top = 0;
   for (int d = tid; d < kPrefixBins; d += NT)
-    if (hist_local[d]) atomicAdd(&H[d], hist_local[d]);
+    if (hist_local[d]) {
+      atomicAdd(&H[d], hist_local[d]);
+      top = (uint32_t)d;
+    }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) top = max(top, __shfl_xor_sync(0xffffffffu, top, o));
+  if (lane == 0 && top) atomicMax(Hmax, top);
   coop_barrier(ctr, (uint32_t)S);
-  // thread t owns bins hi-CH*t-1 .. hi-CH*(t+1) (descending)
-  uint32_t c[CH], sum = 0;
+  if (warp == 0) {
+    const int hi = (int)__ldcg(Hmax);
+    uint32_t above = 0;
+    for (int base = hi; base >= 0; base -= 32) {
+      const int d = base - lane;
+      const uint32_t c = d >= 0 ? __ldcg(H + d) : 0u;
+      uint32_t inc = c;
 #pragma unroll
-  for (int j = 0; j < CH; ++j) {
-    const int d = kPrefixBins - 1 - CH * tid - j;
-    c[j] = d >= 0 ? __ldcg(H + d) : 0u;
-    sum += c[j];
-  }
-  const uint32_t above0 = block_exclusive_scan<NT>(sum, sm.warp_tot, &total);
-  if (above0 < (uint32_t)kk && (uint32_t)kk <= above0 + sum) {
-    uint32_t above = above0;
-#pragma unroll
-    for (int j = 0; j < CH; ++j) {
-      if (above + c[j] >= (uint32_t)kk) {
-        sm.bcast[0] = (uint32_t)(kPrefixBins - 1 - CH * tid - j);
-        sm.bcast[1] = (uint32_t)kk - above;
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, above + inc >= (uint32_t)kk);
+      if (hit) {
+        const int l = __ffs(hit) - 1;
+        if (lane == l) {
+          sm.bcast[0] = (uint32_t)d;
+          sm.bcast[1] = (uint32_t)kk - (above + inc - c);
+        }
         break;
       }
-      above += c[j];
+      above += __shfl_sync(0xffffffffu, inc, 31);
     }
   }
   if (tid < 32) sm.hist[tid] = 0;
@@ -367,22 +379,42 @@ __device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t 
 
   // 2. one pass over the keys: count those above prefix d1, histogram the
   //    suffixes of those inside it, and compact the positions of both (the
-  //    only possible winners) into the warp's part of cand, in order
-  const int span = ((nv + NW - 1) / NW + 31) / 32 * 32;
+  //    only possible winners) into the warp's part of cand, in order.  A lane
+  //    reads 8 consecutive keys (16 bytes) per step.
+  const int span = ((nv + NW - 1) / NW + 255) / 256 * 256;
   const int w0 = min(nv, warp * span), w1 = min(nv, w0 + span);
   uint32_t n_cand = 0, gt1 = 0;
-  for (int base = w0; base < w1; base += 32) {
-    const int p = base + lane;
-    const uint32_t k16 = p < w1 ? kq[p] : 0u;
-    const uint32_t pre = k16 >> 4;
-    const bool hi = p < w1 && pre > d1, mid = p < w1 && pre == d1;
-    const unsigned cm = __ballot_sync(0xffffffffu, hi || mid);
-    if (hi || mid) cand[w0 + n_cand + __popc(cm & lt)] = (uint16_t)p;
-    if (mid) atomicAdd(&sm.hist[k16 & 15u], 1u);
-    n_cand += __popc(cm);
-    gt1 += __popc(__ballot_sync(0xffffffffu, hi));
+  for (int base = w0; base < w1; base += 256) {
+    const int p0 = base + 8 * lane;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (p0 < w1) v = *reinterpret_cast<const uint4*>(kq + p0);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    uint32_t cmask = 0, ngt = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t k16 = (wv[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+      const bool in = p0 + j < w1;
+      const uint32_t pre = k16 >> 4;
+      const bool hi = in && pre > d1, mid = in && pre == d1;
+      cmask |= (hi || mid) ? (1u << j) : 0u;
+      ngt += hi ? 1u : 0u;
+      if (mid) atomicAdd(&sm.hist[k16 & 15u], 1u);
+    }
+    const uint32_t cnt = __popc(cmask);
+    uint32_t inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    uint32_t at = (uint32_t)w0 + n_cand + inc - cnt;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (cmask & (1u << j)) cand[at++] = (uint16_t)(p0 + j);
+    n_cand += __shfl_sync(0xffffffffu, inc, 31);
+    gt1 += ngt;
   }
-  block_exclusive_scan<NT>(lane == 0 ? gt1 : 0u, sm.warp_tot, &total);
+  block_exclusive_scan<NT>(gt1, sm.warp_tot, &total);
   // slot words are stored as value + 1 into a zeroed workspace, so a reader
   // knows a word has arrived when it is nonzero: the exchange needs no
   // barrier, only each reader's bounded poll of the slots it reads

@@ -11,7 +11,7 @@
 // split the CTA finishes the softmax itself.
 //
 // This file holds the SIMT kernel (fp32 FMA): it serves F32 mode (1e-5
-// parity) and every shape the tensor-core kernel (mqa_tc.cu) does not take.
+// parity) and every shape the tensor-core kernel (mqa_umma.cu) does not take.
 #include "csa_internal.cuh"
 #include "mqa_plan.cuh"
 
@@ -262,18 +262,18 @@ cudaError_t launch_mqa_simt(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) 
   return cudaGetLastError();
 }
 
-bool mqa_tc_eligible(const MqaArgs& a);
-MqaPlan make_tc_mqa_plan(const MqaArgs& a);
-cudaError_t launch_mqa_tc(const MqaArgs& a, const MqaPlan& p, cudaStream_t s);
+bool mqa_umma_path(const MqaArgs& a);
+MqaPlan mqa_umma_plan(const MqaArgs& a);
+cudaError_t launch_mqa_umma(const MqaArgs& a, const MqaPlan& p, cudaStream_t s);
 
 size_t mqa_workspace(const MqaArgs& a) {
-  const MqaPlan p = mqa_tc_eligible(a) ? make_tc_mqa_plan(a) : make_simt_mqa_plan(a);
+  const MqaPlan p = mqa_umma_path(a) ? mqa_umma_plan(a) : make_simt_mqa_plan(a);
   return plan_mqa_workspace_bytes(p, a);
 }
 
 cudaError_t launch_mqa(const MqaArgs& a, cudaStream_t s) {
   if ((int64_t)a.batch * a.n_q == 0) return cudaSuccess;
-  if (mqa_tc_eligible(a)) return launch_mqa_tc(a, make_tc_mqa_plan(a), s);
+  if (mqa_umma_path(a)) return launch_mqa_umma(a, mqa_umma_plan(a), s);
   return launch_mqa_simt(a, make_simt_mqa_plan(a), s);
 }
 

@@ -11,7 +11,6 @@ struct MqaPlan {
   int heads_per_cta;
   int n_splits;
   int64_t rows_per_split;
-  int cluster;  // 1: the splits of a query reduce inside a thread block cluster (no partials)
 };
 
 // Rows attended by one query ("DeepSeek-V4 内部机制" 1.2 Step 2 and 1.4): the
@@ -66,7 +65,7 @@ __host__ __device__ __forceinline__ float* plan_partial_ml(const MqaPlan& p, con
 }
 
 inline size_t plan_mqa_workspace_bytes(const MqaPlan& p, const MqaArgs& a) {
-  if (p.n_splits <= 1 || p.cluster) return 0;
+  if (p.n_splits <= 1) return 0;
   const size_t n_bt = (size_t)a.batch * a.n_q;
   return n_bt * p.n_splits * a.n_heads * ((size_t)a.dim + 2) * 4;
 }

@@ -344,7 +344,8 @@ def test_sparse_mqa_matches_oracle(orc, cfg_name, B, T, E, k, q0):
     assert_close(got, want, atol=atol, what=cfg_name)
 
 
-@pytest.mark.parametrize("B,T,E,q0", [(2, 1, 300, 128 * 300 - 1), (1, 8, 40, 128 * 30), (1, 3, 5, 0)])
+@pytest.mark.parametrize("B,T,E,q0", [(2, 1, 300, 128 * 300 - 1), (1, 8, 40, 128 * 30), (1, 3, 5, 0),
+                                      (1, 1, 8192, 128 * 8192 - 1)])  # long rows: split over the GPU
 def test_hca_dense_mqa_matches_oracle(orc, B, T, E, q0):
     got, want, _ = _mqa_case(orc, "hca_decode_bf16", B, T, E, 0, q0, dense=True)
     assert_close(got, want, atol=2e-2, what="hca")
