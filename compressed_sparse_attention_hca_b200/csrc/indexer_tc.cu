@@ -59,9 +59,11 @@ struct Bf16Cfg {
   static_assert(NBUF % 2 == 0, "one epilogue group per buffer");
   static constexpr int TMEM_COLS = 512;
   static constexpr int NT = kThreads;
+  static constexpr int HIST = NQ == 1 ? kPrefixBins * 4 : 0;  // prefix histogram (cooperative select)
   static constexpr int FIXED_SMEM = 1024 + STAGES * K_STAGE + Q_BYTES + NQ * kHI * 4 + 1024 /*barriers*/ +
-                                    (int)sizeof(SelectSmem<NT>) + 1024 /*histogram*/;
-  static constexpr int PER_ENTRY = 2 * NQ;
+                                    (int)sizeof(SelectSmem<NT>) + HIST;
+  // shared memory per slice entry: NQ keys, plus a candidate position (NQ 1)
+  static constexpr int PER_ENTRY = 2 * NQ + (NQ == 1 ? 2 : 0);
   static constexpr uint32_t IDESC = idesc_bf16_f32(kBM, N);
 };
 
@@ -523,7 +525,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* ks = align1024(smem_raw);                        // K ring
   uint8_t* qs = ks + C::STAGES * C::K_STAGE;                // query tile
   uint16_t* keys = reinterpret_cast<uint16_t*>(qs + C::Q_BYTES);
-  float* wsm = reinterpret_cast<float*>(keys + NQ * plan.slice_len);
+  uint16_t* cand = keys + NQ * plan.slice_len;                // [slice_len] candidate positions (NQ 1)
+  float* wsm = reinterpret_cast<float*>(keys + (C::PER_ENTRY / 2) * plan.slice_len);
   uint64_t* full = reinterpret_cast<uint64_t*>(wsm + NQ * kHI);
   uint64_t* empty = full + C::STAGES;
   uint64_t* accf = empty + C::STAGES;
@@ -531,13 +534,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* qbar = acce + C::NBUF;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qbar + 1);
   SelectSmem<kThreads>& sel = *reinterpret_cast<SelectSmem<kThreads>*>(tmem_slot + 4);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(&sel + 1);  // [kPrefixBins] (cooperative select only)
 
   const SliceCtx<NQ> c = slice_ctx<NQ>(a, plan);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool coop = NQ == 1 && plan.coop;
   for (int i = threadIdx.x; i < NQ * kHI; i += kThreads) {
     const int t = c.t0 + i / kHI;
     wsm[i] = t < a.n_q ? a.wI[((int64_t)c.b * a.n_q + t) * kHI + (i % kHI)] : 0.f;
   }
+  if (coop)
+    for (int i = threadIdx.x; i < kPrefixBins; i += kThreads) hist[i] = 0;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int i = 0; i < C::NBUF; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 4); }
@@ -590,12 +597,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= 4) {
-    epilogue_group<NQ, C::N, C::NBUF>(c, a, plan, tmem, accf, acce, wsm, keys, false, nullptr);
+    epilogue_group<NQ, C::N, C::NBUF>(c, a, plan, tmem, accf, acce, wsm, keys, coop, hist);
   }
   scores_tail<NQ, kThreads>(c, a);
   tc_fence_before();
   __syncthreads();
-  slice_select<NQ, kThreads>(c, a, plan, keys, sel);
+  if (coop) {
+    coop_select<kThreads>(keys, cand, c.n_valid[0], c.vis[0], c.s0, c.sl, plan, a, (int64_t)c.b * a.n_q + c.t0, hist,
+                          sel);
+    __syncthreads();
+  } else {
+    slice_select<NQ, kThreads>(c, a, plan, keys, sel);
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
@@ -787,10 +800,23 @@ cudaError_t launch_bf16(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) 
   if (!make_map_2d(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.KI, krows, kDI, 64, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.qI, qrows, kDI, 64, C::N, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
-  const size_t smem = (size_t)C::FIXED_SMEM + (size_t)NQ * p.slice_len * 2;
+  const size_t smem = (size_t)C::FIXED_SMEM + (size_t)C::PER_ENTRY * p.slice_len;
   cudaError_t e = cudaFuncSetAttribute(index_bf16_kernel<NQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_slices, (a.n_q + NQ - 1) / NQ, a.batch);
+  if (p.coop) {
+    // the slices of a row wait on one another: zero their counters and
+    // histograms, and launch cooperatively so that every CTA is resident
+    e = cudaMemsetAsync(a.ws, 0, plan_workspace_bytes(p), s);
+    if (e != cudaSuccess) return e;
+    IndexArgs aa = a;
+    IndexPlan pp = p;
+    CUtensorMap m0 = tmK, m1 = tmQ;
+    void* args[] = {&m0, &m1, &aa, &pp};
+    e = cudaLaunchCooperativeKernel((const void*)index_bf16_kernel<NQ>, grid, dim3(kThreads), args, smem, s);
+    ++launch_counter();
+    return e;
+  }
   index_bf16_kernel<NQ><<<grid, kThreads, smem, s>>>(tmK, tmQ, a, p);
   ++launch_counter();
   return cudaGetLastError();
@@ -885,9 +911,9 @@ IndexPlan make_tc_plan(int batch, int n_q, int64_t n_entries, int k, int dt) {
   p.n_slices = (int)((n_entries + len - 1) / len);
   if (p.n_slices < 1) p.n_slices = 1;
   p.n_rows = (int64_t)batch * n_q;
-  // NVFP4 decode rows split over several slices select cooperatively when the
+  // decode rows split over several slices select cooperatively when the
   // whole grid fits on the GPU at once
-  p.coop = (fp4 && NQ == 1 && p.n_slices > 1 && units * p.n_slices <= sms) ? 1 : 0;
+  p.coop = (NQ == 1 && p.n_slices > 1 && units * p.n_slices <= sms) ? 1 : 0;
   p.cand_cap = (p.n_slices > 1 && !p.coop) ? (int64_t)p.n_slices * k : 0;
   return p;
 }
