@@ -226,6 +226,14 @@ class Step:
         return 2.0 * tot * cfg["n_hI"] * cfg["dI"]
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
+# dominant kernel, from the ncu captures summarised in profiles/
+# (ncu_index_nvf4_csa_decode_1m_mixed.md, ncu_index_bf16_csa_decode_bf16.md).  A
+# change to that kernel makes the figure stale: it is then removed until the next
+# capture.
+NCU_TRAFFIC = {"csa_decode_1m_mixed": 77_656_064, "csa_decode_bf16": 139_616_256}
+
+
 def l2_flush_buffer(device):
     return torch.empty(256 * 1024 * 1024 // 4, device=device, dtype=torch.float32)
 
@@ -461,7 +469,8 @@ def main():
             peak = peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])
             ach = step.index_bytes() / (idx_avg_ms / 1e3) / 1e9
             roof = {"kernel": "csa_index_topk", "bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
-                    "frac": ach / peak, "traffic": None, "algorithmic_bytes": step.index_bytes(),
+                    "frac": ach / peak, "traffic": NCU_TRAFFIC.get(args.config),
+                    "algorithmic_bytes": step.index_bytes(),
                     "avg_launch_ms": idx_avg_ms, "note": f"HBM copy peak, {peaks['source']}"}
     else:
         att_ms = statistics.mean([e[2] - e[1] for e in evs_ms])
