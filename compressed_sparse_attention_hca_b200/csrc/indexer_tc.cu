@@ -536,21 +536,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   SelectSmem<kThreads>& sel = *reinterpret_cast<SelectSmem<kThreads>*>(tmem_slot + 4);
   uint32_t* hist = reinterpret_cast<uint32_t*>(&sel + 1);  // [kPrefixBins] (cooperative select only)
 
-  const SliceCtx<NQ> c = slice_ctx<NQ>(a, plan);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool coop = NQ == 1 && plan.coop;
+  // The queries and the first key tiles do not depend on the query
+  // positions: the producer thread starts them before anything is loaded.
+  const int64_t s0 = (int64_t)blockIdx.x * plan.slice_len;
+  const int len0 = (int)min64(plan.slice_len, a.n_entries - s0);
+  const int pre = min(C::STAGES, (len0 + kBM - 1) / kBM);
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    for (int i = 0; i < C::NBUF; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 4); }
+    mbar_init(qbar, 1);
+    fence_barrier_init();
+    const int qrow = (blockIdx.z * a.n_q + blockIdx.y * NQ) * kHI;
+    mbar_arrive_expect_tx(qbar, C::Q_BYTES);
+    tma_load_2d(qs, &tmQ, qbar, 0, qrow);
+    tma_load_2d(qs + C::N * 128, &tmQ, qbar, 64, qrow);
+    for (int i = 0; i < pre; ++i) {
+      mbar_arrive_expect_tx(&full[i], C::K_STAGE);
+      const int row = (int)((int64_t)blockIdx.z * a.n_entries + s0 + (int64_t)i * kBM);
+      tma_load_2d(ks + i * C::K_STAGE, &tmK, &full[i], 0, row);
+      tma_load_2d(ks + i * C::K_STAGE + kAtom, &tmK, &full[i], 64, row);
+    }
+  }
+  const SliceCtx<NQ> c = slice_ctx<NQ>(a, plan);
   for (int i = threadIdx.x; i < NQ * kHI; i += kThreads) {
     const int t = c.t0 + i / kHI;
     wsm[i] = t < a.n_q ? a.wI[((int64_t)c.b * a.n_q + t) * kHI + (i % kHI)] : 0.f;
   }
   if (coop)
     for (int i = threadIdx.x; i < kPrefixBins; i += kThreads) hist[i] = 0;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
-    for (int i = 0; i < C::NBUF; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 4); }
-    mbar_init(qbar, 1);
-    fence_barrier_init();
-  }
   if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
@@ -559,12 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     if (lane == 0) {
-      tma_prefetch_desc(&tmK);
-      const int qrow = (c.b * a.n_q + c.t0) * kHI;
-      mbar_arrive_expect_tx(qbar, C::Q_BYTES);
-      tma_load_2d(qs, &tmQ, qbar, 0, qrow);
-      tma_load_2d(qs + C::N * 128, &tmQ, qbar, 64, qrow);
-      for (int i = 0; i < c.n_tiles; ++i) {
+      for (int i = pre; i < c.n_tiles; ++i) {
         const int s = i % C::STAGES, j = i / C::STAGES;
         if (j > 0 && !mbar_wait(&empty[s], (j - 1) & 1)) break;
         mbar_arrive_expect_tx(&full[s], C::K_STAGE);
@@ -573,6 +583,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_load_2d(dst, &tmK, &full[s], 0, row);
         tma_load_2d(dst + kAtom, &tmK, &full[s], 64, row);
       }
+      // tiles started early but beyond the visible entries: wait for their
+      // bytes before the CTA moves on
+      for (int i = c.n_tiles; i < pre; ++i) mbar_wait(&full[i], 0);
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -651,16 +664,14 @@ __global__ void __launch_bounds__(Nvf4Cfg<NQ>::NT, 1)
   SelectSmem<C::NT>& sel = *reinterpret_cast<SelectSmem<C::NT>*>(tmem_slot + 4);
   uint32_t* hist = reinterpret_cast<uint32_t*>(&sel + 1);  // [kPrefixBins] (cooperative select only)
 
-  const SliceCtx<NQ> c = slice_ctx<NQ>(a, plan);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool coop = NQ == 1 && plan.coop;
-  const int n_stages = (c.n_tiles + C::TPS - 1) / C::TPS;
-  for (int i = threadIdx.x; i < NQ * kHI; i += C::NT) {
-    const int t = c.t0 + i / kHI;
-    wsm[i] = t < a.n_q ? a.wI[((int64_t)c.b * a.n_q + t) * kHI + (i % kHI)] : 0.f;
-  }
-  if (coop)
-    for (int i = threadIdx.x; i < kPrefixBins; i += C::NT) hist[i] = 0;
+  // The queries and the first stages of key codes do not depend on the query
+  // positions: the producer thread starts them before anything is loaded.
+  const int64_t s0 = (int64_t)blockIdx.x * plan.slice_len;
+  const int len0 = (int)min64(plan.slice_len, a.n_entries - s0);
+  const int pre = min(C::STAGES, ((len0 + kBM - 1) / kBM + C::TPS - 1) / C::TPS);
+  const int b0 = blockIdx.z, t00 = blockIdx.y * NQ;
   if (threadIdx.x == 0) {
     // full: one arrival from each producer (codes, scales); empty: one
     // commit from each issuer (the stage's two tiles)
@@ -669,7 +680,25 @@ __global__ void __launch_bounds__(Nvf4Cfg<NQ>::NT, 1)
     mbar_init(qbar, 1);
     mbar_init(qsf, 1);
     fence_barrier_init();
+    const int qrow = (b0 * a.n_q + t00) * kHI;
+    mbar_arrive_expect_tx(qbar, C::QCODES + C::QRAWSF);
+    tma_load_2d(qreg, &tmQ, qbar, 0, qrow);
+    tma_load_2d(qreg + C::QCODES, &tmQs, qbar, 0, qrow / 2);
+    for (int g = 0; g < pre; ++g) {
+      // a 256-row box: rows past the tensor read as zero, rows of the next
+      // request are never valid positions here
+      mbar_arrive_expect_tx(&full[g], C::TPS * C::CODES);
+      tma_load_2d(st + g * C::STAGE, &tmK, &full[g], 0, (int)((int64_t)b0 * a.n_entries + s0 + (int64_t)g * C::TPS * kBM));
+    }
   }
+  const SliceCtx<NQ> c = slice_ctx<NQ>(a, plan);
+  const int n_stages = (c.n_tiles + C::TPS - 1) / C::TPS;
+  for (int i = threadIdx.x; i < NQ * kHI; i += C::NT) {
+    const int t = c.t0 + i / kHI;
+    wsm[i] = t < a.n_q ? a.wI[((int64_t)c.b * a.n_q + t) * kHI + (i % kHI)] : 0.f;
+  }
+  if (coop)
+    for (int i = threadIdx.x; i < kPrefixBins; i += C::NT) hist[i] = 0;
   if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
@@ -679,18 +708,18 @@ __global__ void __launch_bounds__(Nvf4Cfg<NQ>::NT, 1)
   if (warp == 0) {
     // ------------------------------------------- producer: codes, 2 tiles per copy
     if (lane == 0) {
-      const int qrow = (c.b * a.n_q + c.t0) * kHI;
-      mbar_arrive_expect_tx(qbar, C::QCODES + C::QRAWSF);
-      tma_load_2d(qreg, &tmQ, qbar, 0, qrow);
-      tma_load_2d(qreg + C::QCODES, &tmQs, qbar, 0, qrow / 2);
-      for (int g = 0; g < n_stages; ++g) {
+      for (int g = pre; g < n_stages; ++g) {
         const int s = g % C::STAGES, j = g / C::STAGES;
         if (j > 0 && !mbar_wait(&empty[s], (j - 1) & 1)) break;
-        // a 256-row box: rows past the tensor read as zero, rows of the next
-        // request are never valid positions here
         mbar_arrive_expect_tx(&full[s], C::TPS * C::CODES);
         const int row = (int)((int64_t)c.b * a.n_entries + c.s0 + (int64_t)g * C::TPS * kBM);
         tma_load_2d(st + s * C::STAGE, &tmK, &full[s], 0, row);
+      }
+      // stages started early but beyond the visible entries: add the missing
+      // scale-side arrival and wait for their bytes before the CTA moves on
+      for (int g = n_stages; g < pre; ++g) {
+        mbar_arrive(&full[g]);
+        mbar_wait(&full[g], 0);
       }
     }
   } else if (warp == 2) {

@@ -15,8 +15,9 @@
 //       B = P written by the softmax threads MN-major (a line = the 64 heads
 //       of one row); D = four 128-dim slabs in TMEM (lane = dim).
 // The softmax runs on the 128 threads that own the TMEM lanes: thread r holds
-// row r's 64 scores; per-head maxima and sums across rows are warp
-// reduce-scatters (each lane ends with two heads) combined over four warps.
+// row r's 64 scores; per-head maxima across rows are warp max-reductions
+// (redux.sync) and per-head sums warp reduce-scatters (each lane ends with
+// two heads), both combined over four warps.
 // The running maximum is only raised when a chunk exceeds it by more than
 // 2^8, so O^T is rescaled in TMEM rarely (never within one chunk).
 // FP8MIX rows are expanded to bf16 (value = e4m3 * block scale; RoPE dims
@@ -97,11 +98,17 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// Maximum over the warp's 32 lanes, returned to every lane (sm_100a).
+__device__ __forceinline__ float warp_max_f32(float v) {
+  float r;
+  asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
+  return r;
+}
 // Barrier of the 128 softmax threads (warps 0-3).
 __device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 // Warp reduce-scatter of 64 per-lane values (one per head): afterwards lane l
-// holds the reduction over the warp's 32 lanes for heads 2l and 2l+1.
+// holds the sum (or max) over the warp's 32 lanes for heads 2l and 2l+1.
 template <bool MAX>
 __device__ __forceinline__ void reduce_scatter64(float* v, int lane, float& r0, float& r1) {
 #pragma unroll
@@ -277,13 +284,12 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
       const bool ok = ms.rowp[tid] != nullptr;
 #pragma unroll
       for (int h = 0; h < kHG; ++h) s[h] = ok ? s[h] * sl2 : -INFINITY;
-      float v[kHG];
+      // per-head maximum over the warp's 32 rows (one redux per head)
 #pragma unroll
-      for (int h = 0; h < kHG; ++h) v[h] = s[h];
-      float c0, c1;
-      reduce_scatter64<true>(v, lane, c0, c1);
-      ms.red[warp][2 * lane] = c0;
-      ms.red[warp][2 * lane + 1] = c1;
+      for (int h = 0; h < kHG; ++h) {
+        const float wm = warp_max_f32(s[h]);
+        if (lane == (h >> 1)) ms.red[warp][h] = wm;
+      }
       softmax_sync();
       if (warp == 0) {
         bool raised = false;
@@ -319,6 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
         *reinterpret_cast<uint4*>(Ps + tid * 128 + ((c ^ (tid & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
       }
       // row sums per head of the bf16 probabilities the product will use
+      float v[kHG], c0, c1;
 #pragma unroll
       for (int h = 0; h < kHG; ++h) v[h] = __bfloat162float(__float2bfloat16_rn(s[h]));
       reduce_scatter64<false>(v, lane, c0, c1);
