@@ -140,13 +140,14 @@ class Step:
         return csa.last_launch_count()
 
     def run(self, ev=None):
-        """One step; ev = (start, after_compress, after_index, end) CUDA events.
+        """One step; ev = (start, after_compress, after_index, end) CUDA events
+        (any of them may be None).
 
         CSA: the KV-cache compression does not feed the indexer, so it runs on
         a side stream (a parallel branch of the step's graph) while the index
         keys are compressed and the indexer runs; attention waits for both."""
         s = torch.cuda.current_stream()
-        if ev:
+        if ev and ev[0] is not None:
             ev[0].record(s)
         n = 0
         csa_kind = self.kind.startswith("csa")
@@ -157,16 +158,16 @@ class Step:
             n += self._compress_index_keys()
         else:
             n += self._compress_kv()
-        if ev:
+        if ev and ev[1] is not None:
             ev[1].record(s)
         if csa_kind:
             n += self.index()
-        if ev:
+        if ev and ev[2] is not None:
             ev[2].record(s)
         if csa_kind:
             s.wait_stream(self.side)
         n += self.attend()
-        if ev:
+        if ev and ev[3] is not None:
             ev[3].record(s)
         self.launches = n
 
@@ -421,28 +422,40 @@ def main():
     gev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        step.run(gev)
+        step.run((gev[0], None, None, gev[3]))
     launches_per_step = step.launches
+    # a second graph with event nodes between the phases times the phases
+    pev = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+    pgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(pgraph):
+        step.run(pev)
     for _ in range(3):
         flush_l2(flush)
         graph.replay()
+        flush_l2(flush)
+        pgraph.replay()
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
-    evs_ms = []
+    step_ms = []
     for i in range(args.steps):
         flush_l2(flush)
         graph.replay()
         gev[3].synchronize()
-        evs_ms.append([gev[0].elapsed_time(gev[j]) for j in (1, 2, 3)])
+        step_ms.append(gev[0].elapsed_time(gev[3]))
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     clk = clocks.stop()
+    evs_ms = []
+    for i in range(min(args.steps, 100)):
+        flush_l2(flush)
+        pgraph.replay()
+        pev[3].synchronize()
+        evs_ms.append([pev[0].elapsed_time(pev[j]) for j in (1, 2, 3)])
     launches = launches_per_step * args.steps
-    step_ms = [e[2] for e in evs_ms]
     idx_ms = [e[1] - e[0] for e in evs_ms]
     eager = measure_eager(step, args, flush)
     total_ms = sum(step_ms)
