@@ -62,8 +62,9 @@ struct Bf16Cfg {
   static constexpr int HIST = NQ == 1 ? kPrefixBins * 4 : 0;  // prefix histogram (cooperative select)
   static constexpr int FIXED_SMEM = 1024 + STAGES * K_STAGE + Q_BYTES + NQ * kHI * 4 + 1024 /*barriers*/ +
                                     (int)sizeof(SelectSmem<NT>) + HIST;
-  // shared memory per slice entry: NQ keys, plus a candidate position (NQ 1)
-  static constexpr int PER_ENTRY = 2 * NQ + (NQ == 1 ? 2 : 0);
+  // shared memory per slice entry: NQ keys (the cooperative select's
+  // candidate list reuses the K ring, idle by then)
+  static constexpr int PER_ENTRY = 2 * NQ;
   static constexpr uint32_t IDESC = idesc_bf16_f32(kBM, N);
 };
 
@@ -71,7 +72,7 @@ template <int NQ>
 struct Nvf4Cfg {
   static constexpr int N = kHI * NQ;
   static constexpr int TPS = 2;                         // tiles per stage: one 16 KB code copy
-  static constexpr int STAGES = 8;
+  static constexpr int STAGES = NQ == 1 ? 9 : 8;
   static constexpr int CODES = kBM * kDI / 2;           // 8 KB of E2M1 per tile
   static constexpr int ATOMS = 2 * 512;                 // the tile's two scale atoms
   static constexpr int STAGE = TPS * (CODES + ATOMS);   // 18 KB: codes of both tiles, then their atoms
@@ -95,8 +96,9 @@ struct Nvf4Cfg {
   static constexpr int HIST = NQ == 1 ? kPrefixBins * 4 : 0;  // prefix histogram (cooperative select)
   static constexpr int FIXED_SMEM = 1024 + STAGES * STAGE + QREG + NQ * kHI * 4 + 1024 +
                                     (int)sizeof(SelectSmem<NT>) + HIST;
-  // shared memory per slice entry: NQ keys, plus a candidate position (NQ 1)
-  static constexpr int PER_ENTRY = 2 * NQ + (NQ == 1 ? 2 : 0);
+  // shared memory per slice entry: NQ keys (the cooperative select's
+  // candidate list reuses the stage ring, idle by then)
+  static constexpr int PER_ENTRY = 2 * NQ;
   static constexpr uint32_t IDESC = idesc_nvf4(kBM, N);
 };
 
@@ -525,8 +527,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* ks = align1024(smem_raw);                        // K ring
   uint8_t* qs = ks + C::STAGES * C::K_STAGE;                // query tile
   uint16_t* keys = reinterpret_cast<uint16_t*>(qs + C::Q_BYTES);
-  uint16_t* cand = keys + NQ * plan.slice_len;                // [slice_len] candidate positions (NQ 1)
-  float* wsm = reinterpret_cast<float*>(keys + (C::PER_ENTRY / 2) * plan.slice_len);
+  uint16_t* cand = reinterpret_cast<uint16_t*>(ks);          // [slice_len] candidates, on the idle ring
+  float* wsm = reinterpret_cast<float*>(keys + NQ * plan.slice_len);
   uint64_t* full = reinterpret_cast<uint64_t*>(wsm + NQ * kHI);
   uint64_t* empty = full + C::STAGES;
   uint64_t* accf = empty + C::STAGES;
@@ -652,8 +654,8 @@ __global__ void __launch_bounds__(Nvf4Cfg<NQ>::NT, 1)
   uint8_t* st = align1024(smem_raw);                          // stages: codes x2 | scale atoms x2
   uint8_t* qreg = st + C::STAGES * C::STAGE;                  // q codes | q raw scales | q atoms
   uint16_t* keys = reinterpret_cast<uint16_t*>(qreg + C::QREG);
-  uint16_t* cand = keys + NQ * plan.slice_len;                // [slice_len] candidate positions (NQ 1)
-  float* wsm = reinterpret_cast<float*>(keys + (C::PER_ENTRY / 2) * plan.slice_len);
+  uint16_t* cand = reinterpret_cast<uint16_t*>(st);          // [slice_len] candidates, on the idle ring
+  float* wsm = reinterpret_cast<float*>(keys + NQ * plan.slice_len);
   uint64_t* full = reinterpret_cast<uint64_t*>(wsm + NQ * kHI);
   uint64_t* empty = full + C::STAGES;
   uint64_t* accf = empty + C::STAGES;
@@ -926,6 +928,10 @@ IndexPlan make_tc_plan(int batch, int n_q, int64_t n_entries, int k, int dt) {
                                 : (fp4 ? Nvf4Cfg<2>::PER_ENTRY : Bf16Cfg<2>::PER_ENTRY);
   constexpr int kSmemCap = 227 * 1024;
   int64_t max_slice = ((kSmemCap - fixed) / per_entry) / kBM * kBM;
+  // the cooperative select keeps a 16-bit candidate per entry on the stage ring
+  const int64_t ring = NQ == 1 ? (fp4 ? Nvf4Cfg<1>::STAGES * Nvf4Cfg<1>::STAGE : Bf16Cfg<1>::STAGES * Bf16Cfg<1>::K_STAGE)
+                               : (int64_t)1 << 40;
+  if (max_slice > ring / 2 / kBM * kBM) max_slice = ring / 2 / kBM * kBM;
   const int64_t groups = (n_q + NQ - 1) / NQ;
   const int64_t units = (int64_t)batch * groups;
   const int sms = sm_count();
