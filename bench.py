@@ -98,7 +98,7 @@ class Step:
         if overlap:
             idt = cfg["idx_dt"]
             H = cfg["n_hI"]
-            self.ws_idx = torch.empty(csa.index_topk_workspace_size(B, T, E, cfg["k"], H, cfg["dI"], idt),
+            self.ws_idx = torch.zeros(csa.index_topk_workspace_size(B, T, E, cfg["k"], H, cfg["dI"], idt),
                                       device=device, dtype=torch.uint8)
             self.ws_mqa = torch.empty(csa.sparse_mqa_workspace_size(B, T, cfg["n_h"], c, cfg["k"],
                                                                     cfg["window"], cfg["q_dt"], kv_dt),

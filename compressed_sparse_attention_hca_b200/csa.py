@@ -176,7 +176,7 @@ def index_topk(qI, wI, KI, q_pos, m, k, *, dt=None, qI_sf=None, KI_sf=None, n_he
         sc = torch.empty(B, T, E, device=dev, dtype=torch.float32 if dt == F32 else torch.bfloat16)
     need = index_topk_workspace_size(B, T, E, k, H, dim, dt)
     if ws is None or ws.numel() < need:
-        ws = torch.empty(need, device=dev, dtype=torch.uint8)
+        ws = torch.zeros(need, device=dev, dtype=torch.uint8)  # zero before first use
     _check(load().csa_index_topk(_ptr(qI), _ptr(qI_sf), _ptr(wI), _ptr(KI), _ptr(KI_sf), _ptr(q_pos),
                                  B, T, E, m, H, dim, k, dt, _ptr(idx_out), _ptr(sc), _ptr(ws),
                                  ws.numel(), _stream()))

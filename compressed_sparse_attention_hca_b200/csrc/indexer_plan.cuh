@@ -27,9 +27,9 @@ struct IndexPlan {
 };
 
 // Cooperative selection workspace per query row: 12-bit key-prefix histogram
-// [4096], barrier counter (+pad) [8], per-slice slots [17 * n_slices] (keys
-// above the k-th key's prefix, suffix histogram of keys inside it).  Zeroed
-// before every launch.
+// [4096], counters (+pad) [8], per-slice slots [17 * n_slices] (keys above
+// the k-th key's prefix, suffix histogram of keys inside it).  It must be zero
+// before the first call; every call leaves it at zero.
 __host__ __device__ __forceinline__ int64_t plan_coop_stride(const IndexPlan& p) {
   return (4096 + 8 + 17 * (int64_t)p.n_slices + 7) / 8 * 8;
 }

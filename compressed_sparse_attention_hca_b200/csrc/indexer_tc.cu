@@ -335,7 +335,7 @@ __device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t 
   }
   uint32_t* row = plan_coop_row(plan, a.ws, bt);
   uint32_t* H = row;
-  uint32_t* ctr = row + kPrefixBins;
+  uint32_t* ctr = row + kPrefixBins;       // [0] barrier, [1] highest prefix, [2] completions
   uint32_t* Hmax = row + kPrefixBins + 1;
   uint32_t* slots = row + kPrefixBins + 8;
   uint32_t total;
@@ -452,6 +452,22 @@ __device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t 
     for (int n = 0; n < 16; ++n) {
       h4[n] = h4[n] - 1u;
       if (h4[n]) atomicAdd(&sm.hist[16 + n], h4[n]);
+    }
+  }
+  __syncthreads();
+  // Every slot has arrived, so every CTA of the row is past step 1: the
+  // workspace goes back to zeros for the next call.  This CTA clears its
+  // share of the prefix histogram; the last CTA to get here (all others have
+  // read every slot by then) clears the slots and the counters.
+  for (int d = sl * kPrefixBins / S + tid; d < (sl + 1) * kPrefixBins / S; d += NT) H[d] = 0u;
+  if (tid == 0) sm.bcast[2] = atomicAdd(ctr + 2, 1u) == (uint32_t)S - 1 ? 1u : 0u;
+  __syncthreads();
+  if (sm.bcast[2]) {
+    for (int i = tid; i < S * kSlotWords; i += NT) slots[i] = 0u;
+    if (tid == 0) {
+      ctr[0] = 0u;
+      ctr[1] = 0u;  // the row's highest prefix
+      ctr[2] = 0u;
     }
   }
   __syncthreads();
@@ -836,10 +852,9 @@ cudaError_t launch_bf16(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) 
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_slices, (a.n_q + NQ - 1) / NQ, a.batch);
   if (p.coop) {
-    // the slices of a row wait on one another: zero their counters and
-    // histograms, and launch cooperatively so that every CTA is resident
-    e = cudaMemsetAsync(a.ws, 0, plan_workspace_bytes(p), s);
-    if (e != cudaSuccess) return e;
+    // the slices of a row wait on one another: launch cooperatively so that
+    // every CTA is resident (their counters and histograms start at zero and
+    // the kernel leaves them at zero)
     IndexArgs aa = a;
     IndexPlan pp = p;
     CUtensorMap m0 = tmK, m1 = tmQ;
@@ -873,10 +888,9 @@ cudaError_t launch_nvf4(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) 
   if (e != cudaSuccess) return e;
   dim3 grid(p.n_slices, (a.n_q + NQ - 1) / NQ, a.batch);
   if (p.coop) {
-    // the slices of a row wait on one another: zero their counters and
-    // histograms, and launch cooperatively so that every CTA is resident
-    e = cudaMemsetAsync(a.ws, 0, plan_workspace_bytes(p), s);
-    if (e != cudaSuccess) return e;
+    // the slices of a row wait on one another: launch cooperatively so that
+    // every CTA is resident (their counters and histograms start at zero and
+    // the kernel leaves them at zero)
     IndexArgs aa = a;
     IndexPlan pp = p;
     CUtensorMap m0 = tmK, m1 = tmQ, m2 = tmQs;

@@ -19,7 +19,9 @@
 // array, which keeps whatever the previous call left in it: calls that can
 // overlap on the GPU (different streams, or different host threads) race on
 // it and must be serialised by the caller.  The indexer writes every scratch
-// byte it later reads, so nothing needs to start at zero.
+// byte it later reads, except the cooperative selection's counters and
+// histograms, which must start at zero: the array is zero at load time
+// (static initialisation) and every call leaves them at zero.
 #include <stdio.h>
 
 #include <mutex>

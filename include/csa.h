@@ -174,6 +174,11 @@ csa_status_t csa_compress(const void* Ca, const void* Cb, const void* Za, const 
  *   dt        CSA_F32, CSA_BF16 or CSA_IDX_NVFP4 (qI and KI share it).
  * Limits: 1 <= k <= 2048, dim a multiple of 32 (<= 256; NVFP4: of 64),
  * n_heads <= 128.
+ * Workspace: ws must be zero-filled before its first use with this call
+ * (e.g. one cudaMemset after allocation); every call leaves it zero-filled
+ * again, because decode rows split over several CTAs select together through
+ * counters and histograms kept there.  After CSA_ERR_TIMEOUT from
+ * csa_check_device_status, zero it again.
  */
 size_t csa_index_topk_workspace_size(int batch, int n_q, int64_t n_entries, int k, int n_heads,
                                      int dim, csa_dtype_t dt);
@@ -200,8 +205,9 @@ csa_status_t csa_index_topk(const void* qI, const void* qI_sf, const float* wI, 
  *     array's device address; make that first call before any stream capture.
  *   - All calls on a device share the one array and it keeps the previous
  *     call's contents; calls that may overlap on the GPU (other streams or
- *     host threads) race on it, so serialise them.  Nothing in it needs to
- *     start at zero.
+ *     host threads) race on it, so serialise them.  It starts at zero (static
+ *     initialisation) and every call leaves it at zero, as csa_index_topk
+ *     requires of its workspace.
  */
 csa_status_t csa_index_topk_noalloc(const void* qI, const void* qI_sf, const float* wI,
                                     const void* KI, const void* KI_sf, const int64_t* q_pos,

@@ -39,7 +39,7 @@ def test_graph_replay_matches_eager(idx_dt):
     t = {n: (v.to(dev) if v is not None else None) for n, v in dict(
         qI=qI, qsf=qsf, KI=KI, ksf=ksf, wI=wI, q_pos=q_pos, Q=Q, entries=entries, win=win,
         win_start=win_start, sink=sink).items()}
-    ws_i = torch.empty(csa.index_topk_workspace_size(B, 1, E, k, H, dI, idx_dt), dtype=torch.uint8, device=dev)
+    ws_i = torch.zeros(csa.index_topk_workspace_size(B, 1, E, k, H, dI, idx_dt), dtype=torch.uint8, device=dev)
     ws_a = torch.empty(csa.sparse_mqa_workspace_size(B, 1, n_h, c, k, window, csa.BF16, csa.BF16),
                        dtype=torch.uint8, device=dev)
     idx = torch.empty(B, 1, k, dtype=torch.int32, device=dev)
@@ -65,3 +65,33 @@ def test_graph_replay_matches_eager(idx_dt):
         csa.check_device_status()
         assert torch.equal(idx, idx_eager)
         assert torch.equal(O, O_eager)
+
+
+@pytest.mark.parametrize("idx_dt", [csa.IDX_NVFP4, csa.BF16])
+def test_index_workspace_returns_to_zero(idx_dt):
+    """Decode rows split over several CTAs select through counters and
+    histograms in the workspace; every call must leave it zero-filled so the
+    next call (or graph replay) can use it without clearing it."""
+    if not torch.cuda.is_available():
+        pytest.fail("needs a CUDA device")
+    B, E, k, H, dI, m = 3, 40000, 1024, 64, 128, 4
+    g = W.generator(91)
+    if idx_dt == csa.IDX_NVFP4:
+        qI, qsf = W.nvfp4_rows(g, (B, 1, H), dI)
+        KI, ksf = W.nvfp4_rows(g, (B, E), dI)
+        ksf = W.block_scales(ksf, dI)
+    else:
+        qI, qsf = W.normal(g, (B, 1, H, dI), 1.0, torch.bfloat16), None
+        KI, ksf = W.normal(g, (B, E, dI), 1.0, torch.bfloat16), None
+    wI = W.uniform(g, (B, 1, H))
+    q_pos = torch.tensor([[m * E - 1], [m * E - 1001], [m * 3000]], dtype=torch.int64)
+    cuda = lambda v: None if v is None else v.cuda()  # noqa: E731
+    ws = torch.zeros(csa.index_topk_workspace_size(B, 1, E, k, H, dI, idx_dt), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(3):
+        outs.append(csa.index_topk(cuda(qI), cuda(wI), cuda(KI), cuda(q_pos), m, k, dt=idx_dt, qI_sf=cuda(qsf),
+                                   KI_sf=cuda(ksf), ws=ws))
+        torch.cuda.synchronize()
+        csa.check_device_status()
+        assert int(ws.count_nonzero()) == 0
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
