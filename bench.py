@@ -75,14 +75,16 @@ class Step:
         # newest tokens: the block closed by the last query token (decode), or
         # every new token of the chunk (prefill)
         if self.kind == "csa_prefill":
+            # the chunk's blocks, plus the block before it (overlap) when there is one
             n_new = T
-            self.tok0 = x["q0"] - m
             self.e0 = x["q0"] // m
+            self.tok0 = max(0, x["q0"] - m)
+            rows = n_new + (x["q0"] - self.tok0)
         else:
             n_new = m
             self.tok0 = E * m - (2 * m if self.kind.startswith("csa") else m)
             self.e0 = E - 1
-        rows = n_new + (m if self.kind.startswith("csa") else 0)
+            rows = n_new + (m if self.kind.startswith("csa") else 0)
         overlap = self.kind.startswith("csa")
         self.n_out = n_new // m if self.kind == "csa_prefill" else 1
         self.tok = W.compress_inputs(g, B, rows, c, m, overlap, torch.bfloat16, c_std=cfg["kv_std"],
@@ -235,6 +237,20 @@ class Step:
 NCU_TRAFFIC = {"csa_decode_1m_mixed": 77_656_064, "csa_decode_bf16": 139_616_256}
 
 
+def max_over_ranks(x, dist, device):
+    """The largest x of all ranks (the job's time is its slowest rank's)."""
+    if not dist:
+        return float(x)
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(world, units_per_rank_step, ms_per_step):
+    """Whole-job throughput: every rank processes its own units each step."""
+    return world * units_per_rank_step / (ms_per_step / 1e3)
+
+
 def l2_flush_buffer(device):
     return torch.empty(256 * 1024 * 1024 // 4, device=device, dtype=torch.float32)
 
@@ -259,10 +275,18 @@ class ClockSampler:
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         try:
             self.p = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                       "-lms", "50", "-i", str(gpu_index)], stdout=self.f,
+                                       "-lms", "20", "-i", str(gpu_index)], stdout=self.f,
                                       stderr=subprocess.DEVNULL)
         except OSError:
             self.p = None
+        # nvidia-smi takes a moment to start: wait for its first sample so the
+        # samples cover the timed region
+        t0 = time.time()
+        while self.p is not None and time.time() - t0 < 5.0:
+            self.f.flush()
+            if os.path.getsize(self.f.name) > 0:
+                break
+            time.sleep(0.02)
 
     def stop(self):
         if self.p is None:
@@ -382,7 +406,7 @@ def reference_arm(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--config", default="csa_decode_1m_mixed", choices=sorted(W.CONFIGS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
@@ -458,15 +482,11 @@ def main():
     launches = launches_per_step * args.steps
     idx_ms = [e[1] - e[0] for e in evs_ms]
     eager = measure_eager(step, args, flush)
-    total_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, dev)
     ms_per_step = total_ms / args.steps
     x = step.x
     tokens_per_step = x["B"] * x["T"]
-    value = world * tokens_per_step / (ms_per_step / 1e3)
+    value = job_throughput(world, tokens_per_step, ms_per_step)
 
     # dominant kernel roofline
     kind = step.kind
@@ -591,13 +611,10 @@ def measure_e2e(step, args, flush, dev, dist, world):
         graph.replay()
         e1.synchronize()
         total += e0.elapsed_time(e1)
-    if dist:
-        t = torch.tensor([total], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total = float(t.item())
+    total = max_over_ranks(total, dist, dev)
     ms = total / n
     x = step.x
-    return {"value": world * x["B"] * x["T"] / (ms / 1e3), "unit": "query-tokens/s",
+    return {"value": job_throughput(world, x["B"] * x["T"], ms), "unit": "query-tokens/s",
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms}
 
 

@@ -277,7 +277,8 @@ __global__ void __launch_bounds__(256) compress_tokpar_kernel(CompressArgs a) {
   if (threadIdx.x < 64) {
     const int ch = threadIdx.x;
     float mx = st[0][0][ch], den = st[1][0][ch], acc = st[2][0][ch];
-    for (int l = 1; l < kTokLanes; ++l) merge_state(mx, den, acc, st[0][l][ch], st[1][l][ch], st[2][l][ch]);
+    const int used = U < kTokLanes ? U : kTokLanes;  // lanes that saw a token
+    for (int l = 1; l < used; ++l) merge_state(mx, den, acc, st[0][l][ch], st[1][l][ch], st[2][l][ch]);
     xs[ch] = den > 0.f ? acc / den : 0.f;
   }
   __syncthreads();
