@@ -110,25 +110,11 @@ class Step:
                                                                        cfg["q_dt"], kv_dt),
                                       device=device, dtype=torch.uint8)
         self.launches = 0
-        self.side = torch.cuda.Stream(device=device)
 
     def _compress_kv(self):
         csa, x, cfg, t = self.csa, self.x, self.cfg, self.tok
         csa.compress(t["Ca"], t["Za"], t["Ba"], cfg["m"], t["Cb"], t["Zb"], t["Bb"], tok0=self.tok0, e0=self.e0,
                      n_out=self.n_out, out_dt=cfg["kv_dt"], out=x["entries"], out_row0=self.e0)
-        return csa.last_launch_count()
-
-    def _compress_index_keys(self):
-        csa, x, cfg, it = self.csa, self.x, self.cfg, self.itok
-        csa.compress(it["Ca"], it["Za"], it["Ba"], cfg["m"], it["Cb"], it["Zb"], it["Bb"], tok0=self.tok0,
-                     e0=self.e0, n_out=self.n_out, out_dt=cfg["idx_dt"], out=x["KI"],
-                     out_sf=x.get("KI_sf"), out_row0=self.e0)
-        return csa.last_launch_count()
-
-    def index(self):
-        csa, x, cfg = self.csa, self.x, self.cfg
-        csa.index_topk(x["qI"], x["wI"], x["KI"], x["q_pos"], cfg["m"], cfg["k"], dt=cfg["idx_dt"],
-                       qI_sf=x.get("qI_sf"), KI_sf=x.get("KI_sf"), idx_out=self.idx, ws=self.ws_idx)
         return csa.last_launch_count()
 
     def attend(self):
@@ -141,33 +127,41 @@ class Step:
                               cfg["m"], x["sink"], self.scale, kv_dt=cfg["kv_dt"], O=self.O, ws=self.ws_mqa)
         return csa.last_launch_count()
 
+    def compress_index(self):
+        """The step's compressions (index key and KV entry) fused with the
+        indexer call: one launch on the tensor-core path."""
+        csa, x, cfg, it, t = self.csa, self.x, self.cfg, self.itok, self.tok
+        m = cfg["m"]
+        keys = csa.compress_job(it["Ca"], it["Za"], it["Ba"], m, it["Cb"], it["Zb"], it["Bb"], tok0=self.tok0,
+                                e0=self.e0, n_out=self.n_out, out=x["KI"], out_sf=x.get("KI_sf"),
+                                out_dt=cfg["idx_dt"])
+        kv = csa.compress_job(t["Ca"], t["Za"], t["Ba"], m, t["Cb"], t["Zb"], t["Bb"], tok0=self.tok0, e0=self.e0,
+                              n_out=self.n_out, out=x["entries"], out_dt=cfg["kv_dt"])
+        csa.compress_index_topk(keys, x["qI"], x["wI"], x["KI"], x["q_pos"], m, cfg["k"], extra_job=kv,
+                                dt=cfg["idx_dt"], qI_sf=x.get("qI_sf"), KI_sf=x.get("KI_sf"), idx_out=self.idx,
+                                ws=self.ws_idx)
+        return csa.last_launch_count()
+
     def run(self, ev=None):
         """One step; ev = (start, after_compress, after_index, end) CUDA events
         (any of them may be None).
 
-        CSA: the KV-cache compression does not feed the indexer, so it runs on
-        a side stream (a parallel branch of the step's graph) while the index
-        keys are compressed and the indexer runs; attention waits for both."""
+        CSA: both compressions (index key, KV entry) run inside the indexer
+        call, then attention.  HCA: KV-cache compression, then dense
+        attention."""
         s = torch.cuda.current_stream()
         if ev and ev[0] is not None:
             ev[0].record(s)
         n = 0
         csa_kind = self.kind.startswith("csa")
-        if csa_kind:
-            self.side.wait_stream(s)
-            with torch.cuda.stream(self.side):
-                n += self._compress_kv()
-            n += self._compress_index_keys()
-        else:
+        if not csa_kind:
             n += self._compress_kv()
         if ev and ev[1] is not None:
             ev[1].record(s)
         if csa_kind:
-            n += self.index()
+            n += self.compress_index()
         if ev and ev[2] is not None:
             ev[2].record(s)
-        if csa_kind:
-            s.wait_stream(self.side)
         n += self.attend()
         if ev and ev[3] is not None:
             ev[3].record(s)
@@ -234,7 +228,7 @@ class Step:
 # (ncu_index_nvf4_csa_decode_1m_mixed.md, ncu_index_bf16_csa_decode_bf16.md).  A
 # change to that kernel makes the figure stale: it is then removed until the next
 # capture.
-NCU_TRAFFIC = {"csa_decode_1m_mixed": 77_656_064, "csa_decode_bf16": 139_616_256}
+NCU_TRAFFIC = {}
 
 
 def max_over_ranks(x, dist, device):
@@ -537,8 +531,10 @@ def main():
         "step_hbm": {"algorithmic_bytes": step_bytes, "achieved_gbs": step_gbs,
                      "frac": step_gbs / peaks.get("hbm_gbs", PEAKS_FALLBACK["hbm_gbs"])},
         "phases_ms": phases,
-        "phases_note": ("compress = index-key compression; the KV-cache compression runs beside it and the "
-                        "indexer on a side stream" if kind.startswith("csa") else "compress = KV-cache compression"),
+        "phases_note": ("index_topk includes both compressions (index key and KV entry, fused into the "
+                        "indexer call), so the compress phase is empty" if kind.startswith("csa")
+                        else "compress = KV-cache compression"),
+        "phases_timing": "a second graph with event nodes between the phases (each node adds latency)",
         "launch": "one CUDA graph per step",
         "eager": eager,
         "e2e": e2e,

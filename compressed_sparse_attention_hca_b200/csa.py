@@ -56,6 +56,9 @@ def load():
         "csa_compress": (i32, [P, P, P, P, P, P, i32, i64, i64, i64, i64, i64, i32, i32, i32, P, P,
                                i64, i64, i32, P]),
         "csa_index_topk_workspace_size": (sz, [i32, i32, i64, i32, i32, i32, i32]),
+        "csa_compress_index_topk": (i32, [ctypes.POINTER(CompressJob), ctypes.POINTER(CompressJob),
+                                          P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32, i32,
+                                          P, P, P, sz, P]),
         "csa_index_topk": (i32, [P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32, i32, P, P, P,
                                  sz, P]),
         "csa_sparse_mqa_workspace_size": (sz, [i32, i32, i32, i32, i32, i32, i32, i32]),
@@ -181,6 +184,57 @@ def index_topk(qI, wI, KI, q_pos, m, k, *, dt=None, qI_sf=None, KI_sf=None, n_he
                                  B, T, E, m, H, dim, k, dt, _ptr(idx_out), _ptr(sc), _ptr(ws),
                                  ws.numel(), _stream()))
     return (idx_out, sc) if scores else idx_out
+
+
+class CompressJob(ctypes.Structure):
+    """csa_compress_job_t: one compressor call's arguments (see compress())."""
+    _fields_ = [("Ca", ctypes.c_void_p), ("Cb", ctypes.c_void_p), ("Za", ctypes.c_void_p), ("Zb", ctypes.c_void_p),
+                ("Ba", ctypes.c_void_p), ("Bb", ctypes.c_void_p), ("n_tok", ctypes.c_int64),
+                ("tok0", ctypes.c_int64), ("in_batch_stride", ctypes.c_int64), ("e0", ctypes.c_int64),
+                ("n_out", ctypes.c_int64), ("dim", ctypes.c_int32), ("m", ctypes.c_int32), ("in_dt", ctypes.c_int32),
+                ("out", ctypes.c_void_p), ("out_sf", ctypes.c_void_p), ("out_batch_stride", ctypes.c_int64),
+                ("out_row0", ctypes.c_int64), ("out_dt", ctypes.c_int32)]
+
+
+def compress_job(Ca, Za, Ba, m, Cb=None, Zb=None, Bb=None, *, tok0, e0, n_out, out, out_dt, out_sf=None,
+                 out_row0=None, n_tok=None):
+    """A compressor call's arguments as a CompressJob (entries e0.. written to
+    rows out_row0.. of `out`, out_row0 defaulting to e0)."""
+    _need_cuda(Ca, Za, Ba, Cb, Zb, Bb, out, out_sf)
+    batch, rows, dim = Ca.shape
+    job = CompressJob(
+        Ca=Ca.data_ptr(), Cb=Cb.data_ptr() if Cb is not None else None, Za=Za.data_ptr(),
+        Zb=Zb.data_ptr() if Zb is not None else None, Ba=Ba.data_ptr(), Bb=Bb.data_ptr() if Bb is not None else None,
+        n_tok=rows if n_tok is None else n_tok, tok0=tok0, in_batch_stride=rows, e0=e0, n_out=n_out, dim=dim, m=m,
+        in_dt=_dt_of(Ca), out=out.data_ptr(), out_sf=out_sf.data_ptr() if out_sf is not None else None,
+        out_batch_stride=out.shape[1], out_row0=e0 if out_row0 is None else out_row0, out_dt=out_dt)
+    return job
+
+
+def compress_index_topk(keys_job, qI, wI, KI, q_pos, m, k, *, extra_job=None, dt=None, qI_sf=None, KI_sf=None,
+                        idx_out=None, ws=None):
+    """Run the compressor job `keys_job` (index keys into KI / KI_sf) and, if
+    given, `extra_job` (e.g. the KV cache), then index + top-k over KI: one
+    launch when the tensor-core indexer takes the shape.  Returns idx
+    [B, T, k] int32."""
+    _need_cuda(qI, wI, KI, q_pos, qI_sf, KI_sf)
+    if dt is None:
+        dt = IDX_NVFP4 if qI.dtype == torch.uint8 else _dt_of(qI)
+    B, T, H = wI.shape
+    E = KI.shape[1]
+    dim = qI.shape[-1] * (2 if dt == IDX_NVFP4 else 1)
+    dev = qI.device
+    if idx_out is None:
+        idx_out = torch.empty(B, T, k, device=dev, dtype=torch.int32)
+    need = index_topk_workspace_size(B, T, E, k, H, dim, dt)
+    if ws is None or ws.numel() < need:
+        ws = torch.zeros(need, device=dev, dtype=torch.uint8)  # zero before first use
+    _check(load().csa_compress_index_topk(ctypes.byref(keys_job),
+                                          ctypes.byref(extra_job) if extra_job is not None else None,
+                                          _ptr(qI), _ptr(qI_sf), _ptr(wI), _ptr(KI), _ptr(KI_sf), _ptr(q_pos), B, T,
+                                          E, m, H, dim, k, dt, _ptr(idx_out), None, _ptr(ws), ws.numel(),
+                                          _stream()))
+    return idx_out
 
 
 # -------------------------------------------------------------------- attention

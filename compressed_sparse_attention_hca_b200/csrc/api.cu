@@ -55,6 +55,96 @@ int& csa::launch_counter() { return g_launches; }
 
 csa_status_t csa::set_error(csa_status_t st, const char* msg) { return fail(st, "%s", msg); }
 
+// Validates a compressor call on the host; fills *args, or sets *empty when
+// there is nothing to do.
+static csa_status_t check_compress(const void* Ca, const void* Cb, const void* Za, const void* Zb,
+                                   const float* Ba, const float* Bb, int batch, int64_t n_tok, int64_t tok0,
+                                   int64_t in_batch_stride, int64_t e0, int64_t n_out, int dim, int m,
+                                   csa_dtype_t in_dt, void* out, void* out_sf, int64_t out_batch_stride,
+                                   int64_t out_row0, csa_dtype_t out_dt, csa::CompressArgs* args, bool* empty) {
+  *empty = false;
+  REQUIRE(batch >= 0 && n_tok >= 0 && tok0 >= 0 && e0 >= 0 && n_out >= 0 && out_row0 >= 0,
+          "negative size (batch=%d n_tok=%lld tok0=%lld e0=%lld n_out=%lld out_row0=%lld)", batch,
+          (long long)n_tok, (long long)tok0, (long long)e0, (long long)n_out, (long long)out_row0);
+  REQUIRE(m >= 1 && m <= 4096, "m=%d out of range [1, 4096]", m);
+  REQUIRE(dim >= 8 && dim % 8 == 0, "dim=%d must be a positive multiple of 8", dim);
+  REQUIRE(in_dt == CSA_F32 || in_dt == CSA_BF16, "in_dt must be CSA_F32 or CSA_BF16");
+  REQUIRE(out_dt >= CSA_F32 && out_dt <= CSA_IDX_NVFP4, "unknown out_dt %d", (int)out_dt);
+  if (out_dt == CSA_KV_FP8MIX)
+    REQUIRE(dim >= 128 && (dim - 64) % 64 == 0, "KV_FP8MIX needs dim = 64 + 64*j (j >= 1), got %d", dim);
+  if (out_dt == CSA_IDX_NVFP4) REQUIRE(dim % 64 == 0, "NVFP4 output needs dim %% 64 == 0, got %d", dim);
+  REQUIRE(in_batch_stride >= n_tok, "in_batch_stride %lld < n_tok %lld", (long long)in_batch_stride,
+          (long long)n_tok);
+  REQUIRE(out_batch_stride >= out_row0 + n_out, "out_batch_stride %lld < out_row0 %lld + n_out %lld",
+          (long long)out_batch_stride, (long long)out_row0, (long long)n_out);
+  if ((int64_t)batch * n_out == 0) {
+    *empty = true;
+    return ok();
+  }
+  REQUIRE_PTR(Ca);
+  REQUIRE_PTR(Za);
+  REQUIRE_PTR(Ba);
+  REQUIRE_PTR(out);
+  const bool overlap = Cb != nullptr;
+  if (overlap) {
+    REQUIRE_PTR(Zb);
+    REQUIRE_PTR(Bb);
+    REQUIRE_ALIGNED_OR_NULL(Cb);
+  }
+  if (out_dt == CSA_IDX_NVFP4) {
+    REQUIRE(out_sf != nullptr, "out_sf is NULL for NVFP4 output");
+    REQUIRE_ALIGNED_OR_NULL(out_sf);
+  }
+  const int64_t first = (overlap && e0 >= 1) ? (int64_t)m * (e0 - 1) : (int64_t)m * e0;
+  const int64_t last = (int64_t)m * (e0 + n_out) - 1;
+  REQUIRE(first >= tok0 && last < tok0 + n_tok,
+          "entries [%lld, %lld) need tokens [%lld, %lld] but rows hold [%lld, %lld)",
+          (long long)e0, (long long)(e0 + n_out), (long long)first, (long long)last,
+          (long long)tok0, (long long)(tok0 + n_tok));
+  *args = csa::CompressArgs{Ca, Cb, Za, Zb, Ba, Bb, batch, n_tok, tok0, in_batch_stride, e0, n_out,
+                            dim, m, (int)in_dt, (int)out_dt, out, out_sf, out_batch_stride, out_row0};
+  return ok();
+}
+
+
+// Validates an indexer call on the host; fills *args, or sets *empty when
+// there is nothing to do.
+static csa_status_t check_index(const void* qI, const void* qI_sf, const float* wI, const void* KI,
+                                const void* KI_sf, const int64_t* q_pos, int batch, int n_q, int64_t n_entries,
+                                int m, int n_heads, int dim, int k, csa_dtype_t dt, int32_t* idx_out,
+                                void* scores_out, void* ws, size_t ws_bytes, csa::IndexArgs* args, bool* empty) {
+  *empty = false;
+  REQUIRE(batch >= 0 && n_q >= 0 && n_entries >= 0, "negative size");
+  REQUIRE(n_entries <= (int64_t)1 << 30, "n_entries=%lld too large", (long long)n_entries);
+  REQUIRE(m >= 1, "m=%d must be >= 1", m);
+  REQUIRE(k >= 1 && k <= 2048, "k=%d out of range [1, 2048]", k);
+  REQUIRE(n_heads >= 1 && n_heads <= 128, "n_heads=%d out of range [1, 128]", n_heads);
+  REQUIRE(dim >= 32 && dim <= 256 && dim % 32 == 0, "dim=%d must be a multiple of 32 in [32, 256]", dim);
+  REQUIRE(dt == CSA_F32 || dt == CSA_BF16 || dt == CSA_IDX_NVFP4, "dt must be F32, BF16 or IDX_NVFP4");
+  if ((int64_t)batch * n_q == 0) {
+    *empty = true;
+    return ok();
+  }
+  REQUIRE_PTR(qI);
+  REQUIRE_PTR(wI);
+  REQUIRE_PTR(q_pos);
+  REQUIRE_PTR(idx_out);
+  REQUIRE_ALIGNED_OR_NULL(scores_out);
+  if (n_entries > 0) REQUIRE_PTR(KI);
+  if (dt == CSA_IDX_NVFP4) {
+    REQUIRE(qI_sf != nullptr && (KI_sf != nullptr || n_entries == 0), "NVFP4 needs qI_sf and KI_sf");
+    REQUIRE(dim % 64 == 0, "NVFP4 needs dim %% 64 == 0 (blocked key scales), got %d", dim);
+    REQUIRE_ALIGNED_OR_NULL(KI_sf);
+  }
+  const size_t need = csa_index_topk_workspace_size(batch, n_q, n_entries, k, n_heads, dim, dt);
+  REQUIRE(ws_bytes >= need, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  REQUIRE_PTR(ws);
+  *args = csa::IndexArgs{qI, qI_sf, wI, KI, KI_sf, q_pos, batch, n_q, n_entries, m, n_heads, dim, k,
+                         (int)dt, idx_out, scores_out, ws, ws_bytes, 0, csa::CompressArgs{}};
+  return ok();
+}
+
+
 extern "C" {
 
 const char* csa_last_error(void) { return g_err; }
@@ -91,43 +181,11 @@ csa_status_t csa_compress(const void* Ca, const void* Cb, const void* Za, const 
                           int64_t out_batch_stride, int64_t out_row0, csa_dtype_t out_dt,
                           void* stream) {
   g_launches = 0;
-  REQUIRE(batch >= 0 && n_tok >= 0 && tok0 >= 0 && e0 >= 0 && n_out >= 0 && out_row0 >= 0,
-          "negative size (batch=%d n_tok=%lld tok0=%lld e0=%lld n_out=%lld out_row0=%lld)", batch,
-          (long long)n_tok, (long long)tok0, (long long)e0, (long long)n_out, (long long)out_row0);
-  REQUIRE(m >= 1 && m <= 4096, "m=%d out of range [1, 4096]", m);
-  REQUIRE(dim >= 8 && dim % 8 == 0, "dim=%d must be a positive multiple of 8", dim);
-  REQUIRE(in_dt == CSA_F32 || in_dt == CSA_BF16, "in_dt must be CSA_F32 or CSA_BF16");
-  REQUIRE(out_dt >= CSA_F32 && out_dt <= CSA_IDX_NVFP4, "unknown out_dt %d", (int)out_dt);
-  if (out_dt == CSA_KV_FP8MIX)
-    REQUIRE(dim >= 128 && (dim - 64) % 64 == 0, "KV_FP8MIX needs dim = 64 + 64*j (j >= 1), got %d", dim);
-  if (out_dt == CSA_IDX_NVFP4) REQUIRE(dim % 64 == 0, "NVFP4 output needs dim %% 64 == 0, got %d", dim);
-  REQUIRE(in_batch_stride >= n_tok, "in_batch_stride %lld < n_tok %lld", (long long)in_batch_stride,
-          (long long)n_tok);
-  REQUIRE(out_batch_stride >= out_row0 + n_out, "out_batch_stride %lld < out_row0 %lld + n_out %lld",
-          (long long)out_batch_stride, (long long)out_row0, (long long)n_out);
-  if ((int64_t)batch * n_out == 0) return ok();
-  REQUIRE_PTR(Ca);
-  REQUIRE_PTR(Za);
-  REQUIRE_PTR(Ba);
-  REQUIRE_PTR(out);
-  const bool overlap = Cb != nullptr;
-  if (overlap) {
-    REQUIRE_PTR(Zb);
-    REQUIRE_PTR(Bb);
-    REQUIRE_ALIGNED_OR_NULL(Cb);
-  }
-  if (out_dt == CSA_IDX_NVFP4) {
-    REQUIRE(out_sf != nullptr, "out_sf is NULL for NVFP4 output");
-    REQUIRE_ALIGNED_OR_NULL(out_sf);
-  }
-  const int64_t first = (overlap && e0 >= 1) ? (int64_t)m * (e0 - 1) : (int64_t)m * e0;
-  const int64_t last = (int64_t)m * (e0 + n_out) - 1;
-  REQUIRE(first >= tok0 && last < tok0 + n_tok,
-          "entries [%lld, %lld) need tokens [%lld, %lld] but rows hold [%lld, %lld)",
-          (long long)e0, (long long)(e0 + n_out), (long long)first, (long long)last,
-          (long long)tok0, (long long)(tok0 + n_tok));
-  csa::CompressArgs a{Ca, Cb, Za, Zb, Ba, Bb, batch, n_tok, tok0, in_batch_stride, e0, n_out,
-                      dim, m, (int)in_dt, (int)out_dt, out, out_sf, out_batch_stride, out_row0};
+  csa::CompressArgs a{};
+  bool empty = false;
+  const csa_status_t st = check_compress(Ca, Cb, Za, Zb, Ba, Bb, batch, n_tok, tok0, in_batch_stride, e0, n_out,
+                                         dim, m, in_dt, out, out_sf, out_batch_stride, out_row0, out_dt, &a, &empty);
+  if (st != CSA_OK || empty) return st;
   return cuda_status(csa::launch_compress(a, static_cast<cudaStream_t>(stream)), "csa_compress");
 }
 
@@ -144,31 +202,77 @@ csa_status_t csa_index_topk(const void* qI, const void* qI_sf, const float* wI, 
                             int32_t* idx_out, void* scores_out, void* ws, size_t ws_bytes,
                             void* stream) {
   g_launches = 0;
-  REQUIRE(batch >= 0 && n_q >= 0 && n_entries >= 0, "negative size");
-  REQUIRE(n_entries <= (int64_t)1 << 30, "n_entries=%lld too large", (long long)n_entries);
-  REQUIRE(m >= 1, "m=%d must be >= 1", m);
-  REQUIRE(k >= 1 && k <= 2048, "k=%d out of range [1, 2048]", k);
-  REQUIRE(n_heads >= 1 && n_heads <= 128, "n_heads=%d out of range [1, 128]", n_heads);
-  REQUIRE(dim >= 32 && dim <= 256 && dim % 32 == 0, "dim=%d must be a multiple of 32 in [32, 256]", dim);
-  REQUIRE(dt == CSA_F32 || dt == CSA_BF16 || dt == CSA_IDX_NVFP4, "dt must be F32, BF16 or IDX_NVFP4");
-  if ((int64_t)batch * n_q == 0) return ok();
-  REQUIRE_PTR(qI);
-  REQUIRE_PTR(wI);
-  REQUIRE_PTR(q_pos);
-  REQUIRE_PTR(idx_out);
-  REQUIRE_ALIGNED_OR_NULL(scores_out);
-  if (n_entries > 0) REQUIRE_PTR(KI);
-  if (dt == CSA_IDX_NVFP4) {
-    REQUIRE(qI_sf != nullptr && (KI_sf != nullptr || n_entries == 0), "NVFP4 needs qI_sf and KI_sf");
-    REQUIRE(dim % 64 == 0, "NVFP4 needs dim %% 64 == 0 (blocked key scales), got %d", dim);
-    REQUIRE_ALIGNED_OR_NULL(KI_sf);
-  }
-  const size_t need = csa_index_topk_workspace_size(batch, n_q, n_entries, k, n_heads, dim, dt);
-  REQUIRE(ws_bytes >= need, "workspace too small: %zu < %zu bytes", ws_bytes, need);
-  REQUIRE_PTR(ws);
-  csa::IndexArgs a{qI, qI_sf, wI, KI, KI_sf, q_pos, batch, n_q, n_entries, m, n_heads, dim, k,
-                   (int)dt, idx_out, scores_out, ws, ws_bytes};
+  csa::IndexArgs a{};
+  bool empty = false;
+  const csa_status_t st = check_index(qI, qI_sf, wI, KI, KI_sf, q_pos, batch, n_q, n_entries, m, n_heads, dim, k,
+                                      dt, idx_out, scores_out, ws, ws_bytes, &a, &empty);
+  if (st != CSA_OK || empty) return st;
   return cuda_status(csa::launch_index_topk(a, static_cast<cudaStream_t>(stream)), "csa_index_topk");
+}
+
+csa_status_t csa_compress_index_topk(const csa_compress_job_t* keys, const csa_compress_job_t* extra,
+                                     const void* qI, const void* qI_sf, const float* wI, void* KI, void* KI_sf,
+                                     const int64_t* q_pos, int batch, int n_q, int64_t n_entries, int m,
+                                     int n_heads, int dim, int k, csa_dtype_t dt, int32_t* idx_out,
+                                     void* scores_out, void* ws, size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  REQUIRE(keys != nullptr, "keys is NULL");
+  REQUIRE(keys->out == KI && keys->out_sf == KI_sf && keys->out_dt == dt && keys->dim == dim &&
+              keys->out_batch_stride == n_entries && keys->out_row0 == keys->e0,
+          "keys must write entry i into row i of the indexer's cache (out == KI, out_sf == KI_sf, out_dt == dt, "
+          "dim == dim, out_batch_stride == n_entries, out_row0 == e0)");
+  csa::CompressArgs c{}, c2{};
+  bool c_empty = false, c2_empty = true;
+  csa_status_t st = check_compress(keys->Ca, keys->Cb, keys->Za, keys->Zb, keys->Ba, keys->Bb, batch, keys->n_tok,
+                                   keys->tok0, keys->in_batch_stride, keys->e0, keys->n_out, keys->dim, keys->m,
+                                   keys->in_dt, keys->out, keys->out_sf, keys->out_batch_stride, keys->out_row0,
+                                   keys->out_dt, &c, &c_empty);
+  if (st != CSA_OK) return st;
+  if (extra != nullptr) {
+    REQUIRE(extra->out != KI && (extra->out_sf == nullptr || extra->out_sf != KI_sf),
+            "extra must not write the indexer's cache");
+    st = check_compress(extra->Ca, extra->Cb, extra->Za, extra->Zb, extra->Ba, extra->Bb, batch, extra->n_tok,
+                        extra->tok0, extra->in_batch_stride, extra->e0, extra->n_out, extra->dim, extra->m,
+                        extra->in_dt, extra->out, extra->out_sf, extra->out_batch_stride, extra->out_row0,
+                        extra->out_dt, &c2, &c2_empty);
+    if (st != CSA_OK) return st;
+  }
+  csa::IndexArgs a{};
+  bool i_empty = false;
+  st = check_index(qI, qI_sf, wI, KI, KI_sf, q_pos, batch, n_q, n_entries, m, n_heads, dim, k, dt, idx_out,
+                   scores_out, ws, ws_bytes, &a, &i_empty);
+  if (st != CSA_OK) return st;
+  const cudaStream_t s = static_cast<cudaStream_t>(stream);
+  a.comp = c;
+  a.comp2 = c2;
+  if (c2_empty) a.comp2.n_out = 0;
+  if (!c_empty && !i_empty && csa::index_fusable(a)) {
+    a.fused = 1;
+    return cuda_status(csa::launch_index_topk(a, s), "csa_compress_index_topk");
+  }
+  int launches = 0;
+  const csa::CompressArgs* jobs[2] = {c_empty ? nullptr : &c, c2_empty ? nullptr : &c2};
+  for (const csa::CompressArgs* j : jobs) {
+    if (j == nullptr) continue;
+    g_launches = 0;
+    const cudaError_t e = csa::launch_compress(*j, s);
+    launches += g_launches;
+    if (e != cudaSuccess) {
+      g_launches = launches;
+      return cuda_status(e, "csa_compress_index_topk (compress)");
+    }
+  }
+  if (!i_empty) {
+    g_launches = 0;
+    const cudaError_t e = csa::launch_index_topk(a, s);
+    launches += g_launches;
+    if (e != cudaSuccess) {
+      g_launches = launches;
+      return cuda_status(e, "csa_compress_index_topk (index)");
+    }
+  }
+  g_launches = launches;
+  return ok();
 }
 
 }  // extern "C"

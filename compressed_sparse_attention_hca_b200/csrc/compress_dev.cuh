@@ -1,0 +1,238 @@
+// compress_dev.cuh -- device pieces of the Token-Level Compressor
+// ("DeepSeek-V4 内部机制" 1.2 Step 1 and 1.3; yunpan.plus write-up eq. 6-7 and
+// 10-11) shared by the compressor kernels and by the indexer kernels that
+// compress a decode step's new index key before streaming the cache.
+#pragma once
+
+#include "csa_internal.cuh"
+
+namespace csa {
+namespace {
+
+__device__ __forceinline__ void load8(const void* base, int dt, int64_t elem, float* v) {
+  if (dt == CSA_F32) {
+    const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem);
+    float4 a = __ldg(p), b = __ldg(p + 1);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  } else {
+    uint4 u = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + elem));
+    uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      v[2 * j] = __uint_as_float(w[j] << 16);
+      v[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+    }
+  }
+}
+
+// Writes channels d0 .. d0+7 of entry e0 + ie of request b in the output
+// format.  Called by whole warps: the 8 lanes of a 64-dim FP8 scale block (2
+// lanes of a 16-dim FP4 block) are consecutive and reduce their amax with
+// shuffles; lanes with valid == false take part in the shuffles only.
+__device__ __forceinline__ void store_entry(const CompressArgs& a, int b, int64_t ie, int d0, const float* x,
+                                            bool valid) {
+  const int64_t orow = (int64_t)b * a.out_batch_stride + a.out_row0 + ie;
+  const int64_t rb = row_bytes(a.out_dt, a.dim);
+  uint8_t* row = static_cast<uint8_t*>(a.out) + orow * rb;
+
+  if (a.out_dt == CSA_F32) {
+    if (valid) {
+      float4* p = reinterpret_cast<float4*>(row + 4 * d0);
+      p[0] = make_float4(x[0], x[1], x[2], x[3]);
+      p[1] = make_float4(x[4], x[5], x[6], x[7]);
+    }
+  } else if (a.out_dt == CSA_BF16) {
+    if (valid) {
+      uint32_t w[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
+        memcpy(&w[q], &h, 4);
+      }
+      *reinterpret_cast<uint4*>(row + 2 * d0) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  } else if (a.out_dt == CSA_KV_FP8MIX) {
+    const int n8 = a.dim - kRopeDims;
+    float amax = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) amax = fmaxf(amax, fabsf(x[q]));
+    // 8 consecutive lanes hold one 64-dim scale block
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 4));
+    if (valid) {
+      if (d0 < n8) {
+        const float scale = amax > 0.f ? amax / 448.f : 1.f;
+        uint32_t w[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+              make_float2(x[4 * q] / scale, x[4 * q + 1] / scale), __NV_SATFINITE, __NV_E4M3);
+          __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+              make_float2(x[4 * q + 2] / scale, x[4 * q + 3] / scale), __NV_SATFINITE, __NV_E4M3);
+          w[q] = (uint32_t)lo | ((uint32_t)hi << 16);
+        }
+        *reinterpret_cast<uint2*>(row + d0) = make_uint2(w[0], w[1]);
+        if ((d0 % kFp8Block) == 0)
+          *reinterpret_cast<float*>(row + n8 + 2 * kRopeDims + 4 * (d0 / kFp8Block)) = scale;
+      } else {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(x[2 * q], x[2 * q + 1]);
+          memcpy(&w[q], &h, 4);
+        }
+        *reinterpret_cast<uint4*>(row + n8 + 2 * (d0 - n8)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      if (d0 == 0) {
+        for (int64_t p = n8 + 2 * kRopeDims + 4 * (n8 / kFp8Block); p < rb; ++p) row[p] = 0;
+      }
+    }
+  } else {  // CSA_IDX_NVFP4
+    float amax = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) amax = fmaxf(amax, fabsf(x[q]));
+    amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));  // 2 lanes = 16 values
+    if (valid) {
+      const __nv_fp8_storage_t s8 = __nv_cvt_float_to_fp8(amax / 6.f, __NV_SATFINITE, __NV_E4M3);
+      const float s = e4m3_to_float((uint8_t)s8);
+      uint32_t packed = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        __nv_fp4x2_storage_t p2 = 0;
+        if (s > 0.f)
+          p2 = __nv_cvt_float2_to_fp4x2(make_float2(x[2 * q] / s, x[2 * q + 1] / s), __NV_E2M1,
+                                        cudaRoundNearest);
+        packed |= ((uint32_t)p2) << (8 * q);
+      }
+      *reinterpret_cast<uint32_t*>(row + d0 / 2) = packed;
+      if ((d0 % kFp4Block) == 0) {
+        // key-cache scales live in the blocked scale-factor atom layout
+        const int j = d0 / kFp4Block;
+        const int64_t off = (int64_t)b * nvfp4_blocked_sf_bytes(a.out_batch_stride, a.dim) +
+                            nvfp4_blocked_sf_offset(a.out_row0 + ie, a.dim) + (j / 4) * 512 + (j % 4);
+        static_cast<uint8_t*>(a.out_sf)[off] = (uint8_t)s8;
+      }
+    }
+  }
+}
+
+// ---- the softmax over token positions, in one fixed order ------------------
+// Entry i of a request pools U token positions per channel: u = 0 .. m-1 are
+// tokens m*i + u of the current group (biases B^a[u]); with overlap (CSA,
+// i >= 1) u = m .. 2m-1 are tokens m*(i-1) + u - m of the previous group
+// (biases B^b[u - m]).  Every kernel form computes, per channel,
+//   M   = max_u (z_u + b_u)
+//   e_u = exp((z_u + b_u) - M)
+//   D   = sum over blocks of 32 positions, in order, of (e_u summed in order)
+//   S   = the same with e_u * c_u (fused multiply-add)
+//   out = S / D
+// two passes, so the exponentials of one pass are independent of each other.
+// The form that owns a channel (a thread over 8 channels, a thread per
+// channel, several threads per channel) only changes who computes which
+// block; the operations and their order stay the same, so every form writes
+// the same bytes for the same entry.
+constexpr int kPosBlock = 32;
+
+__device__ __forceinline__ float pos_elem(const uint8_t* base, int dt, int64_t idx) {
+  return dt == CSA_F32 ? reinterpret_cast<const float*>(base)[idx]
+                       : __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(base)[idx] << 16);
+}
+// Running max of channel-relative logits over n rows `stride` elements apart.
+__device__ __forceinline__ float chan_max(const uint8_t* z, const float* bias, int dt, int stride, int n, float M) {
+  for (int u = 0; u < n; ++u) M = fmaxf(M, pos_elem(z, dt, (int64_t)u * stride) + bias[(int64_t)u * stride]);
+  return M;
+}
+// Sums of one block of n <= kPosBlock rows.
+__device__ __forceinline__ void chan_block(const uint8_t* z, const uint8_t* c, const float* bias, int dt, int stride,
+                                           int n, float M, float& d, float& s) {
+  d = 0.f;
+  s = 0.f;
+#pragma unroll 4
+  for (int u = 0; u < n; ++u) {
+    const int64_t k = (int64_t)u * stride;
+    const float e = expf((pos_elem(z, dt, k) + bias[k]) - M);
+    d += e;
+    s = fmaf(e, pos_elem(c, dt, k), s);
+  }
+}
+__device__ __forceinline__ float pooled_value(float D, float S) { return D > 0.f ? S / D : 0.f; }
+
+// ---- staged form (at most kPosBlock positions per entry) --------------------
+// All of an entry's inputs are brought into shared memory with one round of
+// cp.async, so a block that compresses while the rest of the GPU streams pays
+// one memory round trip per call.  Layout of one staged entry (U = 2m with
+// overlap, else m; rows of dim elements):
+//   Z [U][dim] (in_dt) | C [U][dim] (in_dt) | bias [U][dim] f32 | x [dim] f32
+__host__ __device__ __forceinline__ int staged_positions(const CompressArgs& a) {
+  return a.Cb != nullptr ? 2 * a.m : a.m;
+}
+__host__ __device__ __forceinline__ int staged_entry_bytes(const CompressArgs& a) {
+  const int esz = a.in_dt == CSA_F32 ? 4 : 2;
+  const int U = staged_positions(a);
+  return U * a.dim * (2 * esz + 4) + a.dim * 4;
+}
+__device__ __forceinline__ void stage_cp16(uint8_t* dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"((uint32_t)__cvta_generic_to_shared(dst)),
+               "l"(src)
+               : "memory");
+}
+// Issues (without waiting) the cp.async copies of entry e0 + ie of request b.
+template <int NT>
+__device__ void stage_entry(const CompressArgs& a, int b, int64_t ie, uint8_t* buf) {
+  const int esz = a.in_dt == CSA_F32 ? 4 : 2;
+  const int64_t i = a.e0 + ie;
+  const bool two = a.Cb != nullptr && i >= 1;
+  const int U = two ? 2 * a.m : a.m, Umax = staged_positions(a);
+  const int row16 = a.dim * esz / 16;  // 16-byte pieces per input row
+  const int64_t in_base = (int64_t)b * a.in_batch_stride;
+  uint8_t* zb = buf;
+  uint8_t* cb = buf + (size_t)Umax * a.dim * esz;
+  for (int q = threadIdx.x; q < U * row16; q += NT) {
+    const int u = q / row16, p = q % row16;
+    const bool cur = u < a.m;
+    const int64_t tok = cur ? (int64_t)a.m * i + u : (int64_t)a.m * (i - 1) + (u - a.m);
+    const int64_t off = ((in_base + tok - a.tok0) * a.dim) * esz + (int64_t)p * 16;
+    stage_cp16(zb + (size_t)u * a.dim * esz + p * 16, static_cast<const uint8_t*>(cur ? a.Za : a.Zb) + off);
+    stage_cp16(cb + (size_t)u * a.dim * esz + p * 16, static_cast<const uint8_t*>(cur ? a.Ca : a.Cb) + off);
+  }
+  // bias rows in position order: B^a[0..m), then B^b[0..m)
+  uint8_t* bias = buf + (size_t)Umax * a.dim * esz * 2;
+  const int brow16 = a.dim * 4 / 16;
+  for (int q = threadIdx.x; q < U * brow16; q += NT) {
+    const int u = q / brow16, p = q % brow16;
+    const float* src = u < a.m ? a.Ba + (int64_t)u * a.dim : a.Bb + (int64_t)(u - a.m) * a.dim;
+    stage_cp16(bias + ((size_t)u * a.dim) * 4 + p * 16, reinterpret_cast<const uint8_t*>(src) + p * 16);
+  }
+}
+// Channel w of a staged entry (after the copies landed and a block barrier):
+// writes the pooled value into the entry's x row.
+__device__ __forceinline__ void staged_channel(const CompressArgs& a, int64_t ie, uint8_t* buf, int w) {
+  const int esz = a.in_dt == CSA_F32 ? 4 : 2;
+  const int64_t i = a.e0 + ie;
+  const int U = (a.Cb != nullptr && i >= 1) ? 2 * a.m : a.m, Umax = staged_positions(a);
+  const uint8_t* zb = buf + (size_t)w * esz;
+  const uint8_t* cb = buf + (size_t)Umax * a.dim * esz + (size_t)w * esz;
+  const float* bias = reinterpret_cast<const float*>(buf + (size_t)Umax * a.dim * esz * 2) + w;
+  const float M = chan_max(zb, bias, a.in_dt, a.dim, U, -INFINITY);
+  float d, s;
+  chan_block(zb, cb, bias, a.in_dt, a.dim, U, M, d, s);
+  float D = 0.f, S = 0.f;
+  D += d;
+  S += s;
+  reinterpret_cast<float*>(buf + (size_t)Umax * a.dim * (2 * esz + 4))[w] = pooled_value(D, S);
+}
+// Writes the 8-channel chunk ch of a staged entry whose x row is complete.
+// Called by whole warps (valid == false lanes join the shuffles only).
+__device__ __forceinline__ void staged_store(const CompressArgs& a, int b, int64_t ie, const uint8_t* buf, int ch,
+                                             bool valid) {
+  const int esz = a.in_dt == CSA_F32 ? 4 : 2;
+  const float* xr = reinterpret_cast<const float*>(buf + (size_t)staged_positions(a) * a.dim * (2 * esz + 4));
+  float x[8];
+#pragma unroll
+  for (int q = 0; q < 8; ++q) x[q] = valid ? xr[ch * 8 + q] : 0.f;
+  store_entry(a, b, ie, valid ? ch * 8 : 0, x, valid);
+}
+
+}  // namespace
+}  // namespace csa

@@ -183,8 +183,17 @@ struct IndexArgs {
   void* scores_out;
   void* ws;
   size_t ws_bytes;
+  // fused decode form: the CTA whose slice holds the new key rows
+  // comp.e0 .. +n_out compresses them into the key cache (comp.out = KI)
+  // before streaming them, and runs the extra job comp2 (any other cache;
+  // n_out = 0 when absent) for its request
+  int fused;
+  CompressArgs comp, comp2;
 };
 size_t index_topk_workspace(int batch, int n_q, int64_t n_entries, int k, int n_heads, int dim, int dt);
+// Whether the indexer runs the fused decode form (compress the new keys in
+// the indexer launch) for these arguments.
+bool index_fusable(const IndexArgs& a);
 cudaError_t launch_index_topk(const IndexArgs& a, cudaStream_t s);
 
 struct MqaArgs {

@@ -27,6 +27,7 @@
 // for the merge kernel.
 #include <cudaTypedefs.h>
 
+#include "compress_dev.cuh"
 #include "csa_internal.cuh"
 #include "indexer_plan.cuh"
 #include "sm100.cuh"
@@ -533,6 +534,77 @@ __device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t 
   }
 }
 
+// ------------------------------------------------------- fused decode form
+// With a.fused set (one query per CTA, so one CTA per slice of a request):
+// every CTA whose slice holds new key rows a.comp.e0 .. +n_out compresses
+// them into the key cache before its producer loads the stage holding them,
+// and the CTA holding row a.comp.e0 (the lead) also runs the extra job
+// a.comp2 for its request.  The CTA starts the key stages before the first
+// new row, then compresses while they land, in ring stages it has not used.
+template <int NQ>
+__device__ __forceinline__ bool fused_keys(const IndexArgs& a, int64_t s0, int len) {
+  return NQ == 1 && a.fused && s0 < a.comp.e0 + a.comp.n_out && a.comp.e0 < s0 + len;
+}
+template <int NQ>
+__device__ __forceinline__ bool fused_lead(const IndexArgs& a, int64_t s0, int len) {
+  return NQ == 1 && a.fused && s0 <= a.comp.e0 && a.comp.e0 < s0 + len;
+}
+// Shared memory the fused jobs stage (all rows of both jobs at once), and
+// whether the staged form applies (at most 32 token positions per entry).
+__host__ __device__ __forceinline__ int fused_scratch_bytes(const IndexArgs& a) {
+  int need = (int)a.comp.n_out * staged_entry_bytes(a.comp);
+  if (a.comp2.n_out > 0) need += (int)a.comp2.n_out * staged_entry_bytes(a.comp2);
+  return need;
+}
+__host__ __device__ __forceinline__ int fused_scratch_stages(const IndexArgs& a, int stage_bytes) {
+  return (fused_scratch_bytes(a) + stage_bytes - 1) / stage_bytes;
+}
+__host__ __device__ __forceinline__ bool fused_jobs_staged(const IndexArgs& a) {
+  return (a.comp.Cb != nullptr ? 2 : 1) * a.comp.m <= 32 &&
+         (a.comp2.n_out == 0 || (a.comp2.Cb != nullptr ? 2 : 1) * a.comp2.m <= 32);
+}
+template <int NT>
+__device__ void run_fused_jobs(const IndexArgs& a, int b, int64_t s0, int len, uint8_t* scratch, bool keys,
+                               bool lead) {
+  const int64_t lo = keys ? max64(a.comp.e0, s0) : 0, hi = keys ? min64(a.comp.e0 + a.comp.n_out, s0 + len) : 0;
+  const int nk = (int)(hi - lo), nx = lead ? (int)a.comp2.n_out : 0;
+  const int kb = staged_entry_bytes(a.comp), xb = nx > 0 ? staged_entry_bytes(a.comp2) : 0;
+  const int64_t ik = lo - a.comp.e0;  // first key entry of this CTA, relative to e0
+  uint8_t* const xbuf = scratch + (size_t)nk * kb;
+  for (int e = 0; e < nk; ++e) stage_entry<NT>(a.comp, b, ik + e, scratch + (size_t)e * kb);
+  for (int e = 0; e < nx; ++e) stage_entry<NT>(a.comp2, b, e, xbuf + (size_t)e * xb);
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+  __syncthreads();
+  // one channel per thread: the key entries' channels, then the extra job's
+  const int dk = a.comp.dim, dx = a.comp2.dim, ck = nk * dk, cx = nx * dx;
+  for (int g = threadIdx.x; g < ck + cx; g += NT) {
+    if (g < ck) {
+      staged_channel(a.comp, ik + g / dk, scratch + (size_t)(g / dk) * kb, g % dk);
+    } else {
+      const int h = g - ck;
+      staged_channel(a.comp2, h / dx, xbuf + (size_t)(h / dx) * xb, h % dx);
+    }
+  }
+  __syncthreads();
+  // quantise and write, 8 channels per thread (whole warps: the scale blocks
+  // of a row are consecutive lanes)
+  const int qk = nk * (dk / 8), qx = nx * (dx / 8);
+  for (int c0 = 0; c0 < qk; c0 += NT) {
+    const int q = c0 + threadIdx.x;
+    const bool v = q < qk;
+    const int e = v ? q / (dk / 8) : 0;
+    staged_store(a.comp, b, ik + e, scratch + (size_t)e * kb, v ? q % (dk / 8) : 0, v);
+  }
+  for (int c0 = 0; c0 < qx; c0 += NT) {
+    const int q = c0 + threadIdx.x;
+    const bool v = q < qx;
+    const int e = v ? q / (dx / 8) : 0;
+    staged_store(a.comp2, b, e, xbuf + (size_t)e * xb, v ? q % (dx / 8) : 0, v);
+  }
+  fence_proxy_async_global();  // the new key rows are read back by this CTA's TMA
+  __syncthreads();
+}
+
 // ----------------------------------------------------------------- BF16 kernel
 template <int NQ>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -560,7 +632,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // positions: the producer thread starts them before anything is loaded.
   const int64_t s0 = (int64_t)blockIdx.x * plan.slice_len;
   const int len0 = (int)min64(plan.slice_len, a.n_entries - s0);
-  const int pre = min(C::STAGES, (len0 + kBM - 1) / kBM);
+  const bool fkeys = fused_keys<NQ>(a, s0, len0), flead = fused_lead<NQ>(a, s0, len0);
+  const int nscr = (fkeys || flead) ? fused_scratch_stages(a, C::K_STAGE) : 0;
+  int pre = min(C::STAGES - nscr, (len0 + kBM - 1) / kBM);
+  if (fkeys) pre = min(pre, (int)(max64(0, a.comp.e0 - s0) / kBM));
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
     for (int i = 0; i < C::NBUF; ++i) { mbar_init(&accf[i], 1); mbar_init(&acce[i], 4); }
@@ -577,6 +652,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_2d(ks + i * C::K_STAGE + kAtom, &tmK, &full[i], 64, row);
     }
   }
+  if (fkeys || flead)
+    run_fused_jobs<kThreads>(a, blockIdx.z, s0, len0, ks + (C::STAGES - nscr) * C::K_STAGE, fkeys, flead);
   const SliceCtx<NQ> c = slice_ctx<NQ>(a, plan);
   for (int i = threadIdx.x; i < NQ * kHI; i += kThreads) {
     const int t = c.t0 + i / kHI;
@@ -688,8 +765,11 @@ __global__ void __launch_bounds__(Nvf4Cfg<NQ>::NT, 1)
   // positions: the producer thread starts them before anything is loaded.
   const int64_t s0 = (int64_t)blockIdx.x * plan.slice_len;
   const int len0 = (int)min64(plan.slice_len, a.n_entries - s0);
-  const int pre = min(C::STAGES, ((len0 + kBM - 1) / kBM + C::TPS - 1) / C::TPS);
   const int b0 = blockIdx.z, t00 = blockIdx.y * NQ;
+  const bool fkeys = fused_keys<NQ>(a, s0, len0), flead = fused_lead<NQ>(a, s0, len0);
+  const int nscr = (fkeys || flead) ? fused_scratch_stages(a, C::STAGE) : 0;
+  int pre = min(C::STAGES - nscr, ((len0 + kBM - 1) / kBM + C::TPS - 1) / C::TPS);
+  if (fkeys) pre = min(pre, (int)(max64(0, a.comp.e0 - s0) / (C::TPS * kBM)));
   if (threadIdx.x == 0) {
     // full: one arrival from each producer (codes, scales); empty: one
     // commit from each issuer (the stage's two tiles)
@@ -709,6 +789,8 @@ __global__ void __launch_bounds__(Nvf4Cfg<NQ>::NT, 1)
       tma_load_2d(st + g * C::STAGE, &tmK, &full[g], 0, (int)((int64_t)b0 * a.n_entries + s0 + (int64_t)g * C::TPS * kBM));
     }
   }
+  if (fkeys || flead)
+    run_fused_jobs<C::NT>(a, b0, s0, len0, st + (C::STAGES - nscr) * C::STAGE, fkeys, flead);
   const SliceCtx<NQ> c = slice_ctx<NQ>(a, plan);
   const int n_stages = (c.n_tiles + C::TPS - 1) / C::TPS;
   for (int i = threadIdx.x; i < NQ * kHI; i += C::NT) {
@@ -932,6 +1014,13 @@ bool index_tc_eligible(const IndexArgs& a) {
 }
 
 int index_tc_nq(int n_q) { return n_q >= 2 ? 2 : 1; }
+
+bool index_fusable(const IndexArgs& a) {
+  if (!index_tc_eligible(a) || index_tc_nq(a.n_q) != 1 || a.n_entries < 1 || !fused_jobs_staged(a)) return false;
+  // the compress scratch must leave the ring at least one stage
+  if (a.dt == CSA_IDX_NVFP4) return fused_scratch_stages(a, Nvf4Cfg<1>::STAGE) < Nvf4Cfg<1>::STAGES;
+  return fused_scratch_stages(a, Bf16Cfg<1>::K_STAGE) < Bf16Cfg<1>::STAGES;
+}
 
 IndexPlan make_tc_plan(int batch, int n_q, int64_t n_entries, int k, int dt) {
   const int NQ = index_tc_nq(n_q);

@@ -189,6 +189,47 @@ csa_status_t csa_index_topk(const void* qI, const void* qI_sf, const float* wI, 
                             void* stream);
 
 /*
+ * csa_compress_job_t -- the arguments of one csa_compress call, for calls
+ * that run compressions inside another operation's launch.  Field meanings
+ * are those of csa_compress; the request count comes from the enclosing call.
+ */
+typedef struct {
+  const void *Ca, *Cb, *Za, *Zb;
+  const float *Ba, *Bb;
+  int64_t n_tok, tok0, in_batch_stride, e0, n_out;
+  int dim, m;
+  csa_dtype_t in_dt;
+  void *out, *out_sf;
+  int64_t out_batch_stride, out_row0;
+  csa_dtype_t out_dt;
+} csa_compress_job_t;
+
+/*
+ * csa_compress_index_topk -- a decode step's compressions and indexer in one
+ * call ([P5] 1.2 Step 1 and Step 2: the newly closed groups are compressed
+ * into the KV cache and into the index-key cache K^I that the Lightning
+ * Indexer then scores).
+ *
+ * Same results as csa_compress(*keys); csa_compress(*extra) (when extra is not
+ * NULL); csa_index_topk(qI, ..., stream) -- every argument means what it
+ * means there.  `keys` must write into the indexer's cache: keys->out == KI,
+ * keys->out_sf == KI_sf, keys->out_dt == dt, keys->dim == dim,
+ * keys->out_batch_stride == n_entries and keys->out_row0 == keys->e0 (entry i
+ * is cache row i); `extra` (e.g. the KV cache's compression) must not write
+ * what the indexer reads.  With one query per request on the tensor-core
+ * indexer this is one launch: the CTA whose slice of the cache holds the new
+ * key rows starts its first key copies, runs both compressions of its request
+ * while they land, and then streams the rest, so the compressions add no
+ * dependent launch to the step.  Other shapes run the calls in order.  Errors
+ * and workspace rules are those of the underlying calls.
+ */
+csa_status_t csa_compress_index_topk(const csa_compress_job_t* keys, const csa_compress_job_t* extra,
+                                     const void* qI, const void* qI_sf, const float* wI, void* KI, void* KI_sf,
+                                     const int64_t* q_pos, int batch, int n_q, int64_t n_entries, int m,
+                                     int n_heads, int dim, int k, csa_dtype_t dt, int32_t* idx_out,
+                                     void* scores_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * csa_index_topk_noalloc -- csa_index_topk for callers that cannot allocate
  * device memory.  The paper has no counterpart: this is a library service.
  *

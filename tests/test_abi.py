@@ -113,3 +113,28 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         csa.compress(torch.zeros(1, 8, 64), torch.zeros(1, 8, 64), torch.zeros(4, 64), 4)
+
+
+def test_compress_index_topk_rejects_bad_arguments():
+    lib = csa.load()
+    KI = P(8192)
+
+    def job(**kw):
+        j = dict(Ca=4096, Cb=4096, Za=4096, Zb=4096, Ba=4096, Bb=4096, n_tok=8, tok0=56, in_batch_stride=8, e0=15,
+                 n_out=1, dim=32, m=4, in_dt=csa.BF16, out=8192, out_sf=None, out_batch_stride=64, out_row0=15,
+                 out_dt=csa.BF16)
+        j.update(kw)
+        return csa.CompressJob(**j)
+
+    def call(keys, extra=None, dt=csa.BF16, n_entries=64, dim=32):
+        return lib.csa_compress_index_topk(ctypes.byref(keys), ctypes.byref(extra) if extra else None, A, None, A,
+                                           KI, None, A, 1, 1, n_entries, 4, 2, dim, 16, dt, A, None, A, 1 << 20, None)
+    assert call(job(), dt=csa.KV_FP8MIX) == INVALID
+    # the key job must write entry i to row i of the indexer's cache
+    assert call(job(out_row0=3)) == INVALID and "row i" in _err()
+    assert call(job(out=4096)) == INVALID and "row i" in _err()
+    # entry 15 with overlap needs tokens 56..63; rows start at token 60
+    assert call(job(tok0=60, n_tok=4, in_batch_stride=4)) == INVALID and "need tokens" in _err()
+    # the extra job must not write the indexer's cache
+    assert call(job(), extra=job()) == INVALID and "extra" in _err()
+    assert call(job(), dim=48) == INVALID

@@ -57,7 +57,9 @@ def _oracle_compress(orc, x, m, tok0, e0, n_out):
     (1, 64, 128, 4, True, torch.float32, csa.F32, 0, 0, 16),
     (2, 4 * 4800, 64, 4, True, torch.float32, csa.F32, 0, 0, None),  # many entries: thread per entry
     (1, 4 * 10, 72, 4, True, torch.float32, csa.F32, 0, 0, None),    # dim not a multiple of 64
-    (2, 40 * 6, 128, 40, True, torch.bfloat16, csa.BF16, 0, 0, None),  # 2m = 80 tokens over 32 lanes
+    (2, 40 * 6, 128, 40, True, torch.bfloat16, csa.BF16, 0, 0, None),  # 2m = 80 positions, 3 blocks
+    (1, 100 * 4, 64, 100, True, torch.float32, csa.F32, 0, 0, None),     # 2m = 200: two staged chunks
+    (2, 300 * 2 + 5, 128, 300, False, torch.bfloat16, csa.F32, 0, 0, None),  # m' = 300: three chunks
 ])
 def test_compress_matches_oracle(orc, case):
     batch, n_tok, dim, m, overlap, dtype, out_dt, tok0, e0, n_out = case
@@ -74,6 +76,26 @@ def test_compress_matches_oracle(orc, case):
         assert_close(got, want, atol=1e-5, what="compress f32")
     else:
         assert_close(got, want, atol=1e-6, rtol=2.0 ** -8, what="compress bf16")
+
+
+@pytest.mark.parametrize("out_dt", [csa.F32, csa.BF16, csa.KV_FP8MIX, csa.IDX_NVFP4])
+def test_compress_forms_write_the_same_bytes(out_dt):
+    """One call over many entries (a thread per entry and 8 channels) and
+    calls over a few entries each (a block per entry) compute every channel's
+    softmax with the same operations in the same order: the bytes agree."""
+    batch, dim, m, n_out = 2, 128, 4, 2400  # 2 x 2400 x 16 chunks: the thread-per-entry form
+    g = W.generator(4242)
+    x = _cuda(W.compress_inputs(g, batch, m * n_out, dim, m, True, torch.bfloat16))
+    args = (x["Ca"], x["Za"], x["Ba"], m, x["Cb"], x["Zb"], x["Bb"])
+    one = csa.compress(*args, out_dt=out_dt)
+    one, one_sf = one if out_dt == csa.IDX_NVFP4 else (one, None)
+    many = torch.full_like(one, 0x5A if one.dtype == torch.uint8 else 3.0)
+    many_sf = None if one_sf is None else torch.zeros_like(one_sf)
+    for e0 in range(0, n_out, 300):
+        csa.compress(*args, e0=e0, n_out=300, out_dt=out_dt, out=many, out_sf=many_sf, out_row0=e0)
+    assert torch.equal(one, many)
+    if one_sf is not None:
+        assert torch.equal(one_sf, many_sf)
 
 
 def test_compress_writes_into_cache_row(orc):
@@ -367,3 +389,64 @@ def test_mqa_sink_limits_cluster_split(orc):
     got, want, _ = _mqa_case(orc, "csa_decode_bf16", 2, 1, 4000, 512, 4 * 4000 - 1, sink_override=sinks)
     assert_close(got, want, atol=2e-2, what="sink limits, cluster split")
     assert (got[:, :, 0] == 0).all()
+
+
+# ------------------------------------------ fused compressions + indexer
+
+@pytest.mark.parametrize("dt,B,T,E,k", [
+    (csa.IDX_NVFP4, 3, 1, 30000, 1024),   # one launch: the lead CTA compresses while its keys land
+    (csa.BF16, 2, 1, 20000, 512),         # one launch (BF16 keys)
+    (csa.IDX_NVFP4, 2, 1, 300, 128),      # tiny cache: the new row is in the lead slice's first stage
+    (csa.IDX_NVFP4, 2, 3, 5000, 512),     # two queries per CTA: the calls in order
+])
+def test_compress_index_topk_equals_the_separate_calls(orc, dt, B, T, E, k):
+    """The fused call writes the same key-cache and KV-cache bytes and selects
+    the same indices as csa_compress (twice) followed by csa_index_topk, and
+    the new key entry matches the oracle's compression."""
+    m, dI, H, c = 4, 128, 64, 512
+    g = W.generator(500 + E)
+    tok = W.compress_inputs(g, B, 2 * m, dI, m, True, torch.bfloat16)
+    ktok = W.compress_inputs(g, B, 2 * m, c, m, True, torch.bfloat16)
+    if dt == csa.IDX_NVFP4:
+        qI, qsf = W.nvfp4_rows(g, (B, T, H), dI)
+        KI, ksf = W.nvfp4_rows(g, (B, E), dI)
+        ksf = W.block_scales(ksf, dI)
+    else:
+        qI, qsf = W.normal(g, (B, T, H, dI), 1.0, torch.bfloat16), None
+        KI, ksf = W.normal(g, (B, E, dI), 1.0, torch.bfloat16), None
+    wI = W.uniform(g, (B, T, H))
+    kv = torch.randint(0, 256, (B, E, 608), generator=g, dtype=torch.uint8)
+    q_pos = torch.tensor([[m * E - 1 - 13 * t for t in range(T)]] * B, dtype=torch.int64)
+    gt, gk, e0, tok0 = _cuda(tok), _cuda(ktok), E - 1, m * (E - 2)
+    cu = lambda v: None if v is None else v.to(DEV)  # noqa: E731
+    # separate calls
+    K1, S1, V1 = cu(KI).clone(), (cu(ksf).clone() if ksf is not None else None), cu(kv).clone()
+    csa.compress(gt["Ca"], gt["Za"], gt["Ba"], m, gt["Cb"], gt["Zb"], gt["Bb"], tok0=tok0, e0=e0, n_out=1,
+                 out_dt=dt, out=K1, out_sf=S1, out_row0=e0)
+    csa.compress(gk["Ca"], gk["Za"], gk["Ba"], m, gk["Cb"], gk["Zb"], gk["Bb"], tok0=tok0, e0=e0, n_out=1,
+                 out_dt=csa.KV_FP8MIX, out=V1, out_row0=e0)
+    idx1 = csa.index_topk(cu(qI), cu(wI), K1, q_pos.to(DEV), m, k, dt=dt, qI_sf=cu(qsf), KI_sf=S1)
+    # fused
+    K2, S2, V2 = cu(KI).clone(), (cu(ksf).clone() if ksf is not None else None), cu(kv).clone()
+    keys = csa.compress_job(gt["Ca"], gt["Za"], gt["Ba"], m, gt["Cb"], gt["Zb"], gt["Bb"], tok0=tok0, e0=e0,
+                            n_out=1, out=K2, out_sf=S2, out_dt=dt)
+    extra = csa.compress_job(gk["Ca"], gk["Za"], gk["Ba"], m, gk["Cb"], gk["Zb"], gk["Bb"], tok0=tok0, e0=e0,
+                             n_out=1, out=V2, out_dt=csa.KV_FP8MIX)
+    idx2 = csa.compress_index_topk(keys, cu(qI), cu(wI), K2, q_pos.to(DEV), m, k, extra_job=extra, dt=dt,
+                                   qI_sf=cu(qsf), KI_sf=S2)
+    torch.cuda.synchronize()
+    csa.check_device_status()
+    assert torch.equal(K1, K2)
+    if S1 is not None:
+        assert torch.equal(S1, S2)
+    assert torch.equal(V1, V2)
+    assert torch.equal(idx1, idx2)
+    # the new key entry against the oracle's own compression (one quantisation step)
+    want = _oracle_compress(orc, tok, m, tok0, e0, 1)
+    for b in range(B):
+        if dt == csa.IDX_NVFP4:
+            codes = raw(K2[b, e0:e0 + 1])
+            sfr = orc.unblock_scales(raw(S2[b]), E, dI)[e0:e0 + 1]
+            _check_nvfp4_rows(orc, codes, sfr, want[b], dI)
+        else:
+            assert_close(f64(K2[b, e0:e0 + 1]), want[b], atol=1e-6, rtol=2.0 ** -8, what="fused bf16 key")
