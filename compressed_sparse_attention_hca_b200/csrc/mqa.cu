@@ -229,6 +229,74 @@ __global__ void __launch_bounds__(128) mqa_combine_kernel(MqaArgs a, MqaPlan pla
   }
 }
 
+// The same merge for few splits (decode on the tensor-core path): thread t
+// owns dims 4t .. 4t+3 and loads every split's statistics and partial at
+// once, so the kernel waits on one round of loads; the weights are summed in
+// split order.
+constexpr int kFewSplits = 16;
+
+__global__ void __launch_bounds__(128) mqa_combine_few_kernel(MqaArgs a, MqaPlan plan) {
+  const int h = blockIdx.x;
+  const int64_t bt = blockIdx.y;
+  const int S = plan.n_splits;
+  const int d = 4 * threadIdx.x;
+  const bool on = d < a.dim;
+  float2 ml[kFewSplits];
+  float4 o[kFewSplits];
+#pragma unroll
+  for (int s = 0; s < kFewSplits; ++s)
+    if (s < S) {
+      ml[s] = __ldcg(reinterpret_cast<const float2*>(plan_partial_ml(plan, a, bt, s, h)));
+      o[s] = on ? __ldcg(reinterpret_cast<const float4*>(plan_partial_o(plan, a, bt, s, h) + d))
+                : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+  const float sink = a.sink[h];
+  float M = sink;
+#pragma unroll
+  for (int s = 0; s < kFewSplits; ++s)
+    if (s < S) M = fmaxf(M, ml[s].x);
+  const bool zero = (sink == INFINITY) || (M == -INFINITY);
+  float den = 0.f;
+#pragma unroll
+  for (int s = 0; s < kFewSplits; ++s)
+    if (s < S) {
+      ml[s].x = (zero || ml[s].x == -INFINITY) ? 0.f : expf(ml[s].x - M);  // e^{m_s - M}
+      den += ml[s].x > 0.f ? ml[s].y * ml[s].x : 0.f;
+    }
+  if (!zero) den += expf(sink - M);
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int s = 0; s < kFewSplits; ++s)
+    if (s < S) {
+      const float w = zero ? 0.f : ml[s].x / den;
+      acc.x = fmaf(w, o[s].x, acc.x);
+      acc.y = fmaf(w, o[s].y, acc.y);
+      acc.z = fmaf(w, o[s].z, acc.z);
+      acc.w = fmaf(w, o[s].w, acc.w);
+    }
+  if (!on) return;
+  const int64_t ob = (bt * a.n_heads + h) * a.dim + d;
+  if (a.q_dt == CSA_F32) {
+    *reinterpret_cast<float4*>(static_cast<float*>(a.O) + ob) = acc;
+  } else {
+    const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x, acc.y), hi = __floats2bfloat162_rn(acc.z, acc.w);
+    uint2 pk;
+    memcpy(&pk.x, &lo, 4);
+    memcpy(&pk.y, &hi, 4);
+    *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.O) + ob) = pk;
+  }
+}
+
+cudaError_t launch_mqa_combine(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) {
+  const dim3 grid(a.n_heads, (unsigned)((int64_t)a.batch * a.n_q));
+  if (p.n_splits <= kFewSplits && a.dim % 4 == 0 && a.dim <= 512)
+    mqa_combine_few_kernel<<<grid, 128, 0, s>>>(a, p);
+  else
+    mqa_combine_kernel<<<grid, 128, 0, s>>>(a, p);
+  ++launch_counter();
+  return cudaGetLastError();
+}
+
 MqaPlan make_simt_mqa_plan(const MqaArgs& a) {
   MqaPlan p{};
   p.heads_per_cta = (a.n_heads % 8 == 0) ? 8 : (a.n_heads % 4 == 0) ? 4 : (a.n_heads % 2 == 0) ? 2 : 1;
@@ -257,9 +325,7 @@ cudaError_t launch_mqa_simt(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) 
   ++launch_counter();
   e = cudaGetLastError();
   if (e != cudaSuccess || p.n_splits == 1) return e;
-  mqa_combine_kernel<<<dim3(a.n_heads, (unsigned)((int64_t)a.batch * a.n_q)), 128, 0, s>>>(a, p);
-  ++launch_counter();
-  return cudaGetLastError();
+  return launch_mqa_combine(a, p, s);
 }
 
 bool mqa_umma_path(const MqaArgs& a);

@@ -25,8 +25,10 @@
 //
 // With few queries (decode) a query's row chunks are split over several CTAs
 // so that the grid fills the GPU; each writes its unnormalised partial
-// (max, sum, o) to the workspace and mqa_combine_kernel adds them with the
-// sink.
+// (max, sum, o) to the workspace.  When the splits of a query fit one thread
+// block cluster (up to 16 CTAs) they combine the partials themselves after a
+// cluster barrier, each CTA taking a slice of the 512 dims; otherwise
+// mqa_combine_kernel adds them with the sink.
 #include "csa_internal.cuh"
 #include "mqa_plan.cuh"
 #include "sm100.cuh"
@@ -35,7 +37,7 @@ namespace csa {
 
 CSA_DEFINE_STATUS_READER(take_status_mqa_umma)
 
-__global__ void mqa_combine_kernel(MqaArgs a, MqaPlan plan);
+cudaError_t launch_mqa_combine(const MqaArgs& a, const MqaPlan& p, cudaStream_t s);
 
 namespace {
 
@@ -126,7 +128,11 @@ __device__ __forceinline__ void reduce_scatter64(float* v, int lane, float& r0, 
   r1 = v[1];
 }
 
-template <bool FP8, bool SPLIT>
+// How a CTA finishes: the whole query (normalised output) or one split of
+// several (unnormalised partial for the combine kernel).
+enum { kWhole = 0, kSplit = 1 };
+
+template <bool FP8, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPlan plan) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
@@ -393,22 +399,31 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
       for (int h = 0; h < kHG; ++h) o[h] = 0.f;
     }
   };
-  if constexpr (SPLIT) {
-    // one split of many: the unnormalised partial (m, l, o) for the combine kernel
-    if (tid < kHG) {
-      float* ml = plan_partial_ml(plan, a, bt, split, hg * kHG + tid);
-      const float m = ms.m_use[tid];
-      ml[0] = m == -INFINITY ? -INFINITY : m / kLog2e;  // natural-log domain
-      ml[1] = ms.l_run[tid];
-    }
+  if constexpr (MODE != kWhole) {
+    // one split of many: O^T slabs -> the idle row tile as [slab][head][128 dims]
+    float* stg = reinterpret_cast<float*>(KV);
     if (warp < 4) {
 #pragma unroll 1
       for (int sl = 0; sl < 4; ++sl) {
         float o[kHG];
         load_slab(sl, o);
 #pragma unroll
-        for (int h = 0; h < kHG; ++h) plan_partial_o(plan, a, bt, split, hg * kHG + h)[sl * 128 + tid] = o[h];
+        for (int h = 0; h < kHG; ++h) stg[(sl * kHG + h) * 128 + tid] = o[h];
       }
+    }
+    __syncthreads();
+    // the unnormalised partial (m, l, o), written in 16-byte pieces so that
+    // each warp store covers 512 contiguous bytes
+    if (tid < kHG) {
+      float* ml = plan_partial_ml(plan, a, bt, split, hg * kHG + tid);
+      const float m = ms.m_use[tid];
+      ml[0] = m == -INFINITY ? -INFINITY : m / kLog2e;  // natural-log domain
+      ml[1] = ms.l_run[tid];
+    }
+    for (int q = tid; q < kHG * 128; q += kThreads) {
+      const int h = q >> 7, rem = q & 127, sl = rem >> 5, c = rem & 31;
+      const float4 v = *reinterpret_cast<const float4*>(stg + (sl * kHG + h) * 128 + 4 * c);
+      *reinterpret_cast<float4*>(plan_partial_o(plan, a, bt, split, hg * kHG + h) + 4 * rem) = v;
     }
   } else {
     if (tid < kHG) {
@@ -462,24 +477,22 @@ MqaPlan make_umma_mqa_plan(const MqaArgs& a) {
   return p;
 }
 
-template <bool FP8, bool SPLIT>
+template <bool FP8, int MODE>
 cudaError_t launch_umma(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(mqa_umma_kernel<FP8, SPLIT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kSmemBytes);
+  auto kern = mqa_umma_kernel<FP8, MODE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)p.n_splits, a.n_heads / kHG, (unsigned)((int64_t)a.batch * a.n_q));
-  mqa_umma_kernel<FP8, SPLIT><<<grid, kThreads, kSmemBytes, s>>>(a, p);
+  kern<<<grid, kThreads, kSmemBytes, s>>>(a, p);
   ++launch_counter();
   e = cudaGetLastError();
-  if (e != cudaSuccess || !SPLIT) return e;
-  mqa_combine_kernel<<<dim3(a.n_heads, (unsigned)((int64_t)a.batch * a.n_q)), 128, 0, s>>>(a, p);
-  ++launch_counter();
-  return cudaGetLastError();
+  if (e != cudaSuccess || MODE != kSplit) return e;
+  return launch_mqa_combine(a, p, s);
 }
 
 template <bool FP8>
 cudaError_t launch_umma_fmt(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) {
-  return p.n_splits > 1 ? launch_umma<FP8, true>(a, p, s) : launch_umma<FP8, false>(a, p, s);
+  return p.n_splits > 1 ? launch_umma<FP8, kSplit>(a, p, s) : launch_umma<FP8, kWhole>(a, p, s);
 }
 
 }  // namespace
