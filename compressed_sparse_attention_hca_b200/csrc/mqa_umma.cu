@@ -108,6 +108,13 @@ __device__ __forceinline__ float warp_max_f32(float v) {
 }
 // Barrier of the 128 softmax threads (warps 0-3).
 __device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Producer / consumer halves of a named barrier over n threads.
+__device__ __forceinline__ void named_barrier_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void named_barrier_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
 
 // Warp reduce-scatter of 64 per-lane values (one per head): afterwards lane l
 // holds the sum (or max) over the warp's 32 lanes for heads 2l and 2l+1.
@@ -400,8 +407,18 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
     }
   };
   if constexpr (MODE != kWhole) {
-    // one split of many: O^T slabs -> the idle row tile as [slab][head][128 dims]
+    // one split of many: the unnormalised partial (m, l, o).  Warps 0-3 stage
+    // the O^T slabs in the idle row tile as [slab][head][128 dims] while warps
+    // 4-7 write the slabs already staged in 16-byte pieces (each warp store
+    // covers 512 contiguous bytes of one head); named barrier 2 + s marks
+    // slab s staged.
     float* stg = reinterpret_cast<float*>(KV);
+    if (tid < kHG) {
+      float* ml = plan_partial_ml(plan, a, bt, split, hg * kHG + tid);
+      const float m = ms.m_use[tid];
+      ml[0] = m == -INFINITY ? -INFINITY : m / kLog2e;  // natural-log domain
+      ml[1] = ms.l_run[tid];
+    }
     if (warp < 4) {
 #pragma unroll 1
       for (int sl = 0; sl < 4; ++sl) {
@@ -409,21 +426,19 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
         load_slab(sl, o);
 #pragma unroll
         for (int h = 0; h < kHG; ++h) stg[(sl * kHG + h) * 128 + tid] = o[h];
+        named_barrier_arrive(2 + sl, kThreads);
       }
-    }
-    __syncthreads();
-    // the unnormalised partial (m, l, o), written in 16-byte pieces so that
-    // each warp store covers 512 contiguous bytes
-    if (tid < kHG) {
-      float* ml = plan_partial_ml(plan, a, bt, split, hg * kHG + tid);
-      const float m = ms.m_use[tid];
-      ml[0] = m == -INFINITY ? -INFINITY : m / kLog2e;  // natural-log domain
-      ml[1] = ms.l_run[tid];
-    }
-    for (int q = tid; q < kHG * 128; q += kThreads) {
-      const int h = q >> 7, rem = q & 127, sl = rem >> 5, c = rem & 31;
-      const float4 v = *reinterpret_cast<const float4*>(stg + (sl * kHG + h) * 128 + 4 * c);
-      *reinterpret_cast<float4*>(plan_partial_o(plan, a, bt, split, hg * kHG + h) + 4 * rem) = v;
+    } else {
+      const int t = tid - 128;
+#pragma unroll 1
+      for (int sl = 0; sl < 4; ++sl) {
+        named_barrier_sync(2 + sl, kThreads);
+        for (int q = t; q < kHG * 32; q += 128) {
+          const int h = q >> 5, c = q & 31;
+          const float4 v = *reinterpret_cast<const float4*>(stg + (sl * kHG + h) * 128 + 4 * c);
+          *reinterpret_cast<float4*>(plan_partial_o(plan, a, bt, split, hg * kHG + h) + sl * 128 + 4 * c) = v;
+        }
+      }
     }
   } else {
     if (tid < kHG) {

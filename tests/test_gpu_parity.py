@@ -393,20 +393,24 @@ def test_mqa_sink_limits_cluster_split(orc):
 
 # ------------------------------------------ fused compressions + indexer
 
-@pytest.mark.parametrize("dt,B,T,E,k", [
-    (csa.IDX_NVFP4, 3, 1, 30000, 1024),   # one launch: the lead CTA compresses while its keys land
-    (csa.BF16, 2, 1, 20000, 512),         # one launch (BF16 keys)
-    (csa.IDX_NVFP4, 2, 1, 300, 128),      # tiny cache: the new row is in the lead slice's first stage
-    (csa.IDX_NVFP4, 2, 3, 5000, 512),     # two queries per CTA: the calls in order
+@pytest.mark.parametrize("dt,B,T,E,k,n_new", [
+    (csa.IDX_NVFP4, 3, 1, 30000, 1024, 1),   # one launch: the lead CTA compresses while its keys land
+    (csa.BF16, 2, 1, 20000, 512, 1),         # one launch (BF16 keys)
+    (csa.IDX_NVFP4, 2, 1, 300, 128, 1),      # tiny cache: the new row is in the lead slice's first stage
+    (csa.IDX_NVFP4, 2, 3, 5000, 512, 1),     # two queries per CTA: the calls in order
+    # two new rows 19967, 19968 across the boundary of 384-entry slices (2 requests on
+    # 148 SMs): two CTAs compress a key row each, the lead also both KV entries
+    (csa.IDX_NVFP4, 2, 1, 19969, 512, 2),
+    (csa.BF16, 2, 1, 19969, 512, 2),
 ])
-def test_compress_index_topk_equals_the_separate_calls(orc, dt, B, T, E, k):
+def test_compress_index_topk_equals_the_separate_calls(orc, dt, B, T, E, k, n_new):
     """The fused call writes the same key-cache and KV-cache bytes and selects
     the same indices as csa_compress (twice) followed by csa_index_topk, and
     the new key entry matches the oracle's compression."""
     m, dI, H, c = 4, 128, 64, 512
     g = W.generator(500 + E)
-    tok = W.compress_inputs(g, B, 2 * m, dI, m, True, torch.bfloat16)
-    ktok = W.compress_inputs(g, B, 2 * m, c, m, True, torch.bfloat16)
+    tok = W.compress_inputs(g, B, m * (n_new + 1), dI, m, True, torch.bfloat16)
+    ktok = W.compress_inputs(g, B, m * (n_new + 1), c, m, True, torch.bfloat16)
     if dt == csa.IDX_NVFP4:
         qI, qsf = W.nvfp4_rows(g, (B, T, H), dI)
         KI, ksf = W.nvfp4_rows(g, (B, E), dI)
@@ -417,21 +421,22 @@ def test_compress_index_topk_equals_the_separate_calls(orc, dt, B, T, E, k):
     wI = W.uniform(g, (B, T, H))
     kv = torch.randint(0, 256, (B, E, 608), generator=g, dtype=torch.uint8)
     q_pos = torch.tensor([[m * E - 1 - 13 * t for t in range(T)]] * B, dtype=torch.int64)
-    gt, gk, e0, tok0 = _cuda(tok), _cuda(ktok), E - 1, m * (E - 2)
+    gt, gk, e0 = _cuda(tok), _cuda(ktok), E - n_new
+    tok0 = m * (e0 - 1)
     cu = lambda v: None if v is None else v.to(DEV)  # noqa: E731
     # separate calls
     K1, S1, V1 = cu(KI).clone(), (cu(ksf).clone() if ksf is not None else None), cu(kv).clone()
-    csa.compress(gt["Ca"], gt["Za"], gt["Ba"], m, gt["Cb"], gt["Zb"], gt["Bb"], tok0=tok0, e0=e0, n_out=1,
+    csa.compress(gt["Ca"], gt["Za"], gt["Ba"], m, gt["Cb"], gt["Zb"], gt["Bb"], tok0=tok0, e0=e0, n_out=n_new,
                  out_dt=dt, out=K1, out_sf=S1, out_row0=e0)
-    csa.compress(gk["Ca"], gk["Za"], gk["Ba"], m, gk["Cb"], gk["Zb"], gk["Bb"], tok0=tok0, e0=e0, n_out=1,
+    csa.compress(gk["Ca"], gk["Za"], gk["Ba"], m, gk["Cb"], gk["Zb"], gk["Bb"], tok0=tok0, e0=e0, n_out=n_new,
                  out_dt=csa.KV_FP8MIX, out=V1, out_row0=e0)
     idx1 = csa.index_topk(cu(qI), cu(wI), K1, q_pos.to(DEV), m, k, dt=dt, qI_sf=cu(qsf), KI_sf=S1)
     # fused
     K2, S2, V2 = cu(KI).clone(), (cu(ksf).clone() if ksf is not None else None), cu(kv).clone()
     keys = csa.compress_job(gt["Ca"], gt["Za"], gt["Ba"], m, gt["Cb"], gt["Zb"], gt["Bb"], tok0=tok0, e0=e0,
-                            n_out=1, out=K2, out_sf=S2, out_dt=dt)
+                            n_out=n_new, out=K2, out_sf=S2, out_dt=dt)
     extra = csa.compress_job(gk["Ca"], gk["Za"], gk["Ba"], m, gk["Cb"], gk["Zb"], gk["Bb"], tok0=tok0, e0=e0,
-                             n_out=1, out=V2, out_dt=csa.KV_FP8MIX)
+                             n_out=n_new, out=V2, out_dt=csa.KV_FP8MIX)
     idx2 = csa.compress_index_topk(keys, cu(qI), cu(wI), K2, q_pos.to(DEV), m, k, extra_job=extra, dt=dt,
                                    qI_sf=cu(qsf), KI_sf=S2)
     torch.cuda.synchronize()
@@ -442,11 +447,11 @@ def test_compress_index_topk_equals_the_separate_calls(orc, dt, B, T, E, k):
     assert torch.equal(V1, V2)
     assert torch.equal(idx1, idx2)
     # the new key entry against the oracle's own compression (one quantisation step)
-    want = _oracle_compress(orc, tok, m, tok0, e0, 1)
+    want = _oracle_compress(orc, tok, m, tok0, e0, n_new)
     for b in range(B):
         if dt == csa.IDX_NVFP4:
-            codes = raw(K2[b, e0:e0 + 1])
-            sfr = orc.unblock_scales(raw(S2[b]), E, dI)[e0:e0 + 1]
+            codes = raw(K2[b, e0:e0 + n_new])
+            sfr = orc.unblock_scales(raw(S2[b]), E, dI)[e0:e0 + n_new]
             _check_nvfp4_rows(orc, codes, sfr, want[b], dI)
         else:
-            assert_close(f64(K2[b, e0:e0 + 1]), want[b], atol=1e-6, rtol=2.0 ** -8, what="fused bf16 key")
+            assert_close(f64(K2[b, e0:e0 + n_new]), want[b], atol=1e-6, rtol=2.0 ** -8, what="fused bf16 key")
