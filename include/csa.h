@@ -119,6 +119,12 @@ int64_t csa_nvfp4_key_scale_bytes(int64_t n_rows, int dim);
  *   C^Comp[i, d] = sum_j S^a_j C^a[m i + j, d] + sum_j S^b_j C^b[m (i-1) + j, d].
  * Entry 0 has no previous group (its b-branch is absent).  Cb == NULL (and
  * Zb, Bb ignored) selects the HCA form: one branch, no overlap.
+ * Arithmetic is fp32: per channel the largest logit M is found first, then
+ * exp(logit - M) and exp(logit - M) * C are summed over the positions (the
+ * current group's, then the previous group's) in blocks of 32, in order, and
+ * their ratio is converted once to out_dt.  Every call shape takes these
+ * steps in this order, so an entry's bytes do not depend on how many entries
+ * a call produces or on which call (csa_compress_index_topk too) writes it.
  *
  *   Ca, Cb, Za, Zb  [batch][in_batch_stride rows][dim] of in_dt (F32/BF16);
  *                   row r of request b holds absolute token tok0 + r, and
