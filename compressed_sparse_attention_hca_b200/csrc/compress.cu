@@ -4,8 +4,8 @@
 // Prefill form: one thread owns one (request, entry, 8-channel chunk) and
 // streams the entry's 2m (CSA) or m' (HCA) token rows of its chunk with
 // 16-byte loads: a pass over Z and the biases for the max logit, then a pass
-// over Z, C and the biases for the weighted sums (the second read of Z hits
-// L1/L2, so HBM still sees every input byte once).  Lanes that share an FP8
+// over Z, C and the biases for the weighted sums (the second read of Z and
+// the biases normally comes from L1/L2).  Lanes that share an FP8
 // scale block (8 lanes = 64 dims) or an FP4 block (2 lanes = 16 dims) reduce
 // their amax with warp shuffles and quantise in the epilogue.
 #include "compress_dev.cuh"

@@ -1017,6 +1017,9 @@ int index_tc_nq(int n_q) { return n_q >= 2 ? 2 : 1; }
 
 bool index_fusable(const IndexArgs& a) {
   if (!index_tc_eligible(a) || index_tc_nq(a.n_q) != 1 || a.n_entries < 1 || !fused_jobs_staged(a)) return false;
+  // a decode step closes a few groups; larger jobs run as separate launches
+  // (which also keeps the kernel's int scratch arithmetic far from overflow)
+  if (a.comp.n_out > 64 || a.comp2.n_out > 64 || a.comp.dim > 8192 || a.comp2.dim > 8192) return false;
   // the compress scratch must leave the ring at least one stage
   if (a.dt == CSA_IDX_NVFP4) return fused_scratch_stages(a, Nvf4Cfg<1>::STAGE) < Nvf4Cfg<1>::STAGES;
   return fused_scratch_stages(a, Bf16Cfg<1>::K_STAGE) < Bf16Cfg<1>::STAGES;
