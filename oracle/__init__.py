@@ -66,6 +66,8 @@ def _load():
         "orc_topk": (i32, [P, i64, i32, P]),
         "orc_visible_entries": (i64, [i64, i32, i64]),
         "orc_index_topk": (i32, [P, P, P, P, i32, i32, i32, i32, i64, i32, i32, i32, P, P]),
+        "orc_rmsnorm": (i32, [P, i64, i32, P, dbl, P]),
+        "orc_rope_tail": (i32, [P, i64, i32, i32, P, dbl, P]),
         "orc_attend": (None, [P, i32, i32, P, i64, P, dbl, P]),
         "orc_sparse_mqa": (i32, [P, P, i32, i64, P, i32, P, i64, P, P, i32, i32, P, dbl,
                                  i32, i32, i32, i32, P]),
@@ -233,6 +235,27 @@ def index_topk(qI, wI, KI, q_pos, m, k, round_bf16=True, want_scores=True):
     _check(_load().orc_index_topk(_p(qI), _p(wI), _p(KI), _p(q_pos), B, T, H, d, E, m, k,
                                   int(round_bf16), _p(scores), _p(idx)), "index_topk")
     return scores, idx
+
+
+def rmsnorm(x, g=None, eps=1e-6):
+    """RMSNorm of every row (last axis) of x, with per-channel weight g."""
+    x = _f64(x)
+    dim = x.shape[-1]
+    y = np.zeros_like(x)
+    _check(_load().orc_rmsnorm(_p(x), x.size // dim, dim, _p(_f64(g)), eps, _p(y)), "rmsnorm")
+    return y
+
+
+def rope_tail(x, pos, rope_dims=64, base=10000.0):
+    """Partial RoPE of every row (last axis) of x; pos holds one position per
+    row, numpy-broadcast to x.shape[:-1] (e.g. q_pos[..., None] for heads)."""
+    x = _f64(x)
+    dim = x.shape[-1]
+    n = x.size // dim
+    pos = np.ascontiguousarray(np.broadcast_to(np.asarray(pos, np.float64), x.shape[:-1])).reshape(n)
+    y = np.zeros_like(x)
+    _check(_load().orc_rope_tail(_p(x), n, dim, rope_dims, _p(pos), base, _p(y)), "rope_tail")
+    return y
 
 
 def attend(q, KV, sink, scale):

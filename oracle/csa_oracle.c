@@ -484,6 +484,51 @@ void orc_attend(const double* q, int n_h, int dim, const double* KV, int64_t n_r
     free(z);
 }
 
+/* ------------------------------------------------------------------------ */
+/* Q / KV-entry normalisation and partial RoPE ([P5] section 1.4 table:      */
+/* RMSNorm on every query head and on the one compressed KV head before the  */
+/* core attention; RoPE on the last 64 dims of q, of the KV rows and of the  */
+/* output o_{t,i}, the output at position -i; [P2] RoPE paragraph).  The     */
+/* pages give the operations, not their constants; the readings:             */
+/*   - RMSNorm of a row x of c values: y_d = g_d x_d / sqrt(mean_d x_d^2 +   */
+/*     eps), g a per-channel weight (all ones when g is NULL);               */
+/*   - RoPE on the last R dims: pair k (k < R/2) is the adjacent pair        */
+/*     (x_{c-R+2k}, x_{c-R+2k+1}), turned by the angle p * base^(-2k/R) as   */
+/*     the complex number x_{c-R+2k} + i x_{c-R+2k+1} times e^{i angle};     */
+/*     the first c-R dims are left as they are;                              */
+/*   - the output of the query at position t is turned at position -t, so   */
+/*     its RoPE dims carry positions relative to the query.                  */
+/* ------------------------------------------------------------------------ */
+int orc_rmsnorm(const double* x, int64_t n_rows, int dim, const double* g, double eps, double* y) {
+    if (n_rows < 0 || dim < 1 || !(eps >= 0.0)) return -1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const double* xr = x + r * dim;
+        double ss = 0.0;
+        for (int d = 0; d < dim; ++d) ss += xr[d] * xr[d];
+        double inv = 1.0 / sqrt(ss / dim + eps);
+        for (int d = 0; d < dim; ++d) y[r * dim + d] = xr[d] * inv * (g ? g[d] : 1.0);
+    }
+    return 0;
+}
+
+int orc_rope_tail(const double* x, int64_t n_rows, int dim, int rope_dims, const double* pos, double base,
+                  double* y) {
+    if (n_rows < 0 || rope_dims < 0 || rope_dims % 2 || rope_dims > dim || !(base > 0.0)) return -1;
+    for (int64_t r = 0; r < n_rows; ++r) {
+        const double* xr = x + r * dim;
+        double* yr = y + r * dim;
+        for (int d = 0; d < dim; ++d) yr[d] = xr[d];
+        for (int k = 0; k < rope_dims / 2; ++k) {
+            int i0 = dim - rope_dims + 2 * k;
+            double angle = pos[r] * pow(base, -2.0 * k / rope_dims);
+            double c = cos(angle), s = sin(angle);
+            yr[i0] = xr[i0] * c - xr[i0 + 1] * s;
+            yr[i0 + 1] = xr[i0] * s + xr[i0 + 1] * c;
+        }
+    }
+    return 0;
+}
+
 /* Gathers the attended rows of one query: `n_sel` entry rows listed in sel
  * (entries; -1 skipped), then the window tokens max(0,t-W+1)..t.  Returns the
  * row count, or -1 if a listed entry is not visible or a window token is not

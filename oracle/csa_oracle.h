@@ -43,6 +43,10 @@ int orc_index_topk(const double* qI, const double* wI, const double* KI, const i
                    int batch, int n_q, int n_hI, int dI, int64_t n_entries, int m, int k,
                    int round_bf16, double* scores_out, int32_t* idx_out);
 
+int orc_rmsnorm(const double* x, int64_t n_rows, int dim, const double* g, double eps, double* y);
+int orc_rope_tail(const double* x, int64_t n_rows, int dim, int rope_dims, const double* pos, double base,
+                  double* y);
+
 void orc_attend(const double* q, int n_h, int dim, const double* KV, int64_t n_rows,
                 const double* sink, double scale, double* out);
 int orc_sparse_mqa(const double* Q, const void* entries, int kv_dt, int64_t n_entries,
