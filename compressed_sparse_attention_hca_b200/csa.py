@@ -55,6 +55,7 @@ def load():
         "csa_nvfp4_key_scale_bytes": (i64, [i64, i32]),
         "csa_compress": (i32, [P, P, P, P, P, P, i32, i64, i64, i64, i64, i64, i32, i32, i32, P, P,
                                i64, i64, i32, P]),
+        "csa_rmsnorm_rope": (i32, [P, P, i64, i32, P, f32, P, i32, i32, i32, ctypes.c_double, i32, i32, P]),
         "csa_index_topk_workspace_size": (sz, [i32, i32, i64, i32, i32, i32, i32]),
         "csa_compress_index_topk": (i32, [ctypes.POINTER(CompressJob), ctypes.POINTER(CompressJob),
                                           P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32, i32,
@@ -151,6 +152,26 @@ def compress(Ca, Za, Ba, m, Cb=None, Zb=None, Bb=None, *, tok0=0, e0=0, n_out=No
                                tok0, rows, e0, n_out, dim, m, in_dt, _ptr(out), _ptr(out_sf), stride,
                                out_row0, out_dt, _stream()))
     return (out, out_sf) if out_dt == IDX_NVFP4 else out
+
+
+# ------------------------------------------------------ normalisation + partial RoPE
+
+def rmsnorm_rope(x, pos, *, g=None, eps=1e-6, rows_per_pos=1, pos_sign=1, rope_dims=64, base=10000.0,
+                 out=None, out_dt=None):
+    """RMSNorm (when g is given) and RoPE of the last rope_dims dims of every
+    row (last axis) of x; row r uses pos[r // rows_per_pos] (pos int64,
+    flattened).  out defaults to a new tensor of out_dt (x's dtype); out=x
+    works in place."""
+    _need_cuda(x, pos, g, out)
+    dim = x.shape[-1]
+    n_rows = x.numel() // dim
+    in_dt = _dt_of(x)
+    out_dt = in_dt if out_dt is None else out_dt
+    if out is None:
+        out = torch.empty(x.shape, device=x.device, dtype=torch.float32 if out_dt == F32 else torch.bfloat16)
+    _check(load().csa_rmsnorm_rope(_ptr(x), _ptr(out), n_rows, dim, _ptr(g), eps, _ptr(pos), rows_per_pos,
+                                   pos_sign, rope_dims, base, in_dt, out_dt, _stream()))
+    return out
 
 
 # ------------------------------------------------------------------- index top-k

@@ -160,7 +160,7 @@ csa_status_t csa_check_device_status(void) {
   return ok();
 }
 
-int csa_version(void) { return 200; }
+int csa_version(void) { return 201; }
 
 int64_t csa_row_bytes(csa_dtype_t dt, int dim) {
   if (dim <= 0) return -1;
@@ -187,6 +187,31 @@ csa_status_t csa_compress(const void* Ca, const void* Cb, const void* Za, const 
                                          dim, m, in_dt, out, out_sf, out_batch_stride, out_row0, out_dt, &a, &empty);
   if (st != CSA_OK || empty) return st;
   return cuda_status(csa::launch_compress(a, static_cast<cudaStream_t>(stream)), "csa_compress");
+}
+
+csa_status_t csa_rmsnorm_rope(const void* x, void* y, int64_t n_rows, int dim, const float* g, float eps,
+                              const int64_t* pos, int rows_per_pos, int pos_sign, int rope_dims, double base,
+                              csa_dtype_t in_dt, csa_dtype_t out_dt, void* stream) {
+  g_launches = 0;
+  REQUIRE(n_rows >= 0, "n_rows=%lld is negative", (long long)n_rows);
+  REQUIRE(dim >= 8 && dim % 8 == 0, "dim=%d must be a positive multiple of 8", dim);
+  REQUIRE(rope_dims >= 0 && rope_dims % 8 == 0 && rope_dims <= dim,
+          "rope_dims=%d must be a multiple of 8 in [0, dim=%d]", rope_dims, dim);
+  REQUIRE(rows_per_pos >= 1, "rows_per_pos=%d must be >= 1", rows_per_pos);
+  REQUIRE(pos_sign == 1 || pos_sign == -1, "pos_sign=%d must be +1 or -1", pos_sign);
+  REQUIRE(eps >= 0.f, "eps must be >= 0");
+  REQUIRE(base > 0.0, "base must be > 0");
+  REQUIRE(in_dt == CSA_F32 || in_dt == CSA_BF16, "in_dt must be CSA_F32 or CSA_BF16");
+  REQUIRE(out_dt == CSA_F32 || out_dt == CSA_BF16, "out_dt must be CSA_F32 or CSA_BF16");
+  REQUIRE(x != y || in_dt == out_dt, "in place (y == x) needs in_dt == out_dt");
+  if (n_rows == 0) return ok();
+  REQUIRE_PTR(x);
+  REQUIRE_PTR(y);
+  if (rope_dims > 0) REQUIRE(pos != nullptr, "pos is NULL with rope_dims > 0");
+  REQUIRE(n_rows <= ((int64_t)1 << 40), "n_rows=%lld too large", (long long)n_rows);
+  csa::NormRopeArgs a{x, y, n_rows, dim, rows_per_pos, pos_sign, rope_dims, g, eps, pos, base, (int)in_dt,
+                      (int)out_dt};
+  return cuda_status(csa::launch_norm_rope(a, static_cast<cudaStream_t>(stream)), "csa_rmsnorm_rope");
 }
 
 size_t csa_index_topk_workspace_size(int batch, int n_q, int64_t n_entries, int k, int n_heads,

@@ -171,6 +171,19 @@ struct CompressArgs {
 };
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s);
 
+struct NormRopeArgs {
+  const void* x;
+  void* y;
+  int64_t n_rows;
+  int dim, rows_per_pos, pos_sign, rope_dims;
+  const float* g;
+  float eps;
+  const int64_t* pos;
+  double base;
+  int in_dt, out_dt;
+};
+cudaError_t launch_norm_rope(const NormRopeArgs& a, cudaStream_t s);
+
 struct IndexArgs {
   const void *qI, *qI_sf;
   const float* wI;

@@ -153,6 +153,37 @@ csa_status_t csa_compress(const void* Ca, const void* Cb, const void* Za, const 
                           void* stream);
 
 /*
+ * csa_rmsnorm_rope -- Q / KV-entry normalisation and partial RoPE ([P5] 1.4
+ * table: RMSNorm on every query head and on the one compressed KV head
+ * before the core attention, RoPE on the last 64 dims of q, of the KV rows
+ * and of the output, the output at position -i; [P2] RoPE paragraph), in one
+ * pass over rows of dim values:
+ *   g != NULL:  y = rope(g * x / sqrt(mean_d x_d^2 + eps))
+ *   g == NULL:  y = rope(x)            (rotation only: e.g. an output at -t)
+ * rope turns the last rope_dims dims of a row: pair k < rope_dims/2, the
+ * adjacent dims (dim - rope_dims + 2k, dim - rope_dims + 2k + 1), by the
+ * angle pos_sign * p * base^(-2k/rope_dims) (as the complex number
+ * x_{2k} + i x_{2k+1} times e^{i angle}); p = pos[r / rows_per_pos] for row r.
+ * The first dim - rope_dims dims are only normalised.  Normalisation runs in
+ * fp32; angles are reduced in fp64, so large positions keep their accuracy.
+ *
+ *   x, y          [n_rows][dim] of in_dt / out_dt (CSA_F32 or CSA_BF16),
+ *                 16-byte aligned.  y == x (in place) needs in_dt == out_dt;
+ *                 otherwise y must not overlap x.
+ *   g             [dim] fp32 per-channel weight, or NULL (no normalisation).
+ *   pos           [ceil(n_rows / rows_per_pos)] int64 positions (e.g. the
+ *                 query positions with rows_per_pos = n_heads, or the
+ *                 position of each cache row); may be NULL when rope_dims = 0.
+ *   pos_sign      +1, or -1 to turn rows back (the output of the query at t).
+ * Limits: dim a positive multiple of 8; rope_dims a multiple of 8 in
+ * [0, dim]; rows_per_pos >= 1; eps >= 0; base > 0.  Errors:
+ * CSA_ERR_INVALID_ARG before any launch.
+ */
+csa_status_t csa_rmsnorm_rope(const void* x, void* y, int64_t n_rows, int dim, const float* g, float eps,
+                              const int64_t* pos, int rows_per_pos, int pos_sign, int rope_dims, double base,
+                              csa_dtype_t in_dt, csa_dtype_t out_dt, void* stream);
+
+/*
  * csa_index_topk -- Lightning Indexer fused with the top-k selector ([P5] 1.2
  * Step 2; [P1] eq. 8; BF16 scores [P5] 6.2).
  *

@@ -24,7 +24,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_row_bytes():
-    assert csa.load().csa_version() == 200
+    assert csa.load().csa_version() == 201
     assert csa.row_bytes(csa.F32, 512) == 2048
     assert csa.row_bytes(csa.BF16, 512) == 1024
     assert csa.row_bytes(csa.KV_FP8MIX, 512) == 608
@@ -138,3 +138,29 @@ def test_compress_index_topk_rejects_bad_arguments():
     # the extra job must not write the indexer's cache
     assert call(job(), extra=job()) == INVALID and "extra" in _err()
     assert call(job(), dim=48) == INVALID
+
+
+def test_rmsnorm_rope_rejects_bad_arguments():
+    lib = csa.load()
+    F32, BF16 = csa.F32, csa.BF16
+
+    def call(x=A, y=P(8192), n=4, dim=512, g=A, eps=1e-6, pos=A, rpp=1, sign=1, rope=64, base=10000.0,
+             idt=BF16, odt=BF16):
+        return lib.csa_rmsnorm_rope(x, y, n, dim, g, eps, pos, rpp, sign, rope, base, idt, odt, None)
+
+    assert call(n=0) == 0                        # nothing to do
+    assert call(n=-1) == INVALID
+    assert call(dim=500) == INVALID              # not a multiple of 8
+    assert call(rope=60) == INVALID              # rope_dims not a multiple of 8
+    assert call(dim=64, rope=72) == INVALID      # rope_dims > dim
+    assert call(rpp=0) == INVALID
+    assert call(sign=2) == INVALID
+    assert call(eps=-1.0) == INVALID
+    assert call(base=0.0) == INVALID
+    assert call(idt=csa.KV_FP8MIX) == INVALID
+    assert call(odt=csa.IDX_NVFP4) == INVALID
+    assert call(y=A, idt=F32, odt=BF16) == INVALID   # in place needs one dtype
+    assert call(x=P(4100)) == INVALID            # misaligned
+    assert call(x=None) == INVALID
+    assert call(pos=None) == INVALID             # rotation needs positions
+    assert "pos" in csa.load().csa_last_error().decode()

@@ -455,3 +455,52 @@ def test_compress_index_topk_equals_the_separate_calls(orc, dt, B, T, E, k, n_ne
             _check_nvfp4_rows(orc, codes, sfr, want[b], dI)
         else:
             assert_close(f64(K2[b, e0:e0 + n_new]), want[b], atol=1e-6, rtol=2.0 ** -8, what="fused bf16 key")
+
+
+# ------------------------------------------------- Q / KV normalisation + partial RoPE
+
+@pytest.mark.parametrize("case", [
+    # rows, dim, rope_dims, rows_per_pos, in, out, with g, pos_sign, max position
+    (4 * 128, 512, 64, 128, torch.bfloat16, csa.BF16, True, 1, 1 << 20),   # decode queries: 4 x 128 heads
+    (37, 512, 64, 1, torch.bfloat16, csa.BF16, True, 1, 262143),           # ragged cache rows
+    (45, 128, 64, 1, torch.float32, csa.F32, False, -1, 1 << 20),          # rotation only, turned back
+    (16, 448, 0, 1, torch.float32, csa.BF16, True, 1, 10),                 # normalisation only
+    (8, 64, 64, 4, torch.bfloat16, csa.F32, True, 1, 77),                  # every dim rotated
+])
+def test_rmsnorm_rope_matches_oracle(orc, case):
+    n, dim, rope, rpp, dtype, out_dt, with_g, sign, pmax = case
+    g = torch.Generator().manual_seed(900 + n + dim)
+    x = (torch.randn(n, dim, generator=g) * (1 + 3 * torch.rand(n, 1, generator=g))).to(dtype)
+    w = torch.randn(dim, generator=g) if with_g else None
+    pos = torch.randint(0, pmax + 1, ((n + rpp - 1) // rpp,), generator=g, dtype=torch.int64)
+    pos[0] = pmax
+    y = csa.rmsnorm_rope(x.to(DEV), pos.to(DEV), g=None if w is None else w.to(DEV), eps=1e-6, rows_per_pos=rpp,
+                         pos_sign=sign, rope_dims=rope, out_dt=out_dt)
+    torch.cuda.synchronize()
+    want = f64(x)
+    if w is not None:
+        want = orc.rmsnorm(want, f64(w), 1e-6)
+    p_rows = np.repeat(f64(pos), rpp)[:n] * sign
+    want = orc.rope_tail(want, p_rows, rope_dims=rope)
+    got = f64(y)
+    if out_dt == csa.F32:
+        assert_close(got, want, atol=2e-5, rtol=2e-5, what="rmsnorm_rope f32")
+    else:
+        assert_close(got, want, atol=1e-5, rtol=2.0 ** -8, what="rmsnorm_rope bf16")
+
+
+def test_rmsnorm_rope_in_place_and_turn_back():
+    """In place on bf16 rows; turning f32 rows at p and then at -p returns them."""
+    g = torch.Generator().manual_seed(77)
+    x = torch.randn(64, 512, generator=g).to(torch.bfloat16).to(DEV)
+    pos = torch.randint(0, 1 << 20, (64,), generator=g, dtype=torch.int64).to(DEV)
+    w = torch.randn(512, generator=g).to(DEV)
+    ref = csa.rmsnorm_rope(x, pos, g=w)
+    y = x.clone()
+    csa.rmsnorm_rope(y, pos, g=w, out=y)
+    torch.cuda.synchronize()
+    assert torch.equal(y, ref)
+    z = torch.randn(64, 512, generator=g).to(DEV)
+    back = csa.rmsnorm_rope(csa.rmsnorm_rope(z, pos), pos, pos_sign=-1)
+    torch.cuda.synchronize()
+    assert (back - z).abs().max().item() < 1e-5
