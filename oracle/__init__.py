@@ -68,6 +68,7 @@ def _load():
         "orc_index_topk": (i32, [P, P, P, P, i32, i32, i32, i32, i64, i32, i32, i32, P, P]),
         "orc_rmsnorm": (i32, [P, i64, i32, P, dbl, P]),
         "orc_rope_tail": (i32, [P, i64, i32, i32, P, dbl, P]),
+        "orc_grouped_out_proj": (i32, [P, i32, i32, i32, i32, i32, P, P, i32, P]),
         "orc_attend": (None, [P, i32, i32, P, i64, P, dbl, P]),
         "orc_sparse_mqa": (i32, [P, P, i32, i64, P, i32, P, i64, P, P, i32, i32, P, dbl,
                                  i32, i32, i32, i32, P]),
@@ -256,6 +257,17 @@ def rope_tail(x, pos, rope_dims=64, base=10000.0):
     y = np.zeros_like(x)
     _check(_load().orc_rope_tail(_p(x), n, dim, rope_dims, _p(pos), base, _p(y)), "rope_tail")
     return y
+
+
+def grouped_out_proj(O, Wg, Wo):
+    """O [T, n_h, c]; Wg [g, n_h/g * c, d_g]; Wo [g * d_g, d] -> Y [T, d]."""
+    O, Wg, Wo = _f64(O), _f64(Wg), _f64(Wo)
+    T, n_h, c = O.shape
+    g, _, d_g = Wg.shape
+    d = Wo.shape[1]
+    Y = np.zeros((T, d), np.float64)
+    _check(_load().orc_grouped_out_proj(_p(O), T, n_h, c, g, d_g, _p(Wg), _p(Wo), d, _p(Y)), "grouped_out_proj")
+    return Y
 
 
 def attend(q, KV, sink, scale):

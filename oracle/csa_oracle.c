@@ -529,6 +529,42 @@ int orc_rope_tail(const double* x, int64_t n_rows, int dim, int rope_dims, const
     return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Grouped output projection ([P5] section 1.2 Step 3): the n_h head outputs */
+/* of a query are split into g groups of n_h/g consecutive heads; group j's  */
+/* concatenated outputs (n_h/g * c values) are projected to d_g values by    */
+/* its own matrix W_j, and the g results, concatenated, are projected to d   */
+/* values by W_O.  Readings: plain linear maps, no bias, no activation      */
+/* between the two projections, heads grouped in index order.               */
+/*   O [T][n_h][c], Wg [g][n_h/g * c][d_g], Wo [g * d_g][d], Y [T][d].       */
+/* ------------------------------------------------------------------------ */
+int orc_grouped_out_proj(const double* O, int T, int n_h, int c, int g, int d_g, const double* Wg,
+                         const double* Wo, int d, double* Y) {
+    if (T < 0 || n_h < 1 || c < 1 || g < 1 || n_h % g || d_g < 1 || d < 1) return -1;
+    const int64_t in_g = (int64_t)(n_h / g) * c;
+    double* z = (double*)malloc(sizeof(double) * (size_t)g * d_g);
+    if (!z) return -2;
+    for (int t = 0; t < T; ++t) {
+        const double* ot = O + (int64_t)t * n_h * c;
+        for (int j = 0; j < g; ++j) {
+            const double* x = ot + (int64_t)j * in_g;       /* heads j*n_h/g .. of query t */
+            const double* w = Wg + (int64_t)j * in_g * d_g;
+            for (int e = 0; e < d_g; ++e) {
+                double acc = 0.0;
+                for (int64_t i = 0; i < in_g; ++i) acc += x[i] * w[i * d_g + e];
+                z[(int64_t)j * d_g + e] = acc;
+            }
+        }
+        for (int o = 0; o < d; ++o) {
+            double acc = 0.0;
+            for (int64_t i = 0; i < (int64_t)g * d_g; ++i) acc += z[i] * Wo[i * d + o];
+            Y[(int64_t)t * d + o] = acc;
+        }
+    }
+    free(z);
+    return 0;
+}
+
 /* Gathers the attended rows of one query: `n_sel` entry rows listed in sel
  * (entries; -1 skipped), then the window tokens max(0,t-W+1)..t.  Returns the
  * row count, or -1 if a listed entry is not visible or a window token is not

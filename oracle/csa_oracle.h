@@ -47,6 +47,9 @@ int orc_rmsnorm(const double* x, int64_t n_rows, int dim, const double* g, doubl
 int orc_rope_tail(const double* x, int64_t n_rows, int dim, int rope_dims, const double* pos, double base,
                   double* y);
 
+int orc_grouped_out_proj(const double* O, int T, int n_h, int c, int g, int d_g, const double* Wg,
+                         const double* Wo, int d, double* Y);
+
 void orc_attend(const double* q, int n_h, int dim, const double* KV, int64_t n_rows,
                 const double* sink, double scale, double* out);
 int orc_sparse_mqa(const double* Q, const void* entries, int kv_dt, int64_t n_entries,
