@@ -69,6 +69,7 @@ def _load():
         "orc_rmsnorm": (i32, [P, i64, i32, P, dbl, P]),
         "orc_rope_tail": (i32, [P, i64, i32, i32, P, dbl, P]),
         "orc_grouped_out_proj": (i32, [P, i32, i32, i32, i32, i32, P, P, i32, P]),
+        "orc_gather_paged": (i32, [P, i64, i64, i32, P, i32, i32, i64, P]),
         "orc_attend": (None, [P, i32, i32, P, i64, P, dbl, P]),
         "orc_sparse_mqa": (i32, [P, P, i32, i64, P, i32, P, i64, P, P, i32, i32, P, dbl,
                                  i32, i32, i32, i32, P]),
@@ -268,6 +269,19 @@ def grouped_out_proj(O, Wg, Wo):
     Y = np.zeros((T, d), np.float64)
     _check(_load().orc_grouped_out_proj(_p(O), T, n_h, c, g, d_g, _p(Wg), _p(Wo), d, _p(Y)), "grouped_out_proj")
     return Y
+
+
+def gather_paged(pool, table, n_entries):
+    """pool [n_pages, per_page, row_bytes] uint8; table [B, max_pages] int32 ->
+    the contiguous cache [B, n_entries, row_bytes] uint8."""
+    pool = np.ascontiguousarray(pool, dtype=np.uint8)
+    table = _c(table, np.int32)
+    n_pages, per_page, rb = pool.shape
+    B, max_pages = table.shape
+    out = np.zeros((B, n_entries, rb), np.uint8)
+    _check(_load().orc_gather_paged(_p(pool), n_pages, rb, per_page, _p(table), max_pages, B, n_entries, _p(out)),
+           "gather_paged")
+    return out
 
 
 def attend(q, KV, sink, scale):

@@ -565,6 +565,30 @@ int orc_grouped_out_proj(const double* O, int T, int n_h, int c, int g, int d_g,
     return 0;
 }
 
+/* ------------------------------------------------------------------------ */
+/* Paged compressed cache ([P2] cache paragraph; [P5] section 7): the cache */
+/* of every request is stored in fixed pages of lcm(m, m') = 128 tokens,    */
+/* i.e. 32 CSA entries or 1 HCA entry per page, taken from a shared pool    */
+/* through a per-request block table.  Reading: entry i of request b lives  */
+/* in slot i % per_page of pool page table[b][i / per_page].  This gathers  */
+/* the first n_entries entries of every request into a contiguous           */
+/* [batch][n_entries] cache (rows of row_bytes bytes); -1 when a table slot */
+/* is out of the pool.                                                       */
+/* ------------------------------------------------------------------------ */
+int orc_gather_paged(const uint8_t* pool, int64_t n_pages, int64_t row_bytes, int per_page,
+                     const int32_t* table, int max_pages, int batch, int64_t n_entries, uint8_t* out) {
+    if (n_pages < 0 || row_bytes < 1 || per_page < 1 || max_pages < 0 || batch < 0 || n_entries < 0) return -1;
+    if (n_entries > (int64_t)max_pages * per_page) return -1;
+    for (int b = 0; b < batch; ++b)
+        for (int64_t i = 0; i < n_entries; ++i) {
+            int32_t pg = table[(int64_t)b * max_pages + i / per_page];
+            if (pg < 0 || pg >= n_pages) return -1;
+            memcpy(out + ((int64_t)b * n_entries + i) * row_bytes,
+                   pool + ((int64_t)pg * per_page + i % per_page) * row_bytes, (size_t)row_bytes);
+        }
+    return 0;
+}
+
 /* Gathers the attended rows of one query: `n_sel` entry rows listed in sel
  * (entries; -1 skipped), then the window tokens max(0,t-W+1)..t.  Returns the
  * row count, or -1 if a listed entry is not visible or a window token is not

@@ -50,6 +50,9 @@ int orc_rope_tail(const double* x, int64_t n_rows, int dim, int rope_dims, const
 int orc_grouped_out_proj(const double* O, int T, int n_h, int c, int g, int d_g, const double* Wg,
                          const double* Wo, int d, double* Y);
 
+int orc_gather_paged(const uint8_t* pool, int64_t n_pages, int64_t row_bytes, int per_page,
+                     const int32_t* table, int max_pages, int batch, int64_t n_entries, uint8_t* out);
+
 void orc_attend(const double* q, int n_h, int dim, const double* KV, int64_t n_rows,
                 const double* sink, double scale, double* out);
 int orc_sparse_mqa(const double* Q, const void* entries, int kv_dt, int64_t n_entries,
