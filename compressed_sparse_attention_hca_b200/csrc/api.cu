@@ -140,7 +140,7 @@ static csa_status_t check_index(const void* qI, const void* qI_sf, const float* 
   REQUIRE(ws_bytes >= need, "workspace too small: %zu < %zu bytes", ws_bytes, need);
   REQUIRE_PTR(ws);
   *args = csa::IndexArgs{qI, qI_sf, wI, KI, KI_sf, q_pos, batch, n_q, n_entries, m, n_heads, dim, k,
-                         (int)dt, idx_out, scores_out, ws, ws_bytes, 0, csa::CompressArgs{}};
+                         (int)dt, idx_out, scores_out, ws, ws_bytes, 0, csa::CompressArgs{}, csa::CompressArgs{}};
   return ok();
 }
 
