@@ -41,46 +41,70 @@ __device__ __forceinline__ void nr_store8(void* base, int dt, int64_t elem, cons
   }
 }
 
+// Grid-stride over rows, one warp per row at a time.  A lane owns chunks
+// lane, lane + 32, ... of every row, so the frequencies of its (at most
+// kMaxOwn) rotated chunks are computed once, in fp64, before the row loop.
+// Per pair and row: angle = p * theta in fp64, reduced to [-pi, pi] by two-
+// constant Cody-Waite subtraction of the nearest multiple of 2 pi, then
+// sincosf on the fp32 residual.
+constexpr int kMaxOwn = 2;
+
 __global__ void __launch_bounds__(256) norm_rope_kernel(NormRopeArgs a) {
-  const int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
-  if (r >= a.n_rows) return;  // a whole warp per row: the warp leaves together
-  const int nch = a.dim / 8;
-  const int64_t row = r * a.dim;
-  float inv = 1.f;
-  if (a.g != nullptr) {
-    float ss = 0.f;
+  const int64_t warp0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t n_warps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int nch = a.dim / 8, d_rope = a.dim - a.rope_dims;
+  double theta[kMaxOwn][4];
+  int own = 0;
+  for (int c = lane; c < nch && own < kMaxOwn; c += 32) {
+    if (8 * c < d_rope) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) theta[own][j] = pow(a.base, -2.0 * ((8 * c - d_rope) / 2 + j) / a.rope_dims);
+    ++own;
+  }
+  const bool table = (nch - d_rope / 8 + 31) / 32 <= kMaxOwn;  // every lane's rotated chunks fit
+  constexpr double kTwoPiHi = 6.283185307179586232, kTwoPiLo = 2.4492935982947064e-16, kInvTwoPi = 0.15915494309189535;
+  for (int64_t r = warp0; r < a.n_rows; r += n_warps) {
+    const int64_t row = r * a.dim;
+    float inv = 1.f;
+    if (a.g != nullptr) {
+      float ss = 0.f;
+      for (int c = lane; c < nch; c += 32) {
+        float v[8];
+        nr_load8(a.x, a.in_dt, row + 8 * c, v);
+#pragma unroll
+        for (int q = 0; q < 8; ++q) ss = fmaf(v[q], v[q], ss);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      inv = 1.f / sqrtf(ss / (float)a.dim + a.eps);
+    }
+    const double p = a.rope_dims > 0 ? (double)a.pos[r / a.rows_per_pos] * (double)a.pos_sign : 0.0;
+    int slot = 0;
     for (int c = lane; c < nch; c += 32) {
       float v[8];
       nr_load8(a.x, a.in_dt, row + 8 * c, v);
+      if (a.g != nullptr) {
 #pragma unroll
-      for (int q = 0; q < 8; ++q) ss = fmaf(v[q], v[q], ss);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    inv = 1.f / sqrtf(ss / (float)a.dim + a.eps);
-  }
-  const int d_rope = a.dim - a.rope_dims;
-  const double p = a.rope_dims > 0 ? (double)a.pos[r / a.rows_per_pos] * (double)a.pos_sign : 0.0;
-  for (int c = lane; c < nch; c += 32) {
-    float v[8];
-    nr_load8(a.x, a.in_dt, row + 8 * c, v);
-    if (a.g != nullptr) {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) v[q] = v[q] * inv * a.g[8 * c + q];
-    }
-    if (8 * c >= d_rope) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int k = (8 * c - d_rope) / 2 + j;
-        double sd, cd;
-        sincos(p * pow(a.base, -2.0 * k / a.rope_dims), &sd, &cd);
-        const float cs = (float)cd, sn = (float)sd, x0 = v[2 * j], x1 = v[2 * j + 1];
-        v[2 * j] = x0 * cs - x1 * sn;
-        v[2 * j + 1] = x0 * sn + x1 * cs;
+        for (int q = 0; q < 8; ++q) v[q] = v[q] * inv * a.g[8 * c + q];
       }
+      if (8 * c >= d_rope) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const double th = table ? theta[slot][j] : pow(a.base, -2.0 * ((8 * c - d_rope) / 2 + j) / a.rope_dims);
+          const double ang = p * th;
+          const double n = rint(ang * kInvTwoPi);
+          const float red = (float)fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, ang));
+          float sn, cs;
+          sincosf(red, &sn, &cs);
+          const float x0 = v[2 * j], x1 = v[2 * j + 1];
+          v[2 * j] = x0 * cs - x1 * sn;
+          v[2 * j + 1] = x0 * sn + x1 * cs;
+        }
+        if (table) ++slot;
+      }
+      nr_store8(a.y, a.out_dt, row + 8 * c, v);
     }
-    nr_store8(a.y, a.out_dt, row + 8 * c, v);
   }
 }
 
@@ -88,7 +112,9 @@ __global__ void __launch_bounds__(256) norm_rope_kernel(NormRopeArgs a) {
 
 cudaError_t launch_norm_rope(const NormRopeArgs& a, cudaStream_t s) {
   if (a.n_rows == 0) return cudaSuccess;
-  const int64_t blocks = (a.n_rows * 32 + 255) / 256;
+  // one wave of 8-warp blocks (rows beyond it loop), at most one block per 8 rows
+  int64_t blocks = (a.n_rows + 7) / 8;
+  if (blocks > 148 * 8) blocks = 148 * 8;
   norm_rope_kernel<<<(unsigned)blocks, 256, 0, s>>>(a);
   ++launch_counter();
   return cudaGetLastError();
