@@ -1,9 +1,10 @@
 // norm_rope.cu -- Q / KV-entry RMSNorm and partial RoPE ("DeepSeek-V4 内部机制"
-// 1.4 table; admirer.cn article, RoPE paragraph): one warp per row, two passes
-// over the row (sum of squares, then normalise, turn the last rope_dims dims
-// and store), 16-byte loads and stores.  The row is read twice; the second
-// read comes from L1/L2.  Angles are formed and reduced in fp64 (a position
-// of 10^6 times a frequency near 1 leaves fp32 no fractional bits).
+// 1.4 table; admirer.cn article, RoPE paragraph): a warp per row at a time,
+// two passes over the row (sum of squares, then normalise, turn the last
+// rope_dims dims and store), 16-byte loads and stores; the second read of a
+// row comes from L1/L2.  Angles are formed and reduced to [-pi, pi] in fp64
+// (a position of 10^6 times a frequency near 1 leaves fp32 no fractional
+// bits); the sine and cosine of the reduced angle are taken in fp32.
 #include "csa_internal.cuh"
 
 namespace csa {
