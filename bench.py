@@ -224,10 +224,9 @@ class Step:
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the
-# dominant kernel, from the ncu captures summarised in profiles/
-# (ncu_index_nvf4_csa_decode_1m_mixed.md, ncu_index_bf16_csa_decode_bf16.md).  A
-# change to that kernel makes the figure stale: it is then removed until the next
-# capture.
+# dominant kernel, measured by an ncu capture of that kernel on the same
+# workload.  A change to that kernel makes the figure stale: it is then removed
+# until the next capture.
 NCU_TRAFFIC = {"csa_decode_1m_mixed": 78_227_200, "csa_decode_bf16": 138_577_920}
 
 

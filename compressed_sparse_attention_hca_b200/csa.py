@@ -57,6 +57,7 @@ def load():
                                i64, i64, i32, P]),
         "csa_rmsnorm_rope": (i32, [P, P, i64, i32, P, f32, P, i32, i32, i32, ctypes.c_double, i32, i32, P]),
         "csa_index_topk_workspace_size": (sz, [i32, i32, i64, i32, i32, i32, i32]),
+        "csa_index_topk_plan": (i32, [i32, i32, i64, i32, i32, i32, i32, P]),
         "csa_compress_index_topk": (i32, [ctypes.POINTER(CompressJob), ctypes.POINTER(CompressJob),
                                           P, P, P, P, P, P, i32, i32, i64, i32, i32, i32, i32, i32,
                                           P, P, P, sz, P]),
@@ -180,6 +181,15 @@ def index_topk_workspace_size(batch, n_q, n_entries, k, n_heads, dim, dt):
     return int(load().csa_index_topk_workspace_size(batch, n_q, n_entries, k, n_heads, dim, dt))
 
 
+def index_topk_plan(batch, n_q, n_entries, k, n_heads, dim, dt):
+    """How csa_index_topk splits a call of this shape on the current device:
+    dict(slice_len, n_slices, coop, tensor_core, ring_stages, tiles_per_stage)."""
+    out = (ctypes.c_int32 * 6)()
+    _check(load().csa_index_topk_plan(batch, n_q, n_entries, k, n_heads, dim, dt, ctypes.cast(out, ctypes.c_void_p)))
+    keys = ("slice_len", "n_slices", "coop", "tensor_core", "ring_stages", "tiles_per_stage")
+    return dict(zip(keys, [int(v) for v in out]))
+
+
 def index_topk(qI, wI, KI, q_pos, m, k, *, dt=None, qI_sf=None, KI_sf=None, n_heads=None,
                scores=False, idx_out=None, ws=None):
     """Lightning indexer + top-k.  qI [B, T, H, d] (or NVFP4 codes [B, T, H, d/2]),
@@ -233,11 +243,11 @@ def compress_job(Ca, Za, Ba, m, Cb=None, Zb=None, Bb=None, *, tok0, e0, n_out, o
 
 
 def compress_index_topk(keys_job, qI, wI, KI, q_pos, m, k, *, extra_job=None, dt=None, qI_sf=None, KI_sf=None,
-                        idx_out=None, ws=None):
+                        idx_out=None, ws=None, scores=False):
     """Run the compressor job `keys_job` (index keys into KI / KI_sf) and, if
     given, `extra_job` (e.g. the KV cache), then index + top-k over KI: one
     launch when the tensor-core indexer takes the shape.  Returns idx
-    [B, T, k] int32."""
+    [B, T, k] int32 (and the score tensor when scores=True)."""
     _need_cuda(qI, wI, KI, q_pos, qI_sf, KI_sf)
     if dt is None:
         dt = IDX_NVFP4 if qI.dtype == torch.uint8 else _dt_of(qI)
@@ -247,15 +257,18 @@ def compress_index_topk(keys_job, qI, wI, KI, q_pos, m, k, *, extra_job=None, dt
     dev = qI.device
     if idx_out is None:
         idx_out = torch.empty(B, T, k, device=dev, dtype=torch.int32)
+    sc = None
+    if scores:
+        sc = torch.empty(B, T, E, device=dev, dtype=torch.float32 if dt == F32 else torch.bfloat16)
     need = index_topk_workspace_size(B, T, E, k, H, dim, dt)
     if ws is None or ws.numel() < need:
         ws = torch.zeros(need, device=dev, dtype=torch.uint8)  # zero before first use
     _check(load().csa_compress_index_topk(ctypes.byref(keys_job),
                                           ctypes.byref(extra_job) if extra_job is not None else None,
                                           _ptr(qI), _ptr(qI_sf), _ptr(wI), _ptr(KI), _ptr(KI_sf), _ptr(q_pos), B, T,
-                                          E, m, H, dim, k, dt, _ptr(idx_out), None, _ptr(ws), ws.numel(),
+                                          E, m, H, dim, k, dt, _ptr(idx_out), _ptr(sc), _ptr(ws), ws.numel(),
                                           _stream()))
-    return idx_out
+    return (idx_out, sc) if scores else idx_out
 
 
 # -------------------------------------------------------------------- attention

@@ -156,7 +156,13 @@ csa_status_t csa_check_device_status(void) {
   if (e != cudaSuccess) return cuda_status(e, "csa_check_device_status");
   const unsigned int st = csa::take_status_indexer_tc() | csa::take_status_mqa_umma();
   if (st & 2u) return fail(CSA_ERR_CUDA, "csa_check_device_status: status word unreadable");
-  if (st & 1u) return fail(CSA_ERR_TIMEOUT, "a kernel pipeline wait timed out; its results are invalid");
+  if (st & 1u) {
+    // a selection that gave up may have left counters set in the built-in
+    // scratch of csa_index_topk_noalloc: zero it (caller workspaces are the
+    // caller's to zero)
+    csa::reset_static_scratch();
+    return fail(CSA_ERR_TIMEOUT, "a kernel pipeline wait timed out; its results are invalid");
+  }
   return ok();
 }
 
@@ -219,6 +225,19 @@ size_t csa_index_topk_workspace_size(int batch, int n_q, int64_t n_entries, int 
   if (batch <= 0 || n_q <= 0 || n_entries <= 0 || k <= 0) return 256;
   size_t s = csa::index_topk_workspace(batch, n_q, n_entries, k, n_heads, dim, (int)dt);
   return s < 256 ? 256 : s;
+}
+
+csa_status_t csa_index_topk_plan(int batch, int n_q, int64_t n_entries, int k, int n_heads, int dim,
+                                 csa_dtype_t dt, int32_t* out) {
+  REQUIRE(out != nullptr, "out is NULL");
+  REQUIRE(batch >= 1 && n_q >= 1 && n_entries >= 1, "batch, n_q and n_entries must be >= 1");
+  REQUIRE(n_entries <= (int64_t)1 << 30, "n_entries=%lld too large", (long long)n_entries);
+  REQUIRE(k >= 1 && k <= 2048, "k=%d out of range [1, 2048]", k);
+  REQUIRE(n_heads >= 1 && n_heads <= 128, "n_heads=%d out of range [1, 128]", n_heads);
+  REQUIRE(dim >= 32 && dim <= 256 && dim % 32 == 0, "dim=%d must be a multiple of 32 in [32, 256]", dim);
+  REQUIRE(dt == CSA_F32 || dt == CSA_BF16 || dt == CSA_IDX_NVFP4, "dt must be F32, BF16 or IDX_NVFP4");
+  csa::index_topk_plan_info(batch, n_q, n_entries, k, n_heads, dim, (int)dt, out);
+  return ok();
 }
 
 csa_status_t csa_index_topk(const void* qI, const void* qI_sf, const float* wI, const void* KI,

@@ -158,6 +158,9 @@ int& launch_counter();
 // means a wait gave up, 2 means the word could not be read).
 unsigned int take_status_indexer_tc();
 unsigned int take_status_mqa_umma();
+// Zeroes the current device's built-in indexer scratch (csa_index_topk_noalloc)
+// after a timed-out wait; a no-op when the scratch was never used.
+void reset_static_scratch();
 // Records `msg` as the calling thread's last error and returns `st`.
 csa_status_t set_error(csa_status_t st, const char* msg);
 struct CompressArgs {
@@ -204,6 +207,10 @@ struct IndexArgs {
   CompressArgs comp, comp2;
 };
 size_t index_topk_workspace(int batch, int n_q, int64_t n_entries, int k, int n_heads, int dim, int dt);
+// out[0..5]: entries per slice, slices per query row, cooperative selection,
+// tensor-core producer, key stages in the ring, 128-entry tiles per stage.
+void index_topk_plan_info(int batch, int n_q, int64_t n_entries, int k, int n_heads, int dim, int dt,
+                          int32_t* out);
 // Whether the indexer runs the fused decode form (compress the new keys in
 // the indexer launch) for these arguments.
 bool index_fusable(const IndexArgs& a);

@@ -165,6 +165,17 @@ __global__ void __launch_bounds__(kMergeNT) index_merge_kernel(IndexArgs a, Inde
   else
     block_select<kMergeNT>([&](int i) { return ck[i]; }, n, kk, 0, sm, emit, floor);
   for (int j = kk + threadIdx.x; j < a.k; j += kMergeNT) out[j] = -1;
+  // The row's candidates are consumed: zero them (and the per-slice floors),
+  // so that the workspace is all zero again when the call ends, as the
+  // cooperative selection of a later call on the same workspace requires.
+  __syncthreads();
+  uint32_t* ckw = plan_cand_keys(plan, a.ws, bt);
+  int32_t* ciw = plan_cand_idx(plan, a.ws, bt);
+  for (int i = threadIdx.x; i < n; i += kMergeNT) {
+    ckw[i] = 0u;
+    ciw[i] = 0;
+  }
+  for (int j = threadIdx.x; j < plan.n_slices; j += kMergeNT) plan_cand_thr(plan, a.ws, bt)[j] = 0u;
 }
 
 size_t index_merge_smem(const IndexPlan& plan) {
@@ -218,6 +229,23 @@ cudaError_t launch_index_simt(const IndexArgs& a, const IndexPlan& plan, cudaStr
   e = cudaGetLastError();
   if (e != cudaSuccess || plan.n_slices == 1) return e;
   return launch_index_merge(a, plan, s);
+}
+
+void index_topk_plan_info(int batch, int n_q, int64_t n_entries, int k, int n_heads, int dim, int dt,
+                          int32_t* out) {
+  IndexArgs probe{};
+  probe.batch = batch; probe.n_q = n_q; probe.n_entries = n_entries; probe.k = k;
+  probe.n_heads = n_heads; probe.dim = dim; probe.dt = dt;
+  const bool tc = index_tc_eligible(probe);
+  const IndexPlan p = tc ? make_tc_plan(batch, n_q, n_entries, k, dt) : make_simt_plan(batch, n_q, n_entries, k);
+  out[0] = p.slice_len;
+  out[1] = p.n_slices;
+  out[2] = p.coop;
+  out[3] = tc ? 1 : 0;
+  int stages = 0, tiles_per_stage = 1;
+  if (tc) index_tc_ring(n_q, dt, &stages, &tiles_per_stage);
+  out[4] = stages;
+  out[5] = tiles_per_stage;
 }
 
 size_t index_topk_workspace(int batch, int n_q, int64_t n_entries, int k, int n_heads, int dim,

@@ -83,5 +83,8 @@ struct IndexArgs;
 bool index_tc_eligible(const IndexArgs& a);
 IndexPlan make_tc_plan(int batch, int n_q, int64_t n_entries, int k, int dt);
 cudaError_t launch_index_tc(const IndexArgs& a, const IndexPlan& p, cudaStream_t s);
+// Key-stage ring of the tensor-core producer for this query count and dtype:
+// stages in the ring and 128-entry tiles per stage.
+void index_tc_ring(int n_q, int dt, int* stages, int* tiles_per_stage);
 
 }  // namespace csa

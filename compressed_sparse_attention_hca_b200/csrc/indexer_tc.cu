@@ -1059,6 +1059,17 @@ IndexPlan make_tc_plan(int batch, int n_q, int64_t n_entries, int k, int dt) {
   return p;
 }
 
+void index_tc_ring(int n_q, int dt, int* stages, int* tiles_per_stage) {
+  const bool one = index_tc_nq(n_q) == 1;
+  if (dt == CSA_IDX_NVFP4) {
+    *stages = one ? Nvf4Cfg<1>::STAGES : Nvf4Cfg<2>::STAGES;
+    *tiles_per_stage = Nvf4Cfg<1>::TPS;
+  } else {
+    *stages = one ? Bf16Cfg<1>::STAGES : Bf16Cfg<2>::STAGES;
+    *tiles_per_stage = 1;
+  }
+}
+
 cudaError_t launch_index_tc(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) {
   const bool fp4 = a.dt == CSA_IDX_NVFP4;
   if (index_tc_nq(a.n_q) == 1) return fp4 ? launch_nvf4<1>(a, p, s) : launch_bf16<1>(a, p, s);

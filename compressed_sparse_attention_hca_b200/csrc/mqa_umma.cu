@@ -25,10 +25,8 @@
 //
 // With few queries (decode) a query's row chunks are split over several CTAs
 // so that the grid fills the GPU; each writes its unnormalised partial
-// (max, sum, o) to the workspace.  When the splits of a query fit one thread
-// block cluster (up to 16 CTAs) they combine the partials themselves after a
-// cluster barrier, each CTA taking a slice of the 512 dims; otherwise
-// mqa_combine_kernel adds them with the sink.
+// (max, sum, o) to the workspace, and a combine kernel adds them in split
+// order with the sink.
 #include "csa_internal.cuh"
 #include "mqa_plan.cuh"
 #include "sm100.cuh"

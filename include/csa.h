@@ -96,8 +96,10 @@ int csa_last_launch_count(void);
 
 /* Synchronises the current device and reports whether any tensor-core kernel
  * gave up a bounded pipeline wait since the last check (CSA_ERR_TIMEOUT: the
- * results of the affected calls are invalid; the flag is cleared).  Kernels
- * never spin without a limit, so a broken pipeline ends instead of hanging. */
+ * results of the affected calls are invalid; the flag is cleared, and the
+ * built-in scratch of csa_index_topk_noalloc on this device is zeroed again).
+ * Kernels never spin without a limit, so a broken pipeline ends instead of
+ * hanging. */
 csa_status_t csa_check_device_status(void);
 
 /* Bytes per row of format dt at dimension dim (codes only for NVFP4), or -1
@@ -212,10 +214,13 @@ csa_status_t csa_rmsnorm_rope(const void* x, void* y, int64_t n_rows, int dim, c
  * Limits: 1 <= k <= 2048, dim a multiple of 32 (<= 256; NVFP4: of 64),
  * n_heads <= 128.
  * Workspace: ws must be zero-filled before its first use with this call
- * (e.g. one cudaMemset after allocation); every call leaves it zero-filled
- * again, because decode rows split over several CTAs select together through
- * counters and histograms kept there.  After CSA_ERR_TIMEOUT from
- * csa_check_device_status, zero it again.
+ * (e.g. one cudaMemset after allocation), because decode rows split over
+ * several CTAs select together through counters and histograms kept there.
+ * Every call that completes leaves the whole workspace zero-filled again
+ * (the cooperative selection clears its counters, the merge of per-slice
+ * candidates clears the candidate lists), so one workspace, large enough for
+ * each shape, may serve calls of different shapes in turn.  After
+ * CSA_ERR_TIMEOUT from csa_check_device_status, zero it again.
  */
 size_t csa_index_topk_workspace_size(int batch, int n_q, int64_t n_entries, int k, int n_heads,
                                      int dim, csa_dtype_t dt);
@@ -224,6 +229,19 @@ csa_status_t csa_index_topk(const void* qI, const void* qI_sf, const float* wI, 
                             int64_t n_entries, int m, int n_heads, int dim, int k, csa_dtype_t dt,
                             int32_t* idx_out, void* scores_out, void* ws, size_t ws_bytes,
                             void* stream);
+
+/*
+ * csa_index_topk_plan -- how csa_index_topk divides the work of a call of
+ * this shape on the current device (nothing is launched; for tests and
+ * tuning).  out[6] receives: entries per slice, slices per query row, 1 when
+ * the slices of a row select together (cooperative launch, no merge kernel),
+ * 1 when the tensor-core producer runs (0: the SIMT producer), key stages in
+ * the producer's shared-memory ring, and 128-entry tiles per stage.  A slice
+ * of n entries streams ceil(n / (128 * tiles per stage)) stages through that
+ * ring.  Errors: CSA_ERR_INVALID_ARG for the shapes csa_index_topk rejects.
+ */
+csa_status_t csa_index_topk_plan(int batch, int n_q, int64_t n_entries, int k, int n_heads, int dim,
+                                 csa_dtype_t dt, int32_t* out);
 
 /*
  * csa_compress_job_t -- the arguments of one csa_compress call, for calls
@@ -280,12 +298,17 @@ csa_status_t csa_compress_index_topk(const csa_compress_job_t* keys, const csa_c
  *   - Shapes whose csa_index_topk_workspace_size exceeds 4 MiB (4194304
  *     bytes) are rejected with CSA_ERR_INVALID_ARG before any launch.
  *   - The first call on a device (with that device current) looks up the
- *     array's device address; make that first call before any stream capture.
+ *     array's device address and caches it with the device's CUDA context
+ *     (a new context, e.g. after cudaDeviceReset, is looked up again); make
+ *     that first call before any stream capture.
  *   - All calls on a device share the one array and it keeps the previous
  *     call's contents; calls that may overlap on the GPU (other streams or
  *     host threads) race on it, so serialise them.  It starts at zero (static
- *     initialisation) and every call leaves it at zero, as csa_index_topk
- *     requires of its workspace.
+ *     initialisation) and every call that completes leaves it at zero, as
+ *     csa_index_topk requires of its workspace.  A call whose selection timed
+ *     out (CSA_ERR_TIMEOUT from csa_check_device_status) may leave counters
+ *     set: csa_check_device_status zeroes the array of the current device
+ *     when it reports the timeout, with a memset (nothing is allocated).
  */
 csa_status_t csa_index_topk_noalloc(const void* qI, const void* qI_sf, const float* wI,
                                     const void* KI, const void* KI_sf, const int64_t* q_pos,

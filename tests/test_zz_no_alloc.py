@@ -74,6 +74,34 @@ def test_noalloc_matches_workspace_entry_point_twice(dt, B, T, E, k):
         assert torch.equal(out, ref), f"call {call}: differs from csa_index_topk"
 
 
+@pytest.mark.parametrize("merge_first", [True, False])
+def test_noalloc_merge_and_cooperative_calls_in_turn(merge_first):
+    """A call whose rows select through per-slice candidate lists and a merge
+    kernel (two queries per request) and a decode call whose slices select
+    cooperatively (counters and histograms) share the built-in array; in
+    either order each call returns exactly what csa_index_topk returns."""
+    if not torch.cuda.is_available():
+        pytest.fail("needs a CUDA device")
+    merge = dict(dt=csa.IDX_NVFP4, B=2, T=2, E=30000, k=1024)
+    coop = dict(dt=csa.BF16, B=3, T=1, E=20000, k=512)
+    cases = [merge, coop] if merge_first else [coop, merge]
+    fn = _noalloc()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    for rnd in range(2):
+        for c in cases:
+            x = _inputs(c["dt"], c["B"], c["T"], c["E"], seed=c["E"] + rnd)
+            plan = csa.index_topk_plan(c["B"], c["T"], c["E"], c["k"], x["H"], x["d"], c["dt"])
+            assert plan["coop"] == (1 if c is coop else 0) and plan["n_slices"] > 1, plan
+            ref = csa.index_topk(x["qI"], x["wI"], x["KI"], x["q_pos"], 4, c["k"], dt=c["dt"], qI_sf=x["qI_sf"],
+                                 KI_sf=x["KI_sf"])
+            out = torch.full((c["B"], c["T"], c["k"]), -7, device="cuda", dtype=torch.int32)
+            st = fn(_p(x["qI"]), _p(x["qI_sf"]), _p(x["wI"]), _p(x["KI"]), _p(x["KI_sf"]), _p(x["q_pos"]), c["B"],
+                    c["T"], c["E"], 4, x["H"], x["d"], c["k"], c["dt"], _p(out), None, stream)
+            assert st == 0, csa.load().csa_last_error().decode()
+            torch.cuda.synchronize()
+            assert torch.equal(out, ref), f"round {rnd}, {'merge' if c is merge else 'cooperative'} call differs"
+
+
 def test_noalloc_rejects_shapes_beyond_static_scratch():
     if not torch.cuda.is_available():
         pytest.fail("needs a CUDA device")
