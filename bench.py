@@ -102,11 +102,11 @@ class Step:
             H = cfg["n_hI"]
             self.ws_idx = torch.zeros(csa.index_topk_workspace_size(B, T, E, cfg["k"], H, cfg["dI"], idt),
                                       device=device, dtype=torch.uint8)
-            self.ws_mqa = torch.empty(csa.sparse_mqa_workspace_size(B, T, cfg["n_h"], c, cfg["k"],
+            self.ws_mqa = torch.zeros(csa.sparse_mqa_workspace_size(B, T, cfg["n_h"], c, cfg["k"],
                                                                     cfg["window"], cfg["q_dt"], kv_dt),
                                       device=device, dtype=torch.uint8)
         else:
-            self.ws_mqa = torch.empty(csa.hca_dense_mqa_workspace_size(B, T, cfg["n_h"], c, E, cfg["window"],
+            self.ws_mqa = torch.zeros(csa.hca_dense_mqa_workspace_size(B, T, cfg["n_h"], c, E, cfg["window"],
                                                                        cfg["q_dt"], kv_dt),
                                       device=device, dtype=torch.uint8)
         self.launches = 0

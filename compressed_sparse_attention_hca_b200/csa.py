@@ -69,6 +69,11 @@ def load():
         "hca_dense_mqa_workspace_size": (sz, [i32, i32, i32, i32, i64, i32, i32, i32]),
         "hca_dense_mqa": (i32, [P, i32, P, i64, P, i64, P, P, i32, i32, P, f32, i32, i32, i32, i32,
                                 i32, P, P, sz, P]),
+        "csa_mqa_workspace_size": (sz, [i32, i32, i32, i32, i64, i32, i32, ctypes.POINTER(MqaOptions)]),
+        "csa_sparse_mqa_ex": (i32, [P, i32, P, i64, P, i32, P, i64, P, P, i32, i32, P, f32, i32, i32,
+                                    i32, i32, i32, P, P, sz, ctypes.POINTER(MqaOptions), P]),
+        "hca_dense_mqa_ex": (i32, [P, i32, P, i64, P, i64, P, P, i32, i32, P, f32, i32, i32, i32, i32,
+                                   i32, P, P, sz, ctypes.POINTER(MqaOptions), P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -273,6 +278,32 @@ def compress_index_topk(keys_job, qI, wI, KI, q_pos, m, k, *, extra_job=None, dt
 
 # -------------------------------------------------------------------- attention
 
+class MqaOptions(ctypes.Structure):
+    """csa_mqa_options_t: fixed split count (batch-invariant decode), query
+    RMSNorm weights and eps, RoPE dims of the query (at q_pos) and of the
+    output (at -q_pos), RoPE base."""
+    _fields_ = [("splits", ctypes.c_int32), ("q_norm_g", ctypes.c_void_p), ("q_norm_eps", ctypes.c_float),
+                ("q_rope_dims", ctypes.c_int32), ("out_rope_dims", ctypes.c_int32), ("rope_base", ctypes.c_double)]
+
+
+def mqa_options(*, splits=0, q_norm_g=None, q_norm_eps=1e-6, q_rope_dims=0, out_rope_dims=0, rope_base=10000.0):
+    _need_cuda(q_norm_g)
+    o = MqaOptions(splits=splits, q_norm_g=q_norm_g.data_ptr() if q_norm_g is not None else None,
+                   q_norm_eps=q_norm_eps, q_rope_dims=q_rope_dims, out_rope_dims=out_rope_dims,
+                   rope_base=rope_base)
+    o._keep = q_norm_g  # the struct holds a raw pointer: keep the tensor alive with it
+    return o
+
+
+def _opt_ref(options):
+    return ctypes.byref(options) if options is not None else None
+
+
+def mqa_workspace_size(batch, n_q, n_heads, dim, rows_per_query, q_dt, kv_dt, options=None):
+    return int(load().csa_mqa_workspace_size(batch, n_q, n_heads, dim, rows_per_query, q_dt, kv_dt,
+                                             _opt_ref(options)))
+
+
 def _kv_dt(entries, kv_dt):
     if kv_dt is not None:
         return kv_dt
@@ -289,9 +320,11 @@ def hca_dense_mqa_workspace_size(batch, n_q, n_heads, dim, n_entries, window, q_
 
 
 def sparse_mqa(Q, entries, idx, win, win_start, q_pos, window, m, sink, scale, *, kv_dt=None, O=None,
-               ws=None):
+               ws=None, options=None):
     """CSA shared-KV MQA.  Q [B, T, H, c]; entries [B, E, row]; idx [B, T, k] int32;
-    win [B, Lw, row]; win_start [B] int64; q_pos [B, T] int64; sink [H] fp32."""
+    win [B, Lw, row]; win_start [B] int64; q_pos [B, T] int64; sink [H] fp32.
+    options: an MqaOptions (mqa_options()) or None.  A workspace passed in
+    must have been zero-filled before its first use."""
     _need_cuda(Q, entries, idx, win, win_start, q_pos, sink)
     B, T, H, c = Q.shape
     kv_dt = _kv_dt(entries, kv_dt)
@@ -299,18 +332,18 @@ def sparse_mqa(Q, entries, idx, win, win_start, q_pos, window, m, sink, scale, *
     k = idx.shape[-1]
     if O is None:
         O = torch.empty_like(Q)
-    need = sparse_mqa_workspace_size(B, T, H, c, k, window, q_dt, kv_dt)
+    need = mqa_workspace_size(B, T, H, c, k + window, q_dt, kv_dt, options)
     if ws is None or ws.numel() < need:
-        ws = torch.empty(need, device=Q.device, dtype=torch.uint8)
-    _check(load().csa_sparse_mqa(_ptr(Q), q_dt, _ptr(entries), entries.shape[1], _ptr(idx), k, _ptr(win),
-                                 win.shape[1], _ptr(win_start), _ptr(q_pos), window, m, _ptr(sink),
-                                 float(scale), B, T, H, c, kv_dt, _ptr(O), _ptr(ws), ws.numel(),
-                                 _stream()))
+        ws = torch.zeros(need, device=Q.device, dtype=torch.uint8)  # zero before first use
+    _check(load().csa_sparse_mqa_ex(_ptr(Q), q_dt, _ptr(entries), entries.shape[1], _ptr(idx), k, _ptr(win),
+                                    win.shape[1], _ptr(win_start), _ptr(q_pos), window, m, _ptr(sink),
+                                    float(scale), B, T, H, c, kv_dt, _ptr(O), _ptr(ws), ws.numel(),
+                                    _opt_ref(options), _stream()))
     return O
 
 
 def hca_dense_mqa(Q, entries, win, win_start, q_pos, window, m, sink, scale, *, kv_dt=None, O=None,
-                  ws=None):
+                  ws=None, options=None):
     """HCA dense shared-KV MQA over every visible entry plus the window."""
     _need_cuda(Q, entries, win, win_start, q_pos, sink)
     B, T, H, c = Q.shape
@@ -318,10 +351,10 @@ def hca_dense_mqa(Q, entries, win, win_start, q_pos, window, m, sink, scale, *, 
     q_dt = _dt_of(Q)
     if O is None:
         O = torch.empty_like(Q)
-    need = hca_dense_mqa_workspace_size(B, T, H, c, entries.shape[1], window, q_dt, kv_dt)
+    need = mqa_workspace_size(B, T, H, c, entries.shape[1] + window, q_dt, kv_dt, options)
     if ws is None or ws.numel() < need:
-        ws = torch.empty(need, device=Q.device, dtype=torch.uint8)
-    _check(load().hca_dense_mqa(_ptr(Q), q_dt, _ptr(entries), entries.shape[1], _ptr(win), win.shape[1],
-                                _ptr(win_start), _ptr(q_pos), window, m, _ptr(sink), float(scale), B, T,
-                                H, c, kv_dt, _ptr(O), _ptr(ws), ws.numel(), _stream()))
+        ws = torch.zeros(need, device=Q.device, dtype=torch.uint8)  # zero before first use
+    _check(load().hca_dense_mqa_ex(_ptr(Q), q_dt, _ptr(entries), entries.shape[1], _ptr(win), win.shape[1],
+                                   _ptr(win_start), _ptr(q_pos), window, m, _ptr(sink), float(scale), B, T,
+                                   H, c, kv_dt, _ptr(O), _ptr(ws), ws.numel(), _opt_ref(options), _stream()))
     return O

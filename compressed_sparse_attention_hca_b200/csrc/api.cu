@@ -323,6 +323,30 @@ csa_status_t csa_compress_index_topk(const csa_compress_job_t* keys, const csa_c
 
 namespace {
 
+// Copies the attention options into the argument struct (NULL = none).
+csa_status_t apply_mqa_options(csa::MqaArgs& a, const csa_mqa_options_t* opt) {
+  a.splits = 0;
+  a.q_norm_g = nullptr;
+  a.q_norm_eps = 0.f;
+  a.q_rope_dims = a.out_rope_dims = 0;
+  a.rope_base = 10000.0;
+  if (opt == nullptr) return CSA_OK;
+  REQUIRE(opt->splits >= 0 && opt->splits <= 256, "splits=%d out of range [0, 256]", opt->splits);
+  REQUIRE(opt->q_rope_dims >= 0 && opt->q_rope_dims <= 64 && opt->q_rope_dims % 8 == 0,
+          "q_rope_dims=%d must be a multiple of 8 in [0, 64]", opt->q_rope_dims);
+  REQUIRE(opt->out_rope_dims >= 0 && opt->out_rope_dims <= 64 && opt->out_rope_dims % 8 == 0,
+          "out_rope_dims=%d must be a multiple of 8 in [0, 64]", opt->out_rope_dims);
+  REQUIRE(opt->q_norm_g == nullptr || opt->q_norm_eps >= 0.f, "q_norm_eps must be >= 0");
+  REQUIRE(opt->q_rope_dims + opt->out_rope_dims == 0 || opt->rope_base > 0.0, "rope_base must be > 0");
+  a.splits = opt->splits;
+  a.q_norm_g = opt->q_norm_g;
+  a.q_norm_eps = opt->q_norm_eps;
+  a.q_rope_dims = opt->q_rope_dims;
+  a.out_rope_dims = opt->out_rope_dims;
+  a.rope_base = opt->rope_base;
+  return CSA_OK;
+}
+
 csa_status_t check_mqa(const csa::MqaArgs& a) {
   REQUIRE(a.batch >= 0 && a.n_q >= 0 && a.n_entries >= 0 && a.win_len >= 0, "negative size");
   REQUIRE(a.m >= 1, "m=%d must be >= 1", a.m);
@@ -351,6 +375,13 @@ csa_status_t run_mqa(csa::MqaArgs& a, void* stream, const char* name) {
     REQUIRE_PTR(a.win);
     REQUIRE_PTR(a.win_start);
   }
+  if (a.q_norm_g != nullptr || a.q_rope_dims > 0 || a.out_rope_dims > 0) {
+    if (!csa::mqa_tc_path(a))
+      return fail(CSA_ERR_UNSUPPORTED,
+                  "query normalisation / RoPE options need the tensor-core path (bf16 Q, BF16 or KV_FP8MIX rows, "
+                  "dim 512, n_heads a multiple of 64)");
+    if (a.q_norm_g != nullptr) REQUIRE_PTR(a.q_norm_g);
+  }
   const size_t need = csa::mqa_workspace(a);
   REQUIRE(a.ws_bytes >= need, "workspace too small: %zu < %zu bytes", a.ws_bytes, need);
   if (need > 0) REQUIRE_PTR(a.ws);
@@ -367,6 +398,7 @@ csa::MqaArgs mqa_args(const void* Q, csa_dtype_t q_dt, const void* entries, int6
   a.win = win; a.win_len = win_len; a.win_start = win_start; a.q_pos = q_pos; a.window = window;
   a.m = m; a.sink = sink; a.scale = scale; a.batch = batch; a.n_q = n_q; a.n_heads = n_heads;
   a.dim = dim; a.kv_dt = (int)kv_dt; a.O = O; a.ws = ws; a.ws_bytes = ws_bytes;
+  apply_mqa_options(a, nullptr);
   return a;
 }
 
@@ -384,18 +416,42 @@ size_t csa_sparse_mqa_workspace_size(int batch, int n_q, int n_heads, int dim, i
   return s < 256 ? 256 : s;
 }
 
+size_t csa_mqa_workspace_size(int batch, int n_q, int n_heads, int dim, int64_t rows_per_query,
+                              csa_dtype_t q_dt, csa_dtype_t kv_dt, const csa_mqa_options_t* opt) {
+  // a dense call whose row count per query is rows_per_query (window 0)
+  csa::MqaArgs a = mqa_args(nullptr, q_dt, nullptr, rows_per_query < 0 ? 0 : rows_per_query, nullptr, 0, nullptr,
+                            0, nullptr, nullptr, 0, 1, nullptr, 1.f, batch, n_q, n_heads, dim, kv_dt, nullptr,
+                            nullptr, 0);
+  if (apply_mqa_options(a, opt) != CSA_OK || check_mqa(a) != CSA_OK || batch <= 0 || n_q <= 0) return 256;
+  const size_t s = csa::mqa_workspace(a);
+  return s < 256 ? 256 : s;
+}
+
+csa_status_t csa_sparse_mqa_ex(const void* Q, csa_dtype_t q_dt, const void* entries,
+                               int64_t n_entries, const int32_t* idx, int k, const void* win,
+                               int64_t win_len, const int64_t* win_start, const int64_t* q_pos,
+                               int window, int m, const float* sink, float softmax_scale, int batch,
+                               int n_q, int n_heads, int dim, csa_dtype_t kv_dt, void* O, void* ws,
+                               size_t ws_bytes, const csa_mqa_options_t* opt, void* stream) {
+  g_launches = 0;
+  if (idx == nullptr && (int64_t)batch * n_q > 0) return fail(CSA_ERR_INVALID_ARG, "idx is NULL");
+  REQUIRE_ALIGNED_OR_NULL(idx);
+  csa::MqaArgs a = mqa_args(Q, q_dt, entries, n_entries, idx, k, win, win_len, win_start, q_pos,
+                            window, m, sink, softmax_scale, batch, n_q, n_heads, dim, kv_dt, O, ws,
+                            ws_bytes);
+  const csa_status_t st = apply_mqa_options(a, opt);
+  if (st != CSA_OK) return st;
+  return run_mqa(a, stream, "csa_sparse_mqa");
+}
+
 csa_status_t csa_sparse_mqa(const void* Q, csa_dtype_t q_dt, const void* entries,
                             int64_t n_entries, const int32_t* idx, int k, const void* win,
                             int64_t win_len, const int64_t* win_start, const int64_t* q_pos,
                             int window, int m, const float* sink, float softmax_scale, int batch,
                             int n_q, int n_heads, int dim, csa_dtype_t kv_dt, void* O, void* ws,
                             size_t ws_bytes, void* stream) {
-  if (idx == nullptr && (int64_t)batch * n_q > 0) return fail(CSA_ERR_INVALID_ARG, "idx is NULL");
-  REQUIRE_ALIGNED_OR_NULL(idx);
-  csa::MqaArgs a = mqa_args(Q, q_dt, entries, n_entries, idx, k, win, win_len, win_start, q_pos,
-                            window, m, sink, softmax_scale, batch, n_q, n_heads, dim, kv_dt, O, ws,
-                            ws_bytes);
-  return run_mqa(a, stream, "csa_sparse_mqa");
+  return csa_sparse_mqa_ex(Q, q_dt, entries, n_entries, idx, k, win, win_len, win_start, q_pos, window, m, sink,
+                           softmax_scale, batch, n_q, n_heads, dim, kv_dt, O, ws, ws_bytes, nullptr, stream);
 }
 
 size_t hca_dense_mqa_workspace_size(int batch, int n_q, int n_heads, int dim, int64_t n_entries,
@@ -408,16 +464,29 @@ size_t hca_dense_mqa_workspace_size(int batch, int n_q, int n_heads, int dim, in
   return s < 256 ? 256 : s;
 }
 
+csa_status_t hca_dense_mqa_ex(const void* Q, csa_dtype_t q_dt, const void* entries,
+                              int64_t n_entries, const void* win, int64_t win_len,
+                              const int64_t* win_start, const int64_t* q_pos, int window, int m,
+                              const float* sink, float softmax_scale, int batch, int n_q,
+                              int n_heads, int dim, csa_dtype_t kv_dt, void* O, void* ws,
+                              size_t ws_bytes, const csa_mqa_options_t* opt, void* stream) {
+  g_launches = 0;
+  csa::MqaArgs a = mqa_args(Q, q_dt, entries, n_entries, nullptr, 0, win, win_len, win_start, q_pos,
+                            window, m, sink, softmax_scale, batch, n_q, n_heads, dim, kv_dt, O, ws,
+                            ws_bytes);
+  const csa_status_t st = apply_mqa_options(a, opt);
+  if (st != CSA_OK) return st;
+  return run_mqa(a, stream, "hca_dense_mqa");
+}
+
 csa_status_t hca_dense_mqa(const void* Q, csa_dtype_t q_dt, const void* entries,
                            int64_t n_entries, const void* win, int64_t win_len,
                            const int64_t* win_start, const int64_t* q_pos, int window, int m,
                            const float* sink, float softmax_scale, int batch, int n_q,
                            int n_heads, int dim, csa_dtype_t kv_dt, void* O, void* ws,
                            size_t ws_bytes, void* stream) {
-  csa::MqaArgs a = mqa_args(Q, q_dt, entries, n_entries, nullptr, 0, win, win_len, win_start, q_pos,
-                            window, m, sink, softmax_scale, batch, n_q, n_heads, dim, kv_dt, O, ws,
-                            ws_bytes);
-  return run_mqa(a, stream, "hca_dense_mqa");
+  return hca_dense_mqa_ex(Q, q_dt, entries, n_entries, win, win_len, win_start, q_pos, window, m, sink,
+                          softmax_scale, batch, n_q, n_heads, dim, kv_dt, O, ws, ws_bytes, nullptr, stream);
 }
 
 }  // extern "C"

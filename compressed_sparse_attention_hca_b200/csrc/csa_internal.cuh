@@ -234,8 +234,20 @@ struct MqaArgs {
   void* O;
   void* ws;
   size_t ws_bytes;
+  // options (csa_mqa_options_t): a fixed split count per query (0: chosen
+  // from the batch), the query's RMSNorm weights (nullptr: none) and eps, the
+  // RoPE dims turned on the query at q_pos and on the output at -q_pos, and
+  // the RoPE base
+  int splits;
+  const float* q_norm_g;
+  float q_norm_eps;
+  int q_rope_dims, out_rope_dims;
+  double rope_base;
 };
 size_t mqa_workspace(const MqaArgs& a);
+// Whether the tensor-core attention kernel takes these arguments (the query
+// normalisation and RoPE options exist only there).
+bool mqa_tc_path(const MqaArgs& a);
 cudaError_t launch_mqa(const MqaArgs& a, cudaStream_t s);
 
 }  // namespace csa

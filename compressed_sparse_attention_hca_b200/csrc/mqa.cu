@@ -302,7 +302,9 @@ MqaPlan make_simt_mqa_plan(const MqaArgs& a) {
   p.heads_per_cta = (a.n_heads % 8 == 0) ? 8 : (a.n_heads % 4 == 0) ? 4 : (a.n_heads % 2 == 0) ? 2 : 1;
   const int64_t rows_max = max_rows_per_query(a);
   const int64_t units = (int64_t)a.batch * a.n_q * (a.n_heads / p.heads_per_cta);
-  int64_t splits = (296 + units - 1) / units;
+  // automatic: enough splits to cover the GPU about twice; a fixed count
+  // (a.splits) makes the split boundaries depend on the row count only
+  int64_t splits = a.splits > 0 ? a.splits : (296 + units - 1) / units;
   const int64_t max_splits = (rows_max + kRC - 1) / kRC;
   if (splits > max_splits) splits = max_splits;
   if (splits < 1) splits = 1;
@@ -312,6 +314,8 @@ MqaPlan make_simt_mqa_plan(const MqaArgs& a) {
   p.rows_per_split = rps;
   p.n_splits = (int)((rows_max + rps - 1) / rps);
   if (p.n_splits < 1) p.n_splits = 1;
+  p.mode = p.n_splits > 1 ? kMqaSplit : kMqaWhole;
+  p.ws_head = 0;
   return p;
 }
 
@@ -331,6 +335,8 @@ cudaError_t launch_mqa_simt(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) 
 bool mqa_umma_path(const MqaArgs& a);
 MqaPlan mqa_umma_plan(const MqaArgs& a);
 cudaError_t launch_mqa_umma(const MqaArgs& a, const MqaPlan& p, cudaStream_t s);
+
+bool mqa_tc_path(const MqaArgs& a) { return mqa_umma_path(a); }
 
 size_t mqa_workspace(const MqaArgs& a) {
   const MqaPlan p = mqa_umma_path(a) ? mqa_umma_plan(a) : make_simt_mqa_plan(a);

@@ -1,84 +1,100 @@
 // mqa_umma.cu -- shared-KV multi-query attention on the 5th-generation tensor
 // cores (tcgen05.mma, bf16 in, fp32 accumulate in TMEM) for c = 512 and head
 // counts that are a multiple of 64 ("DeepSeek-V4 内部机制" 1.2 Step 2
-// shared-KV MQA, 1.3 HCA, 1.4 window branch and sink equation; yunpan.plus
-// eq. 9).
+// shared-KV MQA, 1.3 HCA, 1.4 window branch, sink equation, and the RMSNorm /
+// partial-RoPE rows of its table; yunpan.plus eq. 9).
 //
 // A CTA owns one query, a group of 64 heads and a range of that query's
-// attended rows, taken 128 at a time.  Each row is both key and value, so one
-// gathered tile serves both products:
+// attended rows, taken 128 at a time (a chunk).  Each row is both key and
+// value, so one gathered tile serves both products:
 //   S^T[128 rows, 64 heads]  = K[128, 512] . Q[64, 512]^T
 //       A = the row tile, K-major (128-byte swizzle, 8 atoms of 64 dims),
 //       B = the query tile, K-major; D in TMEM (lane = row, column = head);
 //   O^T[512 dims, 64 heads] += V^T[512, 128] . P^T[128, 64]
 //       A = the same row tile read MN-major (a line = 64 dims of one row),
 //       B = P written by the softmax threads MN-major (a line = the 64 heads
-//       of one row); D = four 128-dim slabs in TMEM (lane = dim).
-// The softmax runs on the 128 threads that own the TMEM lanes: thread r holds
-// row r's 64 scores; per-head maxima across rows are warp max-reductions
-// (redux.sync) and per-head sums warp reduce-scatters (each lane ends with
-// two heads), both combined over four warps.
-// The running maximum is only raised when a chunk exceeds it by more than
-// 2^8, so O^T is rescaled in TMEM rarely (never within one chunk).
-// FP8MIX rows are expanded to bf16 (value = e4m3 * block scale; RoPE dims
-// copied) on their way into the row tile.
+//       of one row); D = four 128-dim slabs in TMEM (lane = dim);
+//   L[., 64 heads]          += 1[128, 128] . P^T[128, 64]
+//       the per-head sums of P on the tensor core (A = ones kept in TMEM):
+//       every lane of L holds the running denominators.
+// Per chunk: the rows are gathered (FP8MIX rows by one bulk copy each, then
+// expanded to bf16 -- value = e4m3 * block scale, RoPE dims copied -- half
+// the tile at a time, the S^T MMAs of a half issued as soon as it is ready;
+// BF16 rows by cp.async, the S^T MMAs of each 128-dim pair of atoms issued as
+// it lands); eight warps then take the softmax (per-head maxima over the rows
+// by warp max-reductions, P = 2^(s - m) in bf16); the running maximum is only
+// raised when a chunk exceeds it by more than 2^8, so O^T and L are rescaled
+// in TMEM rarely.  A CTA with several BF16 chunks gathers the next chunk's
+// atoms as soon as the products of the current chunk have read them.
 //
-// With few queries (decode) a query's row chunks are split over several CTAs
-// so that the grid fills the GPU; each writes its unnormalised partial
-// (max, sum, o) to the workspace, and a combine kernel adds them in split
-// order with the sink.
+// Rows split over several CTAs (decode: few queries) give partials
+// (max, sum, o) per split.  When the grid fits the GPU at once (cooperative
+// launch) the splits of a (query, head group) wait for one another on a
+// counter and each combines a share of the outputs with the sink; otherwise a
+// separate kernel does the same combine.  Both add the splits in split order
+// with the same arithmetic, and with a fixed split count (an option) the
+// split boundaries depend only on the query's rows: a request's output then
+// does not depend on the batch it runs in.
+//
+// Options: RMSNorm of the query and RoPE of its last dims at the query
+// position (prologue, the same arithmetic as csa_rmsnorm_rope), and RoPE of
+// the output's last dims at minus the query position (output write).
 #include "csa_internal.cuh"
 #include "mqa_plan.cuh"
+#include "rope_dev.cuh"
 #include "sm100.cuh"
 
 namespace csa {
 
 CSA_DEFINE_STATUS_READER(take_status_mqa_umma)
 
-cudaError_t launch_mqa_combine(const MqaArgs& a, const MqaPlan& p, cudaStream_t s);
-
 namespace {
 
 constexpr int kDim = 512;
-constexpr int kHG = 64;          // heads per CTA (N of both products)
+constexpr int kHG = 64;          // heads per CTA (N of the products)
 constexpr int kRows = 128;       // rows per chunk (M of S^T)
 constexpr int kThreads = 256;
-constexpr int kMaxSel = 2048;    // selected entries per query (the top-k limit)
+constexpr int kItems = kHG * kDim / 8;  // output items of a head group: (head, 8 dims)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.f;     // log2 headroom before the running max is raised
+constexpr int kMaxRope = 64;     // RoPE dims the fused options support
 
-// Shared memory (offsets from a 1024-byte aligned base).  The buffers are
-// contiguous so that any descriptor stride stays inside them; the upper half
-// of the row tile and P together stage a chunk of raw FP8MIX rows.
+// Shared memory (offsets from a 1024-byte aligned base).  The upper half of
+// the row tile and P together stage a chunk of raw FP8MIX rows.
+constexpr int kAtom = kRows * 128;               // one 64-dim atom of the row tile
 constexpr int kOffKV = 0;                        // 8 x [128 rows][128 B]    128 KB
-constexpr int kOffP = kOffKV + 8 * kRows * 128;  // [128 rows][128 B]        16 KB
+constexpr int kOffP = kOffKV + 8 * kAtom;        // [128 rows][128 B]        16 KB
 constexpr int kOffQ = kOffP + kRows * 128;       // 8 x [64 heads][128 B]    64 KB
 constexpr int kOffMisc = kOffQ + 8 * kHG * 128;
 constexpr int kRawRow = 608;                     // FP8MIX row at c = 512
-constexpr int kOffRaw = kOffKV + 4 * kRows * 128;  // atoms 4..7 and P
+constexpr int kOffRaw = kOffKV + 4 * kAtom;      // atoms 4..7 and P
 static_assert(kOffRaw + kRows * kRawRow <= kOffQ, "raw staging fits in atoms 4..7 and P");
+static_assert(kHG * kDim * 4 <= 8 * kAtom, "the fp32 output staging fits in the row tile");
 struct Misc {
   float m_use[kHG];    // running max per head (log2 domain)
-  float l_run[kHG];    // running sum per head (relative to m_use)
   float corr[kHG];     // this chunk's rescale factor per head
   float fac[kHG];      // epilogue scale per head
-  float red[4][kHG];   // per-warp partial max / sum
-  const uint8_t* rowp[kRows];
-  int32_t sel[kMaxSel];
-  uint64_t bar_qk, bar_pv;
+  float lsum[kHG];     // final sums per head
+  float red[4][kHG];   // per-quadrant maxima
+  float qcs[kMaxRope / 2], qsn[kMaxRope / 2];  // RoPE at +t (query)
+  float ocs[kMaxRope / 2], osn[kMaxRope / 2];  // RoPE at -t (output)
+  const uint8_t* rowp[2][kRows];               // rows of the current / next chunk
+  uint64_t bar_raw, bar_half[2], bar_pair[4], bar_qk, bar_slab[4], bar_pv;
   uint32_t tmem_slot;
-  int rescale;
 };
 constexpr int kSmemBytes = 1024 + kOffMisc + (int)sizeof(Misc);
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
-// TMEM columns: S^T (64), then O^T slabs s = 0..3 (64 each).
+// TMEM columns: S^T (64), O^T slabs 0..3 (64 each), L (64), ones (32).
 constexpr int kColS = 0;
 constexpr int kColO = 64;
+constexpr int kColL = 320;
+constexpr int kColOnes = 384;
 constexpr int kTmemCols = 512;
 
 constexpr uint32_t kIdescQK = idesc_bf16_f32(kRows, kHG);
 constexpr uint32_t kIdescPV = idesc_bf16_f32_major(128, kHG, 1, 1);
+constexpr uint32_t kIdescL = idesc_bf16_f32_major(128, kHG, 0, 1);
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   const uint32_t a = smem_u32(p);
@@ -86,7 +102,7 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 }
 // Row tile: byte offset of 16-byte chunk g (dims 8g .. 8g+7) of row r.
 __device__ __forceinline__ uint32_t kv_off(int r, int g) {
-  return (uint32_t)((g >> 3) * (kRows * 128) + r * 128 + ((((g & 7) ^ (r & 7))) << 4));
+  return (uint32_t)((g >> 3) * kAtom + r * 128 + ((((g & 7) ^ (r & 7))) << 4));
 }
 // Query tile: byte offset of 16-byte chunk g of head h.
 __device__ __forceinline__ uint32_t q_off(int h, int g) {
@@ -97,59 +113,178 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+// Waits until at most n of this thread's most recent cp.async groups are pending.
+__device__ __forceinline__ void cp_async_wait_pending(int n) {
+  switch (n) {
+    case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+    case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+    case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+    case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+    default: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+  }
+}
 // Maximum over the warp's 32 lanes, returned to every lane (sm_100a).
 __device__ __forceinline__ float warp_max_f32(float v) {
   float r;
   asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
   return r;
 }
-// Barrier of the 128 softmax threads (warps 0-3).
-__device__ __forceinline__ void softmax_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-// Producer / consumer halves of a named barrier over n threads.
-__device__ __forceinline__ void named_barrier_arrive(int id, int n) {
-  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-__device__ __forceinline__ void named_barrier_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
 }
 
-// Warp reduce-scatter of 64 per-lane values (one per head): afterwards lane l
-// holds the sum (or max) over the warp's 32 lanes for heads 2l and 2l+1.
-template <bool MAX>
-__device__ __forceinline__ void reduce_scatter64(float* v, int lane, float& r0, float& r1) {
-#pragma unroll
-  for (int k = 16, n = 32; k >= 1; k >>= 1, n >>= 1) {
-    const bool upper = (lane & k) != 0;
-#pragma unroll
-    for (int j = 0; j < n; ++j) {
-      const float send = upper ? v[j] : v[j + n];
-      const float keep = upper ? v[j + n] : v[j];
-      const float recv = __shfl_xor_sync(0xffffffffu, send, k);
-      v[j] = MAX ? fmaxf(keep, recv) : keep + recv;
+// Address of row r of the query's attended rows when it lies in [.., r_end),
+// else nullptr (absent rows are zero-filled and masked).
+__device__ __forceinline__ const uint8_t* chunk_row(const MqaArgs& a, const RowList& rl, int b, int64_t r,
+                                                    int64_t r_end, int64_t rb) {
+  return r < r_end ? row_ptr(a, rl, b, r, rb) : nullptr;
+}
+
+// BF16 rows: one cp.async commit group per pair of atoms (128 dims).
+__device__ __forceinline__ void gather_bf16(uint8_t* KV, const uint8_t* const* rowp, const void* dummy) {
+  for (int p = 0; p < 4; ++p) {
+    for (int u = threadIdx.x; u < kRows * 16; u += kThreads) {
+      const int r = u >> 4, g = 16 * p + (u & 15);
+      const uint8_t* src = rowp[r];
+      cp_async16(smem_u32(KV + kv_off(r, g)), src ? src + g * 16 : dummy, src != nullptr);
     }
+    cp_async_commit();
   }
-  r0 = v[0];
-  r1 = v[1];
 }
 
-// How a CTA finishes: the whole query (normalised output) or one split of
-// several (unnormalised partial for the combine kernel).
-enum { kWhole = 0, kSplit = 1 };
+// FP8MIX rows: one bulk copy per row into the raw staging area (absent rows
+// zero-filled); threads 0..127 each arrive once on bar_raw.
+__device__ __forceinline__ void gather_fp8(uint8_t* raw, const uint8_t* const* rowp, uint64_t* bar_raw) {
+  const int r = threadIdx.x;
+  if (r >= kRows) return;
+  const uint8_t* src = rowp[r];
+  uint8_t* dst = raw + r * kRawRow;
+  if (src != nullptr) {
+    mbar_arrive_expect_tx(bar_raw, kRawRow);
+    bulk_load(dst, src, kRawRow, bar_raw);
+  } else {
+#pragma unroll 1
+    for (int c = 0; c < kRawRow / 16; ++c) reinterpret_cast<uint4*>(dst)[c] = make_uint4(0u, 0u, 0u, 0u);
+    mbar_arrive(bar_raw);
+  }
+}
+
+// 16-byte chunk g (dims 8g .. 8g+7) of raw FP8MIX row r as bf16.
+__device__ __forceinline__ uint4 expand_fp8(const uint8_t* raw, int r, int g) {
+  const uint8_t* row = raw + r * kRawRow;
+  if (g >= 56) return *reinterpret_cast<const uint4*>(row + 448 + (g - 56) * 16);
+  const uint2 v = *reinterpret_cast<const uint2*>(row + g * 8);
+  const float sc = *reinterpret_cast<const float*>(row + 576 + 4 * (g >> 3));
+  uint32_t w[4];
+  const uint32_t src[2] = {v.x, v.y};
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const float2 lo = e4m3x2_to_float2((uint16_t)(src[q] & 0xFFFF));
+    const float2 hi = e4m3x2_to_float2((uint16_t)(src[q] >> 16));
+    const __nv_bfloat162 x0 = __floats2bfloat162_rn(lo.x * sc, lo.y * sc);
+    const __nv_bfloat162 x1 = __floats2bfloat162_rn(hi.x * sc, hi.y * sc);
+    memcpy(&w[2 * q], &x0, 4);
+    memcpy(&w[2 * q + 1], &x1, 4);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// S^T += K Q^T over atoms [at0, at1) (the first atom of a chunk overwrites).
+__device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t kva, uint32_t qa, int at0, int at1) {
+  for (int at = at0; at < at1; ++at)
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      tc_mma_f16(tmem + kColS, umma_desc_sw128(kva + at * kAtom + kk * 32),
+                 umma_desc_sw128(qa + at * (kHG * 128) + kk * 32), kIdescQK, (at | kk) ? 1u : 0u);
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float* v) {
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+    memcpy(&w[q], &h, 4);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// Output items [i0, i1) of one head group, item = (head, 8 dims): the splits'
+// partials added in split order with the sink, the optional output RoPE,
+// bf16 stores.  W is shared memory for n_splits x 64 weights.
+__device__ void combine_items(const MqaArgs& a, const MqaPlan& plan, int64_t bt, int hg, int i0, int i1, float* W,
+                              const float* ocs, const float* osn) {
+  const int S = plan.n_splits;
+  const int tid = threadIdx.x;
+  if (tid < kHG) {
+    const int h = hg * kHG + tid;
+    const float sink = a.sink[h];
+    float M = sink;
+    for (int j = 0; j < S; ++j) M = fmaxf(M, __ldcg(plan_partial_ml(plan, a, bt, j, h)));
+    const bool zero = (sink == INFINITY) || (M == -INFINITY);
+    float den = 0.f;
+    for (int j = 0; j < S; ++j) {
+      const float* ml = plan_partial_ml(plan, a, bt, j, h);
+      const float mj = __ldcg(ml);
+      const float w = (zero || mj == -INFINITY) ? 0.f : expf(mj - M);
+      W[j * kHG + tid] = w;
+      den += w > 0.f ? __ldcg(ml + 1) * w : 0.f;
+    }
+    if (!zero) den += expf(sink - M);
+    for (int j = 0; j < S; ++j) W[j * kHG + tid] = zero ? 0.f : W[j * kHG + tid] / den;
+  }
+  __syncthreads();
+  const int d_rope = kDim - a.out_rope_dims;
+  for (int it = i0 + tid; it < i1; it += kThreads) {
+    const int h = it >> 6, d0 = 8 * (it & 63);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < S; ++j) {
+      const float* po = plan_partial_o(plan, a, bt, j, hg * kHG + h) + d0;
+      const float4 x0 = __ldcg(reinterpret_cast<const float4*>(po));
+      const float4 x1 = __ldcg(reinterpret_cast<const float4*>(po + 4));
+      const float w = W[j * kHG + h];
+      acc[0] = fmaf(w, x0.x, acc[0]); acc[1] = fmaf(w, x0.y, acc[1]);
+      acc[2] = fmaf(w, x0.z, acc[2]); acc[3] = fmaf(w, x0.w, acc[3]);
+      acc[4] = fmaf(w, x1.x, acc[4]); acc[5] = fmaf(w, x1.y, acc[5]);
+      acc[6] = fmaf(w, x1.z, acc[6]); acc[7] = fmaf(w, x1.w, acc[7]);
+    }
+    if (a.out_rope_dims > 0 && d0 >= d_rope) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int k = (d0 - d_rope) / 2 + q;
+        rope_turn(acc[2 * q], acc[2 * q + 1], ocs[k], osn[k]);
+      }
+    }
+    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + (bt * a.n_heads + (int64_t)hg * kHG + h) * kDim +
+                              d0) = pack_bf16x8(acc);
+  }
+}
+
+// RoPE tables of the query at +t and of the output at -t (threads < 32).
+__device__ __forceinline__ void rope_tables(const MqaArgs& a, int64_t t, float* qcs, float* qsn, float* ocs,
+                                            float* osn) {
+  const int k = threadIdx.x;
+  if (k < a.q_rope_dims / 2) rope_sincos((double)t, rope_theta(a.rope_base, k, a.q_rope_dims), &qsn[k], &qcs[k]);
+  if (k < a.out_rope_dims / 2)
+    rope_sincos((double)t * -1.0, rope_theta(a.rope_base, k, a.out_rope_dims), &osn[k], &ocs[k]);
+}
 
 template <bool FP8, int MODE>
 __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPlan plan) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
-  uint8_t* Ps = base + kOffP;
   uint8_t* KV = base + kOffKV;
+  uint8_t* Ps = base + kOffP;
   uint8_t* Qs = base + kOffQ;
+  uint8_t* raw = base + kOffRaw;
   Misc& ms = *reinterpret_cast<Misc*>(base + kOffMisc);
 
   const int split = blockIdx.x, hg = blockIdx.y;
   const int64_t bt = blockIdx.z;
   const int b = (int)(bt / a.n_q);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int quad = warp & 3, half = warp >> 2;
 
   // query tile (64 heads x 512 dims) -> K-major swizzled atoms, issued first
   // (it depends on nothing)
@@ -172,93 +307,110 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
   const int64_t rb = row_bytes(a.kv_dt, kDim);
 
   if (tid == 0) {
+    mbar_init(&ms.bar_raw, kRows);
+    for (int i = 0; i < 2; ++i) mbar_init(&ms.bar_half[i], kThreads);
+    for (int i = 0; i < 4; ++i) mbar_init(&ms.bar_pair[i], kThreads);
     mbar_init(&ms.bar_qk, 1);
+    for (int i = 0; i < 4; ++i) mbar_init(&ms.bar_slab[i], 1);
     mbar_init(&ms.bar_pv, 1);
     fence_barrier_init();
   }
   if (warp == 0) tmem_alloc(&ms.tmem_slot, kTmemCols);
-  if (tid < kHG) {
-    ms.m_use[tid] = -INFINITY;
-    ms.l_run[tid] = 0.f;
-  }
-  // the selected entry indices of this CTA's rows, fetched once
-  const int64_t sel_end = rl.sel ? min64(r_end, rl.n_sel) : r_begin;
-  for (int64_t r = r_begin + tid; r < sel_end; r += kThreads) ms.sel[r - r_begin] = rl.sel[r];
+  if (tid < kHG) ms.m_use[tid] = -INFINITY;
+  if (tid < 32) rope_tables(a, tq, ms.qcs, ms.qsn, ms.ocs, ms.osn);
+  if (tid < kRows) ms.rowp[0][tid] = n_chunks > 0 ? chunk_row(a, rl, b, r_begin + tid, r_end, rb) : nullptr;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ms.tmem_slot;
+  if (warp < 4) {  // the all-ones A operand of the row-sum product
+    float ones[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) ones[i] = __uint_as_float(0x3F803F80u);
+    tmem_st_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + kColOnes, ones);
+    tmem_st_wait();
+  }
+  // the first chunk's rows are on their way while the query tile is prepared
+  if (n_chunks > 0) {
+    if (FP8) gather_fp8(raw, ms.rowp[0], &ms.bar_raw);
+    else gather_bf16(KV, ms.rowp[0], a.Q);
+  }
+  cp_async_wait_pending((!FP8 && n_chunks > 0) ? 4 : 0);  // the query tile's group
+  fence_proxy_async_smem();
+  __syncthreads();
+  if (a.q_norm_g != nullptr || a.q_rope_dims > 0) {
+    // RMSNorm and RoPE of the query rows in place: warp w takes heads w, w+8,
+    // ...; lane l owns dims 8l..8l+7 and 256+8l..+7 (the order of
+    // csa_rmsnorm_rope, so the bytes agree)
+    const int d_rope = kDim - a.q_rope_dims;
+    for (int h = warp; h < kHG; h += kThreads / 32) {
+      float v[2][8];
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const uint4 u = *reinterpret_cast<const uint4*>(Qs + q_off(h, lane + 32 * k));
+        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          v[k][2 * j] = __uint_as_float(w4[j] << 16);
+          v[k][2 * j + 1] = __uint_as_float(w4[j] & 0xFFFF0000u);
+        }
+      }
+      if (a.q_norm_g != nullptr) {
+        float ss = 0.f;
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) ss = fmaf(v[k][q], v[k][q], ss);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float inv = rms_inv(ss, kDim, a.q_norm_eps);
+#pragma unroll
+        for (int k = 0; k < 2; ++k)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) v[k][q] = __fmul_rn(__fmul_rn(v[k][q], inv), a.q_norm_g[8 * (lane + 32 * k) + q]);
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int d0 = 8 * (lane + 32 * k);
+        if (a.q_rope_dims > 0 && d0 >= d_rope) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int kp = (d0 - d_rope) / 2 + j;
+            rope_turn(v[k][2 * j], v[k][2 * j + 1], ms.qcs[kp], ms.qsn[kp]);
+          }
+        }
+        *reinterpret_cast<uint4*>(Qs + q_off(h, lane + 32 * k)) = pack_bf16x8(v[k]);
+      }
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+  }
   const float sl2 = a.scale * kLog2e;
+  const uint32_t kva = smem_u32(KV), qa = smem_u32(Qs), pa = smem_u32(Ps);
 
   for (int ci = 0; ci < n_chunks; ++ci) {
-    // ---- row pointers and validity
-    if (tid < kRows) {
-      const int64_t r = r_begin + (int64_t)ci * kRows + tid;
-      const uint8_t* p = nullptr;
-      if (r < r_end) {
-        if (r < rl.n_sel) {
-          const int64_t e = rl.sel ? (int64_t)ms.sel[r - r_begin] : r;
-          if (e >= 0 && e < rl.vis) p = static_cast<const uint8_t*>(a.entries) + ((int64_t)b * a.n_entries + e) * rb;
-        } else {
-          p = row_ptr(a, rl, b, r, rb);
-        }
+    const uint32_t par = (uint32_t)(ci & 1);
+    const uint8_t* const* rowp = ms.rowp[ci & 1];
+    // ---- rows -> row tile, S^T = K Q^T issued part by part
+    if (FP8) {
+      mbar_wait(&ms.bar_raw, par);
+      // dims 0..255 straight into atoms 0..3 (no overlap with the staging)
+      for (int u = tid; u < kRows * 32; u += kThreads)
+        *reinterpret_cast<uint4*>(KV + kv_off(u >> 5, u & 31)) = expand_fp8(raw, u >> 5, u & 31);
+      fence_proxy_async_smem();
+      mbar_arrive(&ms.bar_half[0]);
+      if (tid == 0) {
+        mbar_wait(&ms.bar_half[0], par);
+        tc_fence_after();
+        issue_qk(tmem, kva, qa, 0, 4);
       }
-      ms.rowp[tid] = p;
-    }
-    __syncthreads();
-    // ---- gather the rows into the row tile (zeros for absent rows)
-    if (!FP8) {
-      for (int u = tid; u < kRows * 64; u += kThreads) {
-        const int r = u >> 6, g = u & 63;
-        const uint8_t* src = ms.rowp[r];
-        cp_async16(smem_u32(KV + kv_off(r, g)), src ? src + g * 16 : static_cast<const uint8_t*>(a.Q), src != nullptr);
-      }
-      cp_async_commit();
-      cp_async_wait_all();
-    } else {
-      // FP8MIX: the raw rows land in atoms 4..7 + P in one cp.async round
-      // trip, then expand (codes x block scale -> bf16, RoPE dims copied):
-      // dims 0..255 straight into atoms 0..3, dims 256..511 through registers
-      // (their destination overlaps the staging area)
-      uint8_t* raw = base + kOffRaw;
-      for (int u = tid; u < kRows * (kRawRow / 16); u += kThreads) {
-        const int r = u / (kRawRow / 16), c = u % (kRawRow / 16);
-        const uint8_t* src = ms.rowp[r];
-        cp_async16(smem_u32(raw + r * kRawRow + c * 16), src ? src + c * 16 : static_cast<const uint8_t*>(a.Q),
-                   src != nullptr);
-      }
-      cp_async_commit();
-      cp_async_wait_all();
-      __syncthreads();
-      auto expand = [&](int r, int g) -> uint4 {
-        const uint8_t* row = raw + r * kRawRow;
-        if (g >= 56) return *reinterpret_cast<const uint4*>(row + 448 + (g - 56) * 16);
-        const uint2 v = *reinterpret_cast<const uint2*>(row + g * 8);
-        const float sc = *reinterpret_cast<const float*>(row + 576 + 4 * (g >> 3));
-        uint32_t w[4];
-        const uint32_t src[2] = {v.x, v.y};
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const float2 lo = e4m3x2_to_float2((uint16_t)(src[q] & 0xFFFF));
-          const float2 hi = e4m3x2_to_float2((uint16_t)(src[q] >> 16));
-          const __nv_bfloat162 x0 = __floats2bfloat162_rn(lo.x * sc, lo.y * sc);
-          const __nv_bfloat162 x1 = __floats2bfloat162_rn(hi.x * sc, hi.y * sc);
-          memcpy(&w[2 * q], &x0, 4);
-          memcpy(&w[2 * q + 1], &x1, 4);
-        }
-        return make_uint4(w[0], w[1], w[2], w[3]);
-      };
-      // absent rows were zero-filled: zero codes and scales expand to zeros
-      for (int u = tid; u < kRows * 32; u += kThreads) {
-        const int r = u >> 5, g = u & 31;
-        *reinterpret_cast<uint4*>(KV + kv_off(r, g)) = expand(r, g);
-      }
+      // dims 256..511 through registers (their destination overlaps the staging)
       constexpr int kHi = kRows * 32 / kThreads;  // 16 chunks per thread
       uint4 hi[kHi];
 #pragma unroll
       for (int j = 0; j < kHi; ++j) {
         const int u = tid + j * kThreads;
-        hi[j] = expand(u >> 5, 32 + (u & 31));
+        hi[j] = expand_fp8(raw, u >> 5, 32 + (u & 31));
       }
       __syncthreads();
 #pragma unroll
@@ -266,201 +418,163 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
         const int u = tid + j * kThreads;
         *reinterpret_cast<uint4*>(KV + kv_off(u >> 5, 32 + (u & 31))) = hi[j];
       }
+      fence_proxy_async_smem();
+      mbar_arrive(&ms.bar_half[1]);
+      if (tid == 0) {
+        mbar_wait(&ms.bar_half[1], par);
+        tc_fence_after();
+        issue_qk(tmem, kva, qa, 4, 8);
+        tc_commit(&ms.bar_qk);
+      }
+    } else {
+      for (int p = 0; p < 4; ++p) {
+        cp_async_wait_pending(3 - p);
+        fence_proxy_async_smem();
+        mbar_arrive(&ms.bar_pair[p]);
+        if (tid == 0) {
+          mbar_wait(&ms.bar_pair[p], par);
+          tc_fence_after();
+          issue_qk(tmem, kva, qa, 2 * p, 2 * p + 2);
+          if (p == 3) tc_commit(&ms.bar_qk);
+        }
+      }
     }
-    fence_proxy_async_smem();  // generic-proxy tile writes -> tensor core reads
+
+    // ---- softmax: warp (quad, half) owns rows 32 quad.. and heads 32 half..
+    mbar_wait(&ms.bar_qk, par);
+    tc_fence_after();
+    const int r = 32 * quad + lane;
+    const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
+    float s[32];
+    tmem_ld_32x32b_x32(tmem + lane_base + kColS + 32 * half, s);
+    tmem_ld_wait();
+    const bool ok = rowp[r] != nullptr;
+#pragma unroll
+    for (int h = 0; h < 32; ++h) s[h] = ok ? s[h] * sl2 : -INFINITY;
+#pragma unroll
+    for (int h = 0; h < 32; ++h) {
+      const float wm = warp_max_f32(s[h]);
+      if (lane == h) ms.red[quad][32 * half + h] = wm;
+    }
     __syncthreads();
-
-    // ---- S^T = K Q^T
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t kva = smem_u32(KV), qa = smem_u32(Qs);
-#pragma unroll
-      for (int at = 0; at < 8; ++at)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          tc_mma_f16(tmem + kColS, umma_desc_sw128(kva + at * (kRows * 128) + kk * 32),
-                     umma_desc_sw128(qa + at * (kHG * 128) + kk * 32), kIdescQK, (at | kk) ? 1u : 0u);
-      tc_commit(&ms.bar_qk);
+    bool raised = false;
+    if (tid < kHG) {
+      const float cm = fmaxf(fmaxf(ms.red[0][tid], ms.red[1][tid]), fmaxf(ms.red[2][tid], ms.red[3][tid]));
+      const float mold = ms.m_use[tid];
+      float use = mold;
+      if (mold == -INFINITY || cm > mold + kLazy) use = fmaxf(mold, cm);
+      ms.corr[tid] = (mold == -INFINITY || use == mold) ? 1.f : exp2f(mold - use);
+      raised = mold != -INFINITY && use != mold;
+      ms.m_use[tid] = use;
     }
-
-    // ---- softmax on the 128 threads that own the TMEM lanes (row = tid)
-    if (warp < 4) {
-      mbar_wait(&ms.bar_qk, (uint32_t)(ci & 1));
-      tc_fence_after();
-      float s[kHG];
-      const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-      tmem_ld_32x32b_x32(tmem + lane_base + kColS, s);
-      tmem_ld_32x32b_x32(tmem + lane_base + kColS + 32, s + 32);
-      tmem_ld_wait();
-      const bool ok = ms.rowp[tid] != nullptr;
+    const int rescale = __syncthreads_or(raised ? 1 : 0);
+    // P = 2^(s - m) as bf16, MN-major: row r's 128-byte line, heads 32 half..
 #pragma unroll
-      for (int h = 0; h < kHG; ++h) s[h] = ok ? s[h] * sl2 : -INFINITY;
-      // per-head maximum over the warp's 32 rows (one redux per head)
+    for (int h = 0; h < 32; ++h) {
+      const float m = ms.m_use[32 * half + h];
+      s[h] = (s[h] == -INFINITY || m == -INFINITY) ? 0.f : exp2f(s[h] - m);
+    }
 #pragma unroll
-      for (int h = 0; h < kHG; ++h) {
-        const float wm = warp_max_f32(s[h]);
-        if (lane == (h >> 1)) ms.red[warp][h] = wm;
-      }
-      softmax_sync();
-      if (warp == 0) {
-        bool raised = false;
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int h = 2 * lane + j;
-          const float cm = fmaxf(fmaxf(ms.red[0][h], ms.red[1][h]), fmaxf(ms.red[2][h], ms.red[3][h]));
-          const float mold = ms.m_use[h];
-          float use = mold;
-          if (mold == -INFINITY || cm > mold + kLazy) use = fmaxf(mold, cm);
-          ms.corr[h] = (mold == -INFINITY || use == mold) ? 1.f : exp2f(mold - use);
-          raised |= mold != -INFINITY && use != mold;
-          ms.m_use[h] = use;
-        }
-        const unsigned any = __ballot_sync(0xffffffffu, raised);
-        if (lane == 0) ms.rescale = any != 0u;
-      }
-      softmax_sync();
-      // P = 2^(s - m) as bf16, written MN-major (a 128-byte line per row)
-#pragma unroll
-      for (int h = 0; h < kHG; ++h) {
-        const float m = ms.m_use[h];
-        s[h] = (s[h] == -INFINITY || m == -INFINITY) ? 0.f : exp2f(s[h] - m);
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const __nv_bfloat162 x = __floats2bfloat162_rn(s[8 * c + 2 * q], s[8 * c + 2 * q + 1]);
-          memcpy(&w[q], &x, 4);
-        }
-        *reinterpret_cast<uint4*>(Ps + tid * 128 + ((c ^ (tid & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      // row sums per head of the bf16 probabilities the product will use
-      float v[kHG], c0, c1;
-#pragma unroll
-      for (int h = 0; h < kHG; ++h) v[h] = __bfloat162float(__float2bfloat16_rn(s[h]));
-      reduce_scatter64<false>(v, lane, c0, c1);
-      ms.red[warp][2 * lane] = c0;
-      ms.red[warp][2 * lane + 1] = c1;
-      softmax_sync();
-      if (warp == 0) {
-#pragma unroll
-        for (int j = 0; j < 2; ++j) {
-          const int h = 2 * lane + j;
-          const float cs = (ms.red[0][h] + ms.red[1][h]) + (ms.red[2][h] + ms.red[3][h]);
-          ms.l_run[h] = ms.l_run[h] * ms.corr[h] + cs;
-        }
-      }
-      // a raised max rescales the output accumulated so far (lane = dim)
-      if (ci > 0 && ms.rescale) {
+    for (int c4 = 0; c4 < 4; ++c4)
+      *reinterpret_cast<uint4*>(Ps + r * 128 + (((4 * half + c4) ^ (r & 7)) << 4)) = pack_bf16x8(s + 8 * c4);
+    // a raised max rescales what O^T and L accumulated so far (lane = dim)
+    if (ci > 0 && rescale) {
 #pragma unroll 1
-        for (int sl = 0; sl < 4; ++sl) {
-          float o[kHG];
-          const uint32_t ta = tmem + lane_base + kColO + sl * kHG;
-          tmem_ld_32x32b_x32(ta, o);
-          tmem_ld_32x32b_x32(ta + 32, o + 32);
-          tmem_ld_wait();
+      for (int sl = 2 * half; sl < 2 * half + 2 + (half == 0 ? 1 : 0); ++sl) {
+        const uint32_t col = sl < 2 * half + 2 ? kColO + sl * kHG : kColL;
+        float o[kHG];
+        tmem_ld_32x32b_x32(tmem + lane_base + col, o);
+        tmem_ld_32x32b_x32(tmem + lane_base + col + 32, o + 32);
+        tmem_ld_wait();
 #pragma unroll
-          for (int h = 0; h < kHG; ++h) o[h] *= ms.corr[h];
-          tmem_st_32x32b_x32(ta, o);
-          tmem_st_32x32b_x32(ta + 32, o + 32);
-        }
-        tmem_st_wait();
+        for (int h = 0; h < kHG; ++h) o[h] *= ms.corr[h];
+        tmem_st_32x32b_x32(tmem + lane_base + col, o);
+        tmem_st_32x32b_x32(tmem + lane_base + col + 32, o + 32);
       }
-      tc_fence_before();
+      tmem_st_wait();
     }
+    tc_fence_before();
     fence_proxy_async_smem();  // P (generic stores) -> tensor core reads
     __syncthreads();
 
-    // ---- O^T += V^T P^T, four 128-dim slabs
+    // ---- O^T += V^T P^T (slab by slab) and L += 1 P^T
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t kva = smem_u32(KV), pa = smem_u32(Ps);
 #pragma unroll
-      for (int sl = 0; sl < 4; ++sl)
+      for (int sl = 0; sl < 4; ++sl) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          tc_mma_f16(tmem + kColO + sl * kHG,
-                     umma_desc_sw128_mn(kva + (2 * sl) * (kRows * 128) + kk * 2048, kRows * 128, 1024),
-                     umma_desc_sw128_mn(pa + kk * 2048, kRows * 128, 1024), kIdescPV,
-                     (ci > 0 || kk > 0) ? 1u : 0u);
+          tc_mma_f16(tmem + kColO + sl * kHG, umma_desc_sw128_mn(kva + (2 * sl) * kAtom + kk * 2048, kAtom, 1024),
+                     umma_desc_sw128_mn(pa + kk * 2048, kAtom, 1024), kIdescPV, (ci > 0 || kk > 0) ? 1u : 0u);
+        tc_commit(&ms.bar_slab[sl]);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        tc_mma_f16_ta(tmem + kColL, tmem + kColOnes, umma_desc_sw128_mn(pa + kk * 2048, kAtom, 1024), kIdescL,
+                      (ci > 0 || kk > 0) ? 1u : 0u);
       tc_commit(&ms.bar_pv);
     }
-    // the next chunk overwrites the row tile and P: wait for the product
-    mbar_wait(&ms.bar_pv, (uint32_t)(ci & 1));
-    tc_fence_after();
+
+    // ---- the next chunk's rows
+    if (ci + 1 < n_chunks) {
+      if (tid < kRows)
+        ms.rowp[(ci + 1) & 1][tid] = chunk_row(a, rl, b, r_begin + (int64_t)(ci + 1) * kRows + tid, r_end, rb);
+      if (FP8) {
+        // the staging overlaps atoms 4..7 and P: wait for every product
+        mbar_wait(&ms.bar_pv, par);
+        tc_fence_after();
+        __syncthreads();
+        gather_fp8(raw, ms.rowp[(ci + 1) & 1], &ms.bar_raw);
+      } else {
+        __syncthreads();
+        // atoms 2p, 2p+1 are free once the slab-p products have read them
+        for (int p = 0; p < 4; ++p) {
+          mbar_wait(&ms.bar_slab[p], par);
+          const uint8_t* const* nrow = ms.rowp[(ci + 1) & 1];
+          for (int u = tid; u < kRows * 16; u += kThreads) {
+            const int rr = u >> 4, g = 16 * p + (u & 15);
+            const uint8_t* src = nrow[rr];
+            cp_async16(smem_u32(KV + kv_off(rr, g)), src ? src + g * 16 : a.Q, src != nullptr);
+          }
+          cp_async_commit();
+        }
+      }
+    }
   }
-  cp_async_wait_all();
-  __syncthreads();
-  // ---- epilogue: O[h][d] = O^T[d][h] * fac[h]
-  const uint32_t lb = (uint32_t)((warp & 3) * 32) << 16;
-  auto load_slab = [&](int sl, float* o) {  // warps 0-3: lane = dim sl * 128 + tid
+  if (n_chunks > 0) mbar_wait(&ms.bar_pv, (uint32_t)((n_chunks - 1) & 1));
+  tc_fence_after();
+
+  // ---- epilogue: sums, then O^T staged as fp32 [head][512 dims] in the row tile
+  if (warp == 0) {
+    float l[kHG];
     if (n_chunks > 0) {
-      tmem_ld_32x32b_x32(tmem + lb + kColO + sl * kHG, o);
-      tmem_ld_32x32b_x32(tmem + lb + kColO + sl * kHG + 32, o + 32);
+      tmem_ld_32x32b_x32(tmem + kColL, l);
+      tmem_ld_32x32b_x32(tmem + kColL + 32, l + 32);
+      tmem_ld_wait();
+    } else {
+#pragma unroll
+      for (int h = 0; h < kHG; ++h) l[h] = 0.f;
+    }
+    if (lane == 0)
+#pragma unroll
+      for (int h = 0; h < kHG; ++h) ms.lsum[h] = l[h];
+  }
+  float* stg = reinterpret_cast<float*>(KV);
+#pragma unroll 1
+  for (int sl = 2 * half; sl < 2 * half + 2; ++sl) {
+    float o[kHG];
+    if (n_chunks > 0) {
+      const uint32_t ta = tmem + ((uint32_t)(32 * quad) << 16) + kColO + sl * kHG;
+      tmem_ld_32x32b_x32(ta, o);
+      tmem_ld_32x32b_x32(ta + 32, o + 32);
       tmem_ld_wait();
     } else {
 #pragma unroll
       for (int h = 0; h < kHG; ++h) o[h] = 0.f;
     }
-  };
-  if constexpr (MODE != kWhole) {
-    // one split of many: the unnormalised partial (m, l, o).  Warps 0-3 stage
-    // the O^T slabs in the idle row tile as [slab][head][128 dims] while warps
-    // 4-7 write the slabs already staged in 16-byte pieces (each warp store
-    // covers 512 contiguous bytes of one head); named barrier 2 + s marks
-    // slab s staged.
-    float* stg = reinterpret_cast<float*>(KV);
-    if (tid < kHG) {
-      float* ml = plan_partial_ml(plan, a, bt, split, hg * kHG + tid);
-      const float m = ms.m_use[tid];
-      ml[0] = m == -INFINITY ? -INFINITY : m / kLog2e;  // natural-log domain
-      ml[1] = ms.l_run[tid];
-    }
-    if (warp < 4) {
-#pragma unroll 1
-      for (int sl = 0; sl < 4; ++sl) {
-        float o[kHG];
-        load_slab(sl, o);
+    const int d = sl * 128 + 32 * quad + lane;
 #pragma unroll
-        for (int h = 0; h < kHG; ++h) stg[(sl * kHG + h) * 128 + tid] = o[h];
-        named_barrier_arrive(2 + sl, kThreads);
-      }
-    } else {
-      const int t = tid - 128;
-#pragma unroll 1
-      for (int sl = 0; sl < 4; ++sl) {
-        named_barrier_sync(2 + sl, kThreads);
-        for (int q = t; q < kHG * 32; q += 128) {
-          const int h = q >> 5, c = q & 31;
-          const float4 v = *reinterpret_cast<const float4*>(stg + (sl * kHG + h) * 128 + 4 * c);
-          *reinterpret_cast<float4*>(plan_partial_o(plan, a, bt, split, hg * kHG + h) + sl * 128 + 4 * c) = v;
-        }
-      }
-    }
-  } else {
-    if (tid < kHG) {
-      const float sink = a.sink[hg * kHG + tid] * kLog2e;  // log2 domain
-      const float m = ms.m_use[tid];
-      const float M = fmaxf(m, sink);
-      float f = 0.f;
-      if (!(sink == INFINITY) && M != -INFINITY) {
-        const float em = m == -INFINITY ? 0.f : exp2f(m - M);
-        f = em / (ms.l_run[tid] * em + exp2f(sink - M));
-      }
-      ms.fac[tid] = f;
-    }
-    __syncthreads();
-    if (warp < 4) {
-      __nv_bfloat16* ob = static_cast<__nv_bfloat16*>(a.O) + (bt * a.n_heads + (int64_t)hg * kHG) * kDim;
-#pragma unroll 1
-      for (int sl = 0; sl < 4; ++sl) {
-        float o[kHG];
-        load_slab(sl, o);
-#pragma unroll
-        for (int h = 0; h < kHG; ++h) ob[(int64_t)h * kDim + sl * 128 + tid] = __float2bfloat16_rn(o[h] * ms.fac[h]);
-      }
-    }
+    for (int h = 0; h < kHG; ++h) stg[h * kDim + d] = o[h];
   }
   tc_fence_before();
   __syncthreads();
@@ -468,25 +582,126 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+
+  if constexpr (MODE == kMqaWhole) {
+    if (tid < kHG) {
+      const float sink = a.sink[hg * kHG + tid] * kLog2e;  // log2 domain
+      const float m = ms.m_use[tid];
+      const float M = fmaxf(m, sink);
+      float f = 0.f;
+      if (!(sink == INFINITY) && M != -INFINITY) {
+        const float em = m == -INFINITY ? 0.f : exp2f(m - M);
+        f = em / (ms.lsum[tid] * em + exp2f(sink - M));
+      }
+      ms.fac[tid] = f;
+    }
+    __syncthreads();
+    const int d_rope = kDim - a.out_rope_dims;
+    for (int it = tid; it < kItems; it += kThreads) {
+      const int h = it >> 6, d0 = 8 * (it & 63);
+      const float4 x0 = *reinterpret_cast<const float4*>(stg + h * kDim + d0);
+      const float4 x1 = *reinterpret_cast<const float4*>(stg + h * kDim + d0 + 4);
+      const float f = ms.fac[h];
+      float v[8] = {x0.x * f, x0.y * f, x0.z * f, x0.w * f, x1.x * f, x1.y * f, x1.z * f, x1.w * f};
+      if (a.out_rope_dims > 0 && d0 >= d_rope) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int k = (d0 - d_rope) / 2 + q;
+          rope_turn(v[2 * q], v[2 * q + 1], ms.ocs[k], ms.osn[k]);
+        }
+      }
+      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + (bt * a.n_heads + (int64_t)hg * kHG + h) * kDim +
+                                d0) = pack_bf16x8(v);
+    }
+  } else {
+    // one split of several: the unnormalised partial (m, l, o)
+    if (tid < kHG) {
+      float* ml = plan_partial_ml(plan, a, bt, split, hg * kHG + tid);
+      const float m = ms.m_use[tid];
+      ml[0] = m == -INFINITY ? -INFINITY : m / kLog2e;  // natural-log domain
+      ml[1] = ms.lsum[tid];
+    }
+    for (int it = tid; it < kItems; it += kThreads) {
+      const int h = it >> 6, d0 = 8 * (it & 63);
+      float* po = plan_partial_o(plan, a, bt, split, hg * kHG + h) + d0;
+      reinterpret_cast<float4*>(po)[0] = *reinterpret_cast<const float4*>(stg + h * kDim + d0);
+      reinterpret_cast<float4*>(po)[1] = *reinterpret_cast<const float4*>(stg + h * kDim + d0 + 4);
+    }
+    if constexpr (MODE == kMqaCoop) {
+      // the splits of this (query, head group) wait for one another, then
+      // each adds a share of the outputs over all splits
+      __syncthreads();
+      uint32_t* ctr = plan_unit_counters(a, bt * (a.n_heads / kHG) + hg);
+      if (tid == 0) {
+        __threadfence();
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+        const unsigned long long t0 = globaltimer_ns();
+        for (uint32_t it = 1; ld_acquire_gpu(ctr) < (uint32_t)NS; ++it) {
+          if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitTimeoutNs) {
+            atomicOr(&g_device_status, 1u);
+            break;
+          }
+        }
+      }
+      __syncthreads();
+      const int i0 = (int)((int64_t)split * kItems / NS), i1 = (int)((int64_t)(split + 1) * kItems / NS);
+      combine_items(a, plan, bt, hg, i0, i1, stg, ms.ocs, ms.osn);
+      __syncthreads();
+      // the last split to finish leaves the counters at zero for the next call
+      if (tid == 0 && atomicAdd(ctr + 1, 1u) == (uint32_t)NS - 1) {
+        ctr[0] = 0u;
+        ctr[1] = 0u;
+      }
+    }
+  }
+}
+
+// The combine of kMqaSplit mode: one CTA per (head group, query).
+__global__ void __launch_bounds__(kThreads) mqa_umma_combine_kernel(MqaArgs a, MqaPlan plan) {
+  extern __shared__ __align__(16) float cw[];  // [n_splits][64] weights
+  __shared__ float ocs[kMaxRope / 2], osn[kMaxRope / 2], qcs[kMaxRope / 2], qsn[kMaxRope / 2];
+  const int hg = blockIdx.x;
+  const int64_t bt = blockIdx.y;
+  if (threadIdx.x < 32) rope_tables(a, a.q_pos[bt], qcs, qsn, ocs, osn);
+  __syncthreads();
+  combine_items(a, plan, bt, hg, 0, kItems, cw, ocs, osn);
+}
+
+int sm_count_mqa() {
+  static int n = 0;
+  if (n == 0) {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        v <= 0) {
+      cudaGetLastError();
+      return 148;
+    }
+    n = v;
+  }
+  return n;
 }
 
 bool mqa_umma_eligible(const MqaArgs& a) {
   return a.q_dt == CSA_BF16 && (a.kv_dt == CSA_BF16 || a.kv_dt == CSA_KV_FP8MIX) && a.dim == kDim &&
-         a.n_heads % kHG == 0 && (int64_t)a.batch * a.n_q <= 65535 && (a.idx == nullptr || a.k <= kMaxSel);
+         a.n_heads % kHG == 0 && (int64_t)a.batch * a.n_q <= 65535 && (a.idx == nullptr || a.k <= 2048) &&
+         a.q_rope_dims <= kMaxRope && a.out_rope_dims <= kMaxRope;
 }
 
 MqaPlan make_umma_mqa_plan(const MqaArgs& a) {
   MqaPlan p{};
   p.heads_per_cta = kHG;
   p.rows_per_split = 0;
-  // few queries (decode): a query's row chunks are split over CTAs until the
-  // grid fills one wave; the partials are combined by mqa_combine_kernel
+  // automatic: a query's row chunks are split over CTAs until the grid fills
+  // one wave; a fixed count (a.splits) depends on the row count only
+  const int sms = sm_count_mqa();
   const int64_t units = (int64_t)a.batch * a.n_q * (a.n_heads / kHG);
   const int64_t nch = (max_rows_per_query(a) + kRows - 1) / kRows;
-  int64_t ns = 148 / units;
+  int64_t ns = a.splits > 0 ? a.splits : (units >= sms ? 1 : sms / units);
   if (ns > nch) ns = nch;
   if (ns < 1) ns = 1;
   p.n_splits = (int)ns;
+  p.mode = ns == 1 ? kMqaWhole : (units * ns <= sms ? kMqaCoop : kMqaSplit);
+  p.ws_head = ns == 1 ? 0 : kMqaCounterBytes;
   return p;
 }
 
@@ -496,16 +711,33 @@ cudaError_t launch_umma(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) {
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
   const dim3 grid((unsigned)p.n_splits, a.n_heads / kHG, (unsigned)((int64_t)a.batch * a.n_q));
+  if (MODE == kMqaCoop) {
+    // the splits of a (query, head group) wait for one another: every CTA
+    // must be resident at once
+    MqaArgs aa = a;
+    MqaPlan pp = p;
+    void* args[] = {&aa, &pp};
+    e = cudaLaunchCooperativeKernel((const void*)kern, grid, dim3(kThreads), args, kSmemBytes, s);
+    ++launch_counter();
+    return e;
+  }
   kern<<<grid, kThreads, kSmemBytes, s>>>(a, p);
   ++launch_counter();
   e = cudaGetLastError();
-  if (e != cudaSuccess || MODE != kSplit) return e;
-  return launch_mqa_combine(a, p, s);
+  if (e != cudaSuccess || MODE != kMqaSplit) return e;
+  const size_t cs = (size_t)p.n_splits * kHG * sizeof(float);
+  e = cudaFuncSetAttribute(mqa_umma_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cs);
+  if (e != cudaSuccess) return e;
+  mqa_umma_combine_kernel<<<dim3(a.n_heads / kHG, (unsigned)((int64_t)a.batch * a.n_q)), kThreads, cs, s>>>(a, p);
+  ++launch_counter();
+  return cudaGetLastError();
 }
 
 template <bool FP8>
 cudaError_t launch_umma_fmt(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) {
-  return p.n_splits > 1 ? launch_umma<FP8, kSplit>(a, p, s) : launch_umma<FP8, kWhole>(a, p, s);
+  if (p.mode == kMqaCoop) return launch_umma<FP8, kMqaCoop>(a, p, s);
+  if (p.mode == kMqaSplit) return launch_umma<FP8, kMqaSplit>(a, p, s);
+  return launch_umma<FP8, kMqaWhole>(a, p, s);
 }
 
 }  // namespace

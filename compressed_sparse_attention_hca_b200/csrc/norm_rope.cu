@@ -6,6 +6,7 @@
 // (a position of 10^6 times a frequency near 1 leaves fp32 no fractional
 // bits); the sine and cosine of the reduced angle are taken in fp32.
 #include "csa_internal.cuh"
+#include "rope_dev.cuh"
 
 namespace csa {
 namespace {
@@ -60,11 +61,10 @@ __global__ void __launch_bounds__(256) norm_rope_kernel(NormRopeArgs a) {
   for (int c = lane; c < nch && own < kMaxOwn; c += 32) {
     if (8 * c < d_rope) continue;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) theta[own][j] = pow(a.base, -2.0 * ((8 * c - d_rope) / 2 + j) / a.rope_dims);
+    for (int j = 0; j < 4; ++j) theta[own][j] = rope_theta(a.base, (8 * c - d_rope) / 2 + j, a.rope_dims);
     ++own;
   }
   const bool table = (nch - d_rope / 8 + 31) / 32 <= kMaxOwn;  // every lane's rotated chunks fit
-  constexpr double kTwoPiHi = 6.283185307179586232, kTwoPiLo = 2.4492935982947064e-16, kInvTwoPi = 0.15915494309189535;
   for (int64_t r = warp0; r < a.n_rows; r += n_warps) {
     const int64_t row = r * a.dim;
     float inv = 1.f;
@@ -78,7 +78,7 @@ __global__ void __launch_bounds__(256) norm_rope_kernel(NormRopeArgs a) {
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      inv = 1.f / sqrtf(ss / (float)a.dim + a.eps);
+      inv = rms_inv(ss, a.dim, a.eps);
     }
     const double p = a.rope_dims > 0 ? (double)a.pos[r / a.rows_per_pos] * (double)a.pos_sign : 0.0;
     int slot = 0;
@@ -87,20 +87,15 @@ __global__ void __launch_bounds__(256) norm_rope_kernel(NormRopeArgs a) {
       nr_load8(a.x, a.in_dt, row + 8 * c, v);
       if (a.g != nullptr) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) v[q] = v[q] * inv * a.g[8 * c + q];
+        for (int q = 0; q < 8; ++q) v[q] = __fmul_rn(__fmul_rn(v[q], inv), a.g[8 * c + q]);
       }
       if (8 * c >= d_rope) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const double th = table ? theta[slot][j] : pow(a.base, -2.0 * ((8 * c - d_rope) / 2 + j) / a.rope_dims);
-          const double ang = p * th;
-          const double n = rint(ang * kInvTwoPi);
-          const float red = (float)fma(-n, kTwoPiLo, fma(-n, kTwoPiHi, ang));
+          const double th = table ? theta[slot][j] : rope_theta(a.base, (8 * c - d_rope) / 2 + j, a.rope_dims);
           float sn, cs;
-          sincosf(red, &sn, &cs);
-          const float x0 = v[2 * j], x1 = v[2 * j + 1];
-          v[2 * j] = x0 * cs - x1 * sn;
-          v[2 * j + 1] = x0 * sn + x1 * cs;
+          rope_sincos(p, th, &sn, &cs);
+          rope_turn(v[2 * j], v[2 * j + 1], cs, sn);
         }
         if (table) ++slot;
       }

@@ -339,6 +339,8 @@ csa_status_t csa_index_topk_noalloc(const void* qI, const void* qI_sf, const flo
  *             window token of every query must be present.
  *   q_pos     [batch][n_q] int64 (device); sink [n_heads] fp32 (device).
  * Limits: dim a multiple of 64 (<= 512), n_heads <= 128, k <= 2048.
+ * Workspace: zero-filled before its first use (the split counters in its
+ * first 4096 bytes; every call leaves them zero, the rest is scratch).
  */
 size_t csa_sparse_mqa_workspace_size(int batch, int n_q, int n_heads, int dim, int k, int window,
                                      csa_dtype_t q_dt, csa_dtype_t kv_dt);
@@ -348,6 +350,65 @@ csa_status_t csa_sparse_mqa(const void* Q, csa_dtype_t q_dt, const void* entries
                             int window, int m, const float* sink, float softmax_scale, int batch,
                             int n_q, int n_heads, int dim, csa_dtype_t kv_dt, void* O, void* ws,
                             size_t ws_bytes, void* stream);
+
+/*
+ * csa_mqa_options_t -- options of the attention calls (the *_ex variants; a
+ * NULL options pointer, or a zero-filled struct, gives the plain calls).
+ *
+ *   splits      0: the rows of a query are split over as many CTAs as fill
+ *               the GPU for this batch (decode) -- the split count then
+ *               depends on the batch, and so do the last bits of the output.
+ *               n >= 1: batch-invariant decode ([P1] infrastructure section:
+ *               batch-invariant kernels; [P5] 6.3): each query's rows are cut
+ *               into min(n, ceil(rows / 128)) splits of whole 128-row chunks,
+ *               where rows = k + window (sparse) or n_entries + window
+ *               (dense), and the splits are added in split order -- the
+ *               accumulation order of a query depends on its own rows only,
+ *               so a request gives the same bytes in any batch.  n = 1 runs
+ *               each query (per 64 heads) on one SM.  At most 256.
+ *   q_norm_g    NULL, or [dim] fp32 RMSNorm weights applied to every query
+ *               head before attention ([P5] 1.4 table: RMSNorm on the query
+ *               heads): q <- g * q / sqrt(mean(q^2) + q_norm_eps), the
+ *               arithmetic of csa_rmsnorm_rope (so the query the products use
+ *               has exactly the bytes csa_rmsnorm_rope would give it).
+ *   q_rope_dims RoPE dims turned on the query at its position q_pos (after
+ *               the normalisation; 0 = none), as csa_rmsnorm_rope with
+ *               rows_per_pos = n_heads and pos_sign = +1.
+ *   out_rope_dims  RoPE dims of the output turned at -q_pos before the
+ *               output is rounded ([P5] 1.4 table: the output at position
+ *               -i); 0 = none.
+ *   rope_base   RoPE base for both (e.g. 10000).
+ * The normalisation and RoPE options need the tensor-core path (bf16 Q and
+ * O, BF16 or KV_FP8MIX rows, dim 512, n_heads a multiple of 64) and
+ * q_rope_dims, out_rope_dims multiples of 8 in [0, 64]; otherwise
+ * CSA_ERR_UNSUPPORTED / CSA_ERR_INVALID_ARG before any launch.
+ */
+typedef struct {
+  int splits;
+  const float* q_norm_g;
+  float q_norm_eps;
+  int q_rope_dims;
+  int out_rope_dims;
+  double rope_base;
+} csa_mqa_options_t;
+
+/*
+ * csa_mqa_workspace_size -- workspace bytes of an attention call with these
+ * options (rows_per_query = k + window for csa_sparse_mqa_ex, n_entries +
+ * window for hca_dense_mqa_ex).  The workspace must be zero-filled before its
+ * first use (its first 4096 bytes hold the counters with which the splits of
+ * a query meet; every call leaves them zero, the rest is scratch).
+ */
+size_t csa_mqa_workspace_size(int batch, int n_q, int n_heads, int dim, int64_t rows_per_query,
+                              csa_dtype_t q_dt, csa_dtype_t kv_dt, const csa_mqa_options_t* opt);
+
+/* csa_sparse_mqa with options (see csa_mqa_options_t). */
+csa_status_t csa_sparse_mqa_ex(const void* Q, csa_dtype_t q_dt, const void* entries,
+                               int64_t n_entries, const int32_t* idx, int k, const void* win,
+                               int64_t win_len, const int64_t* win_start, const int64_t* q_pos,
+                               int window, int m, const float* sink, float softmax_scale, int batch,
+                               int n_q, int n_heads, int dim, csa_dtype_t kv_dt, void* O, void* ws,
+                               size_t ws_bytes, const csa_mqa_options_t* opt, void* stream);
 
 /*
  * hca_dense_mqa -- HCA core attention ([P5] 1.3: no top-k; every compressed
@@ -363,6 +424,14 @@ csa_status_t hca_dense_mqa(const void* Q, csa_dtype_t q_dt, const void* entries,
                            const float* sink, float softmax_scale, int batch, int n_q,
                            int n_heads, int dim, csa_dtype_t kv_dt, void* O, void* ws,
                            size_t ws_bytes, void* stream);
+
+/* hca_dense_mqa with options (see csa_mqa_options_t). */
+csa_status_t hca_dense_mqa_ex(const void* Q, csa_dtype_t q_dt, const void* entries,
+                              int64_t n_entries, const void* win, int64_t win_len,
+                              const int64_t* win_start, const int64_t* q_pos, int window, int m,
+                              const float* sink, float softmax_scale, int batch, int n_q,
+                              int n_heads, int dim, csa_dtype_t kv_dt, void* O, void* ws,
+                              size_t ws_bytes, const csa_mqa_options_t* opt, void* stream);
 
 #ifdef __cplusplus
 }

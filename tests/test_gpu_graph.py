@@ -14,8 +14,10 @@ from compressed_sparse_attention_hca_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("idx_dt", [csa.IDX_NVFP4, csa.BF16])
-def test_graph_replay_matches_eager(idx_dt):
+@pytest.mark.parametrize("idx_dt,n_h", [(csa.IDX_NVFP4, 16), (csa.BF16, 16), (csa.BF16, 128)])
+def test_graph_replay_matches_eager(idx_dt, n_h):
+    """n_h = 16 runs the SIMT attention with its combine kernel; n_h = 128 the
+    tensor-core attention whose splits combine in one cooperative launch."""
     if not torch.cuda.is_available():
         pytest.fail("needs a CUDA device")
     B, E, k, H, dI, m = 2, 30000, 1024, 64, 128, 4
@@ -29,7 +31,7 @@ def test_graph_replay_matches_eager(idx_dt):
         KI, ksf = W.normal(g, (B, E, dI), 1.0, torch.bfloat16), None
     wI = W.uniform(g, (B, 1, H))
     q_pos = torch.tensor([[m * E - 1], [m * E - 777]], dtype=torch.int64)
-    n_h, c, window = 16, 512, 128
+    c, window = 512, 128
     Q = W.normal(g, (B, 1, n_h, c), 1.0, torch.bfloat16)
     entries = W.normal(g, (B, E, c), 1.0, torch.bfloat16)
     win = W.normal(g, (B, window, c), 1.0, torch.bfloat16)
@@ -40,7 +42,7 @@ def test_graph_replay_matches_eager(idx_dt):
         qI=qI, qsf=qsf, KI=KI, ksf=ksf, wI=wI, q_pos=q_pos, Q=Q, entries=entries, win=win,
         win_start=win_start, sink=sink).items()}
     ws_i = torch.zeros(csa.index_topk_workspace_size(B, 1, E, k, H, dI, idx_dt), dtype=torch.uint8, device=dev)
-    ws_a = torch.empty(csa.sparse_mqa_workspace_size(B, 1, n_h, c, k, window, csa.BF16, csa.BF16),
+    ws_a = torch.zeros(csa.sparse_mqa_workspace_size(B, 1, n_h, c, k, window, csa.BF16, csa.BF16),
                        dtype=torch.uint8, device=dev)
     idx = torch.empty(B, 1, k, dtype=torch.int32, device=dev)
     O = torch.empty(B, 1, n_h, c, dtype=torch.bfloat16, device=dev)
@@ -94,4 +96,31 @@ def test_index_workspace_returns_to_zero(idx_dt):
         torch.cuda.synchronize()
         csa.check_device_status()
         assert int(ws.count_nonzero()) == 0
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+
+
+def test_attention_counters_return_to_zero():
+    """The splits of a decode query meet on counters in the attention
+    workspace; every call leaves them zero, so the same workspace serves the
+    next call."""
+    if not torch.cuda.is_available():
+        pytest.fail("needs a CUDA device")
+    B, E, k, n_h, c, window, m = 2, 3000, 1024, 128, 512, 128, 4
+    g = W.generator(93)
+    q_pos = torch.tensor([[m * E - 1], [m * E - 501]], dtype=torch.int64).cuda()
+    Q = W.normal(g, (B, 1, n_h, c), 1.0, torch.bfloat16).cuda()
+    entries = W.fp8mix_rows(g, (B, E), c).cuda()
+    win = W.fp8mix_rows(g, (B, window), c).cuda()
+    win_start = (q_pos[:, 0] - window + 1).clamp(min=0)
+    sink = W.normal(g, (n_h,), 1.0, torch.float32).cuda()
+    idx = torch.stack([torch.randperm(m * E // m - 200, generator=g)[:k] for _ in range(B)]).view(B, 1, k)
+    idx = idx.to(torch.int32).cuda()
+    ws = torch.zeros(csa.sparse_mqa_workspace_size(B, 1, n_h, c, k, window, csa.BF16, csa.KV_FP8MIX),
+                     dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(3):
+        outs.append(csa.sparse_mqa(Q, entries, idx, win, win_start, q_pos, window, m, sink, c ** -0.5, ws=ws))
+        torch.cuda.synchronize()
+        csa.check_device_status()
+        assert int(ws[:4096].count_nonzero()) == 0
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
