@@ -323,8 +323,7 @@ def sparse_mqa(Q, entries, idx, win, win_start, q_pos, window, m, sink, scale, *
                ws=None, options=None):
     """CSA shared-KV MQA.  Q [B, T, H, c]; entries [B, E, row]; idx [B, T, k] int32;
     win [B, Lw, row]; win_start [B] int64; q_pos [B, T] int64; sink [H] fp32.
-    options: an MqaOptions (mqa_options()) or None.  A workspace passed in
-    must have been zero-filled before its first use."""
+    options: an MqaOptions (mqa_options()) or None."""
     _need_cuda(Q, entries, idx, win, win_start, q_pos, sink)
     B, T, H, c = Q.shape
     kv_dt = _kv_dt(entries, kv_dt)
@@ -334,7 +333,7 @@ def sparse_mqa(Q, entries, idx, win, win_start, q_pos, window, m, sink, scale, *
         O = torch.empty_like(Q)
     need = mqa_workspace_size(B, T, H, c, k + window, q_dt, kv_dt, options)
     if ws is None or ws.numel() < need:
-        ws = torch.zeros(need, device=Q.device, dtype=torch.uint8)  # zero before first use
+        ws = torch.empty(need, device=Q.device, dtype=torch.uint8)
     _check(load().csa_sparse_mqa_ex(_ptr(Q), q_dt, _ptr(entries), entries.shape[1], _ptr(idx), k, _ptr(win),
                                     win.shape[1], _ptr(win_start), _ptr(q_pos), window, m, _ptr(sink),
                                     float(scale), B, T, H, c, kv_dt, _ptr(O), _ptr(ws), ws.numel(),
@@ -353,7 +352,7 @@ def hca_dense_mqa(Q, entries, win, win_start, q_pos, window, m, sink, scale, *, 
         O = torch.empty_like(Q)
     need = mqa_workspace_size(B, T, H, c, entries.shape[1] + window, q_dt, kv_dt, options)
     if ws is None or ws.numel() < need:
-        ws = torch.zeros(need, device=Q.device, dtype=torch.uint8)  # zero before first use
+        ws = torch.empty(need, device=Q.device, dtype=torch.uint8)
     _check(load().hca_dense_mqa_ex(_ptr(Q), q_dt, _ptr(entries), entries.shape[1], _ptr(win), win.shape[1],
                                    _ptr(win_start), _ptr(q_pos), window, m, _ptr(sink), float(scale), B, T,
                                    H, c, kv_dt, _ptr(O), _ptr(ws), ws.numel(), _opt_ref(options), _stream()))

@@ -11,8 +11,6 @@ namespace csa {
 enum MqaMode {
   kMqaWhole = 0,  // one CTA per (query, head group): normalised output directly
   kMqaSplit = 1,  // split rows; partials combined by a separate kernel
-  kMqaCoop = 2,   // split rows; the splits combine their partials in the same
-                  // (cooperative) launch
 };
 
 struct MqaPlan {
@@ -23,12 +21,7 @@ struct MqaPlan {
   int64_t ws_head;         // bytes of the workspace before the partials
 };
 
-// Split counters of the cooperative mode: two words per (query, head group)
-// unit at the start of the workspace, in a fixed region (a cooperative grid
-// has at most one unit per SM), so that workspaces reused across shapes
-// never overlap a partial with a counter.  Zero before the first call; every
-// call leaves them zero.
-constexpr int64_t kMqaCounterBytes = 4096;
+
 
 // Rows attended by one query ("DeepSeek-V4 内部机制" 1.2 Step 2 and 1.4): the
 // selected entries (CSA: k slots, -1 unused; HCA: every visible entry), then
@@ -82,9 +75,6 @@ __host__ __device__ __forceinline__ float* plan_partial_ml(const MqaPlan& p, con
   const int64_t n_bt = (int64_t)a.batch * a.n_q;
   return plan_partials(p, a) + n_bt * p.n_splits * a.n_heads * (int64_t)a.dim +
          ((bt * p.n_splits + s) * a.n_heads + h) * 2;
-}
-__host__ __device__ __forceinline__ uint32_t* plan_unit_counters(const MqaArgs& a, int64_t unit) {
-  return static_cast<uint32_t*>(a.ws) + unit * 2;
 }
 
 inline size_t plan_mqa_workspace_bytes(const MqaPlan& p, const MqaArgs& a) {

@@ -27,14 +27,19 @@
 // in TMEM rarely.  A CTA with several BF16 chunks gathers the next chunk's
 // atoms as soon as the products of the current chunk have read them.
 //
+// The query tile arrives by TMA; the first chunk's entry indices are fetched
+// together with the query position.
+//
 // Rows split over several CTAs (decode: few queries) give partials
-// (max, sum, o) per split.  When the grid fits the GPU at once (cooperative
-// launch) the splits of a (query, head group) wait for one another on a
-// counter and each combines a share of the outputs with the sink; otherwise a
-// separate kernel does the same combine.  Both add the splits in split order
-// with the same arithmetic, and with a fixed split count (an option) the
-// split boundaries depend only on the query's rows: a request's output then
-// does not depend on the batch it runs in.
+// (max, sum, o) per split, staged in shared memory and written by bulk
+// copies; a combine kernel (a CTA per query and head, all of a thread's split
+// operands loaded at once) adds them in split order with the sink.  With a
+// fixed split count (an option) the split boundaries depend only on the
+// query's rows: a request's output then does not depend on the batch it runs
+// in.  (Measured alternatives, removed: the splits meeting on a global
+// counter in one cooperative launch, and a thread block cluster exchanging
+// the partials through distributed shared memory; both spent longer in the
+// exchange than the partial write and the combine launch cost.)
 //
 // Options: RMSNorm of the query and RoPE of its last dims at the query
 // position (prologue, the same arithmetic as csa_rmsnorm_rope), and RoPE of
@@ -58,6 +63,7 @@ constexpr int kItems = kHG * kDim / 8;  // output items of a head group: (head, 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLazy = 8.f;     // log2 headroom before the running max is raised
 constexpr int kMaxRope = 64;     // RoPE dims the fused options support
+constexpr int kMaxSplits = 256;        // splits of a query (the combine's shared memory)
 
 // Shared memory (offsets from a 1024-byte aligned base).  The upper half of
 // the row tile and P together stage a chunk of raw FP8MIX rows.
@@ -79,10 +85,11 @@ struct Misc {
   float qcs[kMaxRope / 2], qsn[kMaxRope / 2];  // RoPE at +t (query)
   float ocs[kMaxRope / 2], osn[kMaxRope / 2];  // RoPE at -t (output)
   const uint8_t* rowp[2][kRows];               // rows of the current / next chunk
-  uint64_t bar_raw, bar_half[2], bar_pair[4], bar_qk, bar_slab[4], bar_pv;
+  uint64_t bar_q, bar_raw, bar_half[2], bar_pair[4], bar_qk, bar_slab[4], bar_pv;
   uint32_t tmem_slot;
 };
 constexpr int kSmemBytes = 1024 + kOffMisc + (int)sizeof(Misc);
+static_assert(kOffMisc % 16 == 0, "bulk-copy sources are 16-byte aligned");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
 // TMEM columns: S^T (64), O^T slabs 0..3 (64 each), L (64), ones (32).
@@ -129,17 +136,22 @@ __device__ __forceinline__ float warp_max_f32(float v) {
   asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v));
   return r;
 }
-__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
 
 // Address of row r of the query's attended rows when it lies in [.., r_end),
 // else nullptr (absent rows are zero-filled and masked).
 __device__ __forceinline__ const uint8_t* chunk_row(const MqaArgs& a, const RowList& rl, int b, int64_t r,
                                                     int64_t r_end, int64_t rb) {
   return r < r_end ? row_ptr(a, rl, b, r, rb) : nullptr;
+}
+
+__device__ __forceinline__ uint4 pack_bf16x8(const float* v) {
+  uint32_t w[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
+    memcpy(&w[q], &h, 4);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
 // BF16 rows: one cp.async commit group per pair of atoms (128 dims).
@@ -171,24 +183,24 @@ __device__ __forceinline__ void gather_fp8(uint8_t* raw, const uint8_t* const* r
   }
 }
 
-// 16-byte chunk g (dims 8g .. 8g+7) of raw FP8MIX row r as bf16.
+// 16-byte chunk g (dims 8g .. 8g+7) of raw FP8MIX row r as bf16: each value
+// is code * scale (the code decoded exactly by the hardware conversion,
+// the product rounded once to fp32), then rounded to bf16.
 __device__ __forceinline__ uint4 expand_fp8(const uint8_t* raw, int r, int g) {
   const uint8_t* row = raw + r * kRawRow;
   if (g >= 56) return *reinterpret_cast<const uint4*>(row + 448 + (g - 56) * 16);
   const uint2 v = *reinterpret_cast<const uint2*>(row + g * 8);
   const float sc = *reinterpret_cast<const float*>(row + 576 + 4 * (g >> 3));
-  uint32_t w[4];
+  float f[8];
   const uint32_t src[2] = {v.x, v.y};
 #pragma unroll
   for (int q = 0; q < 2; ++q) {
     const float2 lo = e4m3x2_to_float2((uint16_t)(src[q] & 0xFFFF));
     const float2 hi = e4m3x2_to_float2((uint16_t)(src[q] >> 16));
-    const __nv_bfloat162 x0 = __floats2bfloat162_rn(lo.x * sc, lo.y * sc);
-    const __nv_bfloat162 x1 = __floats2bfloat162_rn(hi.x * sc, hi.y * sc);
-    memcpy(&w[2 * q], &x0, 4);
-    memcpy(&w[2 * q + 1], &x1, 4);
+    f[4 * q + 0] = lo.x * sc; f[4 * q + 1] = lo.y * sc;
+    f[4 * q + 2] = hi.x * sc; f[4 * q + 3] = hi.y * sc;
   }
-  return make_uint4(w[0], w[1], w[2], w[3]);
+  return pack_bf16x8(f);
 }
 
 // S^T += K Q^T over atoms [at0, at1) (the first atom of a chunk overwrites).
@@ -200,65 +212,40 @@ __device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t kva, uint32_t q
                  umma_desc_sw128(qa + at * (kHG * 128) + kk * 32), kIdescQK, (at | kk) ? 1u : 0u);
 }
 
-__device__ __forceinline__ uint4 pack_bf16x8(const float* v) {
-  uint32_t w[4];
+// The combine of a head group's splits ("DeepSeek-V4 内部机制" sink equation):
+//   M = max(sink, m_j),  w_j = e^{m_j - M},
+//   O = sum_j w_j o_j / (sum_j w_j l_j + e^{sink - M}),
+// with the splits added in split order.  The in-kernel combine (operands in
+// shared memory) and the combine kernel (operands in global memory) run these
+// two functions, so both give the same bytes.
+//
+// Weights of one head: W[j] = w_j / den (0 for an empty split, all 0 when the
+// sink is +inf or nothing is attended).  ml(j) returns (m_j, l_j); callers
+// fetch every split's statistics before calling, so no loads wait here.
+// MAXS > 0: S <= MAXS and the loops are unrolled (ml may index a register
+// array); MAXS = 0: plain loops.  The operations and their order are the
+// same either way.
+template <int MAXS, class ML>
+__device__ __forceinline__ void combine_weights(int S, float sink, const ML& ml, float* W, int stride) {
+  constexpr int kN = MAXS > 0 ? MAXS : 1 << 30;
+  float M = sink;
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * q], v[2 * q + 1]);
-    memcpy(&w[q], &h, 4);
+  for (int j = 0; j < (MAXS > 0 ? MAXS : S); ++j) {
+    if (j >= S || j >= kN) break;
+    M = fmaxf(M, ml(j).x);
   }
-  return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
-// Output items [i0, i1) of one head group, item = (head, 8 dims): the splits'
-// partials added in split order with the sink, the optional output RoPE,
-// bf16 stores.  W is shared memory for n_splits x 64 weights.
-__device__ void combine_items(const MqaArgs& a, const MqaPlan& plan, int64_t bt, int hg, int i0, int i1, float* W,
-                              const float* ocs, const float* osn) {
-  const int S = plan.n_splits;
-  const int tid = threadIdx.x;
-  if (tid < kHG) {
-    const int h = hg * kHG + tid;
-    const float sink = a.sink[h];
-    float M = sink;
-    for (int j = 0; j < S; ++j) M = fmaxf(M, __ldcg(plan_partial_ml(plan, a, bt, j, h)));
-    const bool zero = (sink == INFINITY) || (M == -INFINITY);
-    float den = 0.f;
-    for (int j = 0; j < S; ++j) {
-      const float* ml = plan_partial_ml(plan, a, bt, j, h);
-      const float mj = __ldcg(ml);
-      const float w = (zero || mj == -INFINITY) ? 0.f : expf(mj - M);
-      W[j * kHG + tid] = w;
-      den += w > 0.f ? __ldcg(ml + 1) * w : 0.f;
-    }
-    if (!zero) den += expf(sink - M);
-    for (int j = 0; j < S; ++j) W[j * kHG + tid] = zero ? 0.f : W[j * kHG + tid] / den;
-  }
-  __syncthreads();
-  const int d_rope = kDim - a.out_rope_dims;
-  for (int it = i0 + tid; it < i1; it += kThreads) {
-    const int h = it >> 6, d0 = 8 * (it & 63);
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < S; ++j) {
-      const float* po = plan_partial_o(plan, a, bt, j, hg * kHG + h) + d0;
-      const float4 x0 = __ldcg(reinterpret_cast<const float4*>(po));
-      const float4 x1 = __ldcg(reinterpret_cast<const float4*>(po + 4));
-      const float w = W[j * kHG + h];
-      acc[0] = fmaf(w, x0.x, acc[0]); acc[1] = fmaf(w, x0.y, acc[1]);
-      acc[2] = fmaf(w, x0.z, acc[2]); acc[3] = fmaf(w, x0.w, acc[3]);
-      acc[4] = fmaf(w, x1.x, acc[4]); acc[5] = fmaf(w, x1.y, acc[5]);
-      acc[6] = fmaf(w, x1.z, acc[6]); acc[7] = fmaf(w, x1.w, acc[7]);
-    }
-    if (a.out_rope_dims > 0 && d0 >= d_rope) {
+  const bool zero = (sink == INFINITY) || (M == -INFINITY);
+  float den = 0.f;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int k = (d0 - d_rope) / 2 + q;
-        rope_turn(acc[2 * q], acc[2 * q + 1], ocs[k], osn[k]);
-      }
-    }
-    *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + (bt * a.n_heads + (int64_t)hg * kHG + h) * kDim +
-                              d0) = pack_bf16x8(acc);
+  for (int j = 0; j < (MAXS > 0 ? MAXS : S); ++j) {
+    if (j >= S) break;
+    const float2 v = ml(j);
+    const float w = (zero || v.x == -INFINITY) ? 0.f : expf(v.x - M);
+    W[j * stride] = w;
+    den += w > 0.f ? v.y * w : 0.f;
   }
+  if (!zero) den += expf(sink - M);
+  for (int j = 0; j < S; ++j) W[j * stride] = zero ? 0.f : W[j * stride] / den;
 }
 
 // RoPE tables of the query at +t and of the output at -t (threads < 32).
@@ -271,7 +258,8 @@ __device__ __forceinline__ void rope_tables(const MqaArgs& a, int64_t t, float* 
 }
 
 template <bool FP8, int MODE>
-__global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPlan plan) {
+__global__ void __launch_bounds__(kThreads, 1)
+    mqa_umma_kernel(const __grid_constant__ CUtensorMap tmQ, MqaArgs a, MqaPlan plan) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = align1024(smem_raw);
   uint8_t* KV = base + kOffKV;
@@ -286,27 +274,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int quad = warp & 3, half = warp >> 2;
 
-  // query tile (64 heads x 512 dims) -> K-major swizzled atoms, issued first
-  // (it depends on nothing)
-  {
-    const uint8_t* qg = static_cast<const uint8_t*>(a.Q) + ((bt * a.n_heads + (int64_t)hg * kHG) * kDim) * 2;
-    for (int i = tid; i < kHG * 64; i += kThreads) {
-      const int h = i >> 6, g = i & 63;
-      cp_async16(smem_u32(Qs + q_off(h, g)), qg + (int64_t)h * (kDim * 2) + g * 16, true);
-    }
-    cp_async_commit();
-  }
-  const int64_t tq = a.q_pos[bt];
-  const RowList rl = make_row_list(a, bt, tq);
-  // split s of NS takes chunks [s * nch / NS, (s + 1) * nch / NS) of the rows
-  const int NS = plan.n_splits;
-  const int64_t nch = (rl.n_rows + kRows - 1) / kRows;
-  const int64_t r_begin = (int64_t)split * nch / NS * kRows;
-  const int64_t r_end = min64(rl.n_rows, ((int64_t)split + 1) * nch / NS * kRows);
-  const int n_chunks = r_end > r_begin ? (int)((r_end - r_begin + kRows - 1) / kRows) : 0;
-  const int64_t rb = row_bytes(a.kv_dt, kDim);
-
   if (tid == 0) {
+    mbar_init(&ms.bar_q, 1);
     mbar_init(&ms.bar_raw, kRows);
     for (int i = 0; i < 2; ++i) mbar_init(&ms.bar_half[i], kThreads);
     for (int i = 0; i < 4; ++i) mbar_init(&ms.bar_pair[i], kThreads);
@@ -314,15 +283,56 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
     for (int i = 0; i < 4; ++i) mbar_init(&ms.bar_slab[i], 1);
     mbar_init(&ms.bar_pv, 1);
     fence_barrier_init();
+    // query tile (64 heads x 512 dims): eight TMA boxes of 64 heads x 64 dims
+    // in the 128-byte swizzle, the K-major operand layout (depends on nothing)
+    mbar_arrive_expect_tx(&ms.bar_q, kHG * kDim * 2);
+    const int qrow = (int)(bt * a.n_heads + (int64_t)hg * kHG);
+    for (int at = 0; at < 8; ++at) tma_load_2d(Qs + at * (kHG * 128), &tmQ, &ms.bar_q, 64 * at, qrow);
   }
+  // The first chunk's entry indices are fetched together with the query
+  // position, assuming the query's window is full (decode); a query whose
+  // window is cut by the start of the sequence has fewer rows and fetches its
+  // own range again below.
+  const int NS = plan.n_splits;
+  const int64_t full_rows = a.idx ? (int64_t)a.k + a.window : 0;
+  const int64_t full_nch = (full_rows + kRows - 1) / kRows;
+  const int64_t guess_begin = (int64_t)split * full_nch / NS * kRows;
+  int32_t e_guess = -1;
+  if (a.idx != nullptr && tid < kRows && guess_begin + tid < a.k) e_guess = a.idx[bt * a.k + guess_begin + tid];
+  const int64_t tq = a.q_pos[bt];
+  const RowList rl = make_row_list(a, bt, tq);
+  // split s of NS takes chunks [s * nch / NS, (s + 1) * nch / NS) of the rows
+  const int64_t nch = (rl.n_rows + kRows - 1) / kRows;
+  const int64_t r_begin = (int64_t)split * nch / NS * kRows;
+  const int64_t r_end = min64(rl.n_rows, ((int64_t)split + 1) * nch / NS * kRows);
+  const int n_chunks = r_end > r_begin ? (int)((r_end - r_begin + kRows - 1) / kRows) : 0;
+  const int64_t rb = row_bytes(a.kv_dt, kDim);
+
   if (warp == 0) tmem_alloc(&ms.tmem_slot, kTmemCols);
   if (tid < kHG) ms.m_use[tid] = -INFINITY;
   if (tid < 32) rope_tables(a, tq, ms.qcs, ms.qsn, ms.ocs, ms.osn);
-  if (tid < kRows) ms.rowp[0][tid] = n_chunks > 0 ? chunk_row(a, rl, b, r_begin + tid, r_end, rb) : nullptr;
+  if (tid < kRows) {
+    const int64_t r = r_begin + tid;
+    const uint8_t* p = nullptr;
+    if (n_chunks > 0 && r < r_end) {
+      if (r < rl.n_sel && a.idx != nullptr && r_begin == guess_begin) {
+        const int64_t e = e_guess;
+        if (e >= 0 && e < rl.vis) p = static_cast<const uint8_t*>(a.entries) + ((int64_t)b * a.n_entries + e) * rb;
+      } else {
+        p = row_ptr(a, rl, b, r, rb);
+      }
+    }
+    ms.rowp[0][tid] = p;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = ms.tmem_slot;
+  // the first chunk's rows are on their way while the rest is set up
+  if (n_chunks > 0) {
+    if (FP8) gather_fp8(raw, ms.rowp[0], &ms.bar_raw);
+    else gather_bf16(KV, ms.rowp[0], a.Q);
+  }
   if (warp < 4) {  // the all-ones A operand of the row-sum product
     float ones[32];
 #pragma unroll
@@ -330,14 +340,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
     tmem_st_32x32b_x32(tmem + ((uint32_t)(32 * warp) << 16) + kColOnes, ones);
     tmem_st_wait();
   }
-  // the first chunk's rows are on their way while the query tile is prepared
-  if (n_chunks > 0) {
-    if (FP8) gather_fp8(raw, ms.rowp[0], &ms.bar_raw);
-    else gather_bf16(KV, ms.rowp[0], a.Q);
-  }
-  cp_async_wait_pending((!FP8 && n_chunks > 0) ? 4 : 0);  // the query tile's group
-  fence_proxy_async_smem();
-  __syncthreads();
+  tc_fence_before();
+  if (a.q_norm_g != nullptr || a.q_rope_dims > 0) mbar_wait(&ms.bar_q, 0);
   if (a.q_norm_g != nullptr || a.q_rope_dims > 0) {
     // RMSNorm and RoPE of the query rows in place: warp w takes heads w, w+8,
     // ...; lane l owns dims 8l..8l+7 and 256+8l..+7 (the order of
@@ -385,8 +389,10 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
     fence_proxy_async_smem();
     __syncthreads();
   }
+  if (tid == 0) mbar_wait(&ms.bar_q, 0);  // the query tile, before the first product
   const float sl2 = a.scale * kLog2e;
   const uint32_t kva = smem_u32(KV), qa = smem_u32(Qs), pa = smem_u32(Ps);
+  constexpr int kHalf = kRows * 32 / kThreads;  // 16-byte chunks per thread in half a tile
 
   for (int ci = 0; ci < n_chunks; ++ci) {
     const uint32_t par = (uint32_t)(ci & 1);
@@ -394,9 +400,22 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
     // ---- rows -> row tile, S^T = K Q^T issued part by part
     if (FP8) {
       mbar_wait(&ms.bar_raw, par);
-      // dims 0..255 straight into atoms 0..3 (no overlap with the staging)
-      for (int u = tid; u < kRows * 32; u += kThreads)
-        *reinterpret_cast<uint4*>(KV + kv_off(u >> 5, u & 31)) = expand_fp8(raw, u >> 5, u & 31);
+      // dims 0..255 into atoms 0..3 (no overlap with the staging); every
+      // chunk is decoded before any is stored, so the loads are all in flight
+#pragma unroll 1
+      for (int j0 = 0; j0 < kHalf; j0 += 4) {
+        uint4 lo[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int u = tid + (j0 + j) * kThreads;
+          lo[j] = expand_fp8(raw, u >> 5, u & 31);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int u = tid + (j0 + j) * kThreads;
+          *reinterpret_cast<uint4*>(KV + kv_off(u >> 5, u & 31)) = lo[j];
+        }
+      }
       fence_proxy_async_smem();
       mbar_arrive(&ms.bar_half[0]);
       if (tid == 0) {
@@ -405,16 +424,15 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
         issue_qk(tmem, kva, qa, 0, 4);
       }
       // dims 256..511 through registers (their destination overlaps the staging)
-      constexpr int kHi = kRows * 32 / kThreads;  // 16 chunks per thread
-      uint4 hi[kHi];
+      uint4 hi[kHalf];
 #pragma unroll
-      for (int j = 0; j < kHi; ++j) {
+      for (int j = 0; j < kHalf; ++j) {
         const int u = tid + j * kThreads;
         hi[j] = expand_fp8(raw, u >> 5, 32 + (u & 31));
       }
       __syncthreads();
 #pragma unroll
-      for (int j = 0; j < kHi; ++j) {
+      for (int j = 0; j < kHalf; ++j) {
         const int u = tid + j * kThreads;
         *reinterpret_cast<uint4*>(KV + kv_off(u >> 5, 32 + (u & 31))) = hi[j];
       }
@@ -576,6 +594,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
 #pragma unroll
     for (int h = 0; h < kHG; ++h) stg[h * kDim + d] = o[h];
   }
+  fence_proxy_async_smem();  // the staging is read by bulk copies
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -596,6 +615,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
       ms.fac[tid] = f;
     }
     __syncthreads();
+    // normalised (and optionally turned) bf16 rows [head][512] in the query
+    // region, then one bulk copy per 16 KB to the output
     const int d_rope = kDim - a.out_rope_dims;
     for (int it = tid; it < kItems; it += kThreads) {
       const int h = it >> 6, d0 = 8 * (it & 63);
@@ -610,61 +631,84 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_umma_kernel(MqaArgs a, MqaPla
           rope_turn(v[2 * q], v[2 * q + 1], ms.ocs[k], ms.osn[k]);
         }
       }
-      *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.O) + (bt * a.n_heads + (int64_t)hg * kHG + h) * kDim +
-                                d0) = pack_bf16x8(v);
+      *reinterpret_cast<uint4*>(Qs + it * 16) = pack_bf16x8(v);
+    }
+    fence_proxy_async_smem();
+    __syncthreads();
+    if (tid < 4) {
+      constexpr uint32_t kPiece = kHG * kDim * 2 / 4;
+      bulk_store(static_cast<uint8_t*>(a.O) + (bt * a.n_heads + (int64_t)hg * kHG) * kDim * 2 + tid * kPiece,
+                 Qs + tid * kPiece, kPiece);
+      bulk_commit();
+      bulk_wait_read();  // the shared memory may go once the copy has read it
     }
   } else {
-    // one split of several: the unnormalised partial (m, l, o)
+    // one split of several: the unnormalised partial (m, l, o) for the
+    // combine kernel; o leaves the staging by bulk copies of 8 heads (16 KB)
     if (tid < kHG) {
       float* ml = plan_partial_ml(plan, a, bt, split, hg * kHG + tid);
       const float m = ms.m_use[tid];
       ml[0] = m == -INFINITY ? -INFINITY : m / kLog2e;  // natural-log domain
       ml[1] = ms.lsum[tid];
     }
-    for (int it = tid; it < kItems; it += kThreads) {
-      const int h = it >> 6, d0 = 8 * (it & 63);
-      float* po = plan_partial_o(plan, a, bt, split, hg * kHG + h) + d0;
-      reinterpret_cast<float4*>(po)[0] = *reinterpret_cast<const float4*>(stg + h * kDim + d0);
-      reinterpret_cast<float4*>(po)[1] = *reinterpret_cast<const float4*>(stg + h * kDim + d0 + 4);
-    }
-    if constexpr (MODE == kMqaCoop) {
-      // the splits of this (query, head group) wait for one another, then
-      // each adds a share of the outputs over all splits
-      __syncthreads();
-      uint32_t* ctr = plan_unit_counters(a, bt * (a.n_heads / kHG) + hg);
-      if (tid == 0) {
-        __threadfence();
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
-        const unsigned long long t0 = globaltimer_ns();
-        for (uint32_t it = 1; ld_acquire_gpu(ctr) < (uint32_t)NS; ++it) {
-          if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitTimeoutNs) {
-            atomicOr(&g_device_status, 1u);
-            break;
-          }
-        }
-      }
-      __syncthreads();
-      const int i0 = (int)((int64_t)split * kItems / NS), i1 = (int)((int64_t)(split + 1) * kItems / NS);
-      combine_items(a, plan, bt, hg, i0, i1, stg, ms.ocs, ms.osn);
-      __syncthreads();
-      // the last split to finish leaves the counters at zero for the next call
-      if (tid == 0 && atomicAdd(ctr + 1, 1u) == (uint32_t)NS - 1) {
-        ctr[0] = 0u;
-        ctr[1] = 0u;
-      }
+    if (tid < kHG / 8) {
+      bulk_store(plan_partial_o(plan, a, bt, split, hg * kHG + 8 * tid), stg + 8 * tid * kDim, 8 * kDim * 4);
+      bulk_commit();
+      bulk_wait_read();  // the next kernel sees the writes; the shared memory may go once read
     }
   }
 }
 
-// The combine of kMqaSplit mode: one CTA per (head group, query).
-__global__ void __launch_bounds__(kThreads) mqa_umma_combine_kernel(MqaArgs a, MqaPlan plan) {
-  extern __shared__ __align__(16) float cw[];  // [n_splits][64] weights
+// The combine of kMqaSplit mode: one CTA per (head, query), a thread per 4
+// dims; the splits' statistics go through shared memory once, and each
+// thread's partials are loaded 16 splits at a time, all in flight together.
+constexpr int kCombineThreads = 128;
+constexpr int kLoadSplits = 16;
+__global__ void __launch_bounds__(kCombineThreads) mqa_umma_combine_kernel(MqaArgs a, MqaPlan plan) {
+  __shared__ float2 mls[kMaxSplits];
+  __shared__ float W[kMaxSplits];
   __shared__ float ocs[kMaxRope / 2], osn[kMaxRope / 2], qcs[kMaxRope / 2], qsn[kMaxRope / 2];
-  const int hg = blockIdx.x;
+  const int h = blockIdx.x;
   const int64_t bt = blockIdx.y;
-  if (threadIdx.x < 32) rope_tables(a, a.q_pos[bt], qcs, qsn, ocs, osn);
+  const int S = plan.n_splits, tid = threadIdx.x;
+  if (tid < 32) rope_tables(a, a.q_pos[bt], qcs, qsn, ocs, osn);
+  for (int j = tid; j < S; j += kCombineThreads)
+    mls[j] = __ldcg(reinterpret_cast<const float2*>(plan_partial_ml(plan, a, bt, j, h)));
+  // this thread's 4 dims of the first (up to) 16 splits, loaded while the
+  // weights are formed
+  const int d0 = 4 * tid;
+  float4 x[kLoadSplits];
+#pragma unroll
+  for (int u = 0; u < kLoadSplits; ++u)
+    if (u < S) x[u] = __ldcg(reinterpret_cast<const float4*>(plan_partial_o(plan, a, bt, u, h) + d0));
   __syncthreads();
-  combine_items(a, plan, bt, hg, 0, kItems, cw, ocs, osn);
+  if (tid == 0) combine_weights<0>(S, a.sink[h], [&](int j) { return mls[j]; }, W, 1);
+  __syncthreads();
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int j0 = 0; j0 < S; j0 += kLoadSplits) {
+    if (j0 > 0) {
+#pragma unroll
+      for (int u = 0; u < kLoadSplits; ++u)
+        if (j0 + u < S) x[u] = __ldcg(reinterpret_cast<const float4*>(plan_partial_o(plan, a, bt, j0 + u, h) + d0));
+    }
+#pragma unroll
+    for (int u = 0; u < kLoadSplits; ++u) {
+      if (j0 + u >= S) break;
+      const float w = W[j0 + u];
+      acc[0] = fmaf(w, x[u].x, acc[0]); acc[1] = fmaf(w, x[u].y, acc[1]);
+      acc[2] = fmaf(w, x[u].z, acc[2]); acc[3] = fmaf(w, x[u].w, acc[3]);
+    }
+  }
+  const int d_rope = kDim - a.out_rope_dims;
+  if (a.out_rope_dims > 0 && d0 >= d_rope) {
+    rope_turn(acc[0], acc[1], ocs[(d0 - d_rope) / 2], osn[(d0 - d_rope) / 2]);
+    rope_turn(acc[2], acc[3], ocs[(d0 - d_rope) / 2 + 1], osn[(d0 - d_rope) / 2 + 1]);
+  }
+  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]), hi = __floats2bfloat162_rn(acc[2], acc[3]);
+  uint2 pk;
+  memcpy(&pk.x, &lo, 4);
+  memcpy(&pk.y, &hi, 4);
+  *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.O) + (bt * a.n_heads + h) * kDim + d0) = pk;
 }
 
 int sm_count_mqa() {
@@ -691,6 +735,7 @@ MqaPlan make_umma_mqa_plan(const MqaArgs& a) {
   MqaPlan p{};
   p.heads_per_cta = kHG;
   p.rows_per_split = 0;
+  p.ws_head = 0;
   // automatic: a query's row chunks are split over CTAs until the grid fills
   // one wave; a fixed count (a.splits) depends on the row count only
   const int sms = sm_count_mqa();
@@ -698,10 +743,10 @@ MqaPlan make_umma_mqa_plan(const MqaArgs& a) {
   const int64_t nch = (max_rows_per_query(a) + kRows - 1) / kRows;
   int64_t ns = a.splits > 0 ? a.splits : (units >= sms ? 1 : sms / units);
   if (ns > nch) ns = nch;
+  if (ns > kMaxSplits) ns = kMaxSplits;
   if (ns < 1) ns = 1;
   p.n_splits = (int)ns;
-  p.mode = ns == 1 ? kMqaWhole : (units * ns <= sms ? kMqaCoop : kMqaSplit);
-  p.ws_head = ns == 1 ? 0 : kMqaCounterBytes;
+  p.mode = ns == 1 ? kMqaWhole : kMqaSplit;
   return p;
 }
 
@@ -710,32 +755,23 @@ cudaError_t launch_umma(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) {
   auto kern = mqa_umma_kernel<FP8, MODE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
+  // the queries as [B * T * n_heads rows][512] bf16, boxes of 64 heads x 64 dims
+  CUtensorMap tmQ;
+  if (!make_map_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.Q, (uint64_t)a.batch * a.n_q * a.n_heads, kDim, 64,
+                   kHG, CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
   const dim3 grid((unsigned)p.n_splits, a.n_heads / kHG, (unsigned)((int64_t)a.batch * a.n_q));
-  if (MODE == kMqaCoop) {
-    // the splits of a (query, head group) wait for one another: every CTA
-    // must be resident at once
-    MqaArgs aa = a;
-    MqaPlan pp = p;
-    void* args[] = {&aa, &pp};
-    e = cudaLaunchCooperativeKernel((const void*)kern, grid, dim3(kThreads), args, kSmemBytes, s);
-    ++launch_counter();
-    return e;
-  }
-  kern<<<grid, kThreads, kSmemBytes, s>>>(a, p);
+  kern<<<grid, kThreads, kSmemBytes, s>>>(tmQ, a, p);
   ++launch_counter();
   e = cudaGetLastError();
   if (e != cudaSuccess || MODE != kMqaSplit) return e;
-  const size_t cs = (size_t)p.n_splits * kHG * sizeof(float);
-  e = cudaFuncSetAttribute(mqa_umma_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)cs);
-  if (e != cudaSuccess) return e;
-  mqa_umma_combine_kernel<<<dim3(a.n_heads / kHG, (unsigned)((int64_t)a.batch * a.n_q)), kThreads, cs, s>>>(a, p);
+  mqa_umma_combine_kernel<<<dim3(a.n_heads, (unsigned)((int64_t)a.batch * a.n_q)), kCombineThreads, 0, s>>>(a, p);
   ++launch_counter();
   return cudaGetLastError();
 }
 
 template <bool FP8>
 cudaError_t launch_umma_fmt(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) {
-  if (p.mode == kMqaCoop) return launch_umma<FP8, kMqaCoop>(a, p, s);
   if (p.mode == kMqaSplit) return launch_umma<FP8, kMqaSplit>(a, p, s);
   return launch_umma<FP8, kMqaWhole>(a, p, s);
 }

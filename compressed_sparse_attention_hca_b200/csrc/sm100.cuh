@@ -30,6 +30,12 @@ static __device__ unsigned int g_device_status = 0;
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
 
+// Host: a 2D tiled tensor map over [rows][cols] elements of `esize` bytes (row
+// stride cols * esize) with boxes of box_cols x box_rows (false when the
+// driver entry point is missing or the encoder rejects the shape).
+bool make_map_2d(CUtensorMap* map, CUtensorMapDataType dtype, int esize, const void* base, uint64_t rows,
+                 uint64_t cols, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swizzle);
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -110,6 +116,19 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
+
+// Untiled bulk copy shared -> global of `bytes` (both addresses 16-byte
+// aligned, bytes a multiple of 16), tracked by this thread's bulk group.
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               ::"l"(reinterpret_cast<uint64_t>(dst)), "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Waits until this thread's committed bulk stores have completed (written).
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Waits until this thread's committed bulk stores have read their source.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 // ---------------------------------------------------------------------- TMEM
 // Allocation / release are warp-wide (.sync.aligned): call from one full warp.

@@ -339,8 +339,7 @@ csa_status_t csa_index_topk_noalloc(const void* qI, const void* qI_sf, const flo
  *             window token of every query must be present.
  *   q_pos     [batch][n_q] int64 (device); sink [n_heads] fp32 (device).
  * Limits: dim a multiple of 64 (<= 512), n_heads <= 128, k <= 2048.
- * Workspace: zero-filled before its first use (the split counters in its
- * first 4096 bytes; every call leaves them zero, the rest is scratch).
+ * Workspace: scratch for the split partials; no initialisation needed.
  */
 size_t csa_sparse_mqa_workspace_size(int batch, int n_q, int n_heads, int dim, int k, int window,
                                      csa_dtype_t q_dt, csa_dtype_t kv_dt);
@@ -395,9 +394,7 @@ typedef struct {
 /*
  * csa_mqa_workspace_size -- workspace bytes of an attention call with these
  * options (rows_per_query = k + window for csa_sparse_mqa_ex, n_entries +
- * window for hca_dense_mqa_ex).  The workspace must be zero-filled before its
- * first use (its first 4096 bytes hold the counters with which the splits of
- * a query meet; every call leaves them zero, the rest is scratch).
+ * window for hca_dense_mqa_ex); scratch, no initialisation needed.
  */
 size_t csa_mqa_workspace_size(int batch, int n_q, int n_heads, int dim, int64_t rows_per_query,
                               csa_dtype_t q_dt, csa_dtype_t kv_dt, const csa_mqa_options_t* opt);

@@ -16,8 +16,8 @@ pytestmark = pytest.mark.gpu
 
 @pytest.mark.parametrize("idx_dt,n_h", [(csa.IDX_NVFP4, 16), (csa.BF16, 16), (csa.BF16, 128)])
 def test_graph_replay_matches_eager(idx_dt, n_h):
-    """n_h = 16 runs the SIMT attention with its combine kernel; n_h = 128 the
-    tensor-core attention whose splits combine in one cooperative launch."""
+    """n_h = 16 runs the SIMT attention, n_h = 128 the tensor-core attention
+    (each with its split combine kernel)."""
     if not torch.cuda.is_available():
         pytest.fail("needs a CUDA device")
     B, E, k, H, dI, m = 2, 30000, 1024, 64, 128, 4
@@ -99,10 +99,9 @@ def test_index_workspace_returns_to_zero(idx_dt):
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
 
 
-def test_attention_counters_return_to_zero():
-    """The splits of a decode query meet on counters in the attention
-    workspace; every call leaves them zero, so the same workspace serves the
-    next call."""
+def test_attention_repeated_calls_identical():
+    """The tensor-core attention on a decode batch (split rows, combine
+    kernel): repeated calls on the same workspace give the same bytes."""
     if not torch.cuda.is_available():
         pytest.fail("needs a CUDA device")
     B, E, k, n_h, c, window, m = 2, 3000, 1024, 128, 512, 128, 4
@@ -113,14 +112,13 @@ def test_attention_counters_return_to_zero():
     win = W.fp8mix_rows(g, (B, window), c).cuda()
     win_start = (q_pos[:, 0] - window + 1).clamp(min=0)
     sink = W.normal(g, (n_h,), 1.0, torch.float32).cuda()
-    idx = torch.stack([torch.randperm(m * E // m - 200, generator=g)[:k] for _ in range(B)]).view(B, 1, k)
+    idx = torch.stack([torch.randperm(E - 200, generator=g)[:k] for _ in range(B)]).view(B, 1, k)
     idx = idx.to(torch.int32).cuda()
-    ws = torch.zeros(csa.sparse_mqa_workspace_size(B, 1, n_h, c, k, window, csa.BF16, csa.KV_FP8MIX),
+    ws = torch.empty(csa.sparse_mqa_workspace_size(B, 1, n_h, c, k, window, csa.BF16, csa.KV_FP8MIX),
                      dtype=torch.uint8, device="cuda")
     outs = []
     for _ in range(3):
         outs.append(csa.sparse_mqa(Q, entries, idx, win, win_start, q_pos, window, m, sink, c ** -0.5, ws=ws))
         torch.cuda.synchronize()
         csa.check_device_status()
-        assert int(ws[:4096].count_nonzero()) == 0
     assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])

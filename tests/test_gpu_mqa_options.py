@@ -1,13 +1,12 @@
 """The tensor-core attention's modes and options against the float64 oracle.
 
-  * every way the rows of a query are split and combined -- one CTA per
-    (query, 64 heads), splits that meet in the same cooperative launch, splits
-    combined by a separate kernel -- gives the oracle's output (2e-2 max abs,
-    bf16);
+  * every way the rows of a query are split -- one CTA per (query, 64 heads),
+    several splits combined by the combine kernel, one split or several chunks
+    per CTA -- gives the oracle's output (2e-2 max abs, bf16);
   * batch-invariant decode ("CSA / HCA: 混合稀疏注意力机制", infrastructure
     section; "DeepSeek-V4 内部机制" 6.3): with a fixed split count a request's
-    output is bitwise the same alone and inside batches of 16 and 40 (which
-    runs the other combine), for FP8MIX and BF16 rows and for the dense form;
+    output is bitwise the same alone and inside batches of 16 and 40, for
+    FP8MIX and BF16 rows and for the dense form;
   * the fused query RMSNorm + RoPE and the output turned at -t
     ("DeepSeek-V4 内部机制" 1.4 table) equal the oracle's composition
     rope_tail(attend(rope_tail(rmsnorm(Q), t)), -t), and the fused query
@@ -78,11 +77,11 @@ def _oracle(orc, cfg, x, Q=None):
 
 
 @pytest.mark.parametrize("cfg_name,B,E,T,splits", [
-    ("csa_decode_1m_mixed", 1, 3000, 1, 0),    # automatic: 9 splits meet in one cooperative launch
+    ("csa_decode_1m_mixed", 1, 3000, 1, 0),    # automatic: 9 splits, one chunk each
     ("csa_decode_1m_mixed", 4, 3000, 1, 0),    # automatic, the benchmark's shape of splits
     ("csa_decode_bf16", 3, 3000, 1, 0),        # BF16 rows, automatic
     ("csa_decode_bf16", 2, 3000, 1, 1),        # one CTA per (query, 64 heads)
-    ("csa_decode_1m_mixed", 40, 2000, 1, 3),   # 240 CTAs: partials combined by the separate kernel
+    ("csa_decode_1m_mixed", 40, 2000, 1, 3),   # 240 CTAs, three chunks per split
     ("hca_decode_bf16", 2, 1500, 1, 0),        # dense rows, several chunks per split (prefetch)
     ("hca_decode_bf16", 1, 1500, 1, 2),        # dense rows, long splits
     ("csa_prefill_bf16", 1, 300, 40, 0),       # many queries: one CTA per (query, 64 heads)
@@ -102,9 +101,8 @@ def test_modes_match_oracle(orc, cfg_name, B, E, T, splits):
     ("hca_decode_bf16", 1200, 3),
 ])
 def test_fixed_splits_are_batch_invariant(cfg_name, E, splits):
-    """Requests 0, 7 and 15 of a batch of 16 (and of 40: more CTAs than SMs,
-    so the partials go through the separate combine kernel) give bitwise the
-    outputs they give alone."""
+    """Requests 0, 7 and 15 of a batch of 16 (and of 40: more CTAs than SMs)
+    give bitwise the outputs they give alone."""
     cfg, x = _case(cfg_name, 40, E, seed=23)
     opt = csa.mqa_options(splits=splits)
     o40 = _run(cfg, x, opt)
