@@ -273,12 +273,18 @@ __device__ __forceinline__ void st_relaxed_gpu(uint32_t* p, uint32_t v) {
   asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-__device__ __forceinline__ void coop_barrier(uint32_t* ctr, uint32_t target) {
+// The row's barrier in two halves, so that work needing no other slice runs
+// between them.  Arrive: after a CTA barrier, thread 0 adds 1 with release
+// semantics (this CTA's global writes and atomics, ordered before by the CTA
+// barrier, are visible to every CTA that acquires the counter).  Wait:
+// thread 0 polls the counter with acquire semantics (bounded), then a CTA
+// barrier.
+__device__ __forceinline__ void coop_arrive(uint32_t* ctr) {
   __syncthreads();
+  if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+}
+__device__ __forceinline__ void coop_wait(uint32_t* ctr, uint32_t target) {
   if (threadIdx.x == 0) {
-    // release: this CTA's global writes and atomics (ordered before by the
-    // CTA barrier) are visible to every CTA that acquires the counter
-    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
     const unsigned long long t0 = globaltimer_ns();
     for (uint32_t it = 1; ld_acquire_gpu(ctr) < target; ++it) {
       if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitTimeoutNs) {
@@ -341,9 +347,42 @@ __device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t 
   uint32_t* slots = row + kPrefixBins + 8;
   uint32_t total;
 
-  // 1. prefix histogram (and the row's highest prefix) -> prefix d1 of the
-  //    k-th key; warp 0 walks the bins down from the highest prefix, 32 at a
-  //    time, so only the few bins above the k-th key are read
+  // Warp 0 walks a prefix histogram down from bin `hi`, 32 bins at a time,
+  // to the bin holding the want-th largest key; returns that bin and how many
+  // keys of it are still needed (only the few bins above it are read).
+  auto kth_prefix = [&](const uint32_t* hist, int hi, uint32_t want, bool global, uint32_t* d_out,
+                        uint32_t* rem_out) {
+    uint32_t above = 0;
+    for (int base = hi; base >= 0; base -= 32) {
+      const int d = base - lane;
+      const uint32_t c = d >= 0 ? (global ? __ldcg(hist + d) : hist[d]) : 0u;
+      uint32_t inc = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, above + inc >= want);
+      if (hit) {
+        const int l = __ffs(hit) - 1;
+        if (lane == l) {
+          *d_out = (uint32_t)d;
+          *rem_out = want - (above + inc - c);
+        }
+        return;
+      }
+      above += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) {  // fewer than `want` keys: every bin
+      *d_out = 0u;
+      *rem_out = 0u;
+    }
+  };
+
+  // 1. this slice's prefix histogram into the row's histogram H (and its
+  //    highest prefix into the row's), then arrive on the row's barrier
+  if (tid == 0) sm.hist[64] = 0u;
+  __syncthreads();
   uint32_t top = 0;
   for (int d = tid; d < kPrefixBins; d += NT)
     if (hist_local[d]) {
@@ -352,58 +391,33 @@ __device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t 
     }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) top = max(top, __shfl_xor_sync(0xffffffffu, top, o));
-  if (lane == 0 && top) atomicMax(Hmax, top);
-  coop_barrier(ctr, (uint32_t)S);
-  if (warp == 0) {
-    const int hi = (int)__ldcg(Hmax);
-    uint32_t above = 0;
-    for (int base = hi; base >= 0; base -= 32) {
-      const int d = base - lane;
-      const uint32_t c = d >= 0 ? __ldcg(H + d) : 0u;
-      uint32_t inc = c;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
-        if (lane >= o) inc += y;
-      }
-      const unsigned hit = __ballot_sync(0xffffffffu, above + inc >= (uint32_t)kk);
-      if (hit) {
-        const int l = __ffs(hit) - 1;
-        if (lane == l) {
-          sm.bcast[0] = (uint32_t)d;
-          sm.bcast[1] = (uint32_t)kk - (above + inc - c);
-        }
-        break;
-      }
-      above += __shfl_sync(0xffffffffu, inc, 31);
-    }
+  if (lane == 0 && top) {
+    atomicMax(Hmax, top);
+    atomicMax(&sm.hist[64], top);
   }
-  if (tid < 32) sm.hist[tid] = 0;
-  __syncthreads();
-  const uint32_t d1 = sm.bcast[0], rem1 = sm.bcast[1];
+  coop_arrive(ctr);
 
-  // 2. one pass over the keys: count those above prefix d1, histogram the
-  //    suffixes of those inside it, and compact the positions of both (the
-  //    only possible winners) into the warp's part of cand, in order.  A lane
-  //    reads 8 consecutive keys (16 bytes) per step.
+  // 1b. while the other slices arrive: this slice alone has min(k, nv) keys
+  //     at or above its own k-th key, so the row's k-th key is not below it
+  //     and no key with a smaller prefix L can win; compact the positions of
+  //     the keys with prefix >= L into the warp's part of cand, in order.  A
+  //     lane reads 8 consecutive keys (16 bytes) per step.
+  if (warp == 0) kth_prefix(hist_local, (int)sm.hist[64], (uint32_t)min(a.k, nv), false, &sm.bcast[2], &sm.bcast[3]);
+  __syncthreads();
+  const uint32_t L = sm.bcast[2];
   const int span = ((nv + NW - 1) / NW + 255) / 256 * 256;
   const int w0 = min(nv, warp * span), w1 = min(nv, w0 + span);
-  uint32_t n_cand = 0, gt1 = 0;
+  uint32_t n_cand = 0;
   for (int base = w0; base < w1; base += 256) {
     const int p0 = base + 8 * lane;
     uint4 v = make_uint4(0u, 0u, 0u, 0u);
     if (p0 < w1) v = *reinterpret_cast<const uint4*>(kq + p0);
     const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-    uint32_t cmask = 0, ngt = 0;
+    uint32_t cmask = 0;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       const uint32_t k16 = (wv[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
-      const bool in = p0 + j < w1;
-      const uint32_t pre = k16 >> 4;
-      const bool hi = in && pre > d1, mid = in && pre == d1;
-      cmask |= (hi || mid) ? (1u << j) : 0u;
-      ngt += hi ? 1u : 0u;
-      if (mid) atomicAdd(&sm.hist[k16 & 15u], 1u);
+      cmask |= (p0 + j < w1 && (k16 >> 4) >= L) ? (1u << j) : 0u;
     }
     const uint32_t cnt = __popc(cmask);
     uint32_t inc = cnt;
@@ -417,8 +431,36 @@ __device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t 
     for (int j = 0; j < 8; ++j)
       if (cmask & (1u << j)) cand[at++] = (uint16_t)(p0 + j);
     n_cand += __shfl_sync(0xffffffffu, inc, 31);
-    gt1 += ngt;
   }
+
+  // 1c. every slice has arrived: prefix d1 of the row's k-th key (d1 >= L)
+  coop_wait(ctr, (uint32_t)S);
+  if (warp == 0) kth_prefix(H, (int)__ldcg(Hmax), (uint32_t)kk, true, &sm.bcast[0], &sm.bcast[1]);
+  if (tid < 32) sm.hist[tid] = 0;
+  __syncthreads();
+  const uint32_t d1 = sm.bcast[0], rem1 = sm.bcast[1];
+
+  // 2. the warp's candidates: count those above prefix d1, histogram the
+  //    suffixes of those inside it, and keep both (the only possible
+  //    winners), in order, dropping the others
+  uint16_t* cw0 = cand + w0;
+  uint32_t kept = 0, gt1 = 0;
+  for (int base = 0; base < (int)n_cand; base += 32) {
+    const int j = base + lane;
+    const bool in = j < (int)n_cand;
+    const uint16_t p = in ? cw0[j] : (uint16_t)0;
+    const uint32_t k16 = in ? kq[p] : 0u;
+    const uint32_t pre = k16 >> 4;
+    const bool hi = in && pre > d1, mid = in && pre == d1;
+    if (mid) atomicAdd(&sm.hist[k16 & 15u], 1u);
+    gt1 += hi ? 1u : 0u;
+    const unsigned keep = __ballot_sync(0xffffffffu, hi || mid);
+    __syncwarp();  // every lane has read its entry before any is overwritten
+    if (hi || mid) cw0[kept + __popc(keep & lt)] = p;
+    kept += __popc(keep);
+  }
+  n_cand = kept;
+  __syncthreads();  // the suffix histogram is complete
   block_exclusive_scan<NT>(gt1, sm.warp_tot, &total);
   // slot words are stored as value + 1 into a zeroed workspace, so a reader
   // knows a word has arrived when it is nonzero: the exchange needs no
