@@ -74,6 +74,9 @@ def load():
                                     i32, i32, i32, P, P, sz, ctypes.POINTER(MqaOptions), P]),
         "hca_dense_mqa_ex": (i32, [P, i32, P, i64, P, i64, P, P, i32, i32, P, f32, i32, i32, i32, i32,
                                    i32, P, P, sz, ctypes.POINTER(MqaOptions), P]),
+        "csa_grouped_out_proj_workspace_size": (sz, [i32, i32, i32, i32, i32, i32]),
+        "csa_grouped_out_proj_plan": (i32, [i32, i32, i32, i32, i32, i32, P]),
+        "csa_grouped_out_proj": (i32, [P, P, P, P, i32, i32, i32, i32, i32, i32, P, sz, P]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(lib, name)
@@ -357,3 +360,40 @@ def hca_dense_mqa(Q, entries, win, win_start, q_pos, window, m, sink, scale, *, 
                                    _ptr(win_start), _ptr(q_pos), window, m, _ptr(sink), float(scale), B, T,
                                    H, c, kv_dt, _ptr(O), _ptr(ws), ws.numel(), _opt_ref(options), _stream()))
     return O
+
+
+# ------------------------------------------------------ grouped output projection
+
+def grouped_out_proj_workspace_size(T, n_h, c, g, d_g, d):
+    return int(load().csa_grouped_out_proj_workspace_size(T, n_h, c, g, d_g, d))
+
+
+def grouped_out_proj_plan(T, n_h, c, g, d_g, d):
+    """How csa_grouped_out_proj divides a call of this shape: per projection
+    (group, then output) the tokens per CTA, K slices per tile and CTAs."""
+    out = (ctypes.c_int32 * 6)()
+    _check(load().csa_grouped_out_proj_plan(T, n_h, c, g, d_g, d, ctypes.cast(out, ctypes.c_void_p)))
+    v = [int(x) for x in out]
+    keys = ("tokens_per_cta", "splits", "ctas")
+    return {"group": dict(zip(keys, v[:3])), "output": dict(zip(keys, v[3:]))}
+
+
+def grouped_out_proj(O, Wg, Wo, *, out=None, ws=None):
+    """Grouped output projection.  O [T, n_h, c] bf16, Wg [g, n_h/g * c, d_g]
+    bf16, Wo [g * d_g, d] bf16 -> Y [T, d] bf16.  ws: a workspace of
+    grouped_out_proj_workspace_size bytes whose counters are zero (a fresh
+    zeroed one is made when not given; every call leaves it zero)."""
+    _need_cuda(O, Wg, Wo, out, ws)
+    T, n_h, c = O.shape
+    g, _, d_g = Wg.shape
+    d = Wo.shape[1]
+    if Wg.shape[1] * g != n_h * c or Wo.shape[0] != g * d_g:
+        raise ValueError("Wg must be [g, n_h/g * c, d_g] and Wo [g * d_g, d]")
+    if out is None:
+        out = torch.empty(T, d, device=O.device, dtype=torch.bfloat16)
+    need = grouped_out_proj_workspace_size(T, n_h, c, g, d_g, d)
+    if ws is None:
+        ws = torch.zeros(need, device=O.device, dtype=torch.uint8)
+    _check(load().csa_grouped_out_proj(_ptr(O), _ptr(Wg), _ptr(Wo), _ptr(out), T, n_h, c, g, d_g, d, _ptr(ws),
+                                       ws.numel() * ws.element_size(), _stream()))
+    return out

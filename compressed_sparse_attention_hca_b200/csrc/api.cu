@@ -154,7 +154,7 @@ int csa_last_launch_count(void) { return g_launches; }
 csa_status_t csa_check_device_status(void) {
   const cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_status(e, "csa_check_device_status");
-  const unsigned int st = csa::take_status_indexer_tc() | csa::take_status_mqa_umma();
+  const unsigned int st = csa::take_status_indexer_tc() | csa::take_status_mqa_umma() | csa::take_status_out_proj();
   if (st & 2u) return fail(CSA_ERR_CUDA, "csa_check_device_status: status word unreadable");
   if (st & 1u) {
     // a selection that gave up may have left counters set in the built-in
@@ -487,6 +487,50 @@ csa_status_t hca_dense_mqa(const void* Q, csa_dtype_t q_dt, const void* entries,
                            size_t ws_bytes, void* stream) {
   return hca_dense_mqa_ex(Q, q_dt, entries, n_entries, win, win_len, win_start, q_pos, window, m, sink,
                           softmax_scale, batch, n_q, n_heads, dim, kv_dt, O, ws, ws_bytes, nullptr, stream);
+}
+
+static csa_status_t check_out_proj(int T, int n_h, int c, int g, int d_g, int d) {
+  REQUIRE(T >= 0 && T <= (1 << 24), "T=%d out of range [0, 2^24]", T);
+  REQUIRE(n_h >= 1 && c >= 1 && g >= 1 && n_h % g == 0, "n_h=%d must be a positive multiple of g=%d", n_h, g);
+  REQUIRE((int64_t)(n_h / g) * c % 64 == 0 && (int64_t)n_h * c <= (1 << 20),
+          "n_h/g * c = %lld must be a multiple of 64 (n_h * c <= 2^20)", (long long)(n_h / g) * c);
+  REQUIRE(d_g >= 128 && d_g % 128 == 0 && (int64_t)g * d_g <= (1 << 20),
+          "d_g=%d must be a multiple of 128 (g * d_g <= 2^20)", d_g);
+  REQUIRE(d >= 128 && d % 128 == 0 && d <= (1 << 20), "d=%d must be a multiple of 128 (<= 2^20)", d);
+  return CSA_OK;
+}
+
+size_t csa_grouped_out_proj_workspace_size(int T, int n_h, int c, int g, int d_g, int d) {
+  if (check_out_proj(T, n_h, c, g, d_g, d) != CSA_OK || T == 0) return 256;
+  const size_t s = csa::out_proj_workspace(T, n_h, c, g, d_g, d);
+  return s < 256 ? 256 : s;
+}
+
+csa_status_t csa_grouped_out_proj_plan(int T, int n_h, int c, int g, int d_g, int d, int32_t* out) {
+  REQUIRE(out != nullptr, "out is NULL");
+  const csa_status_t st = check_out_proj(T, n_h, c, g, d_g, d);
+  if (st != CSA_OK) return st;
+  REQUIRE(T >= 1, "T must be >= 1");
+  csa::out_proj_plan_info(T, n_h, c, g, d_g, d, out);
+  return ok();
+}
+
+csa_status_t csa_grouped_out_proj(const void* O, const void* Wg, const void* Wo, void* Y, int T, int n_h, int c,
+                                  int g, int d_g, int d, void* ws, size_t ws_bytes, void* stream) {
+  g_launches = 0;
+  const csa_status_t st = check_out_proj(T, n_h, c, g, d_g, d);
+  if (st != CSA_OK) return st;
+  if (T == 0) return ok();
+  REQUIRE_PTR(O);
+  REQUIRE_PTR(Wg);
+  REQUIRE_PTR(Wo);
+  REQUIRE_PTR(Y);
+  REQUIRE_PTR(ws);
+  const size_t need = csa_grouped_out_proj_workspace_size(T, n_h, c, g, d_g, d);
+  REQUIRE(ws_bytes >= need, "workspace too small: %zu < %zu bytes", ws_bytes, need);
+  REQUIRE(Y != O && Y != ws && O != ws, "Y, O and ws must be distinct buffers");
+  csa::OutProjArgs a{O, Wg, Wo, Y, T, n_h, c, g, d_g, d, ws};
+  return cuda_status(csa::launch_out_proj(a, static_cast<cudaStream_t>(stream)), "csa_grouped_out_proj");
 }
 
 }  // extern "C"

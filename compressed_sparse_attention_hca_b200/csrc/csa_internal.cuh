@@ -158,6 +158,7 @@ int& launch_counter();
 // means a wait gave up, 2 means the word could not be read).
 unsigned int take_status_indexer_tc();
 unsigned int take_status_mqa_umma();
+unsigned int take_status_out_proj();
 // Zeroes the current device's built-in indexer scratch (csa_index_topk_noalloc)
 // after a timed-out wait; a no-op when the scratch was never used.
 void reset_static_scratch();
@@ -249,5 +250,17 @@ size_t mqa_workspace(const MqaArgs& a);
 // normalisation and RoPE options exist only there).
 bool mqa_tc_path(const MqaArgs& a);
 cudaError_t launch_mqa(const MqaArgs& a, cudaStream_t s);
+
+struct OutProjArgs {
+  const void *O, *Wg, *Wo;  // bf16: O [T][n_h][c], Wg [g][n_h/g * c][d_g], Wo [g * d_g][d]
+  void* Y;                  // bf16 [T][d]
+  int T, n_h, c, g, d_g, d;
+  void* ws;
+};
+size_t out_proj_workspace(int T, int n_h, int c, int g, int d_g, int d);
+// out[0..5]: tokens per CTA, K slices and CTAs of the group projection, then
+// the same three for the output projection.
+void out_proj_plan_info(int T, int n_h, int c, int g, int d_g, int d, int32_t* out);
+cudaError_t launch_out_proj(const OutProjArgs& a, cudaStream_t s);
 
 }  // namespace csa

@@ -206,3 +206,20 @@ def attention_inputs(cfg: dict, device="cpu", batch=None, ctx=None, n_q=None, q0
         out["wI"] = uniform(g, (B, T, HI), 0.0, 1.0, device)
     out.update(B=B, T=T, E=E, m=m, c=c, n_h=H, window=W, Lw=Lw, q0=q0)
     return out
+
+
+# V4-Pro grouped output projection ("DeepSeek-V4 内部机制" 1.2 Step 3: g = 16
+# groups, d_g = 1024; model dimension d = 7168 from the page's V4-Pro row).
+OUT_PROJ_V4_PRO = dict(n_h=128, c=512, g=16, d_g=1024, d=7168)
+
+
+def out_proj_inputs(g, T: int, n_h: int, c: int, groups: int, d_g: int, d: int, device="cpu"):
+    """Attention output O [T, n_h, c] (about N(0, 1)) and weights Wg
+    [groups, n_h/groups * c, d_g], Wo [groups * d_g, d] drawn N(0, 1/fan_in),
+    all bf16."""
+    k1 = n_h // groups * c
+    O = normal(g, (T, n_h, c), device=device).to(torch.bfloat16)
+    Wg = normal(g, (groups, k1, d_g), std=1.0 / math.sqrt(k1), device=device).to(torch.bfloat16)
+    Wo = normal(g, (groups * d_g, d), std=1.0 / math.sqrt(groups * d_g), device=device).to(torch.bfloat16)
+    return O, Wg, Wo
+

@@ -7,6 +7,7 @@
  *   [P5] "DeepSeek-V4 内部机制" (LLM-101-CN deep dive):
  *        1.2 Step 1 (compressor equations for S and C^Comp),
  *        1.2 Step 2 (index score I[t,s], top-k, shared-KV MQA),
+ *        1.2 Step 3 (grouped output projection: g groups, d_g each),
  *        1.3 (HCA: m' tokens per entry, no overlap, no top-k),
  *        1.4 table and sink equation (window branch of n_win = 128 raw
  *        tokens, per-head sink logit in the softmax denominator),
@@ -429,6 +430,43 @@ csa_status_t hca_dense_mqa_ex(const void* Q, csa_dtype_t q_dt, const void* entri
                               const float* sink, float softmax_scale, int batch, int n_q,
                               int n_heads, int dim, csa_dtype_t kv_dt, void* O, void* ws,
                               size_t ws_bytes, const csa_mqa_options_t* opt, void* stream);
+
+/*
+ * csa_grouped_out_proj -- grouped output projection after the core attention
+ * ([P5] 1.2 Step 3: the n_h head outputs of a token, c values each, are cut
+ * into g groups of n_h/g consecutive heads; each group is projected to d_g
+ * values, the g results are concatenated and projected to d; V4-Pro: g = 16,
+ * d_g = 1024, d = 7168).
+ *
+ *   Z[t, i*d_g + e] = sum_j O[t, i*(n_h/g)*c + j] * Wg[i][j][e]
+ *   Y[t, o]         = sum_j Z[t, j] * Wo[j][o]
+ *
+ *   O    [T][n_h][c] bf16 (the attention output, heads in index order).
+ *   Wg   [g][(n_h/g) * c][d_g] bf16, group i's weights at i.
+ *   Wo   [g * d_g][d] bf16.
+ *   Y    [T][d] bf16 output; distinct from O and ws.
+ * Products accumulate in fp32; Z is rounded once to bf16 (round to nearest
+ * even) before the second projection, Y once to bf16.  A sum split over
+ * several CTAs adds its slices in a fixed order, so results depend only on
+ * the shape (never on scheduling or on the device).
+ * Limits: (n_h/g) * c a multiple of 64, d_g and d multiples of 128, T <= 2^24.
+ * Workspace: csa_grouped_out_proj_workspace_size() bytes holding Z, fp32
+ * partial sums and one counter per output tile.  The counters must be zero
+ * before the first use (one cudaMemset after allocation); every call that
+ * completes leaves them zero, so the workspace may serve calls of other
+ * shapes in turn.  After CSA_ERR_TIMEOUT from csa_check_device_status, zero
+ * it again.  T = 0 launches nothing.
+ */
+size_t csa_grouped_out_proj_workspace_size(int T, int n_h, int c, int g, int d_g, int d);
+csa_status_t csa_grouped_out_proj(const void* O, const void* Wg, const void* Wo, void* Y, int T, int n_h, int c,
+                                  int g, int d_g, int d, void* ws, size_t ws_bytes, void* stream);
+/*
+ * csa_grouped_out_proj_plan -- how csa_grouped_out_proj divides a call of
+ * this shape (nothing is launched).  out[6] receives, for the group
+ * projection then for the output projection: tokens per CTA, K slices per
+ * output tile, CTAs launched.  Errors: as csa_grouped_out_proj, and T >= 1.
+ */
+csa_status_t csa_grouped_out_proj_plan(int T, int n_h, int c, int g, int d_g, int d, int32_t* out);
 
 #ifdef __cplusplus
 }

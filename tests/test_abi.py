@@ -164,3 +164,39 @@ def test_rmsnorm_rope_rejects_bad_arguments():
     assert call(x=None) == INVALID
     assert call(pos=None) == INVALID             # rotation needs positions
     assert "pos" in csa.load().csa_last_error().decode()
+
+
+def test_grouped_out_proj_rejects_bad_arguments():
+    lib = csa.load()
+
+    def call(O=A, Wg=A, Wo=A, Y=P(8192), T=4, n_h=16, c=64, g=4, d_g=128, d=256, ws=P(16384), wsb=1 << 30):
+        return lib.csa_grouped_out_proj(O, Wg, Wo, Y, T, n_h, c, g, d_g, d, ws, wsb, None)
+
+    assert call(T=0) == 0                       # nothing to do
+    assert call(T=-1) == INVALID
+    assert call(n_h=16, g=3) == INVALID         # groups must divide the heads
+    assert call(c=8) == INVALID                 # n_h/g * c = 32: not a multiple of 64
+    assert call(d_g=96) == INVALID              # not a multiple of 128
+    assert call(d=200) == INVALID
+    assert call(O=None) == INVALID
+    assert call(Wo=P(4104)) == INVALID          # misaligned
+    assert call(Y=A) == INVALID                 # Y aliases O
+    assert call(wsb=256) == INVALID and "workspace too small" in _err()
+
+
+def test_grouped_out_proj_plan():
+    v4 = dict(n_h=128, c=512, g=16, d_g=1024, d=7168)
+    for T in (1, 4, 16):
+        p = csa.grouped_out_proj_plan(T, **v4)
+        # decode reads only weights: K is split until both launches cover the 148 SMs
+        for step in ("group", "output"):
+            assert p[step]["ctas"] >= 148 and p[step]["splits"] > 1, (T, p)
+            assert p[step]["tokens_per_cta"] == 16
+    p = csa.grouped_out_proj_plan(4096, **v4)
+    assert p["group"] == {"tokens_per_cta": 256, "splits": 1, "ctas": 8 * 16 * 16}
+    assert p["output"] == {"tokens_per_cta": 256, "splits": 1, "ctas": 56 * 16}
+    # the workspace holds Z (bf16) at least, and grows with T
+    sizes = [csa.grouped_out_proj_workspace_size(T, **v4) for T in (1, 4, 64, 4096)]
+    assert sizes[-1] >= 4096 * 16 * 1024 * 2 and sizes == sorted(sizes)
+    with pytest.raises(csa.CsaError):
+        csa.grouped_out_proj_plan(0, **v4)
