@@ -74,6 +74,9 @@ def load():
                                     i32, i32, i32, P, P, sz, ctypes.POINTER(MqaOptions), P]),
         "hca_dense_mqa_ex": (i32, [P, i32, P, i64, P, i64, P, P, i32, i32, P, f32, i32, i32, i32, i32,
                                    i32, P, P, sz, ctypes.POINTER(MqaOptions), P]),
+        "csa_compress_ex": (i32, [ctypes.POINTER(CompressJob), i32, P]),
+        "csa_index_topk_paged": (i32, [P, P, P, P, P, ctypes.POINTER(Pages), P, i32, i32, i64, i32, i32, i32, i32,
+                                       i32, P, P, P, sz, P]),
         "csa_grouped_out_proj_workspace_size": (sz, [i32, i32, i32, i32, i32, i32]),
         "csa_grouped_out_proj_plan": (i32, [i32, i32, i32, i32, i32, i32, P]),
         "csa_grouped_out_proj": (i32, [P, P, P, P, i32, i32, i32, i32, i32, i32, P, sz, P]),
@@ -125,6 +128,25 @@ def _need_cuda(*ts):
     for t in ts:
         if t is not None and (not t.is_cuda or not t.is_contiguous()):
             raise ValueError("all tensors must be contiguous CUDA tensors")
+
+
+# ------------------------------------------------------------------ paged cache
+
+class Pages(ctypes.Structure):
+    """csa_pages_t: the block table of a paged cache."""
+    _fields_ = [("table", ctypes.c_void_p), ("max_pages", ctypes.c_int32), ("page_entries", ctypes.c_int32),
+                ("n_pages", ctypes.c_int64)]
+
+
+def pages(table, page_entries, n_pages):
+    """A block table: table [batch, max_pages] int32 (CUDA) of pool pages of
+    page_entries rows each; n_pages pages in the pool."""
+    _need_cuda(table)
+    if table.dtype != torch.int32 or table.dim() != 2:
+        raise ValueError("table must be a [batch, max_pages] int32 tensor")
+    p = Pages(table=table.data_ptr(), max_pages=table.shape[1], page_entries=page_entries, n_pages=n_pages)
+    p._keep = table  # the struct holds a raw pointer: keep the tensor alive with it
+    return p
 
 
 # --------------------------------------------------------------------- compress
@@ -199,16 +221,19 @@ def index_topk_plan(batch, n_q, n_entries, k, n_heads, dim, dt):
 
 
 def index_topk(qI, wI, KI, q_pos, m, k, *, dt=None, qI_sf=None, KI_sf=None, n_heads=None,
-               scores=False, idx_out=None, ws=None):
+               scores=False, idx_out=None, ws=None, key_pages=None, n_entries=None):
     """Lightning indexer + top-k.  qI [B, T, H, d] (or NVFP4 codes [B, T, H, d/2]),
     wI [B, T, H] fp32, KI [B, E, d] (codes [B, E, d/2]), q_pos [B, T] int64.
+    Paged keys: key_pages a Pages (pages()), KI / KI_sf the pool, n_entries = E.
 
     Returns idx [B, T, k] int32 (and the score tensor when scores=True)."""
     _need_cuda(qI, wI, KI, q_pos, qI_sf, KI_sf)
     if dt is None:
         dt = IDX_NVFP4 if qI.dtype == torch.uint8 else _dt_of(qI)
     B, T, H = wI.shape
-    E = KI.shape[1]
+    if key_pages is not None and n_entries is None:
+        raise ValueError("paged keys need n_entries (logical keys per request)")
+    E = KI.shape[1] if n_entries is None else n_entries
     dim = qI.shape[-1] * (2 if dt == IDX_NVFP4 else 1)
     dev = qI.device
     if idx_out is None:
@@ -219,9 +244,10 @@ def index_topk(qI, wI, KI, q_pos, m, k, *, dt=None, qI_sf=None, KI_sf=None, n_he
     need = index_topk_workspace_size(B, T, E, k, H, dim, dt)
     if ws is None or ws.numel() < need:
         ws = torch.zeros(need, device=dev, dtype=torch.uint8)  # zero before first use
-    _check(load().csa_index_topk(_ptr(qI), _ptr(qI_sf), _ptr(wI), _ptr(KI), _ptr(KI_sf), _ptr(q_pos),
-                                 B, T, E, m, H, dim, k, dt, _ptr(idx_out), _ptr(sc), _ptr(ws),
-                                 ws.numel(), _stream()))
+    _check(load().csa_index_topk_paged(_ptr(qI), _ptr(qI_sf), _ptr(wI), _ptr(KI), _ptr(KI_sf),
+                                       ctypes.byref(key_pages) if key_pages is not None else None, _ptr(q_pos),
+                                       B, T, E, m, H, dim, k, dt, _ptr(idx_out), _ptr(sc), _ptr(ws),
+                                       ws.numel(), _stream()))
     return (idx_out, sc) if scores else idx_out
 
 
@@ -232,13 +258,14 @@ class CompressJob(ctypes.Structure):
                 ("tok0", ctypes.c_int64), ("in_batch_stride", ctypes.c_int64), ("e0", ctypes.c_int64),
                 ("n_out", ctypes.c_int64), ("dim", ctypes.c_int32), ("m", ctypes.c_int32), ("in_dt", ctypes.c_int32),
                 ("out", ctypes.c_void_p), ("out_sf", ctypes.c_void_p), ("out_batch_stride", ctypes.c_int64),
-                ("out_row0", ctypes.c_int64), ("out_dt", ctypes.c_int32)]
+                ("out_row0", ctypes.c_int64), ("out_dt", ctypes.c_int32), ("out_pages", ctypes.POINTER(Pages))]
 
 
 def compress_job(Ca, Za, Ba, m, Cb=None, Zb=None, Bb=None, *, tok0, e0, n_out, out, out_dt, out_sf=None,
-                 out_row0=None, n_tok=None):
+                 out_row0=None, n_tok=None, out_pages=None):
     """A compressor call's arguments as a CompressJob (entries e0.. written to
-    rows out_row0.. of `out`, out_row0 defaulting to e0)."""
+    rows out_row0.. of `out`, out_row0 defaulting to e0; with out_pages (a
+    Pages) `out` / `out_sf` are the pool and rows are logical rows)."""
     _need_cuda(Ca, Za, Ba, Cb, Zb, Bb, out, out_sf)
     batch, rows, dim = Ca.shape
     job = CompressJob(
@@ -246,12 +273,19 @@ def compress_job(Ca, Za, Ba, m, Cb=None, Zb=None, Bb=None, *, tok0, e0, n_out, o
         Zb=Zb.data_ptr() if Zb is not None else None, Ba=Ba.data_ptr(), Bb=Bb.data_ptr() if Bb is not None else None,
         n_tok=rows if n_tok is None else n_tok, tok0=tok0, in_batch_stride=rows, e0=e0, n_out=n_out, dim=dim, m=m,
         in_dt=_dt_of(Ca), out=out.data_ptr(), out_sf=out_sf.data_ptr() if out_sf is not None else None,
-        out_batch_stride=out.shape[1], out_row0=e0 if out_row0 is None else out_row0, out_dt=out_dt)
+        out_batch_stride=out.shape[1], out_row0=e0 if out_row0 is None else out_row0, out_dt=out_dt,
+        out_pages=ctypes.pointer(out_pages) if out_pages is not None else None)
+    job._keep = out_pages  # the struct holds a raw pointer: keep the table alive with it
     return job
 
 
+def compress_ex(job, batch):
+    """Runs one CompressJob (compress_job()) on `batch` requests."""
+    _check(load().csa_compress_ex(ctypes.byref(job), batch, _stream()))
+
+
 def compress_index_topk(keys_job, qI, wI, KI, q_pos, m, k, *, extra_job=None, dt=None, qI_sf=None, KI_sf=None,
-                        idx_out=None, ws=None, scores=False):
+                        idx_out=None, ws=None, scores=False, n_entries=None):
     """Run the compressor job `keys_job` (index keys into KI / KI_sf) and, if
     given, `extra_job` (e.g. the KV cache), then index + top-k over KI: one
     launch when the tensor-core indexer takes the shape.  Returns idx
@@ -260,7 +294,9 @@ def compress_index_topk(keys_job, qI, wI, KI, q_pos, m, k, *, extra_job=None, dt
     if dt is None:
         dt = IDX_NVFP4 if qI.dtype == torch.uint8 else _dt_of(qI)
     B, T, H = wI.shape
-    E = KI.shape[1]
+    if keys_job.out_pages and n_entries is None:
+        raise ValueError("a paged key cache needs n_entries (logical keys per request)")
+    E = KI.shape[1] if n_entries is None else n_entries
     dim = qI.shape[-1] * (2 if dt == IDX_NVFP4 else 1)
     dev = qI.device
     if idx_out is None:
@@ -284,18 +320,30 @@ def compress_index_topk(keys_job, qI, wI, KI, q_pos, m, k, *, extra_job=None, dt
 class MqaOptions(ctypes.Structure):
     """csa_mqa_options_t: fixed split count (batch-invariant decode), query
     RMSNorm weights and eps, RoPE dims of the query (at q_pos) and of the
-    output (at -q_pos), RoPE base."""
+    output (at -q_pos), RoPE base, block table of a paged entry cache."""
     _fields_ = [("splits", ctypes.c_int32), ("q_norm_g", ctypes.c_void_p), ("q_norm_eps", ctypes.c_float),
-                ("q_rope_dims", ctypes.c_int32), ("out_rope_dims", ctypes.c_int32), ("rope_base", ctypes.c_double)]
+                ("q_rope_dims", ctypes.c_int32), ("out_rope_dims", ctypes.c_int32), ("rope_base", ctypes.c_double),
+                ("entry_pages", ctypes.POINTER(Pages))]
 
 
-def mqa_options(*, splits=0, q_norm_g=None, q_norm_eps=1e-6, q_rope_dims=0, out_rope_dims=0, rope_base=10000.0):
+def mqa_options(*, splits=0, q_norm_g=None, q_norm_eps=1e-6, q_rope_dims=0, out_rope_dims=0, rope_base=10000.0,
+                entry_pages=None):
+    """Options of the attention calls; entry_pages: a Pages (pages()) when
+    `entries` is the pool of a paged cache."""
     _need_cuda(q_norm_g)
     o = MqaOptions(splits=splits, q_norm_g=q_norm_g.data_ptr() if q_norm_g is not None else None,
                    q_norm_eps=q_norm_eps, q_rope_dims=q_rope_dims, out_rope_dims=out_rope_dims,
-                   rope_base=rope_base)
-    o._keep = q_norm_g  # the struct holds a raw pointer: keep the tensor alive with it
+                   rope_base=rope_base, entry_pages=ctypes.pointer(entry_pages) if entry_pages is not None else None)
+    o._keep = (q_norm_g, entry_pages)  # raw pointers: keep what they point to alive with the struct
     return o
+
+
+def _n_entries(entries, n_entries, options):
+    if options is not None and options.entry_pages:
+        if n_entries is None:
+            raise ValueError("a paged call needs n_entries (logical entries per request)")
+        return n_entries
+    return entries.shape[1] if n_entries is None else n_entries
 
 
 def _opt_ref(options):
@@ -323,9 +371,10 @@ def hca_dense_mqa_workspace_size(batch, n_q, n_heads, dim, n_entries, window, q_
 
 
 def sparse_mqa(Q, entries, idx, win, win_start, q_pos, window, m, sink, scale, *, kv_dt=None, O=None,
-               ws=None, options=None):
-    """CSA shared-KV MQA.  Q [B, T, H, c]; entries [B, E, row]; idx [B, T, k] int32;
-    win [B, Lw, row]; win_start [B] int64; q_pos [B, T] int64; sink [H] fp32.
+               ws=None, options=None, n_entries=None):
+    """CSA shared-KV MQA.  Q [B, T, H, c]; entries [B, E, row] (paged: the
+    pool, with n_entries = E); idx [B, T, k] int32; win [B, Lw, row];
+    win_start [B] int64; q_pos [B, T] int64; sink [H] fp32.
     options: an MqaOptions (mqa_options()) or None."""
     _need_cuda(Q, entries, idx, win, win_start, q_pos, sink)
     B, T, H, c = Q.shape
@@ -337,7 +386,8 @@ def sparse_mqa(Q, entries, idx, win, win_start, q_pos, window, m, sink, scale, *
     need = mqa_workspace_size(B, T, H, c, k + window, q_dt, kv_dt, options)
     if ws is None or ws.numel() < need:
         ws = torch.empty(need, device=Q.device, dtype=torch.uint8)
-    _check(load().csa_sparse_mqa_ex(_ptr(Q), q_dt, _ptr(entries), entries.shape[1], _ptr(idx), k, _ptr(win),
+    _check(load().csa_sparse_mqa_ex(_ptr(Q), q_dt, _ptr(entries), _n_entries(entries, n_entries, options), _ptr(idx),
+                                    k, _ptr(win),
                                     win.shape[1], _ptr(win_start), _ptr(q_pos), window, m, _ptr(sink),
                                     float(scale), B, T, H, c, kv_dt, _ptr(O), _ptr(ws), ws.numel(),
                                     _opt_ref(options), _stream()))
@@ -345,18 +395,20 @@ def sparse_mqa(Q, entries, idx, win, win_start, q_pos, window, m, sink, scale, *
 
 
 def hca_dense_mqa(Q, entries, win, win_start, q_pos, window, m, sink, scale, *, kv_dt=None, O=None,
-                  ws=None, options=None):
-    """HCA dense shared-KV MQA over every visible entry plus the window."""
+                  ws=None, options=None, n_entries=None):
+    """HCA dense shared-KV MQA over every visible entry plus the window
+    (paged: entries is the pool, n_entries the logical entries)."""
     _need_cuda(Q, entries, win, win_start, q_pos, sink)
     B, T, H, c = Q.shape
     kv_dt = _kv_dt(entries, kv_dt)
     q_dt = _dt_of(Q)
     if O is None:
         O = torch.empty_like(Q)
-    need = mqa_workspace_size(B, T, H, c, entries.shape[1] + window, q_dt, kv_dt, options)
+    E = _n_entries(entries, n_entries, options)
+    need = mqa_workspace_size(B, T, H, c, E + window, q_dt, kv_dt, options)
     if ws is None or ws.numel() < need:
         ws = torch.empty(need, device=Q.device, dtype=torch.uint8)
-    _check(load().hca_dense_mqa_ex(_ptr(Q), q_dt, _ptr(entries), entries.shape[1], _ptr(win), win.shape[1],
+    _check(load().hca_dense_mqa_ex(_ptr(Q), q_dt, _ptr(entries), E, _ptr(win), win.shape[1],
                                    _ptr(win_start), _ptr(q_pos), window, m, _ptr(sink), float(scale), B, T,
                                    H, c, kv_dt, _ptr(O), _ptr(ws), ws.numel(), _opt_ref(options), _stream()))
     return O

@@ -49,6 +49,24 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
       return fail(CSA_ERR_INVALID_ARG, "%s is not 16-byte aligned", #p);     \
   } while (0)
 
+// A block table covering `rows` logical rows per request.
+csa_status_t check_pages(const csa_pages_t* p, int64_t rows, const char* what) {
+  REQUIRE(p->table != nullptr, "%s: table is NULL", what);
+  REQUIRE(aligned16(p->table), "%s: table is not 16-byte aligned", what);
+  REQUIRE(p->max_pages >= 1 && p->page_entries >= 1 && p->n_pages >= 1,
+          "%s: max_pages, page_entries and n_pages must be >= 1", what);
+  REQUIRE(p->n_pages <= ((int64_t)1 << 31) && p->n_pages * p->page_entries <= ((int64_t)1 << 40),
+          "%s: pool too large", what);
+  REQUIRE(rows <= (int64_t)p->max_pages * p->page_entries,
+          "%s: %lld rows per request exceed max_pages * page_entries = %lld", what, (long long)rows,
+          (long long)p->max_pages * p->page_entries);
+  return CSA_OK;
+}
+
+csa::PageTable to_pages(const csa_pages_t* p) {
+  return csa::PageTable{p->table, p->max_pages, p->page_entries, p->n_pages};
+}
+
 }  // namespace
 
 int& csa::launch_counter() { return g_launches; }
@@ -61,7 +79,8 @@ static csa_status_t check_compress(const void* Ca, const void* Cb, const void* Z
                                    const float* Ba, const float* Bb, int batch, int64_t n_tok, int64_t tok0,
                                    int64_t in_batch_stride, int64_t e0, int64_t n_out, int dim, int m,
                                    csa_dtype_t in_dt, void* out, void* out_sf, int64_t out_batch_stride,
-                                   int64_t out_row0, csa_dtype_t out_dt, csa::CompressArgs* args, bool* empty) {
+                                   int64_t out_row0, csa_dtype_t out_dt, const csa_pages_t* out_pages,
+                                   csa::CompressArgs* args, bool* empty) {
   *empty = false;
   REQUIRE(batch >= 0 && n_tok >= 0 && tok0 >= 0 && e0 >= 0 && n_out >= 0 && out_row0 >= 0,
           "negative size (batch=%d n_tok=%lld tok0=%lld e0=%lld n_out=%lld out_row0=%lld)", batch,
@@ -75,8 +94,16 @@ static csa_status_t check_compress(const void* Ca, const void* Cb, const void* Z
   if (out_dt == CSA_IDX_NVFP4) REQUIRE(dim % 64 == 0, "NVFP4 output needs dim %% 64 == 0, got %d", dim);
   REQUIRE(in_batch_stride >= n_tok, "in_batch_stride %lld < n_tok %lld", (long long)in_batch_stride,
           (long long)n_tok);
-  REQUIRE(out_batch_stride >= out_row0 + n_out, "out_batch_stride %lld < out_row0 %lld + n_out %lld",
-          (long long)out_batch_stride, (long long)out_row0, (long long)n_out);
+  if (out_pages == nullptr) {
+    REQUIRE(out_batch_stride >= out_row0 + n_out, "out_batch_stride %lld < out_row0 %lld + n_out %lld",
+            (long long)out_batch_stride, (long long)out_row0, (long long)n_out);
+  } else {
+    const csa_status_t st = check_pages(out_pages, out_row0 + n_out, "out_pages");
+    if (st != CSA_OK) return st;
+    if (out_dt == CSA_IDX_NVFP4)
+      REQUIRE(128 % out_pages->page_entries == 0, "paged NVFP4 keys need page_entries dividing 128, got %d",
+              out_pages->page_entries);
+  }
   if ((int64_t)batch * n_out == 0) {
     *empty = true;
     return ok();
@@ -102,7 +129,8 @@ static csa_status_t check_compress(const void* Ca, const void* Cb, const void* Z
           (long long)e0, (long long)(e0 + n_out), (long long)first, (long long)last,
           (long long)tok0, (long long)(tok0 + n_tok));
   *args = csa::CompressArgs{Ca, Cb, Za, Zb, Ba, Bb, batch, n_tok, tok0, in_batch_stride, e0, n_out,
-                            dim, m, (int)in_dt, (int)out_dt, out, out_sf, out_batch_stride, out_row0};
+                            dim, m, (int)in_dt, (int)out_dt, out, out_sf, out_batch_stride, out_row0,
+                            out_pages ? to_pages(out_pages) : csa::PageTable{nullptr, 0, 0, 0}};
   return ok();
 }
 
@@ -112,7 +140,8 @@ static csa_status_t check_compress(const void* Ca, const void* Cb, const void* Z
 static csa_status_t check_index(const void* qI, const void* qI_sf, const float* wI, const void* KI,
                                 const void* KI_sf, const int64_t* q_pos, int batch, int n_q, int64_t n_entries,
                                 int m, int n_heads, int dim, int k, csa_dtype_t dt, int32_t* idx_out,
-                                void* scores_out, void* ws, size_t ws_bytes, csa::IndexArgs* args, bool* empty) {
+                                void* scores_out, void* ws, size_t ws_bytes, const csa_pages_t* key_pages,
+                                csa::IndexArgs* args, bool* empty) {
   *empty = false;
   REQUIRE(batch >= 0 && n_q >= 0 && n_entries >= 0, "negative size");
   REQUIRE(n_entries <= (int64_t)1 << 30, "n_entries=%lld too large", (long long)n_entries);
@@ -136,11 +165,20 @@ static csa_status_t check_index(const void* qI, const void* qI_sf, const float* 
     REQUIRE(dim % 64 == 0, "NVFP4 needs dim %% 64 == 0 (blocked key scales), got %d", dim);
     REQUIRE_ALIGNED_OR_NULL(KI_sf);
   }
+  if (key_pages != nullptr) {
+    const csa_status_t st = check_pages(key_pages, n_entries, "key_pages");
+    if (st != CSA_OK) return st;
+    const int pe = key_pages->page_entries;
+    REQUIRE(pe >= 8 && 128 % pe == 0, "paged keys need page_entries in {8, 16, 32, 64, 128}, got %d", pe);
+    REQUIRE(key_pages->n_pages * pe < ((int64_t)1 << 31), "key pool of %lld rows too large",
+            (long long)(key_pages->n_pages * pe));
+  }
   const size_t need = csa_index_topk_workspace_size(batch, n_q, n_entries, k, n_heads, dim, dt);
   REQUIRE(ws_bytes >= need, "workspace too small: %zu < %zu bytes", ws_bytes, need);
   REQUIRE_PTR(ws);
   *args = csa::IndexArgs{qI, qI_sf, wI, KI, KI_sf, q_pos, batch, n_q, n_entries, m, n_heads, dim, k,
-                         (int)dt, idx_out, scores_out, ws, ws_bytes, 0, csa::CompressArgs{}, csa::CompressArgs{}};
+                         (int)dt, idx_out, scores_out, ws, ws_bytes, 0, csa::CompressArgs{}, csa::CompressArgs{},
+                         key_pages ? to_pages(key_pages) : csa::PageTable{nullptr, 0, 0, 0}};
   return ok();
 }
 
@@ -154,7 +192,8 @@ int csa_last_launch_count(void) { return g_launches; }
 csa_status_t csa_check_device_status(void) {
   const cudaError_t e = cudaDeviceSynchronize();
   if (e != cudaSuccess) return cuda_status(e, "csa_check_device_status");
-  const unsigned int st = csa::take_status_indexer_tc() | csa::take_status_mqa_umma() | csa::take_status_out_proj();
+  const unsigned int st = csa::take_status_indexer_tc() | csa::take_status_mqa_umma() | csa::take_status_out_proj() |
+                          csa::take_status_mqa() | csa::take_status_indexer() | csa::take_status_compress();
   if (st & 2u) return fail(CSA_ERR_CUDA, "csa_check_device_status: status word unreadable");
   if (st & 1u) {
     // a selection that gave up may have left counters set in the built-in
@@ -163,6 +202,7 @@ csa_status_t csa_check_device_status(void) {
     csa::reset_static_scratch();
     return fail(CSA_ERR_TIMEOUT, "a kernel pipeline wait timed out; its results are invalid");
   }
+  if (st & 4u) return fail(CSA_ERR_INVALID_ARG, "a page table named a page outside the pool; rows were dropped");
   return ok();
 }
 
@@ -190,9 +230,23 @@ csa_status_t csa_compress(const void* Ca, const void* Cb, const void* Za, const 
   csa::CompressArgs a{};
   bool empty = false;
   const csa_status_t st = check_compress(Ca, Cb, Za, Zb, Ba, Bb, batch, n_tok, tok0, in_batch_stride, e0, n_out,
-                                         dim, m, in_dt, out, out_sf, out_batch_stride, out_row0, out_dt, &a, &empty);
+                                         dim, m, in_dt, out, out_sf, out_batch_stride, out_row0, out_dt, nullptr, &a,
+                                         &empty);
   if (st != CSA_OK || empty) return st;
   return cuda_status(csa::launch_compress(a, static_cast<cudaStream_t>(stream)), "csa_compress");
+}
+
+csa_status_t csa_compress_ex(const csa_compress_job_t* job, int batch, void* stream) {
+  g_launches = 0;
+  REQUIRE(job != nullptr, "job is NULL");
+  csa::CompressArgs a{};
+  bool empty = false;
+  const csa_status_t st = check_compress(job->Ca, job->Cb, job->Za, job->Zb, job->Ba, job->Bb, batch, job->n_tok,
+                                         job->tok0, job->in_batch_stride, job->e0, job->n_out, job->dim, job->m,
+                                         job->in_dt, job->out, job->out_sf, job->out_batch_stride, job->out_row0,
+                                         job->out_dt, job->out_pages, &a, &empty);
+  if (st != CSA_OK || empty) return st;
+  return cuda_status(csa::launch_compress(a, static_cast<cudaStream_t>(stream)), "csa_compress_ex");
 }
 
 csa_status_t csa_rmsnorm_rope(const void* x, void* y, int64_t n_rows, int dim, const float* g, float eps,
@@ -245,11 +299,19 @@ csa_status_t csa_index_topk(const void* qI, const void* qI_sf, const float* wI, 
                             int64_t n_entries, int m, int n_heads, int dim, int k, csa_dtype_t dt,
                             int32_t* idx_out, void* scores_out, void* ws, size_t ws_bytes,
                             void* stream) {
+  return csa_index_topk_paged(qI, qI_sf, wI, KI, KI_sf, nullptr, q_pos, batch, n_q, n_entries, m, n_heads, dim, k,
+                              dt, idx_out, scores_out, ws, ws_bytes, stream);
+}
+
+csa_status_t csa_index_topk_paged(const void* qI, const void* qI_sf, const float* wI, const void* KI,
+                                  const void* KI_sf, const csa_pages_t* key_pages, const int64_t* q_pos, int batch,
+                                  int n_q, int64_t n_entries, int m, int n_heads, int dim, int k, csa_dtype_t dt,
+                                  int32_t* idx_out, void* scores_out, void* ws, size_t ws_bytes, void* stream) {
   g_launches = 0;
   csa::IndexArgs a{};
   bool empty = false;
   const csa_status_t st = check_index(qI, qI_sf, wI, KI, KI_sf, q_pos, batch, n_q, n_entries, m, n_heads, dim, k,
-                                      dt, idx_out, scores_out, ws, ws_bytes, &a, &empty);
+                                      dt, idx_out, scores_out, ws, ws_bytes, key_pages, &a, &empty);
   if (st != CSA_OK || empty) return st;
   return cuda_status(csa::launch_index_topk(a, static_cast<cudaStream_t>(stream)), "csa_index_topk");
 }
@@ -262,15 +324,15 @@ csa_status_t csa_compress_index_topk(const csa_compress_job_t* keys, const csa_c
   g_launches = 0;
   REQUIRE(keys != nullptr, "keys is NULL");
   REQUIRE(keys->out == KI && keys->out_sf == KI_sf && keys->out_dt == dt && keys->dim == dim &&
-              keys->out_batch_stride == n_entries && keys->out_row0 == keys->e0,
+              (keys->out_pages != nullptr || keys->out_batch_stride == n_entries) && keys->out_row0 == keys->e0,
           "keys must write entry i into row i of the indexer's cache (out == KI, out_sf == KI_sf, out_dt == dt, "
-          "dim == dim, out_batch_stride == n_entries, out_row0 == e0)");
+          "dim == dim, out_batch_stride == n_entries unless paged, out_row0 == e0)");
   csa::CompressArgs c{}, c2{};
   bool c_empty = false, c2_empty = true;
   csa_status_t st = check_compress(keys->Ca, keys->Cb, keys->Za, keys->Zb, keys->Ba, keys->Bb, batch, keys->n_tok,
                                    keys->tok0, keys->in_batch_stride, keys->e0, keys->n_out, keys->dim, keys->m,
                                    keys->in_dt, keys->out, keys->out_sf, keys->out_batch_stride, keys->out_row0,
-                                   keys->out_dt, &c, &c_empty);
+                                   keys->out_dt, keys->out_pages, &c, &c_empty);
   if (st != CSA_OK) return st;
   if (extra != nullptr) {
     REQUIRE(extra->out != KI && (extra->out_sf == nullptr || extra->out_sf != KI_sf),
@@ -278,13 +340,13 @@ csa_status_t csa_compress_index_topk(const csa_compress_job_t* keys, const csa_c
     st = check_compress(extra->Ca, extra->Cb, extra->Za, extra->Zb, extra->Ba, extra->Bb, batch, extra->n_tok,
                         extra->tok0, extra->in_batch_stride, extra->e0, extra->n_out, extra->dim, extra->m,
                         extra->in_dt, extra->out, extra->out_sf, extra->out_batch_stride, extra->out_row0,
-                        extra->out_dt, &c2, &c2_empty);
+                        extra->out_dt, extra->out_pages, &c2, &c2_empty);
     if (st != CSA_OK) return st;
   }
   csa::IndexArgs a{};
   bool i_empty = false;
   st = check_index(qI, qI_sf, wI, KI, KI_sf, q_pos, batch, n_q, n_entries, m, n_heads, dim, k, dt, idx_out,
-                   scores_out, ws, ws_bytes, &a, &i_empty);
+                   scores_out, ws, ws_bytes, keys->out_pages, &a, &i_empty);
   if (st != CSA_OK) return st;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   a.comp = c;
@@ -330,6 +392,7 @@ csa_status_t apply_mqa_options(csa::MqaArgs& a, const csa_mqa_options_t* opt) {
   a.q_norm_eps = 0.f;
   a.q_rope_dims = a.out_rope_dims = 0;
   a.rope_base = 10000.0;
+  a.pages = csa::PageTable{nullptr, 0, 0, 0};
   if (opt == nullptr) return CSA_OK;
   REQUIRE(opt->splits >= 0 && opt->splits <= 256, "splits=%d out of range [0, 256]", opt->splits);
   REQUIRE(opt->q_rope_dims >= 0 && opt->q_rope_dims <= 64 && opt->q_rope_dims % 8 == 0,
@@ -344,6 +407,11 @@ csa_status_t apply_mqa_options(csa::MqaArgs& a, const csa_mqa_options_t* opt) {
   a.q_rope_dims = opt->q_rope_dims;
   a.out_rope_dims = opt->out_rope_dims;
   a.rope_base = opt->rope_base;
+  if (opt->entry_pages != nullptr) {
+    const csa_status_t st = check_pages(opt->entry_pages, a.n_entries, "entry_pages");
+    if (st != CSA_OK) return st;
+    a.pages = to_pages(opt->entry_pages);
+  }
   return CSA_OK;
 }
 
@@ -422,7 +490,15 @@ size_t csa_mqa_workspace_size(int batch, int n_q, int n_heads, int dim, int64_t 
   csa::MqaArgs a = mqa_args(nullptr, q_dt, nullptr, rows_per_query < 0 ? 0 : rows_per_query, nullptr, 0, nullptr,
                             0, nullptr, nullptr, 0, 1, nullptr, 1.f, batch, n_q, n_heads, dim, kv_dt, nullptr,
                             nullptr, 0);
-  if (apply_mqa_options(a, opt) != CSA_OK || check_mqa(a) != CSA_OK || batch <= 0 || n_q <= 0) return 256;
+  // the block table does not change the workspace (rows_per_query is not an
+  // entry count, so the table is not checked against it here)
+  csa_mqa_options_t o{};
+  if (opt != nullptr) {
+    o = *opt;
+    o.entry_pages = nullptr;
+  }
+  if (apply_mqa_options(a, opt ? &o : nullptr) != CSA_OK || check_mqa(a) != CSA_OK || batch <= 0 || n_q <= 0)
+    return 256;
   const size_t s = csa::mqa_workspace(a);
   return s < 256 ? 256 : s;
 }

@@ -9,8 +9,12 @@
 // scale block (8 lanes = 64 dims) or an FP4 block (2 lanes = 16 dims) reduce
 // their amax with warp shuffles and quantise in the epilogue.
 #include "compress_dev.cuh"
+#include "sm100.cuh"
 
 namespace csa {
+
+CSA_DEFINE_STATUS_READER(take_status_compress)
+
 namespace {
 
 __global__ void __launch_bounds__(256) compress_kernel(CompressArgs a) {

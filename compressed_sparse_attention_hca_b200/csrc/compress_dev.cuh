@@ -5,6 +5,7 @@
 #pragma once
 
 #include "csa_internal.cuh"
+#include "sm100.cuh"
 
 namespace csa {
 namespace {
@@ -31,7 +32,17 @@ __device__ __forceinline__ void load8(const void* base, int dt, int64_t elem, fl
 // shuffles; lanes with valid == false take part in the shuffles only.
 __device__ __forceinline__ void store_entry(const CompressArgs& a, int b, int64_t ie, int d0, const float* x,
                                             bool valid) {
-  const int64_t orow = (int64_t)b * a.out_batch_stride + a.out_row0 + ie;
+  const bool paged = a.out_pages.table != nullptr;
+  const int64_t lr = a.out_row0 + ie;  // logical row of the entry in request b's cache
+  int64_t orow = (int64_t)b * a.out_batch_stride + lr;
+  if (paged) {
+    orow = pool_row(a.out_pages, b, lr);
+    if (orow < 0) {
+      if (valid) flag_status(kStatusBadPage);
+      valid = false;  // the lanes still take part in the scale shuffles
+      orow = 0;
+    }
+  }
   const int64_t rb = row_bytes(a.out_dt, a.dim);
   uint8_t* row = static_cast<uint8_t*>(a.out) + orow * rb;
 
@@ -109,9 +120,17 @@ __device__ __forceinline__ void store_entry(const CompressArgs& a, int b, int64_
       if ((d0 % kFp4Block) == 0) {
         // key-cache scales live in the blocked scale-factor atom layout
         const int j = d0 / kFp4Block;
-        const int64_t off = (int64_t)b * nvfp4_blocked_sf_bytes(a.out_batch_stride, a.dim) +
-                            nvfp4_blocked_sf_offset(a.out_row0 + ie, a.dim) + (j / 4) * 512 + (j % 4);
-        static_cast<uint8_t*>(a.out_sf)[off] = (uint8_t)s8;
+        int64_t off = (int64_t)b * nvfp4_blocked_sf_bytes(a.out_batch_stride, a.dim) +
+                      nvfp4_blocked_sf_offset(lr, a.dim);
+        if (paged) {
+          // the page's block (one 128-row block per pool page); the page
+          // holding the codes was in the pool, so is this one unless the
+          // table is inconsistent
+          const int64_t pg = pool_sf_page(a.out_pages, b, lr);
+          off = pg < 0 ? -1 : pg * nvfp4_blocked_sf_bytes(128, a.dim) + nvfp4_blocked_sf_offset(lr % 128, a.dim);
+          if (pg < 0) flag_status(kStatusBadPage);
+        }
+        if (off >= 0) static_cast<uint8_t*>(a.out_sf)[off + (j / 4) * 512 + (j % 4)] = (uint8_t)s8;
       }
     }
   }

@@ -130,6 +130,38 @@ __host__ __device__ __forceinline__ int64_t nvfp4_blocked_sf_bytes(int64_t n_row
   return (n_rows + 127) / 128 * (dim / 64) * 512;
 }
 
+// A paged cache ("CSA / HCA" cache layout: fixed pages of 128 tokens taken
+// from a shared pool through a per-request block table): logical row lr of
+// request b lives in pool row table[b][lr / page_entries] * page_entries +
+// lr % page_entries.  table == nullptr: the contiguous layout, request b's
+// rows at b * (rows per request).
+struct PageTable {
+  const int32_t* table;  // [batch][max_pages]
+  int max_pages;
+  int page_entries;
+  int64_t n_pages;       // pages in the pool
+};
+// Pool page of logical page j of request b, or -1 when the table names a page
+// outside the pool.
+__device__ __forceinline__ int64_t pool_page(const PageTable& pt, int b, int64_t j) {
+  const int32_t pg = __ldg(pt.table + (int64_t)b * pt.max_pages + j);
+  return (pg < 0 || pg >= pt.n_pages) ? -1 : (int64_t)pg;
+}
+// Pool row of logical row lr of request b, or -1 (page outside the pool).
+__device__ __forceinline__ int64_t pool_row(const PageTable& pt, int b, int64_t lr) {
+  const int64_t j = lr / pt.page_entries;
+  const int64_t pg = pool_page(pt, b, j);
+  return pg < 0 ? -1 : pg * pt.page_entries + (lr - j * pt.page_entries);
+}
+// Paged NVFP4 key scales: one blocked 128-row block (dim/64 atoms) per pool
+// page; the 128 logical rows 128 u .. 128 u + 127 (page_entries divides 128)
+// keep theirs in the block of the pool page holding logical row 128 u, at the
+// offset the contiguous layout gives row lr % 128.  Pool page of that block,
+// or -1.
+__device__ __forceinline__ int64_t pool_sf_page(const PageTable& pt, int b, int64_t lr) {
+  return pool_page(pt, b, (lr / 128) * (128 / pt.page_entries));
+}
+
 // Order-preserving key of a float score (larger score -> larger key).
 __device__ __forceinline__ uint32_t f32_key(float s) {
   uint32_t u = __float_as_uint(s);
@@ -159,6 +191,9 @@ int& launch_counter();
 unsigned int take_status_indexer_tc();
 unsigned int take_status_mqa_umma();
 unsigned int take_status_out_proj();
+unsigned int take_status_mqa();
+unsigned int take_status_indexer();
+unsigned int take_status_compress();
 // Zeroes the current device's built-in indexer scratch (csa_index_topk_noalloc)
 // after a timed-out wait; a no-op when the scratch was never used.
 void reset_static_scratch();
@@ -172,6 +207,9 @@ struct CompressArgs {
   int dim, m, in_dt, out_dt;
   void *out, *out_sf;
   int64_t out_batch_stride, out_row0;
+  // output rows through a block table (out_pages.table != nullptr): row
+  // out_row0 + j of request b is logical row out_row0 + j of its pages
+  PageTable out_pages;
 };
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s);
 
@@ -206,6 +244,9 @@ struct IndexArgs {
   // n_out = 0 when absent) for its request
   int fused;
   CompressArgs comp, comp2;
+  // keys through a block table (pages.table != nullptr): KI / KI_sf are the
+  // pool, n_entries the logical entries per request
+  PageTable pages;
 };
 size_t index_topk_workspace(int batch, int n_q, int64_t n_entries, int k, int n_heads, int dim, int dt);
 // out[0..5]: entries per slice, slices per query row, cooperative selection,
@@ -244,6 +285,9 @@ struct MqaArgs {
   float q_norm_eps;
   int q_rope_dims, out_rope_dims;
   double rope_base;
+  // entries through a block table (pages.table != nullptr): `entries` is the
+  // pool, n_entries the logical entries per request
+  PageTable pages;
 };
 size_t mqa_workspace(const MqaArgs& a);
 // Whether the tensor-core attention kernel takes these arguments (the query

@@ -12,10 +12,14 @@
 // (exact-fp32 mode) and for shapes the tensor-core producer does not take;
 // indexer_tc.cu holds the tcgen05 producer for BF16 / NVFP4 inputs.
 #include "csa_internal.cuh"
+#include "sm100.cuh"
 #include "topk_select.cuh"
 #include "indexer_plan.cuh"
 
 namespace csa {
+
+CSA_DEFINE_STATUS_READER(take_status_indexer)
+
 namespace {
 
 constexpr int kNT = 512;
@@ -60,6 +64,17 @@ __global__ void __launch_bounds__(kNT) index_slice_simt_kernel(IndexArgs a, Inde
     if (p < n_valid) {
       const uint8_t* krow = kbase + e * qrb;
       const uint8_t* ksrow = ksf ? ksf + nvfp4_blocked_sf_offset(e, a.dim) : nullptr;
+      if (a.pages.table != nullptr) {
+        // through the block table: the pool row, and the scale block of the
+        // pool page holding row 128 * (e / 128)
+        const int64_t pr = pool_row(a.pages, b, e);
+        const int64_t pg = ksf ? pool_sf_page(a.pages, b, e) : 0;
+        if (pr < 0 || pg < 0) flag_status(kStatusBadPage);
+        krow = static_cast<const uint8_t*>(a.KI) + (pr < 0 ? 0 : pr) * qrb;
+        if (ksf)
+          ksrow = static_cast<const uint8_t*>(a.KI_sf) + (pg < 0 ? 0 : pg) * nvfp4_blocked_sf_bytes(128, a.dim) +
+                  nvfp4_blocked_sf_offset(e % 128, a.dim);
+      }
       float I = 0.f;
       for (int h = 0; h < a.n_heads; ++h) {
         float dot = 0.f;

@@ -583,6 +583,36 @@ __device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t 
 // and the CTA holding row a.comp.e0 (the lead) also runs the extra job
 // a.comp2 for its request.  The CTA starts the key stages before the first
 // new row, then compresses while they land, in ring stages it has not used.
+// TMA row of logical key row lr of request b: the contiguous cache, or the
+// pool row through the block table (rows at or past n_entries, never visible,
+// read pool row 0; a page outside the pool is flagged and read as row 0).
+__device__ __forceinline__ int key_tma_row(const IndexArgs& a, int b, int64_t lr) {
+  if (a.pages.table == nullptr) return (int)((int64_t)b * a.n_entries + lr);
+  if (lr >= a.n_entries) return 0;
+  const int64_t r = pool_row(a.pages, b, lr);
+  if (r < 0) {
+    flag_status(kStatusBadPage);
+    return 0;
+  }
+  return (int)r;
+}
+
+// Loads `rows` key rows of request b from logical row lr0 (a multiple of 128)
+// into dst with the map's boxes: one box of `rows` rows when contiguous, one
+// box per page (page_entries rows, which divides 128) when paged.  Boxes land
+// row_bytes * rows apart, so the smem tile is the one a single box gives.
+// half_bytes > 0: a second box column (x = 64) lands half_bytes after dst.
+__device__ __forceinline__ void load_key_rows(const IndexArgs& a, const CUtensorMap* tm, uint8_t* dst,
+                                              uint64_t* bar, int b, int64_t lr0, int rows, int row_bytes,
+                                              int half_bytes) {
+  const int step = a.pages.table == nullptr ? rows : a.pages.page_entries;
+  for (int q = 0; q < rows; q += step) {
+    const int row = key_tma_row(a, b, lr0 + q);
+    tma_load_2d(dst + q * row_bytes, tm, bar, 0, row);
+    if (half_bytes > 0) tma_load_2d(dst + half_bytes + q * row_bytes, tm, bar, 64, row);
+  }
+}
+
 template <int NQ>
 __device__ __forceinline__ bool fused_keys(const IndexArgs& a, int64_t s0, int len) {
   return NQ == 1 && a.fused && s0 < a.comp.e0 + a.comp.n_out && a.comp.e0 < s0 + len;
@@ -689,9 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_load_2d(qs + C::N * 128, &tmQ, qbar, 64, qrow);
     for (int i = 0; i < pre; ++i) {
       mbar_arrive_expect_tx(&full[i], C::K_STAGE);
-      const int row = (int)((int64_t)blockIdx.z * a.n_entries + s0 + (int64_t)i * kBM);
-      tma_load_2d(ks + i * C::K_STAGE, &tmK, &full[i], 0, row);
-      tma_load_2d(ks + i * C::K_STAGE + kAtom, &tmK, &full[i], 64, row);
+      load_key_rows(a, &tmK, ks + i * C::K_STAGE, &full[i], blockIdx.z, s0 + (int64_t)i * kBM, kBM, 128, kAtom);
     }
   }
   if (fkeys || flead)
@@ -715,10 +743,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int s = i % C::STAGES, j = i / C::STAGES;
         if (j > 0 && !mbar_wait(&empty[s], (j - 1) & 1)) break;
         mbar_arrive_expect_tx(&full[s], C::K_STAGE);
-        const int row = (int)((int64_t)c.b * a.n_entries + c.s0 + (int64_t)i * kBM);
-        uint8_t* dst = ks + s * C::K_STAGE;
-        tma_load_2d(dst, &tmK, &full[s], 0, row);
-        tma_load_2d(dst + kAtom, &tmK, &full[s], 64, row);
+        load_key_rows(a, &tmK, ks + s * C::K_STAGE, &full[s], c.b, c.s0 + (int64_t)i * kBM, kBM, 128, kAtom);
       }
       // tiles started early but beyond the visible entries: wait for their
       // bytes before the CTA moves on
@@ -828,7 +853,7 @@ __global__ void __launch_bounds__(Nvf4Cfg<NQ>::NT, 1)
       // a 256-row box: rows past the tensor read as zero, rows of the next
       // request are never valid positions here
       mbar_arrive_expect_tx(&full[g], C::TPS * C::CODES);
-      tma_load_2d(st + g * C::STAGE, &tmK, &full[g], 0, (int)((int64_t)b0 * a.n_entries + s0 + (int64_t)g * C::TPS * kBM));
+      load_key_rows(a, &tmK, st + g * C::STAGE, &full[g], b0, s0 + (int64_t)g * C::TPS * kBM, C::TPS * kBM, 64, 0);
     }
   }
   if (fkeys || flead)
@@ -854,8 +879,8 @@ __global__ void __launch_bounds__(Nvf4Cfg<NQ>::NT, 1)
         const int s = g % C::STAGES, j = g / C::STAGES;
         if (j > 0 && !mbar_wait(&empty[s], (j - 1) & 1)) break;
         mbar_arrive_expect_tx(&full[s], C::TPS * C::CODES);
-        const int row = (int)((int64_t)c.b * a.n_entries + c.s0 + (int64_t)g * C::TPS * kBM);
-        tma_load_2d(st + s * C::STAGE, &tmK, &full[s], 0, row);
+        load_key_rows(a, &tmK, st + s * C::STAGE, &full[s], c.b, c.s0 + (int64_t)g * C::TPS * kBM, C::TPS * kBM, 64,
+                      0);
       }
       // stages started early but beyond the visible entries: add the missing
       // scale-side arrival and wait for their bytes before the CTA moves on
@@ -873,6 +898,7 @@ __global__ void __launch_bounds__(Nvf4Cfg<NQ>::NT, 1)
       mbar_arrive(qsf);
       // request b's blocked key scales: 1 KB (two atoms) per 128-entry block;
       // slices start on block boundaries, so tile i is block s0/128 + i
+      // (paged: the block of the pool page holding the tile's first row)
       const uint8_t* ksf = static_cast<const uint8_t*>(a.KI_sf) +
                            (int64_t)c.b * nvfp4_blocked_sf_bytes(a.n_entries, kDI) + (c.s0 / kBM) * C::ATOMS;
       for (int g = 0; g < n_stages; ++g) {
@@ -880,8 +906,19 @@ __global__ void __launch_bounds__(Nvf4Cfg<NQ>::NT, 1)
         if (j > 0 && !mbar_wait(&empty[s], (j - 1) & 1)) break;
         const int nt = min(C::TPS, c.n_tiles - g * C::TPS);  // blocks that exist
         mbar_arrive_expect_tx(&full[s], nt * C::ATOMS);
-        bulk_load(st + s * C::STAGE + C::TPS * C::CODES, ksf + (int64_t)g * C::TPS * C::ATOMS, nt * C::ATOMS,
-                  &full[s]);
+        uint8_t* dst = st + s * C::STAGE + C::TPS * C::CODES;
+        if (a.pages.table == nullptr) {
+          bulk_load(dst, ksf + (int64_t)g * C::TPS * C::ATOMS, nt * C::ATOMS, &full[s]);
+        } else {
+          for (int h = 0; h < nt; ++h) {
+            int64_t pg = pool_sf_page(a.pages, c.b, c.s0 + (int64_t)(g * C::TPS + h) * kBM);
+            if (pg < 0) {
+              flag_status(kStatusBadPage);
+              pg = 0;
+            }
+            bulk_load(dst + h * C::ATOMS, static_cast<const uint8_t*>(a.KI_sf) + pg * C::ATOMS, C::ATOMS, &full[s]);
+          }
+        }
       }
     }
   } else if (warp == 1 || warp == 3 || warp >= 12) {
@@ -937,12 +974,23 @@ __global__ void __launch_bounds__(Nvf4Cfg<NQ>::NT, 1)
 
 // ---------------------------------------------------------------- host side
 
+// Rows of the key tensor map: every request's cache, or the pool.
+uint64_t key_map_rows(const IndexArgs& a) {
+  return a.pages.table == nullptr ? (uint64_t)a.batch * a.n_entries
+                                  : (uint64_t)a.pages.n_pages * a.pages.page_entries;
+}
+// Box height of the key map: `rows` (a stage's tiles), or one page.
+uint32_t key_box_rows(const IndexArgs& a, int rows) {
+  return a.pages.table == nullptr ? (uint32_t)rows : (uint32_t)a.pages.page_entries;
+}
+
 template <int NQ>
 cudaError_t launch_bf16(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) {
   using C = Bf16Cfg<NQ>;
   CUtensorMap tmK, tmQ;
-  const uint64_t krows = (uint64_t)a.batch * a.n_entries, qrows = (uint64_t)a.batch * a.n_q * kHI;
-  if (!make_map_2d(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.KI, krows, kDI, 64, kBM, CU_TENSOR_MAP_SWIZZLE_128B) ||
+  const uint64_t krows = key_map_rows(a), qrows = (uint64_t)a.batch * a.n_q * kHI;
+  if (!make_map_2d(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.KI, krows, kDI, 64, key_box_rows(a, kBM),
+                   CU_TENSOR_MAP_SWIZZLE_128B) ||
       !make_map_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, a.qI, qrows, kDI, 64, C::N, CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
   const size_t smem = (size_t)C::FIXED_SMEM + (size_t)C::PER_ENTRY * p.slice_len;
@@ -970,12 +1018,12 @@ template <int NQ>
 cudaError_t launch_nvf4(const IndexArgs& a, const IndexPlan& p, cudaStream_t s) {
   using C = Nvf4Cfg<NQ>;
   CUtensorMap tmK, tmQ, tmQs;
-  const uint64_t krows = (uint64_t)a.batch * a.n_entries, qrows = (uint64_t)a.batch * a.n_q * kHI;
+  const uint64_t krows = key_map_rows(a), qrows = (uint64_t)a.batch * a.n_q * kHI;
   // packed E2M1 rows of 64 bytes in the 64-byte swizzle; query scales as
   // 16-byte lines holding two head rows each (key scales are bulk-copied)
   const bool ok =
-      make_map_2d(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.KI, krows, kDI / 2, kDI / 2, C::TPS * kBM,
-                  CU_TENSOR_MAP_SWIZZLE_64B) &&
+      make_map_2d(&tmK, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.KI, krows, kDI / 2, kDI / 2,
+                  key_box_rows(a, C::TPS * kBM), CU_TENSOR_MAP_SWIZZLE_64B) &&
       make_map_2d(&tmQ, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.qI, qrows, kDI / 2, kDI / 2, C::N,
                   CU_TENSOR_MAP_SWIZZLE_64B) &&
       make_map_2d(&tmQs, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.qI_sf, qrows / 2, 16, 16, C::N / 2,

@@ -16,6 +16,9 @@
 #include "mqa_plan.cuh"
 
 namespace csa {
+
+CSA_DEFINE_STATUS_READER(take_status_mqa)
+
 namespace {
 
 constexpr int kRC = 32;  // rows per chunk (one per lane)

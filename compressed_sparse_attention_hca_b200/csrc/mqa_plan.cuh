@@ -4,6 +4,7 @@
 
 #include "csa_internal.cuh"
 #include "indexer_plan.cuh"
+#include "sm100.cuh"
 
 namespace csa {
 
@@ -42,13 +43,26 @@ __device__ __forceinline__ RowList make_row_list(const MqaArgs& a, int64_t bt, i
   return r;
 }
 
+// Address of entry e of request b (contiguous or through the block table);
+// nullptr, with the bad-page status bit set, when its page is outside the pool.
+__device__ __forceinline__ const uint8_t* entry_row(const MqaArgs& a, int b, int64_t e, int64_t rb) {
+  const uint8_t* base = static_cast<const uint8_t*>(a.entries);
+  if (a.pages.table == nullptr) return base + ((int64_t)b * a.n_entries + e) * rb;
+  const int64_t pr = pool_row(a.pages, b, e);
+  if (pr < 0) {
+    flag_status(kStatusBadPage);
+    return nullptr;
+  }
+  return base + pr * rb;
+}
+
 // Address of attended row r, or nullptr when the slot is unused / invalid.
 __device__ __forceinline__ const uint8_t* row_ptr(const MqaArgs& a, const RowList& rl, int b, int64_t r,
                                                   int64_t rb) {
   if (r < rl.n_sel) {
     const int64_t e = rl.sel ? (int64_t)rl.sel[r] : r;
     if (e < 0 || e >= rl.vis) return nullptr;
-    return static_cast<const uint8_t*>(a.entries) + ((int64_t)b * a.n_entries + e) * rb;
+    return entry_row(a, b, e, rb);
   }
   const int64_t w = rl.win_lo + (r - rl.n_sel) - a.win_start[b];
   if (w < 0 || w >= a.win_len) return nullptr;

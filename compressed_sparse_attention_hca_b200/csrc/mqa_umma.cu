@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (n_chunks > 0 && r < r_end) {
       if (r < rl.n_sel && a.idx != nullptr && r_begin == guess_begin) {
         const int64_t e = e_guess;
-        if (e >= 0 && e < rl.vis) p = static_cast<const uint8_t*>(a.entries) + ((int64_t)b * a.n_entries + e) * rb;
+        if (e >= 0 && e < rl.vis) p = entry_row(a, b, e, rb);
       } else {
         p = row_ptr(a, rl, b, r, rb);
       }

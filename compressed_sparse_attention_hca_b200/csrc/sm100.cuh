@@ -30,6 +30,11 @@ static __device__ unsigned int g_device_status = 0;
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;  // 2 s
 
+// Status bits (bit 1 is the host's "word unreadable").
+constexpr unsigned int kStatusTimeout = 1u;
+constexpr unsigned int kStatusBadPage = 4u;  // a page table named a page outside the pool
+__device__ __forceinline__ void flag_status(unsigned int bit) { atomicOr(&g_device_status, bit); }
+
 // Host: a 2D tiled tensor map over [rows][cols] elements of `esize` bytes (row
 // stride cols * esize) with boxes of box_cols x box_rows (false when the
 // driver entry point is missing or the encoder rejects the shape).
@@ -90,7 +95,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 255u) == 0 && globaltimer_ns() - t0 > kWaitTimeoutNs) {
-      atomicOr(&g_device_status, 1u);
+      flag_status(kStatusTimeout);
       return false;
     }
   }

@@ -112,6 +112,41 @@ int64_t csa_row_bytes(csa_dtype_t dt, int dim);
 int64_t csa_nvfp4_key_scale_bytes(int64_t n_rows, int dim);
 
 /*
+ * csa_pages_t -- a paged compressed cache ([P2] cache paragraph: the
+ * compressed cache is kept in fixed pages of 128 tokens, lcm(m, m') for
+ * m = 4, m' = 128, so a page holds 32 CSA entries or 1 HCA entry; [P5] 7).
+ * The rows of every request live in pages of `page_entries` rows taken from
+ * one pool shared by all requests; logical row r of request b is pool row
+ *   table[b * max_pages + r / page_entries] * page_entries + r % page_entries.
+ *   table         [batch][max_pages] int32 (device): pool page of each of the
+ *                 request's pages.  Every slot j < ceil(rows / page_entries),
+ *                 rows the call's logical rows per request, must hold a page
+ *                 in [0, n_pages).  A kernel that meets a page outside the
+ *                 pool touches no memory outside it (it drops the row, or
+ *                 reads pool page 0 in its place), the call's results are
+ *                 invalid, and csa_check_device_status reports
+ *                 CSA_ERR_INVALID_ARG.
+ *   max_pages     table row length (>= 1).
+ *   page_entries  rows per page (>= 1).
+ *   n_pages       pages in the pool (>= 1).
+ * A paged call takes the POOL in place of the contiguous cache argument
+ * (rows of the same format, n_pages * page_entries of them) and keeps its
+ * logical row count argument (n_entries: rows the table maps per request,
+ * <= max_pages * page_entries).  NVFP4 key scales of a paged key cache: one
+ * blocked 128-row block (dim/64 atoms of 512 bytes) per pool page, so the
+ * scale pool is n_pages * (dim/64) * 512 bytes; the scales of logical rows
+ * 128u .. 128u+127 are kept in the block of the pool page that holds row
+ * 128u, at the offset the contiguous layout gives row r % 128 (page_entries
+ * must divide 128).
+ */
+typedef struct {
+  const int32_t* table;
+  int max_pages;
+  int page_entries;
+  int64_t n_pages;
+} csa_pages_t;
+
+/*
  * csa_compress -- Token-Level Compressor ([P5] 1.2 Step 1; [P1] eq. 6-7;
  * HCA form [P5] 1.3, [P1] eq. 10-11).
  *
@@ -232,6 +267,20 @@ csa_status_t csa_index_topk(const void* qI, const void* qI_sf, const float* wI, 
                             void* stream);
 
 /*
+ * csa_index_topk_paged -- csa_index_topk over a paged key cache: KI (and
+ * NVFP4 KI_sf) are the pool of key_pages (csa_pages_t), n_entries the logical
+ * keys per request.  page_entries must be 8, 16, 32, 64 or 128 (a 128-token
+ * page holds 32 keys at m = 4) and the pool below 2^31 rows.  Results are
+ * those of csa_index_topk on the gathered contiguous cache; the workspace is
+ * the same.  key_pages == NULL is csa_index_topk.
+ */
+csa_status_t csa_index_topk_paged(const void* qI, const void* qI_sf, const float* wI, const void* KI,
+                                  const void* KI_sf, const csa_pages_t* key_pages, const int64_t* q_pos,
+                                  int batch, int n_q, int64_t n_entries, int m, int n_heads, int dim, int k,
+                                  csa_dtype_t dt, int32_t* idx_out, void* scores_out, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/*
  * csa_index_topk_plan -- how csa_index_topk divides the work of a call of
  * this shape on the current device (nothing is launched; for tests and
  * tuning).  out[6] receives: entries per slice, slices per query row, 1 when
@@ -258,7 +307,16 @@ typedef struct {
   void *out, *out_sf;
   int64_t out_batch_stride, out_row0;
   csa_dtype_t out_dt;
+  /* NULL, or the block table of a paged output cache: `out` (and NVFP4
+   * `out_sf`) are then the pool, out_batch_stride is ignored, and entry e0 + j
+   * goes to logical row out_row0 + j of request b's pages (csa_pages_t;
+   * NVFP4 needs page_entries dividing 128). */
+  const csa_pages_t* out_pages;
 } csa_compress_job_t;
+
+/* csa_compress with the arguments of one job (csa_compress_job_t), which may
+ * write a paged cache through out_pages. */
+csa_status_t csa_compress_ex(const csa_compress_job_t* job, int batch, void* stream);
 
 /*
  * csa_compress_index_topk -- a decode step's compressions and indexer in one
@@ -272,7 +330,10 @@ typedef struct {
  * keys->out_sf == KI_sf, keys->out_dt == dt, keys->dim == dim,
  * keys->out_batch_stride == n_entries and keys->out_row0 == keys->e0 (entry i
  * is cache row i); `extra` (e.g. the KV cache's compression) must not write
- * what the indexer reads.  With one query per request on the tensor-core
+ * what the indexer reads.  When keys->out_pages is not NULL the key cache is
+ * paged: KI / KI_sf are its pool and the indexer reads it through that table
+ * (as csa_index_topk_paged; out_batch_stride is then ignored); extra may write
+ * a paged cache of its own.  With one query per request on the tensor-core
  * indexer this is one launch: the CTA whose slice of the cache holds the new
  * key rows starts its first key copies, runs both compressions of its request
  * while they land, and then streams the rest, so the compressions add no
@@ -378,6 +439,10 @@ csa_status_t csa_sparse_mqa(const void* Q, csa_dtype_t q_dt, const void* entries
  *               output is rounded ([P5] 1.4 table: the output at position
  *               -i); 0 = none.
  *   rope_base   RoPE base for both (e.g. 10000).
+ *   entry_pages NULL, or the block table of a paged entry cache (csa_pages_t):
+ *               `entries` is then the pool of n_pages * page_entries rows and
+ *               n_entries the logical entries per request.  The window rows
+ *               (the per-request state cache) stay contiguous.
  * The normalisation and RoPE options need the tensor-core path (bf16 Q and
  * O, BF16 or KV_FP8MIX rows, dim 512, n_heads a multiple of 64) and
  * q_rope_dims, out_rope_dims multiples of 8 in [0, 64]; otherwise
@@ -390,6 +455,7 @@ typedef struct {
   int q_rope_dims;
   int out_rope_dims;
   double rope_base;
+  const csa_pages_t* entry_pages;
 } csa_mqa_options_t;
 
 /*
