@@ -258,15 +258,20 @@ class CompressJob(ctypes.Structure):
                 ("tok0", ctypes.c_int64), ("in_batch_stride", ctypes.c_int64), ("e0", ctypes.c_int64),
                 ("n_out", ctypes.c_int64), ("dim", ctypes.c_int32), ("m", ctypes.c_int32), ("in_dt", ctypes.c_int32),
                 ("out", ctypes.c_void_p), ("out_sf", ctypes.c_void_p), ("out_batch_stride", ctypes.c_int64),
-                ("out_row0", ctypes.c_int64), ("out_dt", ctypes.c_int32), ("out_pages", ctypes.POINTER(Pages))]
+                ("out_row0", ctypes.c_int64), ("out_dt", ctypes.c_int32), ("out_pages", ctypes.POINTER(Pages)),
+                ("norm_g", ctypes.c_void_p), ("norm_eps", ctypes.c_float), ("rope_dims", ctypes.c_int32),
+                ("rope_base", ctypes.c_double), ("pos_stride", ctypes.c_int64), ("pos_offset", ctypes.c_int64)]
 
 
 def compress_job(Ca, Za, Ba, m, Cb=None, Zb=None, Bb=None, *, tok0, e0, n_out, out, out_dt, out_sf=None,
-                 out_row0=None, n_tok=None, out_pages=None):
+                 out_row0=None, n_tok=None, out_pages=None, norm_g=None, norm_eps=1e-6, rope_dims=0,
+                 rope_base=10000.0, pos_stride=None, pos_offset=None):
     """A compressor call's arguments as a CompressJob (entries e0.. written to
     rows out_row0.. of `out`, out_row0 defaulting to e0; with out_pages (a
-    Pages) `out` / `out_sf` are the pool and rows are logical rows)."""
-    _need_cuda(Ca, Za, Ba, Cb, Zb, Bb, out, out_sf)
+    Pages) `out` / `out_sf` are the pool and rows are logical rows).  norm_g /
+    rope_dims: RMSNorm and RoPE of each entry before it is stored, entry i at
+    position pos_stride * i + pos_offset (default m * i + m - 1)."""
+    _need_cuda(Ca, Za, Ba, Cb, Zb, Bb, out, out_sf, norm_g)
     batch, rows, dim = Ca.shape
     job = CompressJob(
         Ca=Ca.data_ptr(), Cb=Cb.data_ptr() if Cb is not None else None, Za=Za.data_ptr(),
@@ -274,8 +279,11 @@ def compress_job(Ca, Za, Ba, m, Cb=None, Zb=None, Bb=None, *, tok0, e0, n_out, o
         n_tok=rows if n_tok is None else n_tok, tok0=tok0, in_batch_stride=rows, e0=e0, n_out=n_out, dim=dim, m=m,
         in_dt=_dt_of(Ca), out=out.data_ptr(), out_sf=out_sf.data_ptr() if out_sf is not None else None,
         out_batch_stride=out.shape[1], out_row0=e0 if out_row0 is None else out_row0, out_dt=out_dt,
-        out_pages=ctypes.pointer(out_pages) if out_pages is not None else None)
-    job._keep = out_pages  # the struct holds a raw pointer: keep the table alive with it
+        out_pages=ctypes.pointer(out_pages) if out_pages is not None else None,
+        norm_g=norm_g.data_ptr() if norm_g is not None else None, norm_eps=norm_eps, rope_dims=rope_dims,
+        rope_base=rope_base, pos_stride=m if pos_stride is None else pos_stride,
+        pos_offset=m - 1 if pos_offset is None else pos_offset)
+    job._keep = (out_pages, norm_g)  # the struct holds raw pointers: keep what they point to alive with it
     return job
 
 

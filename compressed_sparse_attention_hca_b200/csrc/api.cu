@@ -80,7 +80,7 @@ static csa_status_t check_compress(const void* Ca, const void* Cb, const void* Z
                                    int64_t in_batch_stride, int64_t e0, int64_t n_out, int dim, int m,
                                    csa_dtype_t in_dt, void* out, void* out_sf, int64_t out_batch_stride,
                                    int64_t out_row0, csa_dtype_t out_dt, const csa_pages_t* out_pages,
-                                   csa::CompressArgs* args, bool* empty) {
+                                   csa::CompressArgs* args, bool* empty, const csa_compress_job_t* epi = nullptr) {
   *empty = false;
   REQUIRE(batch >= 0 && n_tok >= 0 && tok0 >= 0 && e0 >= 0 && n_out >= 0 && out_row0 >= 0,
           "negative size (batch=%d n_tok=%lld tok0=%lld e0=%lld n_out=%lld out_row0=%lld)", batch,
@@ -131,6 +131,27 @@ static csa_status_t check_compress(const void* Ca, const void* Cb, const void* Z
   *args = csa::CompressArgs{Ca, Cb, Za, Zb, Ba, Bb, batch, n_tok, tok0, in_batch_stride, e0, n_out,
                             dim, m, (int)in_dt, (int)out_dt, out, out_sf, out_batch_stride, out_row0,
                             out_pages ? to_pages(out_pages) : csa::PageTable{nullptr, 0, 0, 0}};
+  args->norm_g = nullptr;
+  args->norm_eps = 0.f;
+  args->rope_dims = 0;
+  args->rope_base = 10000.0;
+  args->pos_stride = m;
+  args->pos_offset = m - 1;
+  if (epi != nullptr && (epi->norm_g != nullptr || epi->rope_dims != 0)) {
+    REQUIRE(epi->rope_dims >= 0 && epi->rope_dims % 8 == 0 && epi->rope_dims <= dim,
+            "rope_dims=%d must be a multiple of 8 in [0, dim=%d]", epi->rope_dims, dim);
+    REQUIRE(epi->norm_g == nullptr || epi->norm_eps >= 0.f, "norm_eps must be >= 0");
+    REQUIRE(epi->rope_dims == 0 || epi->rope_base > 0.0, "rope_base must be > 0");
+    REQUIRE(batch <= 65535, "batch=%d too large for the normalising compressor (<= 65535)", batch);
+    REQUIRE(dim <= 16384, "dim=%d too large for the normalising compressor (<= 16384)", dim);
+    REQUIRE_ALIGNED_OR_NULL(epi->norm_g);
+    args->norm_g = epi->norm_g;
+    args->norm_eps = epi->norm_eps;
+    args->rope_dims = epi->rope_dims;
+    args->rope_base = epi->rope_base;
+    args->pos_stride = epi->pos_stride;
+    args->pos_offset = epi->pos_offset;
+  }
   return ok();
 }
 
@@ -244,7 +265,7 @@ csa_status_t csa_compress_ex(const csa_compress_job_t* job, int batch, void* str
   const csa_status_t st = check_compress(job->Ca, job->Cb, job->Za, job->Zb, job->Ba, job->Bb, batch, job->n_tok,
                                          job->tok0, job->in_batch_stride, job->e0, job->n_out, job->dim, job->m,
                                          job->in_dt, job->out, job->out_sf, job->out_batch_stride, job->out_row0,
-                                         job->out_dt, job->out_pages, &a, &empty);
+                                         job->out_dt, job->out_pages, &a, &empty, job);
   if (st != CSA_OK || empty) return st;
   return cuda_status(csa::launch_compress(a, static_cast<cudaStream_t>(stream)), "csa_compress_ex");
 }
@@ -332,7 +353,7 @@ csa_status_t csa_compress_index_topk(const csa_compress_job_t* keys, const csa_c
   csa_status_t st = check_compress(keys->Ca, keys->Cb, keys->Za, keys->Zb, keys->Ba, keys->Bb, batch, keys->n_tok,
                                    keys->tok0, keys->in_batch_stride, keys->e0, keys->n_out, keys->dim, keys->m,
                                    keys->in_dt, keys->out, keys->out_sf, keys->out_batch_stride, keys->out_row0,
-                                   keys->out_dt, keys->out_pages, &c, &c_empty);
+                                   keys->out_dt, keys->out_pages, &c, &c_empty, keys);
   if (st != CSA_OK) return st;
   if (extra != nullptr) {
     REQUIRE(extra->out != KI && (extra->out_sf == nullptr || extra->out_sf != KI_sf),
@@ -340,7 +361,7 @@ csa_status_t csa_compress_index_topk(const csa_compress_job_t* keys, const csa_c
     st = check_compress(extra->Ca, extra->Cb, extra->Za, extra->Zb, extra->Ba, extra->Bb, batch, extra->n_tok,
                         extra->tok0, extra->in_batch_stride, extra->e0, extra->n_out, extra->dim, extra->m,
                         extra->in_dt, extra->out, extra->out_sf, extra->out_batch_stride, extra->out_row0,
-                        extra->out_dt, extra->out_pages, &c2, &c2_empty);
+                        extra->out_dt, extra->out_pages, &c2, &c2_empty, extra);
     if (st != CSA_OK) return st;
   }
   csa::IndexArgs a{};

@@ -9,6 +9,7 @@
 // scale block (8 lanes = 64 dims) or an FP4 block (2 lanes = 16 dims) reduce
 // their amax with warp shuffles and quantise in the epilogue.
 #include "compress_dev.cuh"
+#include "rope_dev.cuh"
 #include "sm100.cuh"
 
 namespace csa {
@@ -107,16 +108,20 @@ __host__ __device__ __forceinline__ int tokpar_smem_bytes(const CompressArgs& a)
   const int esz = a.in_dt == CSA_F32 ? 4 : 2;
   const int U = staged_positions(a);
   const int P = U < kTpChunk ? U : kTpChunk;
-  return P * kTpW * (2 * esz + 4) + 3 * 4 * kTpW * 4 + kTpW * 4;
+  const int xs = compress_row_epilogue(a) ? a.dim : kTpW;
+  return P * kTpW * (2 * esz + 4) + 3 * 4 * kTpW * 4 + xs * 4;
 }
 
 __global__ void __launch_bounds__(256) compress_tokpar_kernel(CompressArgs a) {
   extern __shared__ __align__(16) uint8_t tsm[];
   const int esz = a.in_dt == CSA_F32 ? 4 : 2;
   const int n_cg = (a.dim + kTpW - 1) / kTpW;
-  const int cg = (int)(blockIdx.x % n_cg), b = blockIdx.y;
-  const int64_t ie = blockIdx.x / n_cg, i = a.e0 + ie;
-  const int c0 = cg * kTpW, W = min(kTpW, a.dim - c0);
+  // row mode (normalisation / RoPE epilogue): the CTA owns every channel
+  // group of its entry, so the whole pooled row is in shared memory at the end
+  const bool rowm = compress_row_epilogue(a);
+  const int b = blockIdx.y;
+  const int64_t ie = rowm ? (int64_t)blockIdx.x : (int64_t)(blockIdx.x / n_cg), i = a.e0 + ie;
+  const int cg_lo = rowm ? 0 : (int)(blockIdx.x % n_cg), cg_hi = rowm ? n_cg : cg_lo + 1;
   const int U = (a.Cb != nullptr && i >= 1) ? 2 * a.m : a.m;
   const int Pmax = min(staged_positions(a), kTpChunk);
   const int P = min(U, kTpChunk);
@@ -127,72 +132,96 @@ __global__ void __launch_bounds__(256) compress_tokpar_kernel(CompressArgs a) {
   float* rmax = bs + (size_t)Pmax * kTpW;  // [4][64]
   float* rd = rmax + 4 * kTpW;             // [4][64]
   float* rs = rd + 4 * kTpW;               // [4][64]
-  float* xs = rs + 4 * kTpW;               // [64]
+  float* xs = rs + 4 * kTpW;               // [64], or [dim] in row mode
   const int w = threadIdx.x % kTpW, k = threadIdx.x / kTpW;
-  const bool ch_ok = w < W;
   const int64_t in_base = (int64_t)b * a.in_batch_stride;
 
-  // positions [u0, u0 + n) of the CTA's channels into shared memory
-  auto stage = [&](int u0, int n, bool with_c) {
-    const int p16 = W * esz / 16;
-    for (int q = threadIdx.x; q < n * p16; q += blockDim.x) {
-      const int r = q / p16, p = q % p16, u = u0 + r;
-      const bool cur = u < a.m;
-      const int64_t tok = cur ? (int64_t)a.m * i + u : (int64_t)a.m * (i - 1) + (u - a.m);
-      const int64_t off = ((in_base + tok - a.tok0) * a.dim + c0) * esz + (int64_t)p * 16;
-      stage_cp16(zs + (size_t)r * kTpW * esz + p * 16, static_cast<const uint8_t*>(cur ? a.Za : a.Zb) + off);
-      if (with_c)
-        stage_cp16(cs + (size_t)r * kTpW * esz + p * 16, static_cast<const uint8_t*>(cur ? a.Ca : a.Cb) + off);
-    }
-    const int b16 = W * 4 / 16;
-    for (int q = threadIdx.x; q < n * b16; q += blockDim.x) {
-      const int r = q / b16, p = q % b16, u = u0 + r;
-      const float* src = (u < a.m ? a.Ba + (int64_t)u * a.dim : a.Bb + (int64_t)(u - a.m) * a.dim) + c0;
-      stage_cp16(reinterpret_cast<uint8_t*>(bs + (size_t)r * kTpW) + p * 16,
-                 reinterpret_cast<const uint8_t*>(src) + p * 16);
-    }
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-    __syncthreads();
-  };
+  for (int cg = cg_lo; cg < cg_hi; ++cg) {
+    const int c0 = cg * kTpW, W = min(kTpW, a.dim - c0);
+    const bool ch_ok = w < W;
+    if (cg > cg_lo) __syncthreads();  // the previous group's staged rows are no longer read
 
-  float M = -INFINITY;  // pass 1: the max logit
-  for (int u0 = 0; u0 < U; u0 += P) {
-    const int n = min(P, U - u0);
-    if (u0 > 0) __syncthreads();
-    stage(u0, n, n_chunks == 1);
-    if (ch_ok)
-      for (int blk = k; blk * kPosBlock < n; blk += 4)
-        M = chan_max(zs + ((size_t)blk * kPosBlock * kTpW + w) * esz, bs + (size_t)blk * kPosBlock * kTpW + w,
-                     a.in_dt, kTpW, min(kPosBlock, n - blk * kPosBlock), M);
-  }
-  rmax[k * kTpW + w] = M;
-  __syncthreads();
-  M = fmaxf(fmaxf(rmax[w], rmax[kTpW + w]), fmaxf(rmax[2 * kTpW + w], rmax[3 * kTpW + w]));
-
-  float D = 0.f, S = 0.f;  // pass 2: block sums, added in block order
-  for (int u0 = 0; u0 < U; u0 += P) {
-    const int n = min(P, U - u0);
-    if (n_chunks > 1) {
-      __syncthreads();
-      stage(u0, n, true);
-    }
-    const int nb = (n + kPosBlock - 1) / kPosBlock;  // <= 4
-    float d = 0.f, s = 0.f;
-    if (ch_ok && k < nb)
-      chan_block(zs + ((size_t)k * kPosBlock * kTpW + w) * esz, cs + ((size_t)k * kPosBlock * kTpW + w) * esz,
-                 bs + (size_t)k * kPosBlock * kTpW + w, a.in_dt, kTpW, min(kPosBlock, n - k * kPosBlock), M, d, s);
-    rd[k * kTpW + w] = d;
-    rs[k * kTpW + w] = s;
-    __syncthreads();
-    if (k == 0)
-      for (int q = 0; q < nb; ++q) {
-        D += rd[q * kTpW + w];
-        S += rs[q * kTpW + w];
+    // positions [u0, u0 + n) of the CTA's channels into shared memory
+    auto stage = [&](int u0, int n, bool with_c) {
+      const int p16 = W * esz / 16;
+      for (int q = threadIdx.x; q < n * p16; q += blockDim.x) {
+        const int r = q / p16, p = q % p16, u = u0 + r;
+        const bool cur = u < a.m;
+        const int64_t tok = cur ? (int64_t)a.m * i + u : (int64_t)a.m * (i - 1) + (u - a.m);
+        const int64_t off = ((in_base + tok - a.tok0) * a.dim + c0) * esz + (int64_t)p * 16;
+        stage_cp16(zs + (size_t)r * kTpW * esz + p * 16, static_cast<const uint8_t*>(cur ? a.Za : a.Zb) + off);
+        if (with_c)
+          stage_cp16(cs + (size_t)r * kTpW * esz + p * 16, static_cast<const uint8_t*>(cur ? a.Ca : a.Cb) + off);
       }
+      const int b16 = W * 4 / 16;
+      for (int q = threadIdx.x; q < n * b16; q += blockDim.x) {
+        const int r = q / b16, p = q % b16, u = u0 + r;
+        const float* src = (u < a.m ? a.Ba + (int64_t)u * a.dim : a.Bb + (int64_t)(u - a.m) * a.dim) + c0;
+        stage_cp16(reinterpret_cast<uint8_t*>(bs + (size_t)r * kTpW) + p * 16,
+                   reinterpret_cast<const uint8_t*>(src) + p * 16);
+      }
+      asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+      __syncthreads();
+    };
+
+    float M = -INFINITY;  // pass 1: the max logit
+    for (int u0 = 0; u0 < U; u0 += P) {
+      const int n = min(P, U - u0);
+      if (u0 > 0) __syncthreads();
+      stage(u0, n, n_chunks == 1);
+      if (ch_ok)
+        for (int blk = k; blk * kPosBlock < n; blk += 4)
+          M = chan_max(zs + ((size_t)blk * kPosBlock * kTpW + w) * esz, bs + (size_t)blk * kPosBlock * kTpW + w,
+                       a.in_dt, kTpW, min(kPosBlock, n - blk * kPosBlock), M);
+    }
+    rmax[k * kTpW + w] = M;
+    __syncthreads();
+    M = fmaxf(fmaxf(rmax[w], rmax[kTpW + w]), fmaxf(rmax[2 * kTpW + w], rmax[3 * kTpW + w]));
+
+    float D = 0.f, S = 0.f;  // pass 2: block sums, added in block order
+    for (int u0 = 0; u0 < U; u0 += P) {
+      const int n = min(P, U - u0);
+      if (n_chunks > 1) {
+        __syncthreads();
+        stage(u0, n, true);
+      }
+      const int nb = (n + kPosBlock - 1) / kPosBlock;  // <= 4
+      float d = 0.f, s = 0.f;
+      if (ch_ok && k < nb)
+        chan_block(zs + ((size_t)k * kPosBlock * kTpW + w) * esz, cs + ((size_t)k * kPosBlock * kTpW + w) * esz,
+                   bs + (size_t)k * kPosBlock * kTpW + w, a.in_dt, kTpW, min(kPosBlock, n - k * kPosBlock), M, d,
+                   s);
+      rd[k * kTpW + w] = d;
+      rs[k * kTpW + w] = s;
+      __syncthreads();
+      if (k == 0)
+        for (int q = 0; q < nb; ++q) {
+          D += rd[q * kTpW + w];
+          S += rs[q * kTpW + w];
+        }
+    }
+    if (k == 0 && ch_ok) xs[(rowm ? c0 : 0) + w] = pooled_value(D, S);
   }
-  if (k == 0) xs[w] = pooled_value(D, S);
   __syncthreads();
+  if (rowm) {
+    // normalise and turn the pooled row, then 8 warps store it
+    if (threadIdx.x < 32)
+      warp_norm_rope_row(xs, a.dim, a.norm_g, a.norm_eps, a.rope_dims, a.rope_base,
+                         (double)(a.pos_stride * i + a.pos_offset), threadIdx.x);
+    __syncthreads();
+    const int nch = a.dim / 8;
+    for (int q0 = 0; q0 < nch; q0 += blockDim.x) {
+      const int ch = q0 + threadIdx.x;
+      const bool valid = ch < nch;
+      float x[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) x[q] = valid ? xs[ch * 8 + q] : 0.f;
+      store_entry(a, b, ie, valid ? ch * 8 : 0, x, valid);
+    }
+    return;
+  }
   if (threadIdx.x < 32) {
+    const int c0 = cg_lo * kTpW;
     const int lane = threadIdx.x;
     const int dl = c0 + (lane & 7) * 8;
     const bool valid = lane < 8 && dl < a.dim;
@@ -210,8 +239,9 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s) {
   if (total == 0) return cudaSuccess;
   // thread per (entry, 8 channels) when the entries alone fill the GPU and
   // each has few tokens; otherwise the token-parallel form
-  const int64_t tokpar_blocks = (int64_t)((a.dim + 63) / 64) * a.n_out;
-  if ((total >= 148 * 512 && a.m <= 8) || a.batch > 65535 || tokpar_blocks >= ((int64_t)1 << 31)) {
+  const bool rowm = compress_row_epilogue(a);  // normalisation / RoPE: a CTA per entry
+  const int64_t tokpar_blocks = rowm ? a.n_out : (int64_t)((a.dim + 63) / 64) * a.n_out;
+  if (!rowm && ((total >= 148 * 512 && a.m <= 8) || a.batch > 65535 || tokpar_blocks >= ((int64_t)1 << 31))) {
     const int threads = 256;
     const int64_t blocks = (total + threads - 1) / threads;
     compress_kernel<<<(unsigned)blocks, threads, 0, s>>>(a);

@@ -210,7 +210,18 @@ struct CompressArgs {
   // output rows through a block table (out_pages.table != nullptr): row
   // out_row0 + j of request b is logical row out_row0 + j of its pages
   PageTable out_pages;
+  // entry normalisation and partial RoPE before the entry is stored: RMSNorm
+  // weights [dim] (nullptr: none) and eps; the last rope_dims dims (0: none)
+  // turned at position pos_stride * i + pos_offset for entry i, base rope_base
+  const float* norm_g;
+  float norm_eps;
+  int rope_dims;
+  double rope_base;
+  int64_t pos_stride, pos_offset;
 };
+__host__ __device__ __forceinline__ bool compress_row_epilogue(const CompressArgs& a) {
+  return a.norm_g != nullptr || a.rope_dims > 0;
+}
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s);
 
 struct NormRopeArgs {

@@ -30,6 +30,7 @@
 #include "compress_dev.cuh"
 #include "csa_internal.cuh"
 #include "indexer_plan.cuh"
+#include "rope_dev.cuh"
 #include "sm100.cuh"
 #include "topk_select.cuh"
 
@@ -658,6 +659,23 @@ __device__ void run_fused_jobs(const IndexArgs& a, int b, int64_t s0, int len, u
     }
   }
   __syncthreads();
+  // normalisation / RoPE epilogue of the pooled rows: a warp per entry
+  const bool nk_row = compress_row_epilogue(a.comp), nx_row = nx > 0 && compress_row_epilogue(a.comp2);
+  if (nk_row || nx_row) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int e = warp; e < nk + nx; e += NT / 32) {
+      const bool key = e < nk;
+      const CompressArgs& c = key ? a.comp : a.comp2;
+      if (key ? !nk_row : !nx_row) continue;
+      const int64_t ie = key ? ik + e : e - nk;
+      uint8_t* buf = key ? scratch + (size_t)e * kb : xbuf + (size_t)(e - nk) * xb;
+      const int esz = c.in_dt == CSA_F32 ? 4 : 2;
+      float* xr = reinterpret_cast<float*>(buf + (size_t)staged_positions(c) * c.dim * (2 * esz + 4));
+      warp_norm_rope_row(xr, c.dim, c.norm_g, c.norm_eps, c.rope_dims, c.rope_base,
+                         (double)(c.pos_stride * (c.e0 + ie) + c.pos_offset), lane);
+    }
+    __syncthreads();
+  }
   // quantise and write, 8 channels per thread (whole warps: the scale blocks
   // of a row are consecutive lanes)
   const int qk = nk * (dk / 8), qx = nx * (dx / 8);

@@ -42,4 +42,46 @@ __device__ __forceinline__ void rope_turn(float& x0, float& x1, float cs, float 
   x1 = __fadd_rn(__fmul_rn(a, sn), __fmul_rn(b, cs));
 }
 
+// One warp normalises (g != nullptr) and turns the last rope_dims dims of an
+// fp32 row x[dim] in shared memory, in place, at position p, with the
+// standalone kernel's arithmetic: lane L sums the squares of chunks L, L+32,
+// ... (8 values each, fused multiply-adds in order), the xor-shuffle tree adds
+// the lanes, every value is multiplied by inv and then by g, and the pairs are
+// turned as rope_turn does.  The row is then the fp32 row csa_rmsnorm_rope
+// would write for the same input.  dim is a multiple of 8.
+__device__ __forceinline__ void warp_norm_rope_row(float* x, int dim, const float* g, float eps, int rope_dims,
+                                                   double base, double p, int lane) {
+  const int nch = dim / 8, d_rope = dim - rope_dims;
+  float inv = 1.f;
+  if (g != nullptr) {
+    float ss = 0.f;
+    for (int c = lane; c < nch; c += 32)
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ss = fmaf(x[8 * c + q], x[8 * c + q], ss);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    inv = rms_inv(ss, dim, eps);
+  }
+  for (int c = lane; c < nch; c += 32) {
+    float v[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v[q] = x[8 * c + q];
+    if (g != nullptr) {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) v[q] = __fmul_rn(__fmul_rn(v[q], inv), g[8 * c + q]);
+    }
+    if (8 * c >= d_rope) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float sn, cs;
+        rope_sincos(p, rope_theta(base, (8 * c - d_rope) / 2 + j, rope_dims), &sn, &cs);
+        rope_turn(v[2 * j], v[2 * j + 1], cs, sn);
+      }
+    }
+#pragma unroll
+    for (int q = 0; q < 8; ++q) x[8 * c + q] = v[q];
+  }
+  __syncwarp();
+}
+
 }  // namespace csa

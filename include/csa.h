@@ -312,6 +312,22 @@ typedef struct {
    * goes to logical row out_row0 + j of request b's pages (csa_pages_t;
    * NVFP4 needs page_entries dividing 128). */
   const csa_pages_t* out_pages;
+  /* Entry normalisation and partial RoPE before the entry is stored ([P5]
+   * 1.4 table: RMSNorm on the compressed KV entries, RoPE on their last 64
+   * dims).  norm_g: NULL or [dim] fp32 RMSNorm weights (x <- g * x /
+   * sqrt(mean(x^2) + norm_eps)); rope_dims: 0 or a multiple of 8 <= dim, the
+   * last rope_dims dims turned at position pos_stride * i + pos_offset for
+   * entry i (pos_stride = m, pos_offset = m - 1 puts an entry at its last
+   * token), base rope_base.  The pooled fp32 row is normalised and turned
+   * with the arithmetic of csa_rmsnorm_rope, then quantised once into out_dt,
+   * so a BF16 entry equals csa_rmsnorm_rope applied to the F32 entry and
+   * rounded.  A zero-filled tail (norm_g NULL, rope_dims 0) stores the
+   * pooled row as csa_compress does. */
+  const float* norm_g;
+  float norm_eps;
+  int rope_dims;
+  double rope_base;
+  int64_t pos_stride, pos_offset;
 } csa_compress_job_t;
 
 /* csa_compress with the arguments of one job (csa_compress_job_t), which may
