@@ -227,7 +227,7 @@ class Step:
 # dominant kernel, measured by an ncu capture of that kernel on the same
 # workload.  A change to that kernel makes the figure stale: it is then removed
 # until the next capture.
-NCU_TRAFFIC = {"csa_decode_1m_mixed": 78_227_200, "csa_decode_bf16": 138_577_920}
+NCU_TRAFFIC = {"csa_decode_1m_mixed": 77_240_000}  # 75.76 MB read + 1.48 MB written (ncu, 2 decimals)
 
 
 def max_over_ranks(x, dist, device):
@@ -448,6 +448,61 @@ def reference_arm(args):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------- grouped output projection
+
+def out_proj_bench(args):
+    """`--op out_proj`: the grouped output projection ("DeepSeek-V4 内部机制"
+    1.2 Step 3) on V4-Pro's shape (n_h = 128, c = 512, g = 16, d_g = 1024,
+    d = 7168) for `--tokens` tokens, L2 flushed before every call.  Decode
+    (few tokens) reads the weights once: HBM-bound; prefill is tensor-bound."""
+    from compressed_sparse_attention_hca_b200 import csa
+    csa.load()
+    dev = torch.device("cuda", 0)
+    s = W.OUT_PROJ_V4_PRO
+    T = args.tokens
+    O, Wg, Wo = (t.to(dev) for t in W.out_proj_inputs(W.generator(1), T, s["n_h"], s["c"], s["g"], s["d_g"],
+                                                         s["d"]))
+    ws = torch.zeros(csa.grouped_out_proj_workspace_size(T, **s), dtype=torch.uint8, device=dev)
+    Y = torch.empty(T, s["d"], dtype=torch.bfloat16, device=dev)
+    flush = l2_flush_buffer(dev)
+    for _ in range(args.warmup):
+        csa.grouped_out_proj(O, Wg, Wo, out=Y, ws=ws)
+    torch.cuda.synchronize()
+    clk = ClockSampler(0)
+    times = []
+    for _ in range(args.steps):
+        flush_l2(flush)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        csa.grouped_out_proj(O, Wg, Wo, out=Y, ws=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    clocks = clk.stop()
+    csa.check_device_status()
+    ms = statistics.mean(times)
+    peaks = load_peaks()
+    weights = (Wg.numel() + Wo.numel()) * 2
+    byts = weights + (O.numel() + Y.numel()) * 2 + 2 * T * s["g"] * s["d_g"] * 2  # + Z written and read
+    flops = 2.0 * T * (Wg.numel() + Wo.numel())
+    hbm = byts / (ms / 1e3) / 1e9
+    tfl = flops / (ms / 1e3) / 1e12
+    tensor = flops / peaks["bf16_tflops"] / 1e12 > byts / peaks["hbm_gbs"] / 1e9
+    roof = ({"bound": "tensor", "achieved": tfl, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+             "frac": tfl / peaks["bf16_tflops"]} if tensor else
+            {"bound": "hbm", "achieved": hbm, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": hbm / peaks["hbm_gbs"]})
+    roof.update({"traffic": None, "algorithmic_bytes": byts, "flops": flops, "note": f"peak {peaks['source']}"})
+    line = {"metric": "grouped output projection tokens/s (V4-Pro shape)", "value": T / (ms / 1e3),
+            "unit": "tokens/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16, fp32 accumulate",
+            "data": "synthetic",
+            "config": {"workload": f"out_proj_v4pro_T{T}", "tokens": T, **s,
+                       "l2": "flushed before every call (256 MiB write then read)"},
+            "plan": csa.grouped_out_proj_plan(T, **s), "roofline": roof, "gpu_launches": 2 * args.steps,
+            "clocks": clocks}
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ GPU side
 
 def main():
@@ -458,10 +513,16 @@ def main():
     ap.add_argument("--config", default="csa_decode_1m_mixed", choices=sorted(W.CONFIGS))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--op", default="step", choices=["step", "out_proj"],
+                    help="step: the hot-path step of --config; out_proj: the grouped output projection")
+    ap.add_argument("--tokens", type=int, default=4, help="tokens of --op out_proj")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.impl == "reference":
         reference_arm(args)
+        return
+    if args.op == "out_proj":
+        out_proj_bench(args)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
