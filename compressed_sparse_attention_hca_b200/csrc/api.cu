@@ -589,6 +589,7 @@ csa_status_t hca_dense_mqa(const void* Q, csa_dtype_t q_dt, const void* entries,
 static csa_status_t check_out_proj(int T, int n_h, int c, int g, int d_g, int d) {
   REQUIRE(T >= 0 && T <= (1 << 24), "T=%d out of range [0, 2^24]", T);
   REQUIRE(n_h >= 1 && c >= 1 && g >= 1 && n_h % g == 0, "n_h=%d must be a positive multiple of g=%d", n_h, g);
+  REQUIRE(g <= 65535, "g=%d too large (<= 65535)", g);
   REQUIRE((int64_t)(n_h / g) * c % 64 == 0 && (int64_t)n_h * c <= (1 << 20),
           "n_h/g * c = %lld must be a multiple of 64 (n_h * c <= 2^20)", (long long)(n_h / g) * c);
   REQUIRE(d_g >= 128 && d_g % 128 == 0 && (int64_t)g * d_g <= (1 << 20),

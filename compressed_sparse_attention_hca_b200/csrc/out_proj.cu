@@ -105,9 +105,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   int* last_flag = reinterpret_cast<int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tiles_n = a.Nw / kBN;
-  const int n_tile = blockIdx.x % tiles_n, split = blockIdx.x / tiles_n;
-  const int n0 = n_tile * kBN, t0 = blockIdx.y * a.nt, grp = blockIdx.z;
+  // token tiles vary fastest, so the CTAs that read one weight strip run
+  // together and the strip comes from HBM once (the token tiles, shared by
+  // every strip of a group, stay in L2)
+  const int tiles_n = a.Nw / kBN, tiles_t = (a.T + a.nt - 1) / a.nt;
+  const int t_tile = (int)(blockIdx.x % tiles_t);
+  const int n_tile = (int)((blockIdx.x / tiles_t) % tiles_n), split = (int)(blockIdx.x / tiles_t / tiles_n);
+  const int n0 = n_tile * kBN, t0 = t_tile * a.nt, grp = blockIdx.y;
   const int n_k = a.K / kBK;
   const int ks0 = (int)((int64_t)split * n_k / a.splits), ks1 = (int)((int64_t)(split + 1) * n_k / a.splits);
   const uint32_t tcols = (uint32_t)tmem_cols_for(a.nt);
@@ -169,7 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t_end = a.T - t0 < a.nt ? a.T - t0 : a.nt;
     mbar_wait(accf, 0);
     tc_fence_after();
-    const int64_t cols = (int64_t)gridDim.z * a.Nw;
+    const int64_t cols = (int64_t)gridDim.y * a.Nw;
     float* part = a.part + (int64_t)split * a.T * cols + col;
     __nv_bfloat16* y = a.Y + col;
     for (int c0 = 0; c0 < t_end; c0 += 32) {
@@ -190,7 +194,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (a.splits > 1) {
       __threadfence();
       epilogue_bar();
-      int* ticket = a.tickets + ((int64_t)blockIdx.z * gridDim.y + blockIdx.y) * tiles_n + n_tile;
+      int* ticket = a.tickets + ((int64_t)grp * tiles_t + t_tile) * tiles_n + n_tile;
       if (threadIdx.x == 64) *last_flag = atomicAdd(ticket, 1) == a.splits - 1;
       epilogue_bar();
       if (*last_flag) {
@@ -230,7 +234,7 @@ cudaError_t launch_projection(const void* W, const void* X, __nv_bfloat16* Y, in
   ProjArgs a{T, K, Nw, p.nt, p.splits, Y, (int64_t)groups * Nw, part, tickets};
   cudaError_t e = cudaFuncSetAttribute(out_proj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)p.smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)(Nw / kBN * p.splits), (unsigned)((T + p.nt - 1) / p.nt), (unsigned)groups);
+  const dim3 grid((unsigned)((int64_t)(Nw / kBN) * p.splits * ((T + p.nt - 1) / p.nt)), (unsigned)groups);
   out_proj_kernel<<<grid, kThreads, p.smem, s>>>(tmW, tmX, a);
   ++launch_counter();
   return cudaGetLastError();
