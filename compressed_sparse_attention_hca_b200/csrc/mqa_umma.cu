@@ -92,8 +92,11 @@ constexpr int kSmemBytes = 1024 + kOffMisc + (int)sizeof(Misc);
 static_assert(kOffMisc % 16 == 0, "bulk-copy sources are 16-byte aligned");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 
-// TMEM columns: S^T (64), O^T slabs 0..3 (64 each), L (64), ones (32).
+// TMEM columns: S^T over the first and the second half of the dims (64
+// each: two threads issue the two halves at once), O^T slabs 0..3 (64 each),
+// L (64), ones (32).
 constexpr int kColS = 0;
+constexpr int kColS2 = 416;
 constexpr int kColO = 64;
 constexpr int kColL = 320;
 constexpr int kColOnes = 384;
@@ -203,13 +206,17 @@ __device__ __forceinline__ uint4 expand_fp8(const uint8_t* raw, int r, int g) {
   return pack_bf16x8(f);
 }
 
-// S^T += K Q^T over atoms [at0, at1) (the first atom of a chunk overwrites).
-__device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t kva, uint32_t qa, int at0, int at1) {
+// Partial S^T += K Q^T over atoms [at0, at1) into TMEM column `col` (atom
+// `first` overwrites).  One thread issues atoms 0..3 into kColS, another
+// atoms 4..7 into kColS2: a tcgen05.mma costs its issuing thread ~0.1 us, so
+// the 32 products of a chunk are issued by two threads at once.
+__device__ __forceinline__ void issue_qk(uint32_t tmem, uint32_t col, uint32_t kva, uint32_t qa, int at0, int at1,
+                                         int first) {
   for (int at = at0; at < at1; ++at)
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      tc_mma_f16(tmem + kColS, umma_desc_sw128(kva + at * kAtom + kk * 32),
-                 umma_desc_sw128(qa + at * (kHG * 128) + kk * 32), kIdescQK, (at | kk) ? 1u : 0u);
+      tc_mma_f16(tmem + col, umma_desc_sw128(kva + at * kAtom + kk * 32),
+                 umma_desc_sw128(qa + at * (kHG * 128) + kk * 32), kIdescQK, (at != first || kk) ? 1u : 0u);
 }
 
 // The combine of a head group's splits ("DeepSeek-V4 内部机制" sink equation):
@@ -279,9 +286,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&ms.bar_raw, kRows);
     for (int i = 0; i < 2; ++i) mbar_init(&ms.bar_half[i], kThreads);
     for (int i = 0; i < 4; ++i) mbar_init(&ms.bar_pair[i], kThreads);
-    mbar_init(&ms.bar_qk, 1);
+    mbar_init(&ms.bar_qk, 2);  // the two half-S^T issuers
     for (int i = 0; i < 4; ++i) mbar_init(&ms.bar_slab[i], 1);
-    mbar_init(&ms.bar_pv, 1);
+    mbar_init(&ms.bar_pv, 5);  // the four slab issuers and the L issuer
     fence_barrier_init();
     // query tile (64 heads x 512 dims): eight TMA boxes of 64 heads x 64 dims
     // in the 128-byte swizzle, the K-major operand layout (depends on nothing)
@@ -421,7 +428,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (tid == 0) {
         mbar_wait(&ms.bar_half[0], par);
         tc_fence_after();
-        issue_qk(tmem, kva, qa, 0, 4);
+        issue_qk(tmem, kColS, kva, qa, 0, 4, 0);
+        tc_commit(&ms.bar_qk);
       }
       // dims 256..511 through registers (their destination overlaps the staging)
       uint4 hi[kHalf];
@@ -438,10 +446,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       fence_proxy_async_smem();
       mbar_arrive(&ms.bar_half[1]);
-      if (tid == 0) {
+      if (tid == 32) {
         mbar_wait(&ms.bar_half[1], par);
         tc_fence_after();
-        issue_qk(tmem, kva, qa, 4, 8);
+        issue_qk(tmem, kColS2, kva, qa, 4, 8, 4);
         tc_commit(&ms.bar_qk);
       }
     } else {
@@ -449,23 +457,30 @@ __global__ void __launch_bounds__(kThreads, 1)
         cp_async_wait_pending(3 - p);
         fence_proxy_async_smem();
         mbar_arrive(&ms.bar_pair[p]);
-        if (tid == 0) {
+        if (tid == (p < 2 ? 0 : 32)) {
           mbar_wait(&ms.bar_pair[p], par);
           tc_fence_after();
-          issue_qk(tmem, kva, qa, 2 * p, 2 * p + 2);
-          if (p == 3) tc_commit(&ms.bar_qk);
+          issue_qk(tmem, p < 2 ? kColS : kColS2, kva, qa, 2 * p, 2 * p + 2, p < 2 ? 0 : 4);
+          if (p == 1 || p == 3) tc_commit(&ms.bar_qk);
         }
       }
     }
 
     // ---- softmax: warp (quad, half) owns rows 32 quad.. and heads 32 half..
     mbar_wait(&ms.bar_qk, par);
+    // P and the O^T / L columns are rewritten below: every product of the
+    // previous chunk must have finished (its five issuers each commit to
+    // bar_pv; the FP8 path already waited for them before its gather)
+    if (!FP8 && ci > 0) mbar_wait(&ms.bar_pv, par ^ 1u);
     tc_fence_after();
     const int r = 32 * quad + lane;
     const uint32_t lane_base = (uint32_t)(32 * quad) << 16;
-    float s[32];
+    float s[32], s2[32];
     tmem_ld_32x32b_x32(tmem + lane_base + kColS + 32 * half, s);
+    tmem_ld_32x32b_x32(tmem + lane_base + kColS2 + 32 * half, s2);
     tmem_ld_wait();
+#pragma unroll
+    for (int h = 0; h < 32; ++h) s[h] += s2[h];
     const bool ok = rowp[r] != nullptr;
 #pragma unroll
     for (int h = 0; h < 32; ++h) s[h] = ok ? s[h] * sl2 : -INFINITY;
@@ -515,21 +530,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_proxy_async_smem();  // P (generic stores) -> tensor core reads
     __syncthreads();
 
-    // ---- O^T += V^T P^T (slab by slab) and L += 1 P^T
-    if (tid == 0) {
+    // ---- O^T += V^T P^T (slab sl issued by warp sl) and L += 1 P^T (warp 4):
+    // five threads issue at once (each product costs its issuer ~0.1 us)
+    if (lane == 0 && warp < 5) {
       tc_fence_after();
-#pragma unroll
-      for (int sl = 0; sl < 4; ++sl) {
+      if (warp < 4) {
+        const int sl = warp;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
           tc_mma_f16(tmem + kColO + sl * kHG, umma_desc_sw128_mn(kva + (2 * sl) * kAtom + kk * 2048, kAtom, 1024),
                      umma_desc_sw128_mn(pa + kk * 2048, kAtom, 1024), kIdescPV, (ci > 0 || kk > 0) ? 1u : 0u);
         tc_commit(&ms.bar_slab[sl]);
-      }
+      } else {
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        tc_mma_f16_ta(tmem + kColL, tmem + kColOnes, umma_desc_sw128_mn(pa + kk * 2048, kAtom, 1024), kIdescL,
-                      (ci > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_f16_ta(tmem + kColL, tmem + kColOnes, umma_desc_sw128_mn(pa + kk * 2048, kAtom, 1024), kIdescL,
+                        (ci > 0 || kk > 0) ? 1u : 0u);
+      }
       tc_commit(&ms.bar_pv);
     }
 
