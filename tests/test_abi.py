@@ -200,3 +200,45 @@ def test_grouped_out_proj_plan():
     assert sizes[-1] >= 4096 * 16 * 1024 * 2 and sizes == sorted(sizes)
     with pytest.raises(csa.CsaError):
         csa.grouped_out_proj_plan(0, **v4)
+
+
+def test_paged_calls_reject_bad_tables():
+    lib = csa.load()
+    pg = csa.Pages(table=4096, max_pages=4, page_entries=32, n_pages=100)
+
+    def index(pages, n_entries=100, dt=csa.BF16):
+        return lib.csa_index_topk_paged(A, None, A, A, None, ctypes.byref(pages) if pages else None, A, 1, 1,
+                                        n_entries, 4, 64, 128, 16, dt, A, None, A, 1 << 30, None)
+    assert index(csa.Pages(table=4096, max_pages=4, page_entries=12, n_pages=100)) == INVALID  # 12 does not divide 128
+    assert index(csa.Pages(table=4096, max_pages=4, page_entries=4, n_pages=100)) == INVALID   # below 8
+    assert index(pg, n_entries=129) == INVALID and "max_pages" in _err()                      # 129 > 4 x 32
+    assert index(csa.Pages(table=None, max_pages=4, page_entries=32, n_pages=100)) == INVALID
+    assert index(csa.Pages(table=4100, max_pages=4, page_entries=32, n_pages=100)) == INVALID  # misaligned
+    assert index(csa.Pages(table=4096, max_pages=4, page_entries=32, n_pages=0)) == INVALID
+
+    def mqa(pages):
+        opt = csa.MqaOptions(entry_pages=ctypes.pointer(pages))
+        return lib.csa_sparse_mqa_ex(A, csa.BF16, A, 100, A, 16, A, 0, A, A, 0, 4, A, 1.0, 1, 1, 64, 512,
+                                     csa.BF16, A, A, 1 << 30, ctypes.byref(opt), None)
+    assert mqa(csa.Pages(table=4096, max_pages=0, page_entries=32, n_pages=10)) == INVALID
+    assert mqa(csa.Pages(table=4096, max_pages=3, page_entries=32, n_pages=10)) == INVALID  # 100 > 96
+
+
+def test_compress_job_rejects_bad_epilogue_and_pages():
+    lib = csa.load()
+
+    def job(**kw):
+        j = csa.CompressJob(Ca=4096, Za=4096, Ba=4096, n_tok=64, tok0=0, in_batch_stride=64, e0=0, n_out=16, dim=128,
+                            m=4, in_dt=csa.F32, out=8192, out_sf=8192, out_batch_stride=16, out_row0=0,
+                            out_dt=csa.F32, rope_base=10000.0, pos_stride=4, pos_offset=3)
+        for k, v in kw.items():
+            setattr(j, k, v)
+        return lib.csa_compress_ex(ctypes.byref(j), 1, None)
+    assert job(rope_dims=12) == INVALID                       # not a multiple of 8
+    assert job(rope_dims=136) == INVALID                      # beyond dim
+    assert job(norm_g=4096, norm_eps=-1.0) == INVALID
+    assert job(rope_dims=64, rope_base=0.0) == INVALID
+    pg = csa.Pages(table=4096, max_pages=1, page_entries=48, n_pages=4)
+    assert job(out_dt=csa.IDX_NVFP4, out_pages=ctypes.pointer(pg)) == INVALID  # 48 does not divide 128
+    pg2 = csa.Pages(table=4096, max_pages=1, page_entries=8, n_pages=4)
+    assert job(out_pages=ctypes.pointer(pg2)) == INVALID      # 16 entries > 1 x 8
