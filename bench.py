@@ -111,11 +111,12 @@ class Step:
                                       device=device, dtype=torch.uint8)
         self.launches = 0
 
-    def _compress_kv(self):
+    def _kv_job(self):
+        """The step's KV-cache compression as a job (built per call: it holds
+        the tensors' current addresses)."""
         csa, x, cfg, t = self.csa, self.x, self.cfg, self.tok
-        csa.compress(t["Ca"], t["Za"], t["Ba"], cfg["m"], t["Cb"], t["Zb"], t["Bb"], tok0=self.tok0, e0=self.e0,
-                     n_out=self.n_out, out_dt=cfg["kv_dt"], out=x["entries"], out_row0=self.e0)
-        return csa.last_launch_count()
+        return csa.compress_job(t["Ca"], t["Za"], t["Ba"], cfg["m"], t["Cb"], t["Zb"], t["Bb"], tok0=self.tok0,
+                                e0=self.e0, n_out=self.n_out, out=x["entries"], out_dt=cfg["kv_dt"])
 
     def attend(self):
         csa, x, cfg = self.csa, self.x, self.cfg
@@ -124,7 +125,8 @@ class Step:
                            cfg["m"], x["sink"], self.scale, kv_dt=cfg["kv_dt"], O=self.O, ws=self.ws_mqa)
         else:
             csa.hca_dense_mqa(x["Q"], x["entries"], x["win"], x["win_start"], x["q_pos"], cfg["window"],
-                              cfg["m"], x["sink"], self.scale, kv_dt=cfg["kv_dt"], O=self.O, ws=self.ws_mqa)
+                              cfg["m"], x["sink"], self.scale, kv_dt=cfg["kv_dt"], O=self.O, ws=self.ws_mqa,
+                              options=csa.mqa_options(compress=self._kv_job()))
         return csa.last_launch_count()
 
     def compress_index(self):
@@ -147,15 +149,13 @@ class Step:
         (any of them may be None).
 
         CSA: both compressions (index key, KV entry) run inside the indexer
-        call, then attention.  HCA: KV-cache compression, then dense
-        attention."""
+        call, then attention.  HCA: one dense attention call that launches the
+        KV-cache compression first."""
         s = torch.cuda.current_stream()
         if ev and ev[0] is not None:
             ev[0].record(s)
         n = 0
         csa_kind = self.kind.startswith("csa")
-        if not csa_kind:
-            n += self._compress_kv()
         if ev and ev[1] is not None:
             ev[1].record(s)
         if csa_kind:
@@ -648,7 +648,8 @@ def main():
         "phases_ms": phases,
         "phases_note": ("index_topk includes both compressions (index key and KV entry, fused into the "
                         "indexer call), so the compress phase is empty" if kind.startswith("csa")
-                        else "compress = KV-cache compression"),
+                        else "the dense attention call launches the KV-cache compression first, so the "
+                        "compress phase is empty and attention includes it"),
         "phases_timing": "a second graph with event nodes between the phases (each node adds latency)",
         "launch": "one CUDA graph per step",
         "eager": eager,

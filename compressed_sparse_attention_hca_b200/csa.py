@@ -331,18 +331,20 @@ class MqaOptions(ctypes.Structure):
     output (at -q_pos), RoPE base, block table of a paged entry cache."""
     _fields_ = [("splits", ctypes.c_int32), ("q_norm_g", ctypes.c_void_p), ("q_norm_eps", ctypes.c_float),
                 ("q_rope_dims", ctypes.c_int32), ("out_rope_dims", ctypes.c_int32), ("rope_base", ctypes.c_double),
-                ("entry_pages", ctypes.POINTER(Pages))]
+                ("entry_pages", ctypes.POINTER(Pages)), ("compress", ctypes.POINTER(CompressJob))]
 
 
 def mqa_options(*, splits=0, q_norm_g=None, q_norm_eps=1e-6, q_rope_dims=0, out_rope_dims=0, rope_base=10000.0,
-                entry_pages=None):
+                entry_pages=None, compress=None):
     """Options of the attention calls; entry_pages: a Pages (pages()) when
-    `entries` is the pool of a paged cache."""
+    `entries` is the pool of a paged cache; compress: a CompressJob
+    (compress_job()) launched before the entries are attended."""
     _need_cuda(q_norm_g)
     o = MqaOptions(splits=splits, q_norm_g=q_norm_g.data_ptr() if q_norm_g is not None else None,
                    q_norm_eps=q_norm_eps, q_rope_dims=q_rope_dims, out_rope_dims=out_rope_dims,
-                   rope_base=rope_base, entry_pages=ctypes.pointer(entry_pages) if entry_pages is not None else None)
-    o._keep = (q_norm_g, entry_pages)  # raw pointers: keep what they point to alive with the struct
+                   rope_base=rope_base, entry_pages=ctypes.pointer(entry_pages) if entry_pages is not None else None,
+                   compress=ctypes.pointer(compress) if compress is not None else None)
+    o._keep = (q_norm_g, entry_pages, compress)  # raw pointers: keep what they point to alive with the struct
     return o
 
 
@@ -415,7 +417,7 @@ def hca_dense_mqa(Q, entries, win, win_start, q_pos, window, m, sink, scale, *, 
     E = _n_entries(entries, n_entries, options)
     need = mqa_workspace_size(B, T, H, c, E + window, q_dt, kv_dt, options)
     if ws is None or ws.numel() < need:
-        ws = torch.empty(need, device=Q.device, dtype=torch.uint8)
+        ws = torch.zeros(need, device=Q.device, dtype=torch.uint8)
     _check(load().hca_dense_mqa_ex(_ptr(Q), q_dt, _ptr(entries), E, _ptr(win), win.shape[1],
                                    _ptr(win_start), _ptr(q_pos), window, m, _ptr(sink), float(scale), B, T,
                                    H, c, kv_dt, _ptr(O), _ptr(ws), ws.numel(), _opt_ref(options), _stream()))

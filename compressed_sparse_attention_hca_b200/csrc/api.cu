@@ -414,6 +414,7 @@ csa_status_t apply_mqa_options(csa::MqaArgs& a, const csa_mqa_options_t* opt) {
   a.q_rope_dims = a.out_rope_dims = 0;
   a.rope_base = 10000.0;
   a.pages = csa::PageTable{nullptr, 0, 0, 0};
+  a.has_comp = 0;
   if (opt == nullptr) return CSA_OK;
   REQUIRE(opt->splits >= 0 && opt->splits <= 256, "splits=%d out of range [0, 256]", opt->splits);
   REQUIRE(opt->q_rope_dims >= 0 && opt->q_rope_dims <= 64 && opt->q_rope_dims % 8 == 0,
@@ -432,6 +433,16 @@ csa_status_t apply_mqa_options(csa::MqaArgs& a, const csa_mqa_options_t* opt) {
     const csa_status_t st = check_pages(opt->entry_pages, a.n_entries, "entry_pages");
     if (st != CSA_OK) return st;
     a.pages = to_pages(opt->entry_pages);
+  }
+  if (opt->compress != nullptr) {
+    const csa_compress_job_t* j = opt->compress;
+    bool empty = false;
+    const csa_status_t st = check_compress(j->Ca, j->Cb, j->Za, j->Zb, j->Ba, j->Bb, a.batch, j->n_tok, j->tok0,
+                                           j->in_batch_stride, j->e0, j->n_out, j->dim, j->m, j->in_dt, j->out,
+                                           j->out_sf, j->out_batch_stride, j->out_row0, j->out_dt, j->out_pages,
+                                           &a.comp, &empty, j);
+    if (st != CSA_OK) return st;
+    a.has_comp = empty ? 0 : 1;
   }
   return CSA_OK;
 }

@@ -299,6 +299,9 @@ struct MqaArgs {
   // entries through a block table (pages.table != nullptr): `entries` is the
   // pool, n_entries the logical entries per request
   PageTable pages;
+  // the step's entry compression (has_comp), launched before the attention
+  int has_comp;
+  CompressArgs comp;
 };
 size_t mqa_workspace(const MqaArgs& a);
 // Whether the tensor-core attention kernel takes these arguments (the query

@@ -347,6 +347,11 @@ size_t mqa_workspace(const MqaArgs& a) {
 }
 
 cudaError_t launch_mqa(const MqaArgs& a, cudaStream_t s) {
+  if (a.has_comp) {
+    // the step's entry compression first, on the same stream
+    const cudaError_t e = launch_compress(a.comp, s);
+    if (e != cudaSuccess) return e;
+  }
   if ((int64_t)a.batch * a.n_q == 0) return cudaSuccess;
   if (mqa_umma_path(a)) return launch_mqa_umma(a, mqa_umma_plan(a), s);
   return launch_mqa_simt(a, make_simt_mqa_plan(a), s);

@@ -459,6 +459,11 @@ csa_status_t csa_sparse_mqa(const void* Q, csa_dtype_t q_dt, const void* entries
  *               `entries` is then the pool of n_pages * page_entries rows and
  *               n_entries the logical entries per request.  The window rows
  *               (the per-request state cache) stay contiguous.
+ *   compress    NULL, or the step's entry compression ([P5] 1.3: the closed
+ *               block of m' tokens becomes the newest HCA entry), launched on
+ *               the same stream before the attention: one call for an HCA
+ *               decode step, the same results as csa_compress_ex(job)
+ *               followed by the attention call.
  * The normalisation and RoPE options need the tensor-core path (bf16 Q and
  * O, BF16 or KV_FP8MIX rows, dim 512, n_heads a multiple of 64) and
  * q_rope_dims, out_rope_dims multiples of 8 in [0, 64]; otherwise
@@ -472,6 +477,7 @@ typedef struct {
   int out_rope_dims;
   double rope_base;
   const csa_pages_t* entry_pages;
+  const csa_compress_job_t* compress;
 } csa_mqa_options_t;
 
 /*
