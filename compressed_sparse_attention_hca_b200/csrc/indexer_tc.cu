@@ -61,7 +61,9 @@ struct Bf16Cfg {
   static_assert(NBUF % 2 == 0, "one epilogue group per buffer");
   static constexpr int TMEM_COLS = 512;
   static constexpr int NT = kThreads;
-  static constexpr int HIST = NQ == 1 ? kPrefixBins * 4 : 0;  // prefix histogram (cooperative select)
+  // prefix histogram: the cooperative select's (NQ 1), or one per query with
+  // two 16-bit counts per word for the one-slice select (NQ 2)
+  static constexpr int HIST = NQ == 1 ? kPrefixBins * 4 : NQ * kPrefixBins * 2;
   static constexpr int FIXED_SMEM = 1024 + STAGES * K_STAGE + Q_BYTES + NQ * kHI * 4 + 1024 /*barriers*/ +
                                     (int)sizeof(SelectSmem<NT>) + HIST;
   // shared memory per slice entry: NQ keys (the cooperative select's
@@ -143,7 +145,7 @@ __device__ __forceinline__ SliceCtx<NQ> slice_ctx(const IndexArgs& a, const Inde
 template <int NQ, int N, int NBUF>
 __device__ __forceinline__ void epilogue_group(const SliceCtx<NQ>& c, const IndexArgs& a, const IndexPlan& plan,
                                                uint32_t tmem, uint64_t* accf, uint64_t* acce, const float* wsm,
-                                               uint16_t* keys, bool coop, uint32_t* hist) {
+                                               uint16_t* keys, bool coop, uint32_t* hist, bool hist2 = false) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int quarter = warp & 3, g = (warp - 4) >> 2;
   const int r = quarter * 32 + lane;
@@ -182,6 +184,7 @@ __device__ __forceinline__ void epilogue_group(const SliceCtx<NQ>& c, const Inde
       const bool valid = pos < c.n_valid[q];
       keys[q * plan.slice_len + pos] = valid ? (uint16_t)(key >> 16) : (uint16_t)0;
       if (coop && valid) atomicAdd(&hist[key >> 20], 1u);
+      if (hist2 && valid) atomicAdd(&hist[q * (kPrefixBins / 2) + (key >> 21)], ((key >> 20) & 1u) ? 0x10000u : 1u);
       if (a.scores_out != nullptr && pos < c.len && c.t0 + q < a.n_q) {
         const float sc = valid ? key_to_f32(key) : -INFINITY;
         static_cast<__nv_bfloat16*>(a.scores_out)[((int64_t)c.b * a.n_q + c.t0 + q) * a.n_entries + c.s0 + pos] =
@@ -206,9 +209,13 @@ __device__ __forceinline__ void scores_tail(const SliceCtx<NQ>& c, const IndexAr
 // Selection by one CTA over its own slice: final indices when it holds the
 // whole row, else the slice's top k as candidates (and its k-th key) for the
 // merge kernel.
+template <int NT>
+__device__ void hist_select(const uint16_t* kq, const uint32_t* h2, uint16_t* cand, int nv, int kk, int64_t s0,
+                            int32_t* out, SelectSmem<NT>& sm);
+
 template <int NQ, int NT>
 __device__ void slice_select(const SliceCtx<NQ>& c, const IndexArgs& a, const IndexPlan& plan, const uint16_t* keys,
-                             SelectSmem<NT>& sel) {
+                             SelectSmem<NT>& sel, const uint32_t* hist2 = nullptr, uint16_t* cand = nullptr) {
   for (int q = 0; q < NQ; ++q) {
     const int t = c.t0 + q;
     if (t >= a.n_q) break;
@@ -219,7 +226,10 @@ __device__ void slice_select(const SliceCtx<NQ>& c, const IndexArgs& a, const In
     auto key_at = [&](int i) { return ((uint32_t)kq[i]) << 16; };
     if (plan.n_slices == 1) {
       int32_t* out = a.idx_out + bt * a.k;
-      block_select<NT>(key_at, nv, kk, 0, sel, [&](int slot, int pos) { out[slot] = (int32_t)(c.s0 + pos); });
+      if (hist2 != nullptr && kk < nv)
+        hist_select<NT>(kq, hist2 + q * (kPrefixBins / 2), cand, nv, kk, c.s0, out, sel);
+      else
+        block_select<NT>(key_at, nv, kk, 0, sel, [&](int slot, int pos) { out[slot] = (int32_t)(c.s0 + pos); });
       for (int j = kk + threadIdx.x; j < a.k; j += NT) out[j] = -1;
     } else {
       const int64_t off = slice_cand_offset(plan, c.sl, c.vis[q], a.n_entries, a.k);
@@ -584,6 +594,128 @@ __device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t 
 // and the CTA holding row a.comp.e0 (the lead) also runs the extra job
 // a.comp2 for its request.  The CTA starts the key stages before the first
 // new row, then compresses while they land, in ring stages it has not used.
+// One query's top k from its whole row in one CTA, with the 12-bit prefix
+// histogram the epilogue built while the keys streamed (two 16-bit counts per
+// word: bin d in half d & 1 of word d >> 1): the prefix d1 of the k-th key
+// from the histogram, one pass over the keys that counts those above d1,
+// histograms the 4-bit suffixes of those at d1 and keeps both as candidates,
+// then the k-th key T and the ordered write over the candidates.  The same
+// order as block_select: (key desc, position asc).  kk < nv.
+template <int NT>
+__device__ void hist_select(const uint16_t* kq, const uint32_t* h2, uint16_t* cand, int nv, int kk, int64_t s0,
+                            int32_t* out, SelectSmem<NT>& sm) {
+  constexpr int NW = NT / 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, tid = threadIdx.x;
+  const unsigned lt = (1u << lane) - 1u;
+  uint32_t total;
+  // 1. prefix d1 of the kk-th key and the keys still needed inside it (warp 0
+  //    walks the bins down, 32 at a time)
+  if (warp == 0) {
+    uint32_t above = 0;
+    bool found = false;
+    for (int base = kPrefixBins - 1; base >= 0 && !found; base -= 32) {
+      const int d = base - lane;
+      const uint32_t c = d >= 0 ? (h2[d >> 1] >> (16 * (d & 1))) & 0xFFFFu : 0u;
+      uint32_t inc = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += y;
+      }
+      const unsigned hit = __ballot_sync(0xffffffffu, above + inc >= (uint32_t)kk);
+      if (hit) {
+        const int l = __ffs(hit) - 1;
+        if (lane == l) {
+          sm.bcast[0] = (uint32_t)d;
+          sm.bcast[1] = (uint32_t)kk - (above + inc - c);
+        }
+        found = true;
+      } else {
+        above += __shfl_sync(0xffffffffu, inc, 31);
+      }
+    }
+  }
+  if (tid < 16) sm.hist[tid] = 0;
+  __syncthreads();
+  const uint32_t d1 = sm.bcast[0], rem1 = sm.bcast[1];
+  // 2. candidates (prefix >= d1) of the warp's span, in order; keys above d1
+  //    counted, suffixes at d1 histogrammed.  A lane reads 8 keys per step.
+  const int span = ((nv + NW - 1) / NW + 255) / 256 * 256;
+  const int w0 = min(nv, warp * span), w1 = min(nv, w0 + span);
+  uint32_t n_cand = 0;
+  for (int base = w0; base < w1; base += 256) {
+    const int p0 = base + 8 * lane;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (p0 < w1) v = *reinterpret_cast<const uint4*>(kq + p0);
+    const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+    uint32_t cmask = 0;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const uint32_t k16 = (wv[j >> 1] >> (16 * (j & 1))) & 0xFFFFu;
+      const bool in = p0 + j < w1 && (k16 >> 4) >= d1;
+      cmask |= in ? (1u << j) : 0u;
+      if (in && (k16 >> 4) == d1) atomicAdd(&sm.hist[k16 & 15u], 1u);
+    }
+    const uint32_t cnt = __popc(cmask);
+    uint32_t inc = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += y;
+    }
+    uint32_t at = (uint32_t)w0 + n_cand + inc - cnt;
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+      if (cmask & (1u << j)) cand[at++] = (uint16_t)(p0 + j);
+    n_cand += __shfl_sync(0xffffffffu, inc, 31);
+  }
+  __syncthreads();  // the suffix histogram is complete
+  // 3. the kk-th key T = (d1 << 4) | d2 and how many keys equal to T to take
+  if (tid == 0) {
+    uint32_t above = 0;
+    for (int n = 15; n >= 0; --n) {
+      if (above + sm.hist[n] >= rem1) {
+        sm.bcast[2] = (uint32_t)n;
+        sm.bcast[3] = rem1 - above;
+        break;
+      }
+      above += sm.hist[n];
+    }
+  }
+  __syncthreads();
+  const uint32_t T = (d1 << 4) | sm.bcast[2];
+  const int need_eq = (int)sm.bcast[3];
+  // 4. per-warp counts over the candidates, offsets, ordered write
+  const uint16_t* cw = cand + w0;
+  uint32_t c_gt = 0, c_eq = 0;
+  for (int base = 0; base < (int)n_cand; base += 32) {
+    const int j = base + lane;
+    const uint32_t k16 = j < (int)n_cand ? kq[cw[j]] : 0u;
+    c_gt += __popc(__ballot_sync(0xffffffffu, j < (int)n_cand && k16 > T));
+    c_eq += __popc(__ballot_sync(0xffffffffu, j < (int)n_cand && k16 == T));
+  }
+  const uint32_t eq_before_w =
+      __shfl_sync(0xffffffffu, block_exclusive_scan<NT>(lane == 0 ? c_eq : 0u, sm.warp_tot, &total), 0);
+  int eq_take_w = need_eq - (int)eq_before_w;
+  eq_take_w = eq_take_w < 0 ? 0 : (eq_take_w > (int)c_eq ? (int)c_eq : eq_take_w);
+  uint32_t o = block_exclusive_scan<NT>(lane == 0 ? c_gt + (uint32_t)eq_take_w : 0u, sm.warp_tot, &total);
+  o = __shfl_sync(0xffffffffu, o, 0);
+  int eq_seen = 0;
+  for (int base = 0; base < (int)n_cand; base += 32) {
+    const int j = base + lane;
+    const bool in = j < (int)n_cand;
+    const int p = in ? cw[j] : 0;
+    const uint32_t k16 = in ? kq[p] : 0u;
+    const unsigned eqm = __ballot_sync(0xffffffffu, in && k16 == T);
+    const bool take = in && (k16 > T || (k16 == T && eq_seen + __popc(eqm & lt) < eq_take_w));
+    const unsigned tm = __ballot_sync(0xffffffffu, take);
+    if (take) out[o + __popc(tm & lt)] = (int32_t)(s0 + p);
+    o += __popc(tm);
+    eq_seen += __popc(eqm);
+  }
+  __syncthreads();  // cand and the histogram are reused by the next query
+}
+
 // TMA row of logical key row lr of request b: the contiguous cache, or the
 // pool row through the block table (rows at or past n_entries, never visible,
 // read pool row 0; a page outside the pool is flagged and read as row 0).
@@ -714,10 +846,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* qbar = acce + C::NBUF;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qbar + 1);
   SelectSmem<kThreads>& sel = *reinterpret_cast<SelectSmem<kThreads>*>(tmem_slot + 4);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(&sel + 1);  // [kPrefixBins] (cooperative select only)
+  uint32_t* hist = reinterpret_cast<uint32_t*>(&sel + 1);  // prefix histogram(s) (HIST bytes)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool coop = NQ == 1 && plan.coop;
+  const bool h2 = NQ == 2 && plan.n_slices == 1;  // one-slice rows select from the epilogue's histograms
   // The queries and the first key tiles do not depend on the query
   // positions: the producer thread starts them before anything is loaded.
   const int64_t s0 = (int64_t)blockIdx.x * plan.slice_len;
@@ -749,6 +882,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (coop)
     for (int i = threadIdx.x; i < kPrefixBins; i += kThreads) hist[i] = 0;
+  if (h2)
+    for (int i = threadIdx.x; i < NQ * kPrefixBins / 2; i += kThreads) hist[i] = 0;
   if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
   tc_fence_before();
   __syncthreads();
@@ -790,7 +925,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= 4) {
-    epilogue_group<NQ, C::N, C::NBUF>(c, a, plan, tmem, accf, acce, wsm, keys, coop, hist);
+    epilogue_group<NQ, C::N, C::NBUF>(c, a, plan, tmem, accf, acce, wsm, keys, coop, hist, h2);
   }
   scores_tail<NQ, kThreads>(c, a);
   tc_fence_before();
@@ -800,7 +935,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                           sel);
     __syncthreads();
   } else {
-    slice_select<NQ, kThreads>(c, a, plan, keys, sel);
+    slice_select<NQ, kThreads>(c, a, plan, keys, sel, h2 ? hist : nullptr, cand);
   }
   if (warp == 1) {
     tc_fence_after();
@@ -842,7 +977,7 @@ __global__ void __launch_bounds__(Nvf4Cfg<NQ>::NT, 1)
   uint64_t* qsf = qbar + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qsf + 1);
   SelectSmem<C::NT>& sel = *reinterpret_cast<SelectSmem<C::NT>*>(tmem_slot + 4);
-  uint32_t* hist = reinterpret_cast<uint32_t*>(&sel + 1);  // [kPrefixBins] (cooperative select only)
+  uint32_t* hist = reinterpret_cast<uint32_t*>(&sel + 1);  // prefix histogram(s) (HIST bytes)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const bool coop = NQ == 1 && plan.coop;
