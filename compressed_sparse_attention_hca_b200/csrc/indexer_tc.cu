@@ -14,17 +14,20 @@
 //     kk).  Key scales are stored in HBM in exactly that layout, so each
 //     tile's two atoms arrive by one 1 KB bulk copy; the query's row-major
 //     scales are permuted once per CTA.
-// Warp roles: 0 TMA producer; 1 TMEM owner and MMA issuer (NVFP4: even
-// tiles, warp 3 the odd ones); 2 query scale atoms (NVFP4); 4-7 and 8-11 two
-// epilogue groups.  The accumulator has NBUF TMEM buffers so that the MMAs
+// Warp roles: 0 TMA producer; 1 TMEM owner and MMA issuer with further
+// issuers taking every other (BF16: warp 2) or every fourth (NVFP4 decode:
+// warps 3, 12, 13) tile, since a tcgen05.mma costs its issuing thread about as
+// long as a tile's data takes to stream; 2 query scale atoms (NVFP4); 4-7 and
+// 8-11 two epilogue groups.  The accumulator has NBUF TMEM buffers so that the MMAs
 // run several tiles ahead of the epilogue; epilogue group g drains the tiles
 // i with i % 2 == g: each thread owns one entry row
 // (one TMEM lane), reads its 64 head scores per query, forms
 // sum_h w_h relu(s_h), rounds to bf16 and stores the 16-bit order key in
 // shared memory.  After the last tile the CTA selects on those keys (the score
 // row never reaches HBM): alone when it holds the whole row, cooperatively
-// with the other slices of the row (NVFP4 decode), or by writing candidates
-// for the merge kernel.
+// with the other slices of the row (decode), or by writing candidates for the
+// merge kernel.  A whole row of several queries (prefill) selects from
+// per-query 12-bit prefix histograms the epilogue builds during the stream.
 #include <cudaTypedefs.h>
 
 #include "compress_dev.cuh"
@@ -58,7 +61,7 @@ struct Bf16Cfg {
   static constexpr int Q_BYTES = N * 2 * kDI;             // two atoms of N rows x 128 B
   static constexpr int K_STAGE = kBM * 2 * kDI;           // two atoms of 128 rows x 128 B
   static constexpr int NBUF = 512 / N;                    // 8 (NQ 1) or 4 (NQ 2)
-  static_assert(NBUF % 2 == 0, "one epilogue group per buffer");
+  static_assert(NBUF % 2 == 0, "one epilogue group and one MMA issuer per buffer");
   static constexpr int TMEM_COLS = 512;
   static constexpr int NT = kThreads;
   // prefix histogram: the cooperative select's (NQ 1), or one per query with
@@ -902,11 +905,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       // bytes before the CTA moves on
       for (int i = c.n_tiles; i < pre; ++i) mbar_wait(&full[i], 0);
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 2) {
+    // MMA issuers: warp 1 issues the even tiles, warp 2 the odd ones (eight
+    // tcgen05.mma per tile cost one issuing thread about as long as the
+    // tile's data takes to stream).  NBUF is even, so a buffer always belongs
+    // to the same issuer and each issuer waits on every phase of its
+    // barriers in order; a stage's uses alternate issuers, but a stage is
+    // refilled only after its previous use committed, so no phase is missed.
     if (lane == 0) {
+      const int w = warp - 1;
       bool ok = mbar_wait(qbar, 0);
       const uint32_t qa = smem_u32(qs);
-      for (int i = 0; ok && i < c.n_tiles; ++i) {
+      for (int i = w; ok && i < c.n_tiles; i += 2) {
         const int s = i % C::STAGES, j = i / C::STAGES, buf = i % C::NBUF, u = i / C::NBUF;
         if (!mbar_wait(&full[s], j & 1)) break;
         if (u > 0 && !mbar_wait(&acce[buf], (u - 1) & 1)) break;
