@@ -31,8 +31,8 @@
 // together with the query position.
 //
 // Rows split over several CTAs (decode: few queries) give partials
-// (max, sum, o) per split, staged in shared memory and written by bulk
-// copies; a combine kernel (a CTA per query and head, all of a thread's split
+// (max, sum, o) per split, o stored from the registers that load it from
+// TMEM; a combine kernel (a CTA per query and head, all of a thread's split
 // operands loaded at once) adds them in split order with the sink.  With a
 // fixed split count (an option) the split boundaries depend only on the
 // query's rows: a request's output then does not depend on the batch it runs
@@ -608,8 +608,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int h = 0; h < kHG; ++h) o[h] = 0.f;
     }
     const int d = sl * 128 + 32 * quad + lane;
+    if constexpr (MODE == kMqaWhole) {
 #pragma unroll
-    for (int h = 0; h < kHG; ++h) stg[h * kDim + d] = o[h];
+      for (int h = 0; h < kHG; ++h) stg[h * kDim + d] = o[h];
+    } else {
+      // a split's partial goes straight from the registers to global memory:
+      // lane = dim, so a warp stores 128 contiguous bytes per head (the
+      // combine reads it from L2)
+      float* po = plan_partial_o(plan, a, bt, split, hg * kHG) + d;
+#pragma unroll
+      for (int h = 0; h < kHG; ++h) po[(int64_t)h * kDim] = o[h];
+    }
   }
   fence_proxy_async_smem();  // the staging is read by bulk copies
   tc_fence_before();
@@ -660,18 +669,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       bulk_wait_read();  // the shared memory may go once the copy has read it
     }
   } else {
-    // one split of several: the unnormalised partial (m, l, o) for the
-    // combine kernel; o leaves the staging by bulk copies of 8 heads (16 KB)
+    // one split of several: the unnormalised partial's statistics (m, l)
+    // for the combine kernel (o was stored above)
     if (tid < kHG) {
       float* ml = plan_partial_ml(plan, a, bt, split, hg * kHG + tid);
       const float m = ms.m_use[tid];
       ml[0] = m == -INFINITY ? -INFINITY : m / kLog2e;  // natural-log domain
       ml[1] = ms.lsum[tid];
-    }
-    if (tid < kHG / 8) {
-      bulk_store(plan_partial_o(plan, a, bt, split, hg * kHG + 8 * tid), stg + 8 * tid * kDim, 8 * kDim * 4);
-      bulk_commit();
-      bulk_wait_read();  // the next kernel sees the writes; the shared memory may go once read
     }
   }
 }
