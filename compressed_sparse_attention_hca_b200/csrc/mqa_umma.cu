@@ -31,9 +31,10 @@
 // together with the query position.
 //
 // Rows split over several CTAs (decode: few queries) give partials
-// (max, sum, o) per split, o stored from the registers that load it from
-// TMEM; a combine kernel (a CTA per query and head, all of a thread's split
-// operands loaded at once) adds them in split order with the sink.  With a
+// (max, sum, o) per split, o stored as bf16 from the registers that load it
+// from TMEM; a combine kernel (a CTA per query and four heads, all of a
+// thread's split operands loaded at once) adds them in split order with the
+// sink.  With a
 // fixed split count (an option) the split boundaries depend only on the
 // query's rows: a request's output then does not depend on the batch it runs
 // in.  (Measured alternatives, removed: the splits meeting on a global
@@ -262,6 +263,18 @@ __device__ __forceinline__ void rope_tables(const MqaArgs& a, int64_t t, float* 
   if (k < a.q_rope_dims / 2) rope_sincos((double)t, rope_theta(a.rope_base, k, a.q_rope_dims), &qsn[k], &qcs[k]);
   if (k < a.out_rope_dims / 2)
     rope_sincos((double)t * -1.0, rope_theta(a.rope_base, k, a.out_rope_dims), &osn[k], &ocs[k]);
+}
+
+// Split partials of this kernel: o of (query bt, split s) as [head quad][512
+// dims][4 heads] bf16 (unnormalised, rounded once from the fp32 TMEM
+// accumulator; four heads of a dim side by side so a thread stores them at
+// once), then (m, l) per head in fp32.  The o region is sized for fp32 rows
+// (the split-KV workspace layout shared with the SIMT kernel); this kernel
+// uses its first half.
+__host__ __device__ __forceinline__ __nv_bfloat16* quad_partial_o(const MqaPlan& p, const MqaArgs& a, int64_t bt,
+                                                                  int s, int hq) {
+  return reinterpret_cast<__nv_bfloat16*>(plan_partials(p, a)) +
+         (((bt * p.n_splits + s) * (a.n_heads / 4)) + hq) * (int64_t)a.dim * 4;
 }
 
 template <bool FP8, int MODE>
@@ -612,12 +625,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int h = 0; h < kHG; ++h) stg[h * kDim + d] = o[h];
     } else {
-      // a split's partial goes straight from the registers to global memory:
-      // lane = dim, so a warp stores 128 contiguous bytes per head (the
-      // combine reads it from L2)
-      float* po = plan_partial_o(plan, a, bt, split, hg * kHG) + d;
+      // a split's partial o goes straight from the registers to global
+      // memory as bf16, four heads interleaved per dim (lane = dim: a warp
+      // stores 256 contiguous bytes per head quad; the combine reads it from
+      // L2)
+      __nv_bfloat16* po = quad_partial_o(plan, a, bt, split, hg * (kHG / 4)) + 4 * d;
 #pragma unroll
-      for (int h = 0; h < kHG; ++h) po[(int64_t)h * kDim] = o[h];
+      for (int q = 0; q < kHG / 4; ++q) {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(o[4 * q], o[4 * q + 1]);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(o[4 * q + 2], o[4 * q + 3]);
+        uint2 pk;
+        memcpy(&pk.x, &lo, 4);
+        memcpy(&pk.y, &hi, 4);
+        *reinterpret_cast<uint2*>(po + (int64_t)q * kDim * 4) = pk;
+      }
     }
   }
   fence_proxy_async_smem();  // the staging is read by bulk copies
@@ -680,56 +701,63 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// The combine of kMqaSplit mode: one CTA per (head, query), a thread per 4
-// dims; the splits' statistics go through shared memory once, and each
-// thread's partials are loaded 16 splits at a time, all in flight together.
-constexpr int kCombineThreads = 128;
+// The combine of kMqaSplit mode: one CTA per (head quad, query), a thread
+// per 2 dims of the four heads; the splits' statistics go through shared
+// memory once, and each thread's partials (16 bytes per split) are loaded 16
+// splits at a time, all in flight together.
+constexpr int kCombineThreads = 256;
 constexpr int kLoadSplits = 16;
 __global__ void __launch_bounds__(kCombineThreads) mqa_umma_combine_kernel(MqaArgs a, MqaPlan plan) {
-  __shared__ float2 mls[kMaxSplits];
-  __shared__ float W[kMaxSplits];
+  __shared__ float2 mls[4][kMaxSplits];
+  __shared__ float W[4][kMaxSplits];
   __shared__ float ocs[kMaxRope / 2], osn[kMaxRope / 2], qcs[kMaxRope / 2], qsn[kMaxRope / 2];
-  const int h = blockIdx.x;
+  const int hq = blockIdx.x;
   const int64_t bt = blockIdx.y;
   const int S = plan.n_splits, tid = threadIdx.x;
   if (tid < 32) rope_tables(a, a.q_pos[bt], qcs, qsn, ocs, osn);
-  for (int j = tid; j < S; j += kCombineThreads)
-    mls[j] = __ldcg(reinterpret_cast<const float2*>(plan_partial_ml(plan, a, bt, j, h)));
-  // this thread's 4 dims of the first (up to) 16 splits, loaded while the
-  // weights are formed
-  const int d0 = 4 * tid;
-  float4 x[kLoadSplits];
+  for (int u = tid; u < 4 * S; u += kCombineThreads)
+    mls[u & 3][u >> 2] = __ldcg(reinterpret_cast<const float2*>(plan_partial_ml(plan, a, bt, u >> 2, 4 * hq + (u & 3))));
+  // this thread's dims d0, d0 + 1 (four heads each, 16 bytes) of the first
+  // (up to) 16 splits, loaded while the weights are formed
+  const int d0 = 2 * tid;
+  uint4 x[kLoadSplits];
 #pragma unroll
   for (int u = 0; u < kLoadSplits; ++u)
-    if (u < S) x[u] = __ldcg(reinterpret_cast<const float4*>(plan_partial_o(plan, a, bt, u, h) + d0));
+    if (u < S) x[u] = __ldcg(reinterpret_cast<const uint4*>(quad_partial_o(plan, a, bt, u, hq) + 4 * d0));
   __syncthreads();
-  if (tid == 0) combine_weights<0>(S, a.sink[h], [&](int j) { return mls[j]; }, W, 1);
+  if (tid < 4) combine_weights<0>(S, a.sink[4 * hq + tid], [&](int j) { return mls[tid][j]; }, W[tid], 1);
   __syncthreads();
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  float acc[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
   for (int j0 = 0; j0 < S; j0 += kLoadSplits) {
     if (j0 > 0) {
 #pragma unroll
       for (int u = 0; u < kLoadSplits; ++u)
-        if (j0 + u < S) x[u] = __ldcg(reinterpret_cast<const float4*>(plan_partial_o(plan, a, bt, j0 + u, h) + d0));
+        if (j0 + u < S) x[u] = __ldcg(reinterpret_cast<const uint4*>(quad_partial_o(plan, a, bt, j0 + u, hq) + 4 * d0));
     }
 #pragma unroll
     for (int u = 0; u < kLoadSplits; ++u) {
       if (j0 + u >= S) break;
-      const float w = W[j0 + u];
-      acc[0] = fmaf(w, x[u].x, acc[0]); acc[1] = fmaf(w, x[u].y, acc[1]);
-      acc[2] = fmaf(w, x[u].z, acc[2]); acc[3] = fmaf(w, x[u].w, acc[3]);
+      // x[u]: (d0, heads 0 1), (d0, heads 2 3), (d0 + 1, heads 0 1), (d0 + 1, heads 2 3)
+      const uint32_t wv[4] = {x[u].x, x[u].y, x[u].z, x[u].w};
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t w = wv[2 * e + (i >> 1)];
+          const float v = __uint_as_float((i & 1) ? (w & 0xFFFF0000u) : (w << 16));
+          acc[i][e] = fmaf(W[i][j0 + u], v, acc[i][e]);
+        }
     }
   }
   const int d_rope = kDim - a.out_rope_dims;
-  if (a.out_rope_dims > 0 && d0 >= d_rope) {
-    rope_turn(acc[0], acc[1], ocs[(d0 - d_rope) / 2], osn[(d0 - d_rope) / 2]);
-    rope_turn(acc[2], acc[3], ocs[(d0 - d_rope) / 2 + 1], osn[(d0 - d_rope) / 2 + 1]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    if (a.out_rope_dims > 0 && d0 >= d_rope)
+      rope_turn(acc[i][0], acc[i][1], ocs[(d0 - d_rope) / 2], osn[(d0 - d_rope) / 2]);
+    const __nv_bfloat162 v = __floats2bfloat162_rn(acc[i][0], acc[i][1]);
+    *reinterpret_cast<__nv_bfloat162*>(static_cast<__nv_bfloat16*>(a.O) + (bt * a.n_heads + 4 * hq + i) * kDim + d0) =
+        v;
   }
-  const __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]), hi = __floats2bfloat162_rn(acc[2], acc[3]);
-  uint2 pk;
-  memcpy(&pk.x, &lo, 4);
-  memcpy(&pk.y, &hi, 4);
-  *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.O) + (bt * a.n_heads + h) * kDim + d0) = pk;
 }
 
 int sm_count_mqa() {
@@ -786,7 +814,7 @@ cudaError_t launch_umma(const MqaArgs& a, const MqaPlan& p, cudaStream_t s) {
   ++launch_counter();
   e = cudaGetLastError();
   if (e != cudaSuccess || MODE != kMqaSplit) return e;
-  mqa_umma_combine_kernel<<<dim3(a.n_heads, (unsigned)((int64_t)a.batch * a.n_q)), kCombineThreads, 0, s>>>(a, p);
+  mqa_umma_combine_kernel<<<dim3(a.n_heads / 4, (unsigned)((int64_t)a.batch * a.n_q)), kCombineThreads, 0, s>>>(a, p);
   ++launch_counter();
   return cudaGetLastError();
 }
