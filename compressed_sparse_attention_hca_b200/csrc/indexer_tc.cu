@@ -512,22 +512,12 @@ __device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t 
     }
   }
   __syncthreads();
-  // Every slot has arrived, so every CTA of the row is past step 1: the
-  // workspace goes back to zeros for the next call.  This CTA clears its
-  // share of the prefix histogram; the last CTA to get here (all others have
-  // read every slot by then) clears the slots and the counters.
-  for (int d = sl * kPrefixBins / S + tid; d < (sl + 1) * kPrefixBins / S; d += NT) H[d] = 0u;
-  if (tid == 0) sm.bcast[2] = atomicAdd(ctr + 2, 1u) == (uint32_t)S - 1 ? 1u : 0u;
-  __syncthreads();
-  if (sm.bcast[2]) {
-    for (int i = tid; i < S * kSlotWords; i += NT) slots[i] = 0u;
-    if (tid == 0) {
-      ctr[0] = 0u;
-      ctr[1] = 0u;  // the row's highest prefix
-      ctr[2] = 0u;
-    }
-  }
-  __syncthreads();
+  // Every slot has arrived, so every CTA of the row is past step 1 and the
+  // workspace can go back to zeros (after the write below).  The ticket that
+  // finds the last CTA is taken now and read at the end, so its round trip
+  // overlaps the write.
+  uint32_t ticket = 0;
+  if (tid == 0) ticket = atomicAdd(ctr + 2, 1u);
   if (tid == 0) {
     uint32_t above = 0;
     for (int n = 15; n >= 0; --n) {
@@ -587,6 +577,21 @@ __device__ void coop_select(const uint16_t* kq, uint16_t* cand, int nv, int64_t 
     if (take) out[o + __popc(tm & lt)] = (int32_t)(s0 + p);
     o += __popc(tm);
     eq_seen += __popc(eqm);
+  }
+
+  // 5. the workspace back to zeros: this CTA's share of the prefix
+  //    histogram; the last CTA to take a ticket (every other has read every
+  //    slot by then) clears the slots and the counters
+  for (int d = sl * kPrefixBins / S + tid; d < (sl + 1) * kPrefixBins / S; d += NT) H[d] = 0u;
+  if (tid == 0) sm.hist[65] = ticket == (uint32_t)S - 1 ? 1u : 0u;
+  __syncthreads();
+  if (sm.hist[65]) {
+    for (int i = tid; i < S * kSlotWords; i += NT) slots[i] = 0u;
+    if (tid == 0) {
+      ctr[0] = 0u;
+      ctr[1] = 0u;  // the row's highest prefix
+      ctr[2] = 0u;
+    }
   }
 }
 
