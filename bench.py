@@ -227,8 +227,8 @@ class Step:
 # dominant kernel, measured by an ncu capture of that kernel on the same
 # workload.  A change to that kernel makes the figure stale: it is then removed
 # until the next capture.
-NCU_TRAFFIC = {"csa_decode_1m_mixed": 77_240_000,   # 75.76 MB read + 1.48 MB written (ncu, 2 decimals)
-               "csa_decode_bf16": 138_160_000}      # 134.98 MB read + 3.18 MB written
+NCU_TRAFFIC = {"csa_decode_1m_mixed": 77_410_000,   # 75.76 MB read + 1.65 MB written (ncu, 2 decimals)
+               "csa_decode_bf16": 135_100_000}      # 134.97 MB read + 0.13 MB written
 
 
 def max_over_ranks(x, dist, device):
